@@ -1,0 +1,123 @@
+"""Paged-attention oracle — TEST INFRASTRUCTURE ONLY.
+
+A ctypes wrapper around ``pa_oracle.cpp``: a plain, slow, single-threaded fp64
+C++ restatement of the KV-cache write and of paged decode attention, written
+from the pages' description of PagedAttention (see the header of
+``pa_oracle.cpp`` for the page titles and sections it follows).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+may import this module.  It does not import the product package, and the
+product package does not import it.  Arrays cross as torch CPU tensors (bf16
+has no numpy dtype); this module does argument marshalling only.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pa_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# Element type codes of the oracle (its own numbering, same meaning as the
+# library's: 0 fp32, 1 fp16, 2 bf16).
+DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+
+ERRORS = {0: "ok", 1: "bad argument", 2: "block id out of range",
+          3: "context length out of range", 4: "slot out of range"}
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def build(src: str = _SRC, out: str = _LIB, force: bool = False) -> str:
+    """Compile the oracle with g++ (-O2, no fast-math: IEEE fp64 throughout)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.run(["g++", "-O2", "-std=c++17", "-fno-fast-math", "-ffp-contract=off",
+                    "-shared", "-fPIC", "-o", tmp, src], check=True)
+    os.replace(tmp, out)
+    return out
+
+
+class Oracle:
+    """One loaded copy of the oracle library (tests may load planted-mistake
+    variants built from a modified copy of the source)."""
+
+    def __init__(self, path: str | None = None):
+        self.path = path or build()
+        lib = ctypes.CDLL(self.path)
+        c = ctypes
+        lib.oracle_reshape_and_cache.restype = c.c_int
+        lib.oracle_reshape_and_cache.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64,
+            c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int]
+        decode_args = [c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                       c.c_float, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
+                       c.c_int64, c.c_int, c.c_void_p, c.c_int]
+        lib.oracle_decode.restype = c.c_int
+        lib.oracle_decode.argtypes = decode_args
+        lib.oracle_decode_partitioned.restype = c.c_int
+        lib.oracle_decode_partitioned.argtypes = decode_args + [c.c_int]
+        lib.oracle_pool_index.restype = c.c_int64
+        lib.oracle_pool_index.argtypes = [c.c_int64, c.c_int, c.c_int, c.c_int, c.c_int,
+                                          c.c_int, c.c_int, c.c_int]
+        self.lib = lib
+
+    @staticmethod
+    def _check(rc: int):
+        if rc != 0:
+            raise OracleError(f"oracle returned {rc}: {ERRORS.get(rc, 'unknown')}")
+
+    def reshape_and_cache(self, key, value, k_cache, v_cache, slot_mapping, block_size):
+        """In-place write of key/value [T, Hkv, D] into the CPU pools."""
+        for t in (key, value, k_cache, v_cache):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        slots = slot_mapping.to(torch.int64).contiguous()
+        T, Hkv, D = key.shape
+        num_blocks = k_cache.shape[0]
+        self._check(self.lib.oracle_reshape_and_cache(
+            key.data_ptr(), value.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            slots.data_ptr(), T, Hkv, D, block_size, num_blocks, DTYPE_CODE[key.dtype]))
+
+    def decode(self, q, k_cache, v_cache, block_tables, context_lens, scale, block_size,
+               num_kv_heads, seqs=None, partition_size=None) -> np.ndarray:
+        """fp64 attention output [len(seqs) or S, Hq, D] as a numpy array."""
+        for t in (q, k_cache, v_cache):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        bt = block_tables.to(torch.int32).contiguous()
+        cl = context_lens.to(torch.int32).contiguous()
+        S, Hq, D = q.shape
+        n = S if seqs is None else len(seqs)
+        out = np.zeros((n, Hq, D), dtype=np.float64)
+        sel = None if seqs is None else np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        args = [out.ctypes.data, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                bt.data_ptr(), cl.data_ptr(), float(scale), block_size, S, Hq, num_kv_heads, D,
+                bt.shape[1], k_cache.shape[0], DTYPE_CODE[q.dtype],
+                None if sel is None else sel.ctypes.data, n]
+        if partition_size is None:
+            self._check(self.lib.oracle_decode(*args))
+        else:
+            self._check(self.lib.oracle_decode_partitioned(*args, int(partition_size)))
+        return out
+
+    def pool_index(self, block, head, token, dim, num_kv_heads, block_size, head_dim, dtype):
+        return int(self.lib.oracle_pool_index(block, head, token, dim, num_kv_heads,
+                                              block_size, head_dim, DTYPE_CODE[dtype]))
+
+
+_default: Oracle | None = None
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

@@ -1,0 +1,336 @@
+"""Pins for the oracle: checks against things other than the oracle itself —
+hand-derived golden values, closed forms, exact special cases, invariants the
+pages fix, long-double brute force on tiny inputs, and library routines for the
+number formats.  Each pin takes an ``oracle.Oracle`` so the same suite can be
+run against copies of the oracle with planted mistakes (test_oracle_mutants).
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import workloads
+from pagedutil import (as_f64, brute_force, logical_kv, materialize_shared, permute_physical,
+                       rel_err, relayout_block_size)
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _decode(orc, b, **kw):
+    return orc.decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale,
+                      b.block_size, b.num_kv_heads, **kw)
+
+
+def _empty_batch(dtype, lens, Hq, Hkv, D, B, N, tables, scale=1.0):
+    x = workloads.vec_elems(dtype)
+    S = len(lens)
+    return workloads.Batch(
+        name="hand", dtype=dtype, num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+        block_size=B, num_blocks=N, scale=scale,
+        context_lens=torch.tensor(lens, dtype=torch.int32),
+        block_tables=torch.tensor(tables, dtype=torch.int32),
+        q=torch.zeros((S, Hq, D), dtype=dtype),
+        k_cache=torch.zeros((N, Hkv, D // x, B, x), dtype=dtype),
+        v_cache=torch.zeros((N, Hkv, D // x, B, x), dtype=dtype),
+        new_key=torch.zeros((0, Hkv, D), dtype=dtype), new_value=torch.zeros((0, Hkv, D), dtype=dtype),
+        slot_mapping=torch.zeros((0,), dtype=torch.int64))
+
+
+# ---------------------------------------------------------------------------- layout & slots
+
+def pin_layout_golden(orc):
+    """Hand-derived element offsets of the pool layout; the oracle's reshape
+    must put a written element exactly there and touch nothing else."""
+    for c in _golden("pool_layout.json")["cases"]:
+        dt = DT[c["dtype"]]
+        Hkv, B, D = c["Hkv"], c["B"], c["D"]
+        assert orc.pool_index(c["b"], c["h"], c["t"], c["d"], Hkv, B, D, dt) == c["index"], c
+        x = workloads.vec_elems(dt)
+        N = c["b"] + 1
+        k = torch.zeros((N, Hkv, D // x, B, x), dtype=dt)
+        v = torch.zeros_like(k)
+        key = torch.zeros((1, Hkv, D), dtype=dt)
+        key[0, c["h"], c["d"]] = 3.0
+        val = torch.zeros_like(key)
+        val[0, c["h"], c["d"]] = -5.0
+        orc.reshape_and_cache(key, val, k, v, torch.tensor([c["b"] * B + c["t"]]), B)
+        kf, vf = k.reshape(-1), v.reshape(-1)
+        nz = torch.nonzero(kf).flatten().tolist()
+        assert nz == [c["index"]], (c, nz)
+        assert float(kf[c["index"]]) == 3.0 and float(vf[c["index"]]) == -5.0
+        assert torch.nonzero(vf).flatten().tolist() == [c["index"]]
+
+
+def pin_slot_golden(orc):
+    """The append_token walkthrough: the generator's decode slots and the
+    oracle's gather both follow slot = table[p // B] * B + p % B."""
+    g = _golden("slot_mapping.json")
+    B, row = g["block_size"], g["block_table_row"]
+    for p, want in zip(g["positions"], g["slots"]):
+        tables = np.array([row], dtype=np.int32)
+        assert int(workloads._decode_slots(tables, [p + 1], B)[0]) == want
+    for n, want in zip(g["appended"], g["blocks_in_use"]):
+        assert (n + B - 1) // B == want
+    # Needle through the oracle: write a marked token at the golden slot with
+    # the oracle's reshape, then decode must fetch it at that logical position.
+    D, N = 8, 16
+    for p, slot in zip(g["positions"], g["slots"]):
+        b = _empty_batch(torch.float32, [p + 1], 1, 1, D, B, N, [row], scale=1.0)
+        key = torch.zeros((1, 1, D)); key[0, 0, 0] = 64.0
+        val = torch.arange(1, D + 1, dtype=torch.float32).reshape(1, 1, D) * (p + 1)
+        orc.reshape_and_cache(key, val, b.k_cache, b.v_cache, torch.tensor([slot]), B)
+        b.q[0, 0, 0] = 64.0
+        out = _decode(orc, b)
+        assert np.array_equal(out[0, 0], val[0, 0].double().numpy()), (p, out[0, 0])
+
+
+# ---------------------------------------------------------------------------- attention
+
+def _tiny_cases():
+    cases = []
+    for seed, (dt, B, lens, Hq, Hkv, D) in enumerate([
+        (torch.float32, 1, (3, 1, 7), 1, 1, 8),
+        (torch.float32, 2, (5, 4, 0, 9), 4, 2, 16),
+        (torch.float32, 16, (1, 17, 33, 40), 4, 4, 64),
+        (torch.bfloat16, 8, (40, 3, 12), 8, 2, 16),
+        (torch.float16, 16, (2, 31, 16), 8, 1, 64),
+        (torch.bfloat16, 16, (1, 25), 4, 1, 128),
+        (torch.float16, 8, (9, 40, 16, 1), 8, 8, 8),
+    ]):
+        cases.append(workloads.random_small(seed=seed, dtype=dt, lens=lens, num_q_heads=Hq,
+                                            num_kv_heads=Hkv, head_dim=D, block_size=B,
+                                            extra_blocks=5))
+    return cases
+
+
+def pin_brute_force(orc):
+    """Oracle vs long-double dense attention over the logical K/V (numpy view of
+    the layout), tiny inputs: <= 1e-12 relative."""
+    for b in _tiny_cases():
+        got = _decode(orc, b)
+        ref = brute_force(b)
+        assert rel_err(got, ref) <= 1e-12, (b.name, rel_err(got, ref))
+
+
+def pin_dense_equality(orc):
+    """Dense K/V written into a shuffled paged pool with the oracle's own
+    reshape (slot by slot), vs the same K/V as one contiguous block per
+    sequence: bit-identical outputs, and equal to brute force."""
+    rng = np.random.default_rng(7)
+    S, Hq, Hkv, D, B = 3, 4, 2, 16, 8
+    lens = [13, 1, 24]
+    dt = torch.bfloat16
+    dense_k = [torch.randn(L, Hkv, D).to(dt) for L in lens]
+    dense_v = [torch.randn(L, Hkv, D).to(dt) for L in lens]
+    q = torch.randn(S, Hq, D).to(dt)
+    # paged
+    nblk = [(L + B - 1) // B for L in lens]
+    N = sum(nblk) + 4
+    ids = rng.permutation(N)
+    tables = np.full((S, max(nblk)), -1, dtype=np.int32)
+    cur = 0
+    for s in range(S):
+        tables[s, :nblk[s]] = ids[cur:cur + nblk[s]]
+        cur += nblk[s]
+    paged = _empty_batch(dt, lens, Hq, Hkv, D, B, N, tables, scale=0.25)
+    paged.q.copy_(q)
+    for s in range(S):
+        slots = torch.tensor([int(tables[s, t // B]) * B + t % B for t in range(lens[s])])
+        orc.reshape_and_cache(dense_k[s].contiguous(), dense_v[s].contiguous(), paged.k_cache,
+                              paged.v_cache, slots, B)
+    # contiguous: block size = longest context, block s holds sequence s
+    Bc = 24
+    cont = _empty_batch(dt, lens, Hq, Hkv, D, Bc, S, [[s] for s in range(S)], scale=0.25)
+    cont.q.copy_(q)
+    for s in range(S):
+        orc.reshape_and_cache(dense_k[s].contiguous(), dense_v[s].contiguous(), cont.k_cache,
+                              cont.v_cache, torch.arange(lens[s]) + s * Bc, Bc)
+    a, c = _decode(orc, paged), _decode(orc, cont)
+    assert np.array_equal(a, c)
+    # and the dense definition, straight from the dense arrays
+    for s in range(S):
+        for h in range(Hq):
+            kvh = h // (Hq // Hkv)
+            K = as_f64(dense_k[s][:, kvh]).astype(np.longdouble)
+            V = as_f64(dense_v[s][:, kvh]).astype(np.longdouble)
+            z = np.longdouble(0.25) * (K @ as_f64(q[s, h]).astype(np.longdouble))
+            w = np.exp(z - z.max())
+            ref = (w[:, None] * V).sum(0) / w.sum()
+            assert np.max(np.abs(a[s, h] - ref.astype(np.float64))) <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def pin_permutation_invariance(orc):
+    for b in _tiny_cases()[2:5]:
+        assert np.array_equal(_decode(orc, b), _decode(orc, permute_physical(b, seed=11)))
+
+
+def pin_block_size_invariance(orc):
+    b = workloads.random_small(seed=21, dtype=torch.float16, lens=(70, 1, 33, 16), num_q_heads=8,
+                               num_kv_heads=2, head_dim=64, block_size=16)
+    ref = _decode(orc, b)
+    for nb in (8, 32):
+        assert np.array_equal(ref, _decode(orc, relayout_block_size(b, nb)))
+
+
+def pin_shared_vs_copied(orc):
+    for prefix in (32, 40):  # 40: the prefix ends inside a block (copy-on-write block)
+        b = workloads.prefix_sharing(seed=3, prefix_len=prefix, num_seqs=3, suffix_range=(1, 20))
+        twin = materialize_shared(b)
+        assert twin.num_blocks > b.num_blocks
+        assert np.array_equal(_decode(orc, b), _decode(orc, twin))
+
+
+def pin_closed_forms(orc):
+    # L = 1: the output is V[0] exactly.
+    b = workloads.random_small(seed=31, dtype=torch.bfloat16, lens=(1, 1, 1), num_q_heads=4,
+                               num_kv_heads=2, head_dim=16, block_size=8)
+    out = _decode(orc, b)
+    for s in range(3):
+        for h in range(4):
+            _, V = logical_kv(b, s, h // 2)
+            assert np.array_equal(out[s, h], V[0])
+    # q = 0: uniform weights, the output is the mean of V over the context.
+    b = workloads.random_small(seed=32, dtype=torch.float32, lens=(5, 12, 33), num_q_heads=2,
+                               num_kv_heads=1, head_dim=8, block_size=8)
+    b.q.zero_()
+    out = _decode(orc, b)
+    for s in range(3):
+        _, V = logical_kv(b, s, 0)
+        assert np.max(np.abs(out[s, 0] - V.mean(axis=0))) <= 1e-14
+    # two tokens with scores 0 and 1: logistic weights (golden).
+    g = _golden("two_token_logistic.json")
+    D = g["head_dim"]
+    tb = _empty_batch(torch.float32, [2], 1, 1, D, 16, 1, [[0]], scale=g["scale"])
+    tb.q[0, 0] = torch.tensor(g["q"], dtype=torch.float32)
+    orc.reshape_and_cache(torch.tensor(g["keys"], dtype=torch.float32).reshape(2, 1, D),
+                          torch.tensor(g["values"], dtype=torch.float32).reshape(2, 1, D),
+                          tb.k_cache, tb.v_cache, torch.tensor([0, 1]), 16)
+    out = _decode(orc, tb)
+    assert np.max(np.abs(out[0, 0] - np.array(g["out"]))) <= g["abs_tol"], out[0, 0]
+    # empty context: zeros.
+    b = workloads.random_small(seed=33, dtype=torch.float16, lens=(0, 4), num_q_heads=2,
+                               num_kv_heads=1, head_dim=8, block_size=8)
+    out = _decode(orc, b)
+    assert np.array_equal(out[0], np.zeros_like(out[0])) and np.any(out[1] != 0)
+
+
+def pin_needle(orc):
+    """q and one key aligned with score 4096 at position t*: every other weight
+    is exp(-4096) = 0 in fp64, so the output is V[t*] exactly.  The needle sits
+    in one kv head only; the other head's queries see no needle."""
+    b = workloads.random_small(seed=41, dtype=torch.bfloat16, lens=(37, 8, 1), num_q_heads=4,
+                               num_kv_heads=2, head_dim=16, block_size=8)
+    b.scale = 1.0
+    B = b.block_size
+    for s in range(b.num_seqs):
+        for t in range(int(b.context_lens[s])):
+            c = permute_physical(b, seed=t)  # fresh copy
+            c.k_cache.zero_()
+            c.q.zero_()
+            c.q[s, 0:2, 0] = 64.0                      # q heads 0,1 -> kv head 0
+            blk = int(c.block_tables[s, t // B])
+            c.k_cache[blk, 0, 0, t % B, 0] = 64.0      # dim 0 of token t, kv head 0
+            out = _decode(orc, c, seqs=[s])
+            _, V = logical_kv(c, s, 0)
+            assert np.array_equal(out[0, 0], V[t]) and np.array_equal(out[0, 1], V[t]), (s, t)
+            _, V1 = logical_kv(c, s, 1)
+            assert np.max(np.abs(out[0, 2] - V1.mean(axis=0))) <= 1e-14   # no needle in head 1
+
+
+def pin_partitioned(orc):
+    """Partition + log-sum-exp merge (fp64) equals the plain definition."""
+    for b in _tiny_cases():
+        plain = _decode(orc, b)
+        for part in (1, 3, 8, 16, 512):
+            got = _decode(orc, b, partition_size=part)
+            assert rel_err(got, plain) <= 1e-13, (b.name, part)
+
+
+def pin_reshape_scatter(orc):
+    """Reshape vs an independent numpy scatter through the 5-D pool view;
+    untouched bytes stay as they were; padding slots (-1) write nothing."""
+    for dt, B, D in ((torch.bfloat16, 16, 128), (torch.float32, 8, 64), (torch.float16, 32, 64)):
+        b = workloads.random_small(seed=51, dtype=dt, lens=(20, 5), num_q_heads=4, num_kv_heads=2,
+                                   head_dim=D, block_size=B, extra_blocks=4, new_tokens=12)
+        k0, v0 = b.k_cache.clone(), b.v_cache.clone()
+        orc.reshape_and_cache(b.new_key, b.new_value, b.k_cache, b.v_cache, b.slot_mapping, B)
+        x = workloads.vec_elems(dt)
+        for i, slot in enumerate(b.slot_mapping.tolist()):
+            if slot < 0:
+                continue
+            k0[slot // B, :, :, slot % B, :] = b.new_key[i].reshape(b.num_kv_heads, D // x, x)
+            v0[slot // B, :, :, slot % B, :] = b.new_value[i].reshape(b.num_kv_heads, D // x, x)
+        kb = k0.view(-1).view(torch.int16 if dt != torch.float32 else torch.int32)
+        gb = b.k_cache.view(-1).view(kb.dtype)
+        assert torch.equal(kb, gb) and torch.equal(
+            v0.view(-1).view(kb.dtype), b.v_cache.view(-1).view(kb.dtype))
+
+
+def pin_errors(orc):
+    from oracle import OracleError
+    b = workloads.random_small(seed=61, dtype=torch.float16, lens=(9, 3), num_q_heads=2,
+                               num_kv_heads=1, head_dim=8, block_size=8)
+    bad = b.block_tables.clone()
+    bad[0, 1] = b.num_blocks          # out of range
+    for tables, lens, code in ((bad, b.context_lens, "block id"),
+                               (b.block_tables, torch.tensor([9, 100], dtype=torch.int32), "context")):
+        try:
+            orc.decode(b.q, b.k_cache, b.v_cache, tables, lens, b.scale, 8, 1)
+        except OracleError as e:
+            assert code in str(e)
+        else:
+            raise AssertionError("oracle accepted bad input")
+    try:
+        orc.reshape_and_cache(b.new_key, b.new_value, b.k_cache, b.v_cache,
+                              torch.tensor([b.num_blocks * 8] * b.new_key.shape[0]), 8)
+    except OracleError as e:
+        assert "slot" in str(e)
+    else:
+        raise AssertionError("oracle accepted a slot past the pool")
+
+
+def pin_number_formats(orc):
+    """Every fp16 and bf16 bit pattern, and a sample of fp32 patterns, widen
+    exactly: L = 1 with q = 0 returns V[0] itself; compared with numpy's
+    float16 and torch's bfloat16 conversions to float64."""
+    D = 64
+    for dt in (torch.float16, torch.bfloat16):
+        bits = torch.arange(-32768, 32768, dtype=torch.int32).to(torch.int16)
+        vals = bits.view(dt)
+        S = vals.numel() // D
+        x = workloads.vec_elems(dt)
+        b = _empty_batch(dt, [1] * S, 1, 1, D, 8, S, [[s] for s in range(S)])
+        rows = vals.reshape(S, D)
+        orc.reshape_and_cache(torch.zeros((S, 1, D), dtype=dt), rows.reshape(S, 1, D).contiguous(),
+                              b.k_cache, b.v_cache, torch.arange(S) * 8, 8)
+        out = _decode(orc, b)[:, 0]
+        if dt == torch.float16:
+            ref = rows.numpy().view(np.float16).astype(np.float64)
+        else:
+            ref = rows.to(torch.float64).numpy()
+        np.testing.assert_array_equal(out, ref)
+    rng = np.random.default_rng(5)
+    f32 = rng.integers(0, 2**32, size=64 * D, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    f32 = np.where(np.isfinite(f32), f32, 0).astype(np.float32)
+    S = f32.size // D
+    b = _empty_batch(torch.float32, [1] * S, 1, 1, D, 8, S, [[s] for s in range(S)])
+    rows = torch.from_numpy(f32.reshape(S, 1, D).copy())
+    orc.reshape_and_cache(torch.zeros_like(rows), rows, b.k_cache, b.v_cache, torch.arange(S) * 8, 8)
+    np.testing.assert_array_equal(_decode(orc, b)[:, 0], f32.reshape(S, D).astype(np.float64))
+
+
+PINS = [pin_layout_golden, pin_slot_golden, pin_brute_force, pin_dense_equality,
+        pin_permutation_invariance, pin_block_size_invariance, pin_shared_vs_copied,
+        pin_closed_forms, pin_needle, pin_partitioned, pin_reshape_scatter, pin_errors,
+        pin_number_formats]

@@ -1,0 +1,175 @@
+"""Test-side helpers: an independent numpy formulation of the pool layout (used
+to read logical K/V and to build twin pools), a long-double brute-force
+attention, and the tolerance checks.  Nothing here is imported by the product
+or by the oracle."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import workloads
+
+
+def as_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def logical_kv(batch, s: int, kvh: int):
+    """Logical K, V of (sequence s, kv head kvh) as fp64 [L, D], read through the
+    block table with numpy indexing of the 5-D pool view [N, Hkv, D/x, B, x]."""
+    B, D = batch.block_size, batch.head_dim
+    L = int(batch.context_lens[s])
+    kc = batch.k_cache.detach().cpu()
+    vc = batch.v_cache.detach().cpu()
+    K = np.zeros((L, D))
+    V = np.zeros((L, D))
+    for t in range(L):
+        blk = int(batch.block_tables[s, t // B])
+        K[t] = as_f64(kc[blk, kvh, :, t % B, :].reshape(D))
+        V[t] = as_f64(vc[blk, kvh, :, t % B, :].reshape(D))
+    return K, V
+
+
+def brute_force(batch, seqs=None) -> np.ndarray:
+    """Dense softmax(scale q K^T) V per (seq, q head) over the logical K/V, in
+    numpy long double, normalising after the weighted sum."""
+    S, Hq, D, g = batch.num_seqs, batch.num_q_heads, batch.head_dim, batch.group
+    seqs = list(range(S)) if seqs is None else list(seqs)
+    q = as_f64(batch.q)
+    out = np.zeros((len(seqs), Hq, D), dtype=np.float64)
+    scale = np.longdouble(np.float32(batch.scale))
+    for i, s in enumerate(seqs):
+        for kvh in range(batch.num_kv_heads):
+            K, V = logical_kv(batch, s, kvh)
+            if K.shape[0] == 0:
+                continue
+            Kl, Vl = K.astype(np.longdouble), V.astype(np.longdouble)
+            for j in range(g):
+                h = kvh * g + j
+                z = scale * (Kl @ q[s, h].astype(np.longdouble))
+                w = np.exp(z - z.max())
+                out[i, h] = ((w[:, None] * Vl).sum(axis=0) / w.sum()).astype(np.float64)
+    return out
+
+
+def rel_err(got: np.ndarray, ref: np.ndarray) -> float:
+    scale = max(1e-300, float(np.max(np.abs(ref))) if ref.size else 1.0)
+    return float(np.max(np.abs(got - ref))) / scale if ref.size else 0.0
+
+
+# ----------------------------------------------------------------------------
+# twins (same logical K/V, different physical arrangement)
+
+def clone_batch(batch, **changes):
+    fields = dict(batch.__dict__)
+    for k in ("q", "k_cache", "v_cache", "new_key", "new_value", "context_lens",
+              "block_tables", "slot_mapping"):
+        fields[k] = fields[k].clone()
+    fields["meta"] = dict(batch.meta)
+    fields.update(changes)
+    return workloads.Batch(**fields)
+
+
+def permute_physical(batch, seed=1):
+    """Move every block to a new physical id (a random permutation of the pool)
+    and rewrite the block tables to match."""
+    rng = np.random.default_rng(seed)
+    N = batch.num_blocks
+    perm = torch.from_numpy(rng.permutation(N).astype(np.int64))   # old id -> new id
+    k = torch.empty_like(batch.k_cache)
+    v = torch.empty_like(batch.v_cache)
+    k[perm.to(k.device)] = batch.k_cache
+    v[perm.to(v.device)] = batch.v_cache
+    bt = batch.block_tables.clone()
+    valid = bt >= 0
+    bt[valid] = perm[bt[valid].to(torch.int64)].to(torch.int32)
+    slots = batch.slot_mapping.clone()
+    ok = slots >= 0
+    B = batch.block_size
+    slots[ok] = perm[slots[ok] // B] * B + slots[ok] % B
+    return clone_batch(batch, k_cache=k, v_cache=v, block_tables=bt, slot_mapping=slots)
+
+
+def materialize_shared(batch):
+    """Give every sequence private copies of the blocks it shares with others
+    (whole-tile copies), leaving its logical K/V unchanged."""
+    bt = batch.block_tables.clone()
+    counts = {}
+    for x in bt[bt >= 0].tolist():
+        counts[x] = counts.get(x, 0) + 1
+    src, dst = [], []
+    nxt = batch.num_blocks
+    for s in range(bt.shape[0]):
+        for j in range(bt.shape[1]):
+            x = int(bt[s, j])
+            if x >= 0 and counts[x] > 1:
+                src.append(x)
+                dst.append(nxt)
+                bt[s, j] = nxt
+                nxt += 1
+    if not src:
+        return clone_batch(batch)
+    idx = torch.tensor(src, device=batch.k_cache.device)
+    k = torch.cat([batch.k_cache, batch.k_cache[idx]])
+    v = torch.cat([batch.v_cache, batch.v_cache[idx]])
+    return clone_batch(batch, k_cache=k, v_cache=v, block_tables=bt, num_blocks=nxt)
+
+
+def relayout_block_size(batch, new_B, seed=2):
+    """The same logical K/V stored with another block size: tokens are copied
+    row by row (through the numpy view of the layout) into freshly allocated,
+    shuffled blocks."""
+    rng = np.random.default_rng(seed)
+    S, Hkv, D = batch.num_seqs, batch.num_kv_heads, batch.head_dim
+    lens = [int(x) for x in batch.context_lens]
+    nblk = [(L + new_B - 1) // new_B for L in lens]
+    N = sum(nblk) + 3
+    ids = rng.permutation(N).astype(np.int32)
+    tables = np.full((S, max(1, max(nblk))), -1, dtype=np.int32)
+    x = workloads.vec_elems(batch.dtype)
+    k = torch.zeros((N, Hkv, D // x, new_B, x), dtype=batch.dtype)
+    v = torch.zeros_like(k)
+    kc, vc = batch.k_cache.cpu(), batch.v_cache.cpu()
+    cur = 0
+    for s in range(S):
+        tables[s, :nblk[s]] = ids[cur:cur + nblk[s]]
+        cur += nblk[s]
+        for t in range(lens[s]):
+            ob = int(batch.block_tables[s, t // batch.block_size])
+            nb = int(tables[s, t // new_B])
+            k[nb, :, :, t % new_B, :] = kc[ob, :, :, t % batch.block_size, :]
+            v[nb, :, :, t % new_B, :] = vc[ob, :, :, t % batch.block_size, :]
+    dev = batch.k_cache.device
+    return clone_batch(batch, k_cache=k.to(dev), v_cache=v.to(dev), block_size=new_B, num_blocks=N,
+                       block_tables=torch.from_numpy(tables),
+                       slot_mapping=torch.full_like(batch.slot_mapping, -1))
+
+
+# ----------------------------------------------------------------------------
+# tolerances
+
+def check_tolerance(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype):
+    """The pass criteria:
+      fp32:      |g - r| <= 1e-5 |r| + 1e-5 max_d |r[s,h,:]|   (1e-5 relative)
+      fp16/bf16: |g - r| <= 2e-2 + 2e-2 |r|                      (2e-2 abs + 2e-2 rel)
+    Returns a dict of diagnostics; raises AssertionError on failure."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "non-finite output"
+    err = np.abs(got - ref)
+    if dtype == torch.float32:
+        row_max = np.max(np.abs(ref), axis=-1, keepdims=True)
+        bound = 1e-5 * np.abs(ref) + 1e-5 * row_max
+    else:
+        bound = 2e-2 + 2e-2 * np.abs(ref)
+    worst = float(np.max(err / bound)) if err.size else 0.0
+    rms = math.sqrt(float(np.mean(err ** 2))) if err.size else 0.0
+    rms_ref = math.sqrt(float(np.mean(ref ** 2))) if ref.size else 0.0
+    diag = {"max_abs_err": float(err.max()) if err.size else 0.0, "worst_frac_of_bound": worst,
+            "rms_err_over_rms_ref": rms / rms_ref if rms_ref else 0.0}
+    assert worst <= 1.0, f"tolerance exceeded: {diag}"
+    return diag

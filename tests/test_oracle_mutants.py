@@ -1,0 +1,85 @@
+"""Planted mistakes: each entry copies the oracle source, plants one plausible
+error (a dropped term, a wrong sign or index, a transposed operand), builds it
+on the CPU, and runs the pin suite against it.  At least one pin must fail for
+every mutant — otherwise the pins would not notice that mistake in the oracle.
+"""
+
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+from oracle_pins import PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.cpp")
+
+MUTANTS = {
+    "gqa_interleaved_heads": ("const int h = kvh * group + j;",
+                              "const int h = j * sh.num_kv_heads + kvh;"),
+    "layout_token_outer": ("return (vector * block_size + token) * vec + dim % vec;",
+                           "return ((tile * block_size + token) * (head_dim / vec) + dim / vec) * vec + dim % vec;"),
+    "offset_off_by_one": ("const int offset = t % sh.block_size;",
+                          "const int offset = (t + 1) % sh.block_size;"),
+    "logical_block_off_by_one": ("table_row[t / sh.block_size]", "table_row[(t + 1) / sh.block_size]"),
+    "softmax_sign": ("w[t] = std::exp(z[t] - zmax);", "w[t] = std::exp(zmax - z[t]);"),
+    "dropped_scale": ("z[t] = scale * dot;", "z[t] = dot;"),
+    "missing_normalisation": ("const double p = w[t] / denom;", "const double p = w[t];"),
+    "merge_weight_dropped": ("const double w = std::exp(m[p] - big) / denom;",
+                             "const double w = 1.0 / denom;"),
+    "partition_end_short": ("const int t1 = std::min(context_len, t0 + part);",
+                            "const int t1 = std::min(context_len, t0 + part - 1);"),
+    "reshape_block_shift": ("const int64_t block = slot / block_size;",
+                            "const int64_t block = (slot + 1) / block_size;"),
+    "reshape_kv_swapped": ("static_cast<const uint8_t*>(value) + src * es, es);",
+                           "static_cast<const uint8_t*>(key) + src * es, es);"),
+    "reshape_skips_slot_zero": ("if (slot < 0) continue;", "if (slot <= 0) continue;"),
+    "f16_exponent_bias": ("exponent - 25);", "exponent - 24);"),
+    "bf16_wrong_half": ("static_cast<uint32_t>(bits) << 16);", "static_cast<uint32_t>(bits) << 15);"),
+    "context_len_short": ("attend_plain(qrow.data(), keys, values, len, D, scale_d, dst);",
+                          "attend_plain(qrow.data(), keys, values, len > 1 ? len - 1 : len, D, scale_d, dst);"),
+    "q_from_wrong_head": ("(static_cast<int64_t>(s) * sh.num_q_heads + h) * D + d",
+                          "(static_cast<int64_t>(s) * sh.num_q_heads + kvh) * D + d"),
+}
+
+
+# Runs the pins against one oracle build in a child process: a planted
+# indexing mistake may read or write outside an array, and a crash of the
+# child counts as a pin failing.
+_CHILD = """
+import sys
+sys.path[:0] = [{root!r}, {tests!r}]
+import oracle
+from oracle_pins import PINS
+orc = oracle.Oracle({lib!r})
+failed = []
+for pin in PINS:
+    try:
+        pin(orc)
+    except Exception as e:
+        failed.append(pin.__name__)
+print("FAILED:" + ",".join(failed))
+"""
+
+
+def _pins_failed(lib):
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = _CHILD.format(root=os.path.dirname(here), tests=here, lib=lib)
+    proc = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    if proc.returncode != 0:
+        return [f"child exited with {proc.returncode}"]
+    line = [l for l in proc.stdout.splitlines() if l.startswith("FAILED:")][-1]
+    return [x for x in line[len("FAILED:"):].split(",") if x]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found exactly once: {old!r}"
+    mutant_src = tmp_path / "pa_oracle_mutant.cpp"
+    mutant_src.write_text(src.replace(old, new))
+    lib = oracle.build(str(mutant_src), str(tmp_path / "liboracle_mutant.so"), force=True)
+    failed = _pins_failed(lib)
+    assert failed, f"no pin caught the planted mistake {name}"
