@@ -1,0 +1,483 @@
+"""Benchmark of the paged decode hot path: one step = write the newest token of
+every sequence into the KV pool (pa_reshape_and_cache) + paged decode attention
+over every sequence's whole context (pa_decode / pa_decode_splitk).
+
+Default workload: Llama-3-8B-shaped single-layer decode, bf16 — 64 sequences,
+32 q / 8 kv heads, head_dim 128, block size 16, context lengths uniform on
+[128, 2048], a 16384-block pool with shuffled ids, synthetic N(0,1) data.
+
+Prints one JSON line (rank 0).  `value` is KV GB/s over the whole step:
+algorithmic bytes (sum_s L_s*Hkv*D*2*e + Q + out + block-table entries +
+context_lens, plus the new tokens' K/V read and written) / step time, summed
+over ranks and divided by the max-over-ranks time.  Timing: CUDA events per
+step on the launching stream, L2 flushed (a 256 MiB write) between steps.
+
+Multi-GPU: sequences are independent, so each rank runs its own batch (weak
+scaling, no data-path collective); only the timing reduction crosses ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference available: the
+pages ship no code) on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+METRIC = "paged decode KV GB/s & tokens/s (Llama-3-8B shape) as % of B200 HBM peak"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama3_8b_decode",
+                    choices=["tiny_mha_f32", "llama3_8b_decode", "continuous_batching_mix", "prefix_sharing",
+                             "llama3_70b_long"])
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--mode", choices=["single", "splitk"], default=None,
+                    help="decode entry point (default: splitk for long contexts, else single)")
+    ap.add_argument("--partition-size", type=int, default=512)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between steps")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def make_workload(name, seed, device, block_size=None):
+    import workloads
+    kw = {"seed": seed, "device": device}
+    if block_size is not None and name != "tiny_mha_f32":
+        kw["block_size"] = block_size
+    return workloads.CONFIGS[name](**kw)
+
+
+def step_bytes(batch):
+    """Algorithmic bytes of one step: the decode's (K/V + Q + out + block-table
+    entries + context_lens) and the reshape's (new K/V read + written, slots)."""
+    decode = batch.algorithmic_bytes()
+    T = int(batch.slot_mapping.numel())
+    reshape = 2 * 2 * T * batch.num_kv_heads * batch.head_dim * batch.elem_bytes + 8 * T
+    return decode, reshape
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not getattr(self, "lines", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max of a scalar over ranks (timing only; not on the data path)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- the GPU arm
+
+class Step:
+    """One hot-path step through the C ABI on device-resident inputs."""
+
+    def __init__(self, batch, mode, partition_size):
+        import paged_kv_cache_449_b200 as pa
+        self.pa = pa
+        self.b = batch
+        self.mode = mode
+        self.part = partition_size
+        dev = "cuda"
+        self.q = batch.q.to(dev).contiguous()
+        self.k = batch.k_cache.to(dev).contiguous()
+        self.v = batch.v_cache.to(dev).contiguous()
+        self.bt = batch.block_tables.to(dev).contiguous()
+        self.cl = batch.context_lens.to(dev).contiguous()
+        self.nk = batch.new_key.to(dev).contiguous()
+        self.nv = batch.new_value.to(dev).contiguous()
+        self.slots = batch.slot_mapping.to(dev).contiguous()
+        self.out = torch.empty_like(self.q)
+        self.mcl = batch.max_context_len
+        need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
+                                                  self.part)
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        self.kernels_per_step = 1 + (2 if mode == "splitk" else 1)
+
+    def reshape(self, stream):
+        self.pa.pa_reshape_and_cache(self.nk, self.nv, self.k, self.v, self.slots, stream=stream)
+
+    def decode(self, stream):
+        if self.mode == "splitk":
+            self.pa.pa_decode_splitk(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale, self.mcl,
+                                     partition_size=self.part, workspace=self.ws, stream=stream)
+        else:
+            self.pa.pa_decode(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale,
+                              max_context_len=self.mcl, stream=stream)
+
+
+def run_gpu(args, world, rank, local):
+    import paged_kv_cache_449_b200 as pa
+    from paged_kv_cache_449_b200 import build as pabuild
+    pabuild.build()
+    pa.load()
+    batch = make_workload(args.workload, args.seed + rank, "cuda", args.block_size)
+    mode = args.mode or ("splitk" if batch.max_context_len > 4096 else "single")
+    step = Step(batch, mode, args.partition_size)
+    stream = torch.cuda.current_stream()
+    flush = None if args.no_flush else torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    decode_bytes, reshape_bytes = step_bytes(batch)
+
+    def one(timed_events=None):
+        if timed_events is None:
+            step.reshape(stream)
+            step.decode(stream)
+            return
+        e0, e1, e2 = timed_events
+        e0.record(stream)
+        step.reshape(stream)
+        e1.record(stream)
+        step.decode(stream)
+        e2.record(stream)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        time.sleep(0.3)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            one(events[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [e[0].elapsed_time(e[2]) for e in events]
+    decode_ms = [e[1].elapsed_time(e[2]) for e in events]
+    reshape_ms = [e[0].elapsed_time(e[1]) for e in events]
+    local_step = sum(step_ms) / len(step_ms)
+    local_decode = sum(decode_ms) / len(decode_ms)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+
+    # ---- end to end through the public API: pinned host inputs -> device -> step -> host output
+    e2e = None
+    if not args.no_e2e:
+        host = {name: t.cpu().pin_memory() for name, t in (
+            ("q", step.q), ("nk", step.nk), ("nv", step.nv), ("slots", step.slots), ("bt", step.bt),
+            ("cl", step.cl))}
+        host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = host_out.numel() * host_out.element_size()
+        e2e_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+        def e2e_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            step.q.copy_(host["q"], non_blocking=True)
+            step.nk.copy_(host["nk"], non_blocking=True)
+            step.nv.copy_(host["nv"], non_blocking=True)
+            step.slots.copy_(host["slots"], non_blocking=True)
+            step.bt.copy_(host["bt"], non_blocking=True)
+            step.cl.copy_(host["cl"], non_blocking=True)
+            step.reshape(stream)
+            step.decode(stream)
+            host_out.copy_(step.out, non_blocking=True)
+            if ev is not None:
+                ev[1].record(stream)
+
+        for _ in range(args.warmup):
+            if flush is not None:
+                flush.zero_()
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            e2e_step(e2e_events[i])
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_events) / args.steps
+        e2e_ms_max = reduce_max(e2e_ms, world)
+        e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e2e_ms_max, "_local_bytes": decode_bytes + reshape_bytes}
+
+    step_ms_max = reduce_max(local_step, world)
+    decode_ms_max = reduce_max(local_decode, world)
+    total_bytes = reduce_sum(decode_bytes + reshape_bytes, world)
+    total_decode_bytes = reduce_sum(decode_bytes, world)
+    total_seqs = reduce_sum(batch.num_seqs, world)
+    if e2e is not None:
+        e2e["value"] = total_bytes / (e2e["ms_per_step"] * 1e-3) / 1e9
+        e2e.pop("_local_bytes")
+    clk = clocks.summary()
+    peak, peak_kind = measured_peaks()
+    achieved = decode_bytes / (local_decode * 1e-3) / 1e9
+    value = total_bytes / (step_ms_max * 1e-3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms_max, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[batch.dtype],
+        "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and shuffled block ids)",
+        "config": {
+            "workload": batch.name,
+            "global_batch": int(total_seqs),
+            "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
+            "head_dim": batch.head_dim, "block_size": batch.block_size, "num_blocks": batch.num_blocks,
+            "context_len_mean": float(batch.context_lens.float().mean()),
+            "context_len_max": batch.max_context_len,
+            "decode_entry": "pa_decode_splitk" if mode == "splitk" else "pa_decode",
+            "partition_size": args.partition_size if mode == "splitk" else None,
+            "parallelism": f"replicas x{world} (sequence batches, no collective)",
+            "l2": "flushed between steps (256 MiB write), per-step CUDA events" if flush is not None
+            else "not flushed",
+            "step": "pa_reshape_and_cache (newest token of every sequence) + decode",
+        },
+        "tokens_per_s": round(total_seqs / (step_ms_max * 1e-3), 1),
+        "decode_ms": round(decode_ms_max, 5),
+        "reshape_ms": round(sum(reshape_ms) / len(reshape_ms), 5),
+        "decode_gbs": round(total_decode_bytes / (decode_ms_max * 1e-3) / 1e9, 2),
+        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        "pct_of_spec_8tbs": round(100 * value / world / SPEC_HBM_GBS, 2),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode (partition + merge kernels)" if mode == "splitk" else "pa_decode_kernel",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
+            "algorithmic_bytes_per_launch": int(decode_bytes),
+            "traffic": None,
+        },
+        "gpu_launches": int(step.kernels_per_step * args.steps),
+        "clocks": clk,
+    }
+    if e2e is not None:
+        result["e2e"] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in e2e.items()}
+    return result, batch
+
+
+# ----------------------------------------------------------------------------- the oracle (CPU)
+
+def oracle_sample(batch, seconds_target, seed=0):
+    """Times the oracle on a bounded sample of the batch's sequences; returns
+    (GB/s over the sample's algorithmic bytes, description, threads)."""
+    import oracle
+    orc = oracle.default()
+    rng = np.random.default_rng(seed)
+    order = list(rng.permutation(batch.num_seqs))
+    # estimate the cost of one sequence from a first one, then size the sample
+    taken, spent, nbytes = [], 0.0, 0
+    e = batch.elem_bytes
+    per_seq_fixed = 2 * batch.num_q_heads * batch.head_dim * e + 4
+    for s in order:
+        seqs = [int(s)]
+        q, k, v, bt, cl = _compact(batch, seqs)
+        t0 = time.perf_counter()
+        orc.decode(q, k, v, bt, cl, batch.scale, batch.block_size, batch.num_kv_heads)
+        spent += time.perf_counter() - t0
+        L = int(batch.context_lens[s])
+        nbytes += L * batch.num_kv_heads * batch.head_dim * 2 * e + per_seq_fixed + \
+            ((L + batch.block_size - 1) // batch.block_size) * 4
+        taken.append(int(s))
+        if spent >= seconds_target:
+            break
+    gbs = nbytes / spent / 1e9
+    desc = (f"{len(taken)} of {batch.num_seqs} sequences (seeded sample, "
+            f"{sum(int(batch.context_lens[s]) for s in taken)} tokens), single-threaded fp64, {spent:.1f} s")
+    return gbs, desc, spent, len(taken)
+
+
+def _compact(batch, seqs):
+    bt = batch.block_tables[seqs]
+    used = sorted(set(int(x) for x in bt[bt >= 0].tolist()))
+    remap = {old: new for new, old in enumerate(used)}
+    nbt = bt.clone()
+    flat = nbt.view(-1)
+    for i in range(flat.numel()):
+        x = int(flat[i])
+        if x >= 0:
+            flat[i] = remap[x]
+    idx = torch.tensor(used if used else [0], dtype=torch.int64, device=batch.k_cache.device)
+    return (batch.q[seqs].cpu().contiguous(), batch.k_cache[idx].cpu().contiguous(),
+            batch.v_cache[idx].cpu().contiguous(), nbt.contiguous(), batch.context_lens[seqs].contiguous())
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle on the host cores, bounded sample per step."""
+    if rank != 0:
+        return None
+    import workloads
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    batch = make_workload(args.workload, args.seed, device, args.block_size)
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    times, gbs_list, desc = [], [], ""
+    for i in range(args.warmup + args.steps):
+        gbs, desc, spent, n = oracle_sample(batch, per_step, seed=i)
+        if i >= args.warmup:
+            times.append(spent)
+            gbs_list.append(gbs)
+    value = statistics.mean(gbs_list)
+    return {
+        "metric": METRIC, "impl": "reference", "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (same seeded workload as the GPU arm)",
+        "config": {"workload": batch.name, "global_batch": batch.num_seqs},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+            if res is not None:
+                print(json.dumps(res), flush=True)
+            return
+        res, batch = run_gpu(args, world, rank, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                gbs, desc, spent, n = oracle_sample(batch, args.cpu_sample_seconds)
+                res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                       "sample": desc}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

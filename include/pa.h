@@ -1,0 +1,173 @@
+/*
+ * pa.h — C ABI of the B200 paged KV-cache attention library (libpa.so).
+ *
+ * What the library computes (page titles and sections):
+ *   [P1] "vLLM核心架构总览：PagedAttention、Continuous Batching、分布式推理等核心组件",
+ *        §4.1 PagedAttention — the KV cache of every sequence lives in fixed-size
+ *        physical blocks of one pool; logically contiguous KV is physically
+ *        scattered; a block table maps logical to physical blocks; prefix blocks
+ *        can be shared between sequences.
+ *   [P3] "从源码剖析 vLLM 的显存管理与连续批处理",
+ *        §2.1 BlockTable.append_token — a token's KV is written at the physical
+ *             block address plus its offset in the block;
+ *        §2.2 one pool, preallocated once and carved into equal blocks;
+ *        §2.3 attention takes block tables instead of a (batch, seq, dim) tensor
+ *             and gathers K/V through them.
+ *   [P4] "vLLM框架解析：PagedAttention技术如何实现LLM推理20倍加速",
+ *        §2.3 blocks shared by reference count; copy-on-write for isolation.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Ownership.  Every pointer argument is device memory owned by the caller (for
+ *   example allocated by PyTorch).  The library allocates and frees nothing and
+ *   keeps no state except one device-side error word per GPU (see
+ *   pa_get_device_error).  All calls are asynchronous on `stream` (a
+ *   cudaStream_t passed as void*; NULL = the legacy default stream) and return
+ *   once the work is enqueued.
+ * Alignment.  q, out, key, value, both pools and the workspace must be
+ *   16-byte aligned; slot_mapping 8-byte, block_tables and context_lens
+ *   4-byte aligned.
+ * Element types.  q, out, key, value and both pools share one pa_dtype.
+ * Pool layout.  k_cache and v_cache are each an array
+ *       [num_blocks][num_kv_heads][head_dim / X][block_size][X],  X = 16 / sizeof(elem)
+ *   (X = 8 for fp16/bf16, 4 for fp32): the tile of one (block, kv head) is
+ *   contiguous (block_size * head_dim elements) and split along head_dim into
+ *   16-byte vectors, vector index outer, token inner.
+ * Slots.  slot = physical_block * block_size + offset_in_block; slot < 0 marks
+ *   a padding token that is skipped.
+ * Block tables.  block_tables is int32 [num_seqs][max_blocks_per_seq]; entry
+ *   [s][j] is the physical block holding logical tokens [j*B, (j+1)*B) of
+ *   sequence s.  Entries at j >= ceil(context_lens[s] / B) are never read.
+ *   Several rows may name the same physical block (shared prefix).
+ * Context lengths.  context_lens[s] (int32) counts every token of sequence s,
+ *   including the one just written by pa_reshape_and_cache; 0 gives an
+ *   all-zero output row.
+ * GQA.  num_q_heads is a multiple of num_kv_heads; query head h reads kv head
+ *   h / (num_q_heads / num_kv_heads).
+ * Supported shapes.  head_dim in {64, 128}; block_size in {8, 16, 32};
+ *   num_q_heads / num_kv_heads in {1, 2, 4, 8}.
+ * Arithmetic.  Scores, softmax and the weighted sum accumulate in fp32 (online
+ *   softmax); the output is rounded once (round to nearest even) to the dtype.
+ * Errors.  Host-side checks (null pointers, unsupported shapes, misalignment,
+ *   a workspace too small) return a non-zero pa_status before anything is
+ *   launched.  A launch failure returns PA_ERR_CUDA.  Device data that
+ *   violates the conventions (a block id outside [0, num_blocks), a slot past
+ *   the pool, a context length above min(max_context_len,
+ *   max_blocks_per_seq * block_size)) is never dereferenced: the kernel skips
+ *   the offending access and sets a bit in the device error word, readable with
+ *   pa_get_device_error.  The library never traps and never waits without a
+ *   bound.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer */
+    PA_ERR_UNSUPPORTED = 2,   /* head_dim / block_size / group / dtype not supported */
+    PA_ERR_WORKSPACE = 3,     /* split-K workspace missing or too small */
+    PA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Bits of the device error word. */
+#define PA_DEVERR_BLOCK_ID     1  /* a block-table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN  2  /* a context length < 0 or above the stated maximum */
+#define PA_DEVERR_SLOT         4  /* a slot >= num_blocks * block_size */
+#define PA_DEVERR_TIMEOUT      8  /* an asynchronous copy did not complete in time */
+
+/*
+ * pa_reshape_and_cache — write the K/V of new tokens into the pools.
+ * [P3] §2.1 (append_token: physical address = block address + offset).
+ *
+ *   key, value     [num_tokens][num_kv_heads][head_dim], contiguous, read only
+ *   k_cache,
+ *   v_cache        pools of num_blocks blocks (layout above), written in place
+ *   slot_mapping   int64 [num_tokens]; token i goes to block slot/B, offset
+ *                  slot%B; slot < 0 skips the token
+ *   The copy is bit-exact.  Two tokens naming the same slot is the caller's
+ *   error (the result then holds one of them).  num_tokens == 0 is a no-op.
+ */
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int64_t num_tokens, int num_kv_heads,
+                               int head_dim, int block_size, int64_t num_blocks, pa_dtype dtype,
+                               void* stream);
+
+/*
+ * pa_decode — one query token per sequence attends over its whole paged
+ * context, in one launch (one pass over each sequence's KV).
+ * [P3] §2.3 (block tables in, gather by index remapping); [P1] §4.1.
+ *
+ *   out            [num_seqs][num_q_heads][head_dim], written
+ *   q              [num_seqs][num_q_heads][head_dim]
+ *   k_cache,
+ *   v_cache        pools (layout above), read only
+ *   block_tables   int32 [num_seqs][max_blocks_per_seq]
+ *   context_lens   int32 [num_seqs]
+ *   scale          softmax scale applied to q.k (typically 1/sqrt(head_dim))
+ *   max_context_len  an upper bound of context_lens (used for validation)
+ *   out[s,h,:] = sum_t softmax_t(scale * q[s,h,:].K[s,t,:]) V[s,t,:].
+ *   num_seqs == 0 is a no-op.
+ */
+pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* block_tables, const int32_t* context_lens, float scale,
+                    int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                    void* stream);
+
+/*
+ * pa_decode_splitk_workspace_size — bytes of workspace pa_decode_splitk needs:
+ * per (sequence, query head, partition) an fp32 partial output of head_dim
+ * values plus its running max and sum, for ceil(max_context_len /
+ * partition_size) partitions.
+ */
+pa_status pa_decode_splitk_workspace_size(int num_seqs, int num_q_heads, int head_dim,
+                                          int max_context_len, int partition_size, size_t* bytes);
+
+/*
+ * pa_decode_splitk — the same result as pa_decode, computed for long contexts
+ * by token partitions: kernel 1 handles each (sequence, kv head, partition of
+ * partition_size tokens) on its own and writes fp32 partials (unnormalised
+ * output, max, sum) to `workspace`; kernel 2 merges the partitions of each
+ * (sequence, query head) with log-sum-exp weights exp(m_p - max_p m_p) and
+ * writes `out`.  Two launches on `stream`, no inter-CTA waiting.
+ *
+ *   partition_size  tokens per partition; a positive multiple of 16 and of
+ *                   block_size (512 is the usual choice)
+ *   workspace       device scratch of at least
+ *                   pa_decode_splitk_workspace_size(...) bytes, 16-byte
+ *                   aligned; its contents need no initialisation and are
+ *                   clobbered
+ *   Other arguments as in pa_decode; here max_context_len also sizes the
+ *   partition grid, so every context_lens[s] must be <= max_context_len.
+ */
+pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, float scale,
+                           int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                           int head_dim, int max_blocks_per_seq, int max_context_len,
+                           int64_t num_blocks, pa_dtype dtype, int partition_size, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * pa_get_device_error — read and clear the device error word of the current
+ * GPU.  Synchronises `stream` first, so it reports every launch enqueued on it
+ * before the call.  *code receives an OR of PA_DEVERR_* bits (0 = no error).
+ */
+pa_status pa_get_device_error(void* stream, int32_t* code);
+
+/* pa_status_string — a static, human-readable name of a status. */
+const char* pa_status_string(pa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,168 @@
+"""Python binding of libpa — B200 paged KV-cache attention (C ABI in include/pa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libpa.so.  There is no fallback; if the library is missing the
+calls raise.  Tensors are torch CUDA tensors; pools are shaped
+[num_blocks, num_kv_heads, head_dim // X, block_size, X] (X = 16 bytes /
+element size), so block_size, num_blocks and the head counts are read off the
+tensor shapes.  Calls run on the current torch CUDA stream unless `stream`
+(a torch.cuda.Stream or a raw cudaStream_t int) is given.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
+           "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
+           "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+_DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE", 4: "PA_ERR_CUDA"}
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load libpa.so (built in-tree by paged_kv_cache_449_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libpa.so is not built ({_LIB_PATH}); run paged_kv_cache_449_b200/build.py")
+    lib = ctypes.CDLL(_LIB_PATH)
+    c = ctypes
+    P, I, I64, F, SZ = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
+    lib.pa_reshape_and_cache.restype = I
+    lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I, P]
+    decode_args = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I64, I]
+    lib.pa_decode.restype = I
+    lib.pa_decode.argtypes = decode_args + [P]
+    lib.pa_decode_splitk_workspace_size.restype = I
+    lib.pa_decode_splitk_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
+    lib.pa_decode_splitk.restype = I
+    lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P]
+    lib.pa_get_device_error.restype = I
+    lib.pa_get_device_error.argtypes = [P, c.POINTER(c.c_int32)]
+    lib.pa_status_string.restype = c.c_char_p
+    lib.pa_status_string.argtypes = [I]
+    _lib = lib
+    return lib
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise PagedAttentionError(status, what)
+
+
+def pool_shape(num_blocks: int, num_kv_heads: int, head_dim: int, block_size: int, dtype: torch.dtype):
+    x = 16 // torch.tensor([], dtype=dtype).element_size()
+    return (num_blocks, num_kv_heads, head_dim // x, block_size, x)
+
+
+def _pool_dims(k_cache: torch.Tensor):
+    if k_cache.dim() != 5:
+        raise ValueError("pools must be shaped [num_blocks, num_kv_heads, head_dim // X, block_size, X]")
+    n, hkv, dv, b, x = k_cache.shape
+    return n, hkv, dv * x, b
+
+
+def _dev_ptr(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def pa_status_string(status: int) -> str:
+    return load().pa_status_string(int(status)).decode()
+
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
+    """Write key/value [T, Hkv, D] into the pools at slot_mapping (int64 [T])."""
+    lib = load()
+    n, hkv, d, b = _pool_dims(k_cache)
+    T = key.shape[0]
+    _check(lib.pa_reshape_and_cache(
+        _dev_ptr(key, "key"), _dev_ptr(value, "value"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(slot_mapping, "slot_mapping"), T, hkv, d, b, n,
+        _DTYPE[key.dtype], _stream(stream)), "pa_reshape_and_cache")
+
+
+def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len):
+    n, hkv, d, b = _pool_dims(k_cache)
+    S, Hq, D = q.shape
+    if max_context_len is None:
+        max_context_len = int(block_tables.shape[1]) * b
+    return [_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+            _dev_ptr(block_tables, "block_tables"), _dev_ptr(context_lens, "context_lens"), float(scale), b, S,
+            Hq, hkv, D, int(block_tables.shape[1]), int(max_context_len), n, _DTYPE[q.dtype]]
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None, stream=None):
+    """Paged decode attention, one launch.  out, q: [S, Hq, D]; block_tables
+    int32 [S, max_blocks]; context_lens int32 [S]."""
+    lib = load()
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode(*args, _stream(stream)), "pa_decode")
+
+
+def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size=512) -> int:
+    lib = load()
+    size = ctypes.c_size_t(0)
+    _check(lib.pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                               partition_size, ctypes.byref(size)),
+           "pa_decode_splitk_workspace_size")
+    return int(size.value)
+
+
+def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                     partition_size=512, workspace=None, stream=None):
+    """Split-K paged decode (partitions of partition_size tokens + log-sum-exp
+    merge).  `workspace` is a CUDA uint8 tensor of at least
+    pa_decode_splitk_workspace_size(...) bytes; allocated here if None."""
+    lib = load()
+    S, Hq, D = q.shape
+    need = pa_decode_splitk_workspace_size(S, Hq, D, int(max_context_len), partition_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_splitk(*args, int(partition_size), _dev_ptr(workspace, "workspace"),
+                                workspace.numel() * workspace.element_size(), _stream(stream)),
+           "pa_decode_splitk")
+
+
+def pa_get_device_error(stream=None) -> int:
+    """Read and clear the device error word (synchronises the stream)."""
+    lib = load()
+    code = ctypes.c_int32(0)
+    _check(lib.pa_get_device_error(_stream(stream), ctypes.byref(code)), "pa_get_device_error")
+    return int(code.value)

@@ -173,3 +173,59 @@ def check_tolerance(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype):
             "rms_err_over_rms_ref": rms / rms_ref if rms_ref else 0.0}
     assert worst <= 1.0, f"tolerance exceeded: {diag}"
     return diag
+
+
+# ----------------------------------------------------------------------------
+# GPU runs through the C ABI and sampled oracle references
+
+def device_batch(batch, device="cuda"):
+    """Tensors the kernels read, on the device (pools may already be there)."""
+    return {
+        "q": batch.q.to(device).contiguous(),
+        "k_cache": batch.k_cache.to(device).contiguous(),
+        "v_cache": batch.v_cache.to(device).contiguous(),
+        "block_tables": batch.block_tables.to(device).contiguous(),
+        "context_lens": batch.context_lens.to(device).contiguous(),
+    }
+
+
+def gpu_decode(batch, mode="single", partition_size=512, dev=None, max_context_len=None):
+    import paged_kv_cache_449_b200 as pa
+    dev = dev or device_batch(batch)
+    out = torch.full_like(dev["q"], float("nan"))
+    mcl = batch.max_context_len if max_context_len is None else max_context_len
+    if mode == "single":
+        pa.pa_decode(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"], dev["context_lens"],
+                     batch.scale, max_context_len=mcl)
+    else:
+        pa.pa_decode_splitk(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"],
+                            dev["context_lens"], batch.scale, mcl, partition_size=partition_size)
+    torch.cuda.synchronize()
+    return out
+
+
+def compact_for_oracle(batch, seqs):
+    """The sampled sequences with only the blocks they reference, moved to the
+    CPU (whole tiles gathered, tables renumbered) — what the oracle needs to
+    compute their outputs one by one."""
+    seqs = list(seqs)
+    bt = batch.block_tables[seqs]
+    used = sorted(set(int(x) for x in bt[bt >= 0].tolist()))
+    remap = {old: new for new, old in enumerate(used)}
+    nbt = bt.clone()
+    for i in range(nbt.shape[0]):
+        for j in range(nbt.shape[1]):
+            x = int(nbt[i, j])
+            if x >= 0:
+                nbt[i, j] = remap[x]
+    idx = torch.tensor(used if used else [0], dtype=torch.int64, device=batch.k_cache.device)
+    k = batch.k_cache[idx].cpu().contiguous()
+    v = batch.v_cache[idx].cpu().contiguous()
+    q = batch.q[seqs].cpu().contiguous()
+    return q, k, v, nbt.contiguous(), batch.context_lens[seqs].contiguous()
+
+
+def oracle_decode_sampled(orc, batch, seqs, partition_size=None):
+    q, k, v, bt, cl = compact_for_oracle(batch, seqs)
+    return orc.decode(q, k, v, bt, cl, batch.scale, batch.block_size, batch.num_kv_heads,
+                      partition_size=partition_size)

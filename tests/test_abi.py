@@ -1,0 +1,105 @@
+"""The C ABI library on the CPU: it builds, loads without a GPU, exports every
+function include/pa.h declares, and its host-side checks and helpers behave
+as documented.  No kernel is launched here."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_cache_449_b200 as pa
+from paged_kv_cache_449_b200 import build as pabuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pabuild.build()
+    return pa.load()
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted([
+        "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size", "pa_get_device_error",
+        "pa_reshape_and_cache", "pa_status_string"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT\s+(\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_library_needs_no_cuda_driver_or_shared_cudart(lib):
+    deps = subprocess.run(["ldd", pa.library_path()], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in deps and "libcudart.so" not in deps
+
+
+def test_status_strings(lib):
+    assert pa.pa_status_string(0) == "PA_OK"
+    assert pa.pa_status_string(3) == "PA_ERR_WORKSPACE"
+    assert pa.pa_status_string(99) == "PA_UNKNOWN_STATUS"
+
+
+def test_workspace_size(lib):
+    # S * Hq * ceil(max_len / part) * (D + 2) * 4 bytes
+    assert pa.pa_decode_splitk_workspace_size(32, 64, 128, 32768, 512) == 32 * 64 * 64 * 130 * 4
+    assert pa.pa_decode_splitk_workspace_size(4, 4, 64, 100, 512) == 4 * 4 * 1 * 66 * 4
+    assert pa.pa_decode_splitk_workspace_size(4, 4, 64, 0, 512) == 0
+    with pytest.raises(pa.PagedAttentionError):
+        pa.pa_decode_splitk_workspace_size(4, 4, 64, 100, 0)
+
+
+P = ctypes.c_void_p
+
+
+def _decode(lib, **kw):
+    a = dict(out=16, q=16, k=16, v=16, bt=16, cl=16, scale=0.125, B=16, S=4, Hq=4, Hkv=4, D=64, mb=7, mcl=100,
+             N=64, dt=0)
+    a.update(kw)
+    return lib.pa_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["scale"], a["B"], a["S"], a["Hq"],
+                         a["Hkv"], a["D"], a["mb"], a["mcl"], a["N"], a["dt"], None)
+
+
+def test_host_validation_rejects_before_launch(lib):
+    # Every case here fails validation, so nothing reaches the (absent) GPU.
+    assert _decode(lib, D=96) == 2                 # unsupported head_dim
+    assert _decode(lib, B=12) == 2                 # unsupported block_size
+    assert _decode(lib, Hq=12, Hkv=4) == 2         # group 3
+    assert _decode(lib, Hq=6, Hkv=4) == 1          # not a multiple
+    assert _decode(lib, dt=7) == 2                 # unknown dtype
+    assert _decode(lib, q=0) == 1                  # null pointer
+    assert _decode(lib, k=24) == 1                 # misaligned pool
+    assert _decode(lib, N=0) == 1                  # empty pool
+    assert _decode(lib, scale=float("nan")) == 1
+    assert _decode(lib, S=0) == 0                  # empty batch: a no-op
+    assert lib.pa_reshape_and_cache(16, 16, 16, 16, 16, 4, 8, 100, 16, 10, 2, None) == 2   # 200 B rows
+    assert lib.pa_reshape_and_cache(16, 16, 16, 16, 12, 4, 8, 128, 16, 10, 2, None) == 1   # slots misaligned
+    assert lib.pa_reshape_and_cache(0, 0, 0, 0, 0, 0, 8, 128, 16, 10, 2, None) == 0        # no tokens
+    args = [16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 64, 0]
+    assert lib.pa_decode_splitk(*args, 500, 16, 1 << 20, None) == 1   # partition not a multiple of 16
+    assert lib.pa_decode_splitk(*args, 512, 16, 100, None) == 3       # workspace too small
+    assert lib.pa_decode_splitk(*args, 512, 0, 1 << 20, None) == 3    # no workspace
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(pa, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(pa, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        pa.load()
