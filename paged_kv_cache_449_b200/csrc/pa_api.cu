@@ -26,10 +26,14 @@ namespace {
 
 template <typename T, int D, int B>
 struct DecodeConfig {
-    static constexpr int kWarps = PA_DECODE_WARPS;
     static constexpr int kStageBytes = 2 * B * D * static_cast<int>(sizeof(T));  // K + V tile
+    static constexpr int kRingCap = 200 * 1024;                                   // ring bytes per CTA at most
+    static constexpr int kMaxWarps = kRingCap / kStageBytes;
+    static constexpr int kWarps = PA_DECODE_WARPS < kMaxWarps ? PA_DECODE_WARPS : kMaxWarps;
     static constexpr int kRaw = PA_RING_BYTES_PER_WARP / kStageBytes;
-    static constexpr int kStages = kRaw < 1 ? 1 : (kRaw > 16 ? 16 : kRaw);
+    static constexpr int kFit = kRingCap / (kWarps * kStageBytes);
+    static constexpr int kStages0 = kRaw < 1 ? 1 : (kRaw > 16 ? 16 : kRaw);
+    static constexpr int kStages = kStages0 < kFit ? kStages0 : kFit;
     using Smem = pa::DecodeSmem<T, D, B, kWarps, kStages>;
     static_assert(Smem::kTotal <= 227 * 1024, "shared memory per CTA");
 };

@@ -166,7 +166,8 @@ def check_tolerance(got: np.ndarray, ref: np.ndarray, dtype: torch.dtype):
         bound = 1e-5 * np.abs(ref) + 1e-5 * row_max
     else:
         bound = 2e-2 + 2e-2 * np.abs(ref)
-    worst = float(np.max(err / bound)) if err.size else 0.0
+    ratio = np.where(bound > 0, err / np.where(bound > 0, bound, 1.0), np.where(err > 0, np.inf, 0.0))
+    worst = float(np.max(ratio)) if err.size else 0.0
     rms = math.sqrt(float(np.mean(err ** 2))) if err.size else 0.0
     rms_ref = math.sqrt(float(np.mean(ref ** 2))) if ref.size else 0.0
     diag = {"max_abs_err": float(err.max()) if err.size else 0.0, "worst_frac_of_bound": worst,
