@@ -1,6 +1,7 @@
 """Benchmark of the paged decode hot path: one step = write the newest token of
 every sequence into the KV pool (pa_reshape_and_cache) + paged decode attention
-over every sequence's whole context (pa_decode / pa_decode_splitk).
+over every sequence's whole context (pa_decode, pa_decode_splitk or
+pa_decode_streamk, --mode).
 
 Default workload: Llama-3-8B-shaped single-layer decode, bf16 — 64 sequences,
 32 q / 8 kv heads, head_dim 128, block size 16, context lengths uniform on
@@ -52,9 +53,9 @@ def parse_args(argv=None):
                     choices=["tiny_mha_f32", "llama3_8b_decode", "continuous_batching_mix", "prefix_sharing",
                              "llama3_70b_long"])
     ap.add_argument("--block-size", type=int, default=None)
-    ap.add_argument("--mode", choices=["single", "splitk"], default=None,
-                    help="decode entry point (default: splitk for long contexts, else single)")
-    ap.add_argument("--partition-size", type=int, default=512)
+    ap.add_argument("--mode", choices=["single", "splitk", "splitk2", "streamk"], default="single",
+                    help="decode entry point: pa_decode, pa_decode_splitk or pa_decode_streamk")
+    ap.add_argument("--partition-size", type=int, default=1024)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between steps")
     ap.add_argument("--no-e2e", action="store_true")
@@ -212,15 +213,21 @@ class Step:
         need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
                                                   self.part)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        self.kernels_per_step = 1 + (2 if mode == "splitk" else 1)
+        self.sk_ws = pa.StreamKWorkspace()
+        self.counters = pa.Counters()
+        self.kernels_per_step = 1 + (2 if mode == "splitk2" else 1)
 
     def reshape(self, stream):
         self.pa.pa_reshape_and_cache(self.nk, self.nv, self.k, self.v, self.slots, stream=stream)
 
     def decode(self, stream):
-        if self.mode == "splitk":
+        if self.mode == "streamk":
+            self.pa.pa_decode_streamk(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale,
+                                      max_context_len=self.mcl, workspace=self.sk_ws, stream=stream)
+        elif self.mode in ("splitk", "splitk2"):
             self.pa.pa_decode_splitk(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale, self.mcl,
-                                     partition_size=self.part, workspace=self.ws, stream=stream)
+                                     partition_size=self.part, workspace=self.ws, fused=(self.mode == "splitk"),
+                                     counters=self.counters, stream=stream)
         else:
             self.pa.pa_decode(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale,
                               max_context_len=self.mcl, stream=stream)
@@ -232,7 +239,7 @@ def run_gpu(args, world, rank, local):
     pabuild.build()
     pa.load()
     batch = make_workload(args.workload, args.seed + rank, "cuda", args.block_size)
-    mode = args.mode or ("splitk" if batch.max_context_len > 4096 else "single")
+    mode = args.mode
     step = Step(batch, mode, args.partition_size)
     stream = torch.cuda.current_stream()
     flush = None if args.no_flush else torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -352,8 +359,9 @@ def run_gpu(args, world, rank, local):
             "head_dim": batch.head_dim, "block_size": batch.block_size, "num_blocks": batch.num_blocks,
             "context_len_mean": float(batch.context_lens.float().mean()),
             "context_len_max": batch.max_context_len,
-            "decode_entry": "pa_decode_splitk" if mode == "splitk" else "pa_decode",
-            "partition_size": args.partition_size if mode == "splitk" else None,
+            "decode_entry": {"splitk": "pa_decode_splitk (fused merge)", "splitk2": "pa_decode_splitk (merge kernel)",
+                             "streamk": "pa_decode_streamk"}.get(mode, "pa_decode"),
+            "partition_size": args.partition_size if mode.startswith("splitk") else None,
             "parallelism": f"replicas x{world} (sequence batches, no collective)",
             "l2": "flushed between steps (256 MiB write), per-step CUDA events" if flush is not None
             else "not flushed",
@@ -367,7 +375,9 @@ def run_gpu(args, world, rank, local):
         "pct_of_spec_8tbs": round(100 * value / world / SPEC_HBM_GBS, 2),
         "roofline": {
             "bound": "hbm",
-            "kernel": "decode (partition + merge kernels)" if mode == "splitk" else "pa_decode_kernel",
+            "kernel": {"splitk": "pa_decode_kernel<split, fused merge>",
+                       "splitk2": "pa_decode_kernel<split> + pa_merge_kernel",
+                       "streamk": "pa_decode_streamk_kernel"}.get(mode, "pa_decode_kernel"),
             "achieved": round(achieved, 2),
             "peak": peak,
             "peak_kind": f"{peak_kind} copy bandwidth (burst)",

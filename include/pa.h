@@ -136,9 +136,13 @@ pa_status pa_decode_splitk_workspace_size(int num_seqs, int num_q_heads, int hea
  * pa_decode_splitk — the same result as pa_decode, computed for long contexts
  * by token partitions: kernel 1 handles each (sequence, kv head, partition of
  * partition_size tokens) on its own and writes fp32 partials (unnormalised
- * output, max, sum) to `workspace`; kernel 2 merges the partitions of each
- * (sequence, query head) with log-sum-exp weights exp(m_p - max_p m_p) and
- * writes `out`.  Two launches on `stream`, no inter-CTA waiting.
+ * output, max, sum) to `workspace`; the partitions of each (sequence, query
+ * head) are then merged with log-sum-exp weights exp(m_p - max_p m_p):
+ *   counters == NULL   by kernel 2 (two launches on `stream`);
+ *   counters != NULL   inside kernel 1 (one launch): the CTA that records the
+ *                      last partition of a (sequence, kv head) merges them,
+ *                      and a sequence with one partition is finished directly.
+ * No thread waits for another CTA in either form.
  *
  *   partition_size  tokens per partition; a positive multiple of 16 and of
  *                   block_size (512 is the usual choice)
@@ -146,15 +150,68 @@ pa_status pa_decode_splitk_workspace_size(int num_seqs, int num_q_heads, int hea
  *                   pa_decode_splitk_workspace_size(...) bytes, 16-byte
  *                   aligned; its contents need no initialisation and are
  *                   clobbered
+ *   counters        NULL, or an int32 array of num_counters >= num_seqs *
+ *                   num_kv_heads arrival counters (entry s*Hkv + kvh), all
+ *                   zero before the first call (allocate it zeroed); every
+ *                   completed call leaves the entries it used at zero, so one
+ *                   array serves successive calls of any shape.  Zero it again
+ *                   after a call that reported PA_DEVERR_TIMEOUT.
  *   Other arguments as in pa_decode; here max_context_len also sizes the
  *   partition grid, so every context_lens[s] must be <= max_context_len.
+ *   Calls that may run concurrently on the GPU need their own workspace and
+ *   counters.
  */
 pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const void* v_cache,
                            const int32_t* block_tables, const int32_t* context_lens, float scale,
                            int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
                            int head_dim, int max_blocks_per_seq, int max_context_len,
                            int64_t num_blocks, pa_dtype dtype, int partition_size, void* workspace,
-                           size_t workspace_bytes, void* stream);
+                           size_t workspace_bytes, int32_t* counters, int64_t num_counters,
+                           void* stream);
+
+/*
+ * pa_decode_streamk_workspace_size — bytes of scratch pa_decode_streamk needs
+ * on the current device for its partial records: per worker warp of the
+ * persistent grid two records, each holding fp32 head_dim outputs plus the
+ * running max and sum of the g query heads of one kv head (padded to 16
+ * bytes).  The worker count follows the device's SM count and the kernel's
+ * occupancy, so the size depends on the GPU (and slightly on num_seqs).
+ */
+pa_status pa_decode_streamk_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                           int block_size, pa_dtype dtype, size_t* bytes);
+
+/*
+ * pa_decode_streamk — the same result as pa_decode, scheduled for batches
+ * whose context lengths differ widely ([P1] §4.2: sequences of every length
+ * share each decode iteration).  The (sequence, kv head, logical block) tiles
+ * of the batch, in that order, are cut into equal contiguous ranges, one per
+ * warp of a grid sized to one full wave.  A sequence lying inside one range is
+ * finished there; one cut by range boundaries leaves a partial result per
+ * piece, and the piece that completes last merges them in a fixed order with
+ * log-sum-exp weights.  One launch; no thread waits for another CTA; results
+ * are bitwise reproducible on a given GPU model.
+ *
+ *   workspace        device scratch of at least
+ *                    pa_decode_streamk_workspace_size(...) bytes, 16-byte
+ *                    aligned; no initialisation needed, contents clobbered.
+ *   counters         int32 device array of num_counters >= num_seqs *
+ *                    num_kv_heads arrival counters, entry s*Hkv + kvh for
+ *                    (sequence s, kv head kvh).  Must be all zero before the
+ *                    first call (allocate it zeroed); every completed call
+ *                    leaves the entries it used at zero, so one array serves
+ *                    successive calls of any shape.  Zero it again after a
+ *                    call that reported PA_DEVERR_TIMEOUT.
+ *   Calls that may run concurrently on the GPU need their own workspace and
+ *   counters.
+ *   num_seqs         at most 16384 (PA_ERR_UNSUPPORTED above).
+ *   Other arguments as in pa_decode.
+ */
+pa_status pa_decode_streamk(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens, float scale,
+                            int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                            int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                            void* workspace, size_t workspace_bytes, int32_t* counters,
+                            int64_t num_counters, void* stream);
 
 /*
  * pa_get_device_error — read and clear the device error word of the current

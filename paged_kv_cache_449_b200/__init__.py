@@ -17,6 +17,7 @@ import os
 import torch
 
 __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
+           "pa_decode_streamk", "pa_decode_streamk_workspace_size", "StreamKWorkspace", "Counters",
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT"]
 
@@ -60,7 +61,11 @@ def load() -> ctypes.CDLL:
     lib.pa_decode_splitk_workspace_size.restype = I
     lib.pa_decode_splitk_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
     lib.pa_decode_splitk.restype = I
-    lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P]
+    lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P, I64, P]
+    lib.pa_decode_streamk_workspace_size.restype = I
+    lib.pa_decode_streamk_workspace_size.argtypes = [I, I, I, I, I, I, c.POINTER(SZ)]
+    lib.pa_decode_streamk.restype = I
+    lib.pa_decode_streamk.argtypes = decode_args + [P, SZ, P, I64, P]
     lib.pa_get_device_error.restype = I
     lib.pa_get_device_error.argtypes = [P, c.POINTER(c.c_int32)]
     lib.pa_status_string.restype = c.c_char_p
@@ -144,20 +149,105 @@ def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context
     return int(size.value)
 
 
+class Counters:
+    """Zero-initialised int32 arrival counters for the fused merges
+    (pa_decode_splitk with fused=True, pa_decode_streamk); the kernels leave
+    them at zero, so one array is reused across calls of any shape on a
+    stream.  Grows on demand."""
+
+    def __init__(self):
+        self.buf = None
+
+    def get(self, n: int, device) -> torch.Tensor:
+        device = torch.device(device)
+        if self.buf is None or self.buf.numel() < n or self.buf.device != device:
+            self.buf = torch.zeros(max(n, 4), dtype=torch.int32, device=device)
+        return self.buf
+
+
+_default_counters: dict = {}
+_splitk_ws_cache: dict = {}
+
+
 def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
-                     partition_size=512, workspace=None, stream=None):
+                     partition_size=512, workspace=None, fused=True, counters=None, stream=None):
     """Split-K paged decode (partitions of partition_size tokens + log-sum-exp
     merge).  `workspace` is a CUDA uint8 tensor of at least
-    pa_decode_splitk_workspace_size(...) bytes; allocated here if None."""
+    pa_decode_splitk_workspace_size(...) bytes (allocated here if None).
+    fused=True merges inside the partition kernel using `counters` (a
+    Counters; a per-device default if None); fused=False launches the
+    separate merge kernel."""
     lib = load()
     S, Hq, D = q.shape
-    need = pa_decode_splitk_workspace_size(S, Hq, D, int(max_context_len), partition_size)
+    hkv = k_cache.shape[1]
+    key = (S, Hq, D, int(max_context_len), partition_size)
+    need = _splitk_ws_cache.get(key)
+    if need is None:
+        need = _splitk_ws_cache[key] = pa_decode_splitk_workspace_size(S, Hq, D, int(max_context_len),
+                                                                        partition_size)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    cptr, ncount = None, 0
+    if fused:
+        if counters is None:
+            counters = _default_counters.setdefault(q.device.index, Counters())
+        buf = counters.get(S * hkv, q.device) if isinstance(counters, Counters) else counters
+        cptr, ncount = _dev_ptr(buf, "counters"), buf.numel()
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_splitk(*args, int(partition_size), _dev_ptr(workspace, "workspace"),
-                                workspace.numel() * workspace.element_size(), _stream(stream)),
+                                workspace.numel() * workspace.element_size(), cptr, ncount, _stream(stream)),
            "pa_decode_splitk")
+
+
+def pa_decode_streamk_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, dtype) -> int:
+    """Workspace bytes of pa_decode_streamk on the current device."""
+    lib = load()
+    size = ctypes.c_size_t(0)
+    _check(lib.pa_decode_streamk_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                                _DTYPE[dtype], ctypes.byref(size)),
+           "pa_decode_streamk_workspace_size")
+    return int(size.value)
+
+
+class StreamKWorkspace:
+    """Scratch for pa_decode_streamk on one device and stream: the partial
+    records (uninitialised) and the arrival counters (zero-initialised; the
+    kernel leaves them at zero, so they are reused across calls of any
+    shape).  Grows on demand."""
+
+    def __init__(self):
+        self.records = None
+        self.counters = None
+
+    def get(self, record_bytes: int, num_counters: int, device):
+        device = torch.device(device)
+        if self.records is None or self.records.numel() < record_bytes or self.records.device != device:
+            self.records = torch.empty(max(record_bytes, 16), dtype=torch.uint8, device=device)
+        if self.counters is None or self.counters.numel() < num_counters or self.counters.device != device:
+            self.counters = torch.zeros(max(num_counters, 4), dtype=torch.int32, device=device)
+        return self.records, self.counters
+
+
+_default_streamk_ws: dict = {}
+
+
+def pa_decode_streamk(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
+                      workspace=None, stream=None):
+    """Work-balanced paged decode: equal contiguous ranges of (sequence, kv
+    head, block) tiles per warp of a persistent grid, with log-sum-exp merges
+    of the sequences cut by range boundaries.  `workspace` is a
+    StreamKWorkspace (a per-device default is used if None)."""
+    lib = load()
+    n, hkv, d, b = _pool_dims(k_cache)
+    S, Hq, D = q.shape
+    need = pa_decode_streamk_workspace_size(S, Hq, hkv, D, b, q.dtype)
+    if workspace is None:
+        workspace = _default_streamk_ws.setdefault(q.device.index, StreamKWorkspace())
+    records, counters = workspace.get(need, S * hkv, q.device)
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_streamk(*args, _dev_ptr(records, "workspace"), records.numel(),
+                                 _dev_ptr(counters, "counters"), counters.numel(), _stream(stream)),
+           "pa_decode_streamk")
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -9,28 +9,64 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "pa.h"
 #include "pa_decode.cuh"
 #include "pa_reshape.cuh"
+#include "pa_streamk.cuh"
 
-// Per-warp shared-memory ring size and warps per CTA of the decode kernel.
-#ifndef PA_DECODE_WARPS
-#define PA_DECODE_WARPS 4
+// Warps per CTA and per-warp shared-memory ring bytes of each decode entry
+// point (measured on B200 over the benchmark workloads): the one-pass kernel
+// streams a whole sequence per CTA and wants more warps in flight per CTA; the
+// split-K kernel runs many short CTAs and wants more CTAs per SM.
+#ifndef PA_SINGLE_WARPS
+#define PA_SINGLE_WARPS 8
 #endif
-#ifndef PA_RING_BYTES_PER_WARP
-#define PA_RING_BYTES_PER_WARP 32768
+#ifndef PA_SINGLE_RING
+#define PA_SINGLE_RING 16384
+#endif
+#ifndef PA_SPLIT_WARPS
+#define PA_SPLIT_WARPS 4
+#endif
+#ifndef PA_SPLIT_RING
+#define PA_SPLIT_RING 12288
+#endif
+#ifndef PA_STREAM_WARPS
+#define PA_STREAM_WARPS 4
+#endif
+#ifndef PA_STREAM_RING
+#define PA_STREAM_RING 16384
 #endif
 
 namespace {
 
-template <typename T, int D, int B>
+enum class Kind { kSingle, kSplit, kStream };
+
+template <Kind K>
+struct KindTuning;
+template <>
+struct KindTuning<Kind::kSingle> {
+    static constexpr int kWarps = PA_SINGLE_WARPS, kRing = PA_SINGLE_RING;
+};
+template <>
+struct KindTuning<Kind::kSplit> {
+    static constexpr int kWarps = PA_SPLIT_WARPS, kRing = PA_SPLIT_RING;
+};
+template <>
+struct KindTuning<Kind::kStream> {
+    static constexpr int kWarps = PA_STREAM_WARPS, kRing = PA_STREAM_RING;
+};
+
+template <typename T, int D, int B, Kind K>
 struct DecodeConfig {
     static constexpr int kStageBytes = 2 * B * D * static_cast<int>(sizeof(T));  // K + V tile
     static constexpr int kRingCap = 200 * 1024;                                   // ring bytes per CTA at most
     static constexpr int kMaxWarps = kRingCap / kStageBytes;
-    static constexpr int kWarps = PA_DECODE_WARPS < kMaxWarps ? PA_DECODE_WARPS : kMaxWarps;
-    static constexpr int kRaw = PA_RING_BYTES_PER_WARP / kStageBytes;
+    static constexpr int kWarps = KindTuning<K>::kWarps < kMaxWarps ? KindTuning<K>::kWarps : kMaxWarps;
+    static constexpr int kRaw = KindTuning<K>::kRing / kStageBytes;
     static constexpr int kFit = kRingCap / (kWarps * kStageBytes);
     static constexpr int kStages0 = kRaw < 1 ? 1 : (kRaw > 16 ? 16 : kRaw);
     static constexpr int kStages = kStages0 < kFit ? kStages0 : kFit;
@@ -45,58 +81,139 @@ int elem_size(pa_dtype dt) { return dt == PA_F32 ? 4 : 2; }
 
 bool dtype_ok(int dt) { return dt == PA_F32 || dt == PA_F16 || dt == PA_BF16; }
 
-// Raises the dynamic shared-memory limit of one kernel once per device.
-template <typename Kernel>
-cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask) {
-    if (bytes <= 48 * 1024) return cudaSuccess;
+// Raises the dynamic shared-memory limit of `kernel` on the current device to
+// the device's opt-in maximum, once per (kernel, device).  Setting it to the
+// largest value (rather than to one launch's size) keeps every later launch
+// of any size within the limit.
+cudaError_t ensure_smem(const void* kernel) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, bool> done;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
-    if (bit && (done_mask.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && bit) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kernel, dev})) return cudaSuccess;
+    int optin = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes attr{};
+    e = cudaFuncGetAttributes(&attr, kernel);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - static_cast<int>(attr.sharedSizeBytes));
+    if (e == cudaSuccess) done[{kernel, dev}] = true;
     return e;
+}
+
+template <typename T>
+struct TypeTag {
+    using type = T;
+};
+template <int V>
+struct IntTag {
+    static constexpr int value = V;
+};
+
+// Calls f(TypeTag<T>, IntTag<D>, IntTag<B>) for the kernel variant of
+// (dtype, head_dim, block_size); the shape has been validated already.
+template <typename F>
+cudaError_t with_variant(pa_dtype dt, int D, int B, F&& f) {
+    auto by_block = [&](auto tt, auto dd) -> cudaError_t {
+        switch (B) {
+            case 8: return f(tt, dd, IntTag<8>{});
+            case 16: return f(tt, dd, IntTag<16>{});
+            case 32: return f(tt, dd, IntTag<32>{});
+            default: return cudaErrorInvalidValue;
+        }
+    };
+    auto by_dim = [&](auto tt) -> cudaError_t {
+        switch (D) {
+            case 64: return by_block(tt, IntTag<64>{});
+            case 128: return by_block(tt, IntTag<128>{});
+            default: return cudaErrorInvalidValue;
+        }
+    };
+    switch (dt) {
+        case PA_F32: return by_dim(TypeTag<float>{});
+        case PA_F16: return by_dim(TypeTag<__half>{});
+        case PA_BF16: return by_dim(TypeTag<__nv_bfloat16>{});
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 template <typename T, int D, int B, bool SPLIT>
 cudaError_t launch_decode(const pa::DecodeParams& p, dim3 grid, cudaStream_t stream) {
-    using C = DecodeConfig<T, D, B>;
+    using C = DecodeConfig<T, D, B, SPLIT ? Kind::kSplit : Kind::kSingle>;
     auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT>;
-    static std::atomic<uint64_t> done{0};
-    cudaError_t e = ensure_smem(kernel, C::Smem::kTotal, done);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
     kernel<<<grid, C::kWarps * 32, C::Smem::kTotal, stream>>>(p);
     return cudaGetLastError();
 }
 
-template <typename T, int D, bool SPLIT>
-cudaError_t decode_by_block(int B, const pa::DecodeParams& p, dim3 grid, cudaStream_t st) {
-    switch (B) {
-        case 8: return launch_decode<T, D, 8, SPLIT>(p, grid, st);
-        case 16: return launch_decode<T, D, 16, SPLIT>(p, grid, st);
-        case 32: return launch_decode<T, D, 32, SPLIT>(p, grid, st);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
-template <typename T, bool SPLIT>
-cudaError_t decode_by_dim(int D, int B, const pa::DecodeParams& p, dim3 grid, cudaStream_t st) {
-    switch (D) {
-        case 64: return decode_by_block<T, 64, SPLIT>(B, p, grid, st);
-        case 128: return decode_by_block<T, 128, SPLIT>(B, p, grid, st);
-        default: return cudaErrorInvalidValue;
-    }
-}
-
 template <bool SPLIT>
 cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p, dim3 grid, cudaStream_t st) {
-    switch (dt) {
-        case PA_F32: return decode_by_dim<float, SPLIT>(D, B, p, grid, st);
-        case PA_F16: return decode_by_dim<__half, SPLIT>(D, B, p, grid, st);
-        case PA_BF16: return decode_by_dim<__nv_bfloat16, SPLIT>(D, B, p, grid, st);
-        default: return cudaErrorInvalidValue;
+    return with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) {
+        using T = typename decltype(tt)::type;
+        return launch_decode<T, decltype(dd)::value, decltype(bb)::value, SPLIT>(p, grid, st);
+    });
+}
+
+// ---- stream-K: persistent grid sized to one full wave
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+// CTAs per SM of `kernel` at `smem` bytes, cached per (kernel, device, smem).
+template <typename Kernel>
+int resident_ctas(Kernel kernel, int threads, int smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, int>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const auto key = std::make_tuple(reinterpret_cast<const void*>(kernel), dev, smem);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) return it->second;
     }
+    if (ensure_smem(reinterpret_cast<const void*>(kernel)) != cudaSuccess) return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = n;
+    return n;
+}
+
+struct StreamPlan {
+    int grid = 0, threads = 0, smem = 0, workers = 0;
+};
+
+template <typename T, int D, int B>
+StreamPlan streamk_plan(int num_seqs) {
+    using C = DecodeConfig<T, D, B, Kind::kStream>;
+    using Smem = pa::StreamSmem<T, D, B, C::kWarps, C::kStages>;
+    auto kernel = pa::pa_decode_streamk_kernel<T, D, B, C::kWarps, C::kStages>;
+    StreamPlan plan;
+    plan.threads = C::kWarps * 32;
+    plan.smem = Smem::total(num_seqs);
+    const int per_sm = resident_ctas(kernel, plan.threads, plan.smem);
+    plan.grid = per_sm * sm_count();
+    plan.workers = plan.grid * C::kWarps;
+    return plan;
+}
+
+template <typename T, int D, int B>
+cudaError_t launch_streamk(pa::StreamParams p, const StreamPlan& plan, cudaStream_t stream) {
+    using C = DecodeConfig<T, D, B, Kind::kStream>;
+    auto kernel = pa::pa_decode_streamk_kernel<T, D, B, C::kWarps, C::kStages>;
+    p.workers = plan.workers;
+    kernel<<<plan.grid, plan.threads, plan.smem, stream>>>(p);
+    return cudaGetLastError();
 }
 
 template <typename T, int D>
@@ -179,6 +296,22 @@ size_t splitk_bytes(long long seqs, long long heads, long long parts, long long 
     return static_cast<size_t>(seqs * heads * parts * (head_dim + 2) * 4);
 }
 
+constexpr int kStreamMaxSeqs = 16384;  // per-CTA length prefix lives in shared memory
+
+// Stream-K workspace: partial records [workers][2][record_floats(g, D)] fp32.
+size_t streamk_bytes(long long workers, int group, int head_dim) {
+    return static_cast<size_t>(workers * 2 * pa::record_floats(group, head_dim) * 4);
+}
+
+bool streamk_plan_for(pa_dtype dt, int D, int B, int num_seqs, StreamPlan* plan) {
+    const cudaError_t e = with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) {
+        using T = typename decltype(tt)::type;
+        *plan = streamk_plan<T, decltype(dd)::value, decltype(bb)::value>(num_seqs);
+        return cudaSuccess;
+    });
+    return e == cudaSuccess && plan->grid > 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -244,7 +377,8 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
                            const int32_t* block_tables, const int32_t* context_lens, float scale,
                            int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                            int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
-                           int partition_size, void* workspace, size_t workspace_bytes, void* stream) {
+                           int partition_size, void* workspace, size_t workspace_bytes, int32_t* counters,
+                           int64_t num_counters, void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
@@ -264,11 +398,17 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
     p.part_ml = acc + static_cast<size_t>(num_seqs) * num_q_heads * parts * head_dim;
     p.partition_blocks = pb;
     p.num_partitions = static_cast<int>(parts);
+    if (counters != nullptr) {
+        if (!aligned4(counters) || num_counters < static_cast<int64_t>(num_seqs) * num_kv_heads)
+            return PA_ERR_WORKSPACE;
+        p.counters = counters;
+    }
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (parts > 0) {
         const dim3 grid(static_cast<unsigned>(parts), num_kv_heads, num_seqs);
         const cudaError_t e = decode_dispatch<true>(dtype, head_dim, block_size, p, grid, s);
         if (e != cudaSuccess) return PA_ERR_CUDA;
+        if (counters != nullptr) return PA_OK;  // merged inside the partition kernel
     }
     pa::MergeParams m{};
     m.out = out;
@@ -282,6 +422,68 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
     m.partition_blocks = pb;
     m.num_partitions = static_cast<int>(parts);
     return merge_dispatch(dtype, head_dim, m, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_streamk_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                           int block_size, pa_dtype dtype, size_t* bytes) {
+    if (!bytes || num_seqs < 0) return PA_ERR_INVALID_ARG;
+    // Shape checks only (an empty batch needs no pointers).
+    const DecodeShape shape_only{block_size, 0, num_q_heads, num_kv_heads, head_dim, 0, 0, 1, static_cast<int>(dtype)};
+    const pa_status st = check_decode(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 1.f, shape_only);
+    if (st != PA_OK) return st;
+    if (num_seqs > kStreamMaxSeqs) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) {
+        *bytes = 0;
+        return PA_OK;
+    }
+    StreamPlan plan;
+    if (!streamk_plan_for(dtype, head_dim, block_size, num_seqs, &plan)) return PA_ERR_CUDA;
+    *bytes = streamk_bytes(plan.workers, num_q_heads / num_kv_heads, head_dim);
+    return PA_OK;
+}
+
+pa_status pa_decode_streamk(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens, float scale, int block_size,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                            int max_context_len, int64_t num_blocks, pa_dtype dtype, void* workspace,
+                            size_t workspace_bytes, int32_t* counters, int64_t num_counters, void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (st != PA_OK) return st;
+    if (num_seqs > kStreamMaxSeqs) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (!counters || !aligned4(counters) || num_counters < static_cast<int64_t>(num_seqs) * num_kv_heads)
+        return PA_ERR_WORKSPACE;
+    StreamPlan plan;
+    if (!streamk_plan_for(dtype, head_dim, block_size, num_seqs, &plan)) return PA_ERR_CUDA;
+    const int group = num_q_heads / num_kv_heads;
+    const size_t need = streamk_bytes(plan.workers, group, head_dim);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
+    const pa::DecodeParams d = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    pa::StreamParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.records = static_cast<float*>(workspace);
+    p.counters = counters;
+    p.score_scale = d.score_scale;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = group;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.context_cap = d.context_cap;
+    p.num_blocks = num_blocks;
+    const cudaError_t e = with_variant(dtype, head_dim, block_size, [&](auto tt, auto dd, auto bb) {
+        using T = typename decltype(tt)::type;
+        return launch_streamk<T, decltype(dd)::value, decltype(bb)::value>(p, plan,
+                                                                           static_cast<cudaStream_t>(stream));
+    });
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(void* stream, int32_t* code) {

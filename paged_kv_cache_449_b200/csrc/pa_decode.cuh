@@ -31,7 +31,7 @@
 //    (acc, m, l) to the workspace and pa_merge_kernel combines partitions.
 #pragma once
 
-#include "pa_device.cuh"
+#include "pa_warp.cuh"
 
 namespace pa {
 
@@ -54,19 +54,48 @@ struct DecodeParams {
     long long num_blocks;
     int partition_blocks;  // split: blocks per partition
     int num_partitions;    // split: P
+    int* counters;         // split, fused merge: [S*Hkv] arrival counters (zero between calls); null = merge kernel
 };
 
-constexpr int kMaxGroup = 8;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait, far above any copy time
+// Fused split-K merge, run by the CTA that completes the last partition of
+// (sequence s, kv head kvh): combines the np partial results of each of the
+// group's query heads in partition order with a running maximum (the
+// log-sum-exp merge) and writes the output rows.  Threads own 16-byte slices.
+template <typename T, int D, bool LOG2, int THREADS>
+__device__ __forceinline__ void merge_partitions_cta(const DecodeParams& p, int s, int kvh, int np) {
+    const int group = p.group;
+    const int slices = group * D / 4;
+    for (int v = threadIdx.x; v < slices; v += THREADS) {
+        const int r = (4 * v) / D;
+        const long long row = static_cast<long long>(s) * p.num_q_heads + kvh * group + r;
+        const float* ml = p.part_ml + row * p.num_partitions * 2;
+        const float4* acc = reinterpret_cast<const float4*>(p.part_acc + row * p.num_partitions * D) + (v % (D / 4));
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        float M = kNegInf, den = 0.f;
+#pragma unroll 4
+        for (int q = 0; q < np; ++q) {
+            const float m = __ldcg(ml + 2 * q), l = __ldcg(ml + 2 * q + 1);
+            const float4 x = __ldcg(acc + static_cast<long long>(q) * (D / 4));
+            const float mn = fmaxf(M, m);
+            if (mn != kNegInf) {
+                const float sa = softmax_exp<LOG2>(M - mn), sb = softmax_exp<LOG2>(m - mn);
+                a.x = fmaf(a.x, sa, x.x * sb);
+                a.y = fmaf(a.y, sa, x.y * sb);
+                a.z = fmaf(a.z, sa, x.z * sb);
+                a.w = fmaf(a.w, sa, x.w * sb);
+                den = fmaf(den, sa, l * sb);
+                M = mn;
+            }
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        T* dst = reinterpret_cast<T*>(p.out) + row * D + 4 * (v % (D / 4));
+        dst[0] = from_float<T>(a.x * inv);
+        dst[1] = from_float<T>(a.y * inv);
+        dst[2] = from_float<T>(a.z * inv);
+        dst[3] = from_float<T>(a.w * inv);
+    }
+}
 
-template <typename T>
-struct IsF32 {
-    static constexpr bool value = false;
-};
-template <>
-struct IsF32<float> {
-    static constexpr bool value = true;
-};
 
 template <typename T, int D, int B, int NW, int STAGES>
 struct DecodeSmem {
@@ -78,292 +107,6 @@ struct DecodeSmem {
     static constexpr int kBars = (NW * STAGES * 8 + 15) / 16 * 16;  // keeps what follows 16-byte aligned
     static constexpr int kQ = IsF32<T>::value ? kMaxGroup * D * 4 : 0;
     static constexpr int kTotal = kArea + kBars + kQ;
-};
-
-// ----------------------------------------------------------------------------
-// Per-warp accumulator state and block computation, 16-bit inputs (tensor cores)
-
-template <typename T, int D, int B>
-struct WarpMma {
-    static constexpr int kNt = B / 8;  // 8-token n-tiles per block
-    float o[D / 8][4];                 // out^ rows (r, r+8) x d-tile
-    uint32_t qa[D / 16][2];            // Q A-fragments: row r, k = 2c.., 8+2c..
-    float m_run = kNegInf;             // row r, score domain (base 2)
-    float l_run = 0.f;                 // this thread's share of row r's sum
-
-    __device__ __forceinline__ void init(const T* q_rows, int group, int lane) {
-        const int r = lane >> 2, c = lane & 3;
-#pragma unroll
-        for (int j = 0; j < D / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            if (r < group) {
-                const T* row = q_rows + r * D + ks * 16 + 2 * c;
-                qa[ks][0] = *reinterpret_cast<const uint32_t*>(row);
-                qa[ks][1] = *reinterpret_cast<const uint32_t*>(row + 8);
-            } else {
-                qa[ks][0] = qa[ks][1] = 0u;
-            }
-        }
-    }
-
-    // Zero the 16-bit halves of a V fragment register that belong to tokens
-    // >= valid (token `tok` in the low half, tok+1 in the high half).
-    static __device__ __forceinline__ uint32_t mask_pair(uint32_t v, int tok, int valid) {
-        const uint32_t keep = (tok < valid ? 0x0000ffffu : 0u) | (tok + 1 < valid ? 0xffff0000u : 0u);
-        return v & keep;
-    }
-
-    __device__ __forceinline__ void block(uint32_t kbase, uint32_t vbase, int valid, int group, float scale_log2,
-                                          int lane) {
-        const int r = lane >> 2, c = lane & 3;
-        const int mtx = lane >> 3, row = lane & 7;
-        float sc[kNt][4];
-#pragma unroll
-        for (int nt = 0; nt < kNt; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-
-        // S = Q K^T: M = query rows, N = tokens, K = head dim.
-        if constexpr (B >= 16) {
-#pragma unroll
-            for (int np = 0; np < kNt / 2; ++np) {
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const int tok = np * 16 + (mtx >> 1) * 8 + row;
-                    const int chunk = 2 * ks + (mtx & 1);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kbase + (chunk * B + tok) * 16, b0, b1, b2, b3);
-                    Mma<T>::k16(sc[2 * np], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-                    Mma<T>::k16(sc[2 * np + 1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int kq = 0; kq < D / 32; ++kq) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kbase + ((4 * kq + mtx) * 8 + row) * 16, b0, b1, b2, b3);
-                Mma<T>::k16(sc[0], qa[2 * kq][0], 0u, qa[2 * kq][1], 0u, b0, b1);
-                Mma<T>::k16(sc[0], qa[2 * kq + 1][0], 0u, qa[2 * kq + 1][1], 0u, b2, b3);
-            }
-        }
-
-        // Online softmax on row r (rows r+8 are padding and stay zero).
-        const bool row_ok = r < group;
-        float mx = kNegInf;
-#pragma unroll
-        for (int nt = 0; nt < kNt; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int tok = nt * 8 + 2 * c + e;
-                const float x = (row_ok && tok < valid) ? sc[nt][e] * scale_log2 : kNegInf;
-                sc[nt][e] = x;
-                mx = fmaxf(mx, x);
-            }
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run, mx);
-        const float m_use = (m_new == kNegInf) ? 0.f : m_new;
-        const float alpha = exp2_approx(m_run - m_use);
-        float rs = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < kNt; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float pv = exp2_approx(sc[nt][e] - m_use);
-                sc[nt][e] = pv;
-                rs += pv;
-            }
-        }
-        l_run = l_run * alpha + rs;
-        m_run = m_new;
-#pragma unroll
-        for (int j = 0; j < D / 8; ++j) {
-            o[j][0] *= alpha;
-            o[j][1] *= alpha;
-        }
-
-        // O += P V: M = query rows, N = head dim, K = tokens.
-        const bool partial = valid < B;
-        if constexpr (B >= 16) {
-#pragma unroll
-            for (int kp = 0; kp < kNt / 2; ++kp) {
-                const uint32_t a0 = Mma<T>::pack(sc[2 * kp][0], sc[2 * kp][1]);
-                const uint32_t a2 = Mma<T>::pack(sc[2 * kp + 1][0], sc[2 * kp + 1][1]);
-                const int tlo = kp * 16 + 2 * c, thi = kp * 16 + 8 + 2 * c;
-#pragma unroll
-                for (int dj = 0; dj < D / 16; ++dj) {
-                    const int tok = kp * 16 + (mtx & 1) * 8 + row;
-                    const int chunk = 2 * dj + (mtx >> 1);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(vbase + (chunk * B + tok) * 16, b0, b1, b2, b3);
-                    if (partial) {
-                        b0 = mask_pair(b0, tlo, valid);
-                        b1 = mask_pair(b1, thi, valid);
-                        b2 = mask_pair(b2, tlo, valid);
-                        b3 = mask_pair(b3, thi, valid);
-                    }
-                    Mma<T>::k16(o[2 * dj], a0, 0u, a2, 0u, b0, b1);
-                    Mma<T>::k16(o[2 * dj + 1], a0, 0u, a2, 0u, b2, b3);
-                }
-            }
-        } else {
-            const uint32_t a0 = Mma<T>::pack(sc[0][0], sc[0][1]);
-#pragma unroll
-            for (int dq = 0; dq < D / 32; ++dq) {
-                uint32_t b[4];
-                ldsm_x4_trans(vbase + ((4 * dq + mtx) * 8 + row) * 16, b[0], b[1], b[2], b[3]);
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    if (partial) b[m] = mask_pair(b[m], 2 * c, valid);
-                    Mma<T>::k8(o[4 * dq + m], a0, 0u, b[m]);
-                }
-            }
-        }
-    }
-
-    // Writes this warp's (m, l, o) for its valid rows into the merge area.
-    __device__ __forceinline__ void store(float* mo, float* mml, int warp, int group, int lane) {
-        const int r = lane >> 2, c = lane & 3;
-        float l = l_run;
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        if (r < group) {
-            float* dst = mo + (warp * kMaxGroup + r) * D;
-#pragma unroll
-            for (int j = 0; j < D / 8; ++j) {
-                dst[8 * j + 2 * c] = o[j][0];
-                dst[8 * j + 2 * c + 1] = o[j][1];
-            }
-            if (c == 0) {
-                mml[(warp * kMaxGroup + r) * 2] = m_run;
-                mml[(warp * kMaxGroup + r) * 2 + 1] = l;
-            }
-        }
-    }
-};
-
-// ----------------------------------------------------------------------------
-// fp32 inputs (CUDA cores)
-
-template <int D, int B>
-struct WarpF32 {
-    static constexpr int kC = D / 4;          // 16-byte vectors per token row
-    static constexpr int kTg = 32 / B;        // lanes sharing one token in QK^T
-    static constexpr int kCpp = kC / kTg;     // vectors per lane in QK^T
-    static constexpr int kGrp = 32 / kC;      // token groups in PV (1 for D=128, 2 for D=64)
-    float o[kMaxGroup][4];
-    float m_run[kMaxGroup];
-    float l_run[kMaxGroup];
-
-    __device__ __forceinline__ void init() {
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
-            m_run[h] = kNegInf;
-            l_run[h] = 0.f;
-        }
-    }
-
-    __device__ __forceinline__ void block(const float* ktile, const float* vtile, const float* qs, int valid,
-                                          int group, float scale, int lane) {
-        const int t = lane % B, part = lane / B;
-        float s[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) s[h] = 0.f;
-#pragma unroll 4
-        for (int cc = 0; cc < kCpp; ++cc) {
-            const int chunk = part * kCpp + cc;
-            const float4 kv = *reinterpret_cast<const float4*>(ktile + (chunk * B + t) * 4);
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) {
-                if (h < group) {
-                    const float4 qv = *reinterpret_cast<const float4*>(qs + h * D + chunk * 4);
-                    s[h] = fmaf(qv.x, kv.x, s[h]);
-                    s[h] = fmaf(qv.y, kv.y, s[h]);
-                    s[h] = fmaf(qv.z, kv.z, s[h]);
-                    s[h] = fmaf(qv.w, kv.w, s[h]);
-                }
-            }
-        }
-        float p[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h >= group) {
-                p[h] = 0.f;
-                continue;
-            }
-#pragma unroll
-            for (int off = B; off < 32; off <<= 1) s[h] += __shfl_xor_sync(0xffffffffu, s[h], off);
-            const float x = (t < valid) ? s[h] * scale : kNegInf;
-            float mx = x;
-#pragma unroll
-            for (int off = 1; off < B; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float m_new = fmaxf(m_run[h], mx);
-            const float m_use = (m_new == kNegInf) ? 0.f : m_new;
-            const float alpha = expf(m_run[h] - m_use);
-            const float pv = expf(x - m_use);
-            float sum = (part == 0) ? pv : 0.f;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            l_run[h] = l_run[h] * alpha + sum;
-            m_run[h] = m_new;
-            o[h][0] *= alpha;
-            o[h][1] *= alpha;
-            o[h][2] *= alpha;
-            o[h][3] *= alpha;
-            p[h] = pv;
-        }
-        // PV: lane owns vector cj of D for the tokens of group tg.
-        const int cj = lane % kC, tg = lane / kC;
-        constexpr int kPer = B / kGrp;
-#pragma unroll 4
-        for (int ii = 0; ii < kPer; ++ii) {
-            const int tt = ((ii + cj) % kPer) * kGrp + tg;  // rotated so a quarter-warp hits 8 banks
-            float4 vv = *reinterpret_cast<const float4*>(vtile + (cj * B + tt) * 4);
-            if (tt >= valid) vv = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) {
-                const float ph = __shfl_sync(0xffffffffu, p[h], tt);
-                if (h < group) {
-                    o[h][0] = fmaf(ph, vv.x, o[h][0]);
-                    o[h][1] = fmaf(ph, vv.y, o[h][1]);
-                    o[h][2] = fmaf(ph, vv.z, o[h][2]);
-                    o[h][3] = fmaf(ph, vv.w, o[h][3]);
-                }
-            }
-        }
-    }
-
-    __device__ __forceinline__ void store(float* mo, float* mml, int warp, int group, int lane) {
-        const int cj = lane % kC, tg = lane / kC;
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if constexpr (kGrp == 2) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], 16);
-            }
-            if (h < group && tg == 0) {
-                float* dst = mo + (warp * kMaxGroup + h) * D + cj * 4;
-                dst[0] = o[h][0];
-                dst[1] = o[h][1];
-                dst[2] = o[h][2];
-                dst[3] = o[h][3];
-            }
-            if (h < group && lane == 0) {
-                mml[(warp * kMaxGroup + h) * 2] = m_run[h];
-                mml[(warp * kMaxGroup + h) * 2 + 1] = l_run[h];
-            }
-        }
-    }
-};
-
-template <typename T, int D, int B>
-struct WarpState {
-    using type = WarpMma<T, D, B>;
-};
-template <int D, int B>
-struct WarpState<float, D, B> {
-    using type = WarpF32<D, B>;
 };
 
 // ----------------------------------------------------------------------------
@@ -396,6 +139,12 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     int b0 = 0, b1 = nblk;
     if constexpr (SPLIT) {
         b0 = part * p.partition_blocks;
+        if (nblk == 0 && part == 0 && p.counters != nullptr) {
+            // Fused merge: no partition runs for an empty context, so its
+            // output rows are zeroed here.
+            T* out = reinterpret_cast<T*>(p.out) + (static_cast<long long>(s) * p.num_q_heads + kvh * group) * D;
+            for (int i = threadIdx.x; i < group * D; i += NW * 32) out[i] = from_float<T>(0.f);
+        }
         if (b0 >= nblk) return;  // this partition is past the end of the sequence
         b1 = min(nblk, b0 + p.partition_blocks);
     }
@@ -467,10 +216,11 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     };
 
     typename WarpState<T, D, B>::type acc;
+    acc.reset();
     if constexpr (kF32) {
-        acc.init();
+        acc.qs = qs;
     } else {
-        acc.init(qrows, group, lane);
+        acc.load_q(qrows, group, lane);
     }
 
     int issued = n_w < STAGES ? n_w : STAGES;
@@ -493,8 +243,8 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         const int valid = id < 0 ? 0 : min(B, L - j * B);
         uint8_t* stage = wring + st * 2 * kTile;
         if constexpr (kF32) {
-            acc.block(reinterpret_cast<const float*>(stage), reinterpret_cast<const float*>(stage + kTile), qs,
-                      valid, group, p.score_scale, lane);
+            acc.block(reinterpret_cast<const float*>(stage), reinterpret_cast<const float*>(stage + kTile), valid,
+                      group, p.score_scale, lane);
         } else {
             acc.block(smem_u32(stage), smem_u32(stage + kTile), valid, group, p.score_scale, lane);
         }
@@ -515,10 +265,14 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     // ---- merge the warps' states (the ring is free now)
     float* mo = reinterpret_cast<float*>(smem);
     float* mml = mo + NW * kMaxGroup * D;
-    acc.store(mo, mml, warp, group, lane);
+    acc.store_smem(mo, mml, warp, group, lane);
     __syncthreads();
 
     constexpr bool kLog2 = !kF32;
+    // Split mode writes fp32 partials, except that with the fused merge a
+    // sequence with a single partition is finished here.
+    const int num_parts = SPLIT ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
+    const bool to_workspace = SPLIT && !(p.counters != nullptr && num_parts == 1);
     for (int idx = threadIdx.x; idx < group * D; idx += NW * 32) {
         const int r = idx / D, d = idx - r * D;
         float M = kNegInf;
@@ -534,7 +288,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
             }
         }
         const int h = kvh * group + r;
-        if constexpr (SPLIT) {
+        if (to_workspace) {
             const long long slot = (static_cast<long long>(s) * p.num_q_heads + h) * p.num_partitions + part;
             p.part_acc[slot * D + d] = num;
             if (d == 0) {
@@ -544,6 +298,24 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         } else {
             T* out = reinterpret_cast<T*>(p.out) + (static_cast<long long>(s) * p.num_q_heads + h) * D;
             out[d] = from_float<T>(den > 0.f ? num / den : 0.f);
+        }
+    }
+    if constexpr (SPLIT) {
+        if (p.counters != nullptr && to_workspace) {
+            // Fused merge: the CTA that records the last partition merges them.
+            __shared__ int last_arrival;
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                const int old = atomicAdd(p.counters + static_cast<long long>(s) * p.num_kv_heads + kvh, 1);
+                last_arrival = old == num_parts - 1;
+            }
+            __syncthreads();
+            if (last_arrival) {
+                __threadfence();
+                merge_partitions_cta<T, D, kLog2, NW * 32>(p, s, kvh, num_parts);
+                if (threadIdx.x == 0) p.counters[static_cast<long long>(s) * p.num_kv_heads + kvh] = 0;
+            }
         }
     }
 }

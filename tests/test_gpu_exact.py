@@ -135,7 +135,7 @@ def test_needle_every_position(dtype, B, mode, part):
 def test_permutation_invariance_bit_exact():
     b = workloads.continuous_batching_mix(seed=2, device="cuda", num_seqs=40)
     c = permute_physical(b, seed=9)
-    for mode in ("single", "splitk"):
+    for mode in ("single", "splitk", "splitk2", "streamk"):
         assert torch.equal(_bits(gpu_decode(b, mode)), _bits(gpu_decode(c, mode)))
 
 
@@ -144,7 +144,7 @@ def test_shared_vs_copied_bit_exact(prefix_len):
     b = workloads.prefix_sharing(seed=1, device="cuda", prefix_len=prefix_len, num_seqs=16)
     twin = materialize_shared(b)
     assert twin.num_blocks > b.num_blocks
-    for mode in ("single", "splitk"):
+    for mode in ("single", "splitk", "splitk2", "streamk"):
         assert torch.equal(_bits(gpu_decode(b, mode)), _bits(gpu_decode(twin, mode)))
 
 
@@ -154,14 +154,14 @@ def test_block_size_within_tolerance(orc):
     ref = orc.decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale, 16, 8)
     for nb in (8, 32):
         c = relayout_block_size(b, nb)
-        for mode in ("single", "splitk"):
+        for mode in ("single", "splitk", "splitk2", "streamk"):
             check_tolerance(as_f64(gpu_decode(c, mode)), ref, b.dtype)
 
 
 def test_run_to_run_deterministic():
     b = workloads.llama3_8b_decode(seed=3, device="cuda", num_seqs=16, num_blocks=4096)
     dev = device_batch(b)
-    for mode in ("single", "splitk"):
+    for mode in ("single", "splitk", "splitk2", "streamk"):
         first = gpu_decode(b, mode, dev=dev)
         for _ in range(3):
             assert torch.equal(_bits(first), _bits(gpu_decode(b, mode, dev=dev)))
@@ -177,7 +177,7 @@ def test_out_of_range_block_id_is_flagged_not_read():
     bad[0, 1] = b.num_blocks + 1000
     bad[1, 0] = -7
     c = b.__class__(**{**b.__dict__, "block_tables": bad})
-    for mode in ("single", "splitk"):
+    for mode in ("single", "splitk", "splitk2", "streamk"):
         out = gpu_decode(c, mode)
         assert torch.isfinite(out.float()).all()
         assert pa.pa_get_device_error() & pa.DEVERR_BLOCK_ID
