@@ -214,6 +214,42 @@ pa_status pa_decode_streamk(void* out, const void* q, const void* k_cache, const
                             int64_t num_counters, void* stream);
 
 /*
+ * pa_decode_splitk_static — pa_decode_splitk for callers that cannot
+ * allocate device memory when they launch work (for example a plugin of an
+ * inference runtime that is handed only its inputs and outputs at enqueue
+ * time, or a latency-critical loop where cudaMalloc's implicit device
+ * synchronisation would stall other streams).  The pages describe no such
+ * entry point; it exists for those callers only.
+ *
+ * The caller passes inputs and outputs exactly as for pa_decode_splitk, but
+ * no workspace: the fp32 partials are kept in one fixed array of
+ * PA_SPLITK_STATIC_SCRATCH_BYTES bytes inside the library's device image,
+ * which every GPU that loads the library holds until the process exits.  The
+ * library allocates nothing.  The merge runs as the second kernel (the form
+ * of pa_decode_splitk without counters), so nothing in the array has to start
+ * at zero and the contents left by an earlier call are never read.
+ *
+ *   Requests whose partials need more than PA_SPLITK_STATIC_SCRATCH_BYTES
+ *   (num_seqs * num_q_heads * ceil(max_context_len / partition_size) *
+ *   (head_dim + 2) * 4 bytes) are refused with PA_ERR_WORKSPACE before any
+ *   device work; use a larger partition_size or pa_decode_splitk.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture.
+ *   Every call on a device shares the one array: calls that may overlap on
+ *   the GPU (different streams without ordering between them) race on it and
+ *   must not be issued.
+ *   Other arguments, results and errors as in pa_decode_splitk.
+ */
+#define PA_SPLITK_STATIC_SCRATCH_BYTES (16u << 20)
+
+pa_status pa_decode_splitk_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                  int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int max_blocks_per_seq, int max_context_len,
+                                  int64_t num_blocks, pa_dtype dtype, int partition_size, void* stream);
+
+/*
  * pa_get_device_error — read and clear the device error word of the current
  * GPU.  Synchronises `stream` first, so it reports every launch enqueued on it
  * before the call.  *code receives an OR of PA_DEVERR_* bits (0 = no error).

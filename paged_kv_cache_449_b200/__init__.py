@@ -18,6 +18,7 @@ import torch
 
 __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
            "pa_decode_streamk", "pa_decode_streamk_workspace_size", "StreamKWorkspace", "Counters",
+           "pa_decode_splitk_static", "SPLITK_STATIC_SCRATCH_BYTES",
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT"]
 
@@ -66,6 +67,8 @@ def load() -> ctypes.CDLL:
     lib.pa_decode_streamk_workspace_size.argtypes = [I, I, I, I, I, I, c.POINTER(SZ)]
     lib.pa_decode_streamk.restype = I
     lib.pa_decode_streamk.argtypes = decode_args + [P, SZ, P, I64, P]
+    lib.pa_decode_splitk_static.restype = I
+    lib.pa_decode_splitk_static.argtypes = decode_args + [I, P]
     lib.pa_get_device_error.restype = I
     lib.pa_get_device_error.argtypes = [P, c.POINTER(c.c_int32)]
     lib.pa_status_string.restype = c.c_char_p
@@ -248,6 +251,25 @@ def pa_decode_streamk(out, q, k_cache, v_cache, block_tables, context_lens, scal
     _check(lib.pa_decode_streamk(*args, _dev_ptr(records, "workspace"), records.numel(),
                                  _dev_ptr(counters, "counters"), counters.numel(), _stream(stream)),
            "pa_decode_streamk")
+
+
+SPLITK_STATIC_SCRATCH_BYTES = 16 << 20
+
+
+def pa_decode_splitk_static(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                            partition_size=512, stream=None):
+    """Split-K paged decode that allocates nothing: for callers that cannot
+    allocate device memory when they launch work (runtime plugins handed only
+    inputs and outputs, latency-critical loops that must not trigger
+    cudaMalloc's implicit synchronisation).  The partials live in a fixed
+    SPLITK_STATIC_SCRATCH_BYTES array inside libpa's device image; larger
+    requests raise PagedAttentionError (PA_ERR_WORKSPACE).  All calls on a
+    device share that array, so calls must not overlap on the GPU.  The first
+    call on a device resolves the array's address; make it before any stream
+    capture."""
+    lib = load()
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_splitk_static(*args, int(partition_size), _stream(stream)), "pa_decode_splitk_static")
 
 
 def pa_get_device_error(stream=None) -> int:

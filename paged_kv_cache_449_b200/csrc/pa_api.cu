@@ -509,3 +509,62 @@ const char* pa_status_string(pa_status status) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Split-K decode with library-owned scratch (no allocation by the caller or
+// the library).  Some callers cannot allocate device memory when they launch
+// work: plugins of inference runtimes that are handed only their inputs and
+// outputs at enqueue time, or latency-critical loops where cudaMalloc's
+// implicit device synchronisation would stall other streams.  For them, the
+// fp32 partial results live in one fixed array in the library's device image.
+
+namespace {
+
+// The array is part of the module, so every GPU that loads the library holds
+// it until the process exits.
+constexpr size_t kStaticScratchBytes = PA_SPLITK_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) float g_splitk_scratch[kStaticScratchBytes / sizeof(float)];
+
+// Device address of g_splitk_scratch on the current device.  In host code
+// the name g_splitk_scratch is only a host-side stand-in, so the address is
+// looked up once per device (with that device current) and cached.
+pa_status static_scratch_address(void** ptr) {
+    static std::mutex mu;
+    static void* cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_splitk_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+        cached[dev] = p;
+    }
+    *ptr = cached[dev];
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_splitk_static(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                             const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                             int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                                             int head_dim, int max_blocks_per_seq, int max_context_len,
+                                             int64_t num_blocks, pa_dtype dtype, int partition_size,
+                                             void* stream) {
+    // Requests whose partials do not fit the fixed array are refused before
+    // any device work.
+    size_t need = 0;
+    const pa_status size_status =
+        pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size, &need);
+    if (size_status != PA_OK) return size_status;
+    if (need > kStaticScratchBytes) return PA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const pa_status addr_status = static_scratch_address(&scratch);
+    if (addr_status != PA_OK) return addr_status;
+    // Two-launch form (no arrival counters): the partition kernel writes every
+    // partial that the merge kernel reads, so no part of the array has to
+    // start at zero, and the previous call's leftovers are never read.
+    return pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size, num_seqs,
+                            num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, max_context_len, num_blocks,
+                            dtype, partition_size, scratch, kStaticScratchBytes, nullptr, 0, stream);
+}

@@ -34,7 +34,7 @@ def lib():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size", "pa_decode_streamk",
-        "pa_decode_streamk_workspace_size", "pa_get_device_error",
+        "pa_decode_streamk_workspace_size", "pa_decode_splitk_static", "pa_get_device_error",
         "pa_reshape_and_cache", "pa_status_string"])
 
 
