@@ -83,6 +83,29 @@ def make_workload(name, seed, device, block_size=None):
     return workloads.CONFIGS[name](**kw)
 
 
+# DRAM bytes (read + write) per launch of the timed decode kernel, from one
+# Nsight Compute capture (dram__bytes_read.sum + dram__bytes_write.sum; summaries
+# in profiles/).  Keyed by a hash of the kernel sources: once the kernels change,
+# the figure no longer describes them and the bench reports null.
+NCU_TRAFFIC = {
+    "2fdb1e40bbfedd82": {
+        ("llama3_8b_decode_bf16", "single"): 292.467712e6 + 4.382976e6,
+        ("llama3_70b_long_bf16", "splitk"): 2.519324e9 + 8.799488e6,
+    },
+}
+
+
+def kernel_source_hash():
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_kv_cache_449_b200", "csrc", "*.cu*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def step_bytes(batch):
     """Algorithmic bytes of one step: the decode's (K/V + Q + out + block-table
     entries + context_lens) and the reshape's (new K/V read + written, slots)."""
@@ -385,7 +408,7 @@ def run_gpu(args, world, rank, local):
             "frac": round(achieved / peak, 4),
             "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
             "algorithmic_bytes_per_launch": int(decode_bytes),
-            "traffic": None,
+            "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get((batch.name, mode)),
         },
         "gpu_launches": int(step.kernels_per_step * args.steps),
         "clocks": clk,
