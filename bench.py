@@ -1,7 +1,7 @@
 """Benchmark of the paged decode hot path: one step = write the newest token of
 every sequence into the KV pool (pa_reshape_and_cache) + paged decode attention
-over every sequence's whole context (pa_decode, pa_decode_splitk or
-pa_decode_streamk, --mode).
+over every sequence's whole context (pa_decode_append by default: both in one
+launch; or pa_reshape_and_cache followed by pa_decode / pa_decode_splitk, --mode).
 
 Default workload: Llama-3-8B-shaped single-layer decode, bf16 — 64 sequences,
 32 q / 8 kv heads, head_dim 128, block size 16, context lengths uniform on
@@ -53,8 +53,10 @@ def parse_args(argv=None):
                     choices=["tiny_mha_f32", "llama3_8b_decode", "continuous_batching_mix", "prefix_sharing",
                              "llama3_70b_long"])
     ap.add_argument("--block-size", type=int, default=None)
-    ap.add_argument("--mode", choices=["single", "splitk", "splitk2", "streamk"], default="single",
-                    help="decode entry point: pa_decode, pa_decode_splitk or pa_decode_streamk")
+    ap.add_argument("--mode", choices=["append", "single", "splitk", "splitk2"], default="append",
+                    help="append: one pa_decode_append launch per step (write + decode); the others launch "
+                         "pa_reshape_and_cache then pa_decode (single) or pa_decode_splitk with fused (splitk) or "
+                         "kernel (splitk2) merge")
     ap.add_argument("--partition-size", type=int, default=1024)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between steps")
@@ -236,17 +238,18 @@ class Step:
         need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
                                                   self.part)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-        self.sk_ws = pa.StreamKWorkspace()
         self.counters = pa.Counters()
-        self.kernels_per_step = 1 + (2 if mode == "splitk2" else 1)
+        self.kernels_per_step = {"append": 1, "splitk2": 3}.get(mode, 2)
 
     def reshape(self, stream):
+        if self.mode == "append":
+            return  # the newest token is written by the decode launch itself
         self.pa.pa_reshape_and_cache(self.nk, self.nv, self.k, self.v, self.slots, stream=stream)
 
     def decode(self, stream):
-        if self.mode == "streamk":
-            self.pa.pa_decode_streamk(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale,
-                                      max_context_len=self.mcl, workspace=self.sk_ws, stream=stream)
+        if self.mode == "append":
+            self.pa.pa_decode_append(self.out, self.q, self.nk, self.nv, self.k, self.v, self.bt, self.cl, self.b.scale,
+                                     max_context_len=self.mcl, stream=stream)
         elif self.mode in ("splitk", "splitk2"):
             self.pa.pa_decode_splitk(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale, self.mcl,
                                      partition_size=self.part, workspace=self.ws, fused=(self.mode == "splitk"),
@@ -275,8 +278,9 @@ def run_gpu(args, world, rank, local):
             return
         e0, e1, e2 = timed_events
         e0.record(stream)
-        step.reshape(stream)
-        e1.record(stream)
+        if step.mode != "append":  # append: the whole step is the decode launch
+            step.reshape(stream)
+            e1.record(stream)
         step.decode(stream)
         e2.record(stream)
 
@@ -300,8 +304,12 @@ def run_gpu(args, world, rank, local):
         torch.cuda.synchronize()
     barrier(world)
     step_ms = [e[0].elapsed_time(e[2]) for e in events]
-    decode_ms = [e[1].elapsed_time(e[2]) for e in events]
-    reshape_ms = [e[0].elapsed_time(e[1]) for e in events]
+    if mode == "append":
+        decode_ms = step_ms
+        reshape_ms = [0.0 for _ in events]
+    else:
+        decode_ms = [e[1].elapsed_time(e[2]) for e in events]
+        reshape_ms = [e[0].elapsed_time(e[1]) for e in events]
     local_step = sum(step_ms) / len(step_ms)
     local_decode = sum(decode_ms) / len(decode_ms)
     if pa.pa_get_device_error() != 0:
@@ -383,12 +391,13 @@ def run_gpu(args, world, rank, local):
             "context_len_mean": float(batch.context_lens.float().mean()),
             "context_len_max": batch.max_context_len,
             "decode_entry": {"splitk": "pa_decode_splitk (fused merge)", "splitk2": "pa_decode_splitk (merge kernel)",
-                             "streamk": "pa_decode_streamk"}.get(mode, "pa_decode"),
+                             "append": "pa_decode_append"}.get(mode, "pa_decode"),
             "partition_size": args.partition_size if mode.startswith("splitk") else None,
             "parallelism": f"replicas x{world} (sequence batches, no collective)",
             "l2": "flushed between steps (256 MiB write), per-step CUDA events" if flush is not None
             else "not flushed",
-            "step": "pa_reshape_and_cache (newest token of every sequence) + decode",
+            "step": ("pa_decode_append: newest token of every sequence written + decode, one launch" if mode == "append"
+                     else "pa_reshape_and_cache (newest token of every sequence) + decode"),
         },
         "tokens_per_s": round(total_seqs / (step_ms_max * 1e-3), 1),
         "decode_ms": round(decode_ms_max, 5),
@@ -398,9 +407,9 @@ def run_gpu(args, world, rank, local):
         "pct_of_spec_8tbs": round(100 * value / world / SPEC_HBM_GBS, 2),
         "roofline": {
             "bound": "hbm",
-            "kernel": {"splitk": "pa_decode_kernel<split, fused merge>",
+            "kernel": {"append": "pa_decode_kernel (append)", "splitk": "pa_decode_kernel<split, fused merge>",
                        "splitk2": "pa_decode_kernel<split> + pa_merge_kernel",
-                       "streamk": "pa_decode_streamk_kernel"}.get(mode, "pa_decode_kernel"),
+                       }.get(mode, "pa_decode_kernel"),
             "achieved": round(achieved, 2),
             "peak": peak,
             "peak_kind": f"{peak_kind} copy bandwidth (burst)",

@@ -37,7 +37,9 @@
  *   a padding token that is skipped.
  * Block tables.  block_tables is int32 [num_seqs][max_blocks_per_seq]; entry
  *   [s][j] is the physical block holding logical tokens [j*B, (j+1)*B) of
- *   sequence s.  Entries at j >= ceil(context_lens[s] / B) are never read.
+ *   sequence s.  Entries at j >= ceil(context_lens[s] / B) are ignored (a
+ *   kernel may load them early and discard them, so the whole
+ *   [num_seqs][max_blocks_per_seq] array must be readable device memory).
  *   Several rows may name the same physical block (shared prefix).
  * Context lengths.  context_lens[s] (int32) counts every token of sequence s,
  *   including the one just written by pa_reshape_and_cache; 0 gives an
@@ -124,6 +126,29 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream);
 
 /*
+ * pa_decode_append — one decode step in one launch: for every sequence s with
+ * context_lens[s] = L > 0, write key[s] / value[s] (the newest token) at
+ * logical position L-1, i.e. at block block_tables[s][(L-1)/B], offset
+ * (L-1)%B ([P3] §2.1 append_token), then attend over all L tokens ([P3] §2.3).
+ * The result, and every pool byte, equal pa_reshape_and_cache with that slot
+ * per sequence followed by pa_decode.  The CTA that computes a sequence's last
+ * block patches the new row into the block it has staged and into the pool.
+ *
+ *   key, value     [num_seqs][num_kv_heads][head_dim], one new token per
+ *                  sequence, 16-byte aligned
+ *   k_cache,
+ *   v_cache        written at the new tokens' rows, read everywhere else
+ *   The block holding position L-1 must belong to sequence s alone (a block
+ *   shared with other sequences is copied before it is written, as
+ *   copy-on-write requires, [P4] §2.3).  Other arguments as in pa_decode.
+ */
+pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value, void* k_cache,
+                           void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                           float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                           int head_dim, int max_blocks_per_seq, int max_context_len, int64_t num_blocks,
+                           pa_dtype dtype, void* stream);
+
+/*
  * pa_decode_splitk_workspace_size — bytes of workspace pa_decode_splitk needs:
  * per (sequence, query head, partition) an fp32 partial output of head_dim
  * values plus its running max and sum, for ceil(max_context_len /
@@ -168,50 +193,6 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
                            int64_t num_blocks, pa_dtype dtype, int partition_size, void* workspace,
                            size_t workspace_bytes, int32_t* counters, int64_t num_counters,
                            void* stream);
-
-/*
- * pa_decode_streamk_workspace_size — bytes of scratch pa_decode_streamk needs
- * on the current device for its partial records: per worker warp of the
- * persistent grid two records, each holding fp32 head_dim outputs plus the
- * running max and sum of the g query heads of one kv head (padded to 16
- * bytes).  The worker count follows the device's SM count and the kernel's
- * occupancy, so the size depends on the GPU (and slightly on num_seqs).
- */
-pa_status pa_decode_streamk_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                                           int block_size, pa_dtype dtype, size_t* bytes);
-
-/*
- * pa_decode_streamk — the same result as pa_decode, scheduled for batches
- * whose context lengths differ widely ([P1] §4.2: sequences of every length
- * share each decode iteration).  The (sequence, kv head, logical block) tiles
- * of the batch, in that order, are cut into equal contiguous ranges, one per
- * warp of a grid sized to one full wave.  A sequence lying inside one range is
- * finished there; one cut by range boundaries leaves a partial result per
- * piece, and the piece that completes last merges them in a fixed order with
- * log-sum-exp weights.  One launch; no thread waits for another CTA; results
- * are bitwise reproducible on a given GPU model.
- *
- *   workspace        device scratch of at least
- *                    pa_decode_streamk_workspace_size(...) bytes, 16-byte
- *                    aligned; no initialisation needed, contents clobbered.
- *   counters         int32 device array of num_counters >= num_seqs *
- *                    num_kv_heads arrival counters, entry s*Hkv + kvh for
- *                    (sequence s, kv head kvh).  Must be all zero before the
- *                    first call (allocate it zeroed); every completed call
- *                    leaves the entries it used at zero, so one array serves
- *                    successive calls of any shape.  Zero it again after a
- *                    call that reported PA_DEVERR_TIMEOUT.
- *   Calls that may run concurrently on the GPU need their own workspace and
- *   counters.
- *   num_seqs         at most 16384 (PA_ERR_UNSUPPORTED above).
- *   Other arguments as in pa_decode.
- */
-pa_status pa_decode_streamk(void* out, const void* q, const void* k_cache, const void* v_cache,
-                            const int32_t* block_tables, const int32_t* context_lens, float scale,
-                            int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                            int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
-                            void* workspace, size_t workspace_bytes, int32_t* counters,
-                            int64_t num_counters, void* stream);
 
 /*
  * pa_decode_splitk_static — pa_decode_splitk for callers that cannot

@@ -16,8 +16,9 @@ import os
 
 import torch
 
-__all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
-           "pa_decode_streamk", "pa_decode_streamk_workspace_size", "StreamKWorkspace", "Counters",
+__all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_splitk",
+           "pa_decode_splitk_workspace_size",
+           "Counters",
            "pa_decode_splitk_static", "SPLITK_STATIC_SCRATCH_BYTES",
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT"]
@@ -59,14 +60,12 @@ def load() -> ctypes.CDLL:
     decode_args = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I64, I]
     lib.pa_decode.restype = I
     lib.pa_decode.argtypes = decode_args + [P]
+    lib.pa_decode_append.restype = I
+    lib.pa_decode_append.argtypes = [P, P, P, P] + decode_args[2:] + [P]
     lib.pa_decode_splitk_workspace_size.restype = I
     lib.pa_decode_splitk_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
     lib.pa_decode_splitk.restype = I
     lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P, I64, P]
-    lib.pa_decode_streamk_workspace_size.restype = I
-    lib.pa_decode_streamk_workspace_size.argtypes = [I, I, I, I, I, I, c.POINTER(SZ)]
-    lib.pa_decode_streamk.restype = I
-    lib.pa_decode_streamk.argtypes = decode_args + [P, SZ, P, I64, P]
     lib.pa_decode_splitk_static.restype = I
     lib.pa_decode_splitk_static.argtypes = decode_args + [I, P]
     lib.pa_get_device_error.restype = I
@@ -143,6 +142,16 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_c
     _check(lib.pa_decode(*args, _stream(stream)), "pa_decode")
 
 
+def pa_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
+                     stream=None):
+    """One decode step: write each sequence's newest token (key/value [S, Hkv,
+    D]) at position context_lens[s]-1, then attend over the whole context."""
+    lib = load()
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_append(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
+                                _stream(stream)), "pa_decode_append")
+
+
 def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size=512) -> int:
     lib = load()
     size = ctypes.c_size_t(0)
@@ -153,8 +162,8 @@ def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context
 
 
 class Counters:
-    """Zero-initialised int32 arrival counters for the fused merges
-    (pa_decode_splitk with fused=True, pa_decode_streamk); the kernels leave
+    """Zero-initialised int32 arrival counters for the fused split-K merge
+    (pa_decode_splitk with fused=True); the kernels leave
     them at zero, so one array is reused across calls of any shape on a
     stream.  Grows on demand."""
 
@@ -200,57 +209,6 @@ def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale
     _check(lib.pa_decode_splitk(*args, int(partition_size), _dev_ptr(workspace, "workspace"),
                                 workspace.numel() * workspace.element_size(), cptr, ncount, _stream(stream)),
            "pa_decode_splitk")
-
-
-def pa_decode_streamk_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, dtype) -> int:
-    """Workspace bytes of pa_decode_streamk on the current device."""
-    lib = load()
-    size = ctypes.c_size_t(0)
-    _check(lib.pa_decode_streamk_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                                                _DTYPE[dtype], ctypes.byref(size)),
-           "pa_decode_streamk_workspace_size")
-    return int(size.value)
-
-
-class StreamKWorkspace:
-    """Scratch for pa_decode_streamk on one device and stream: the partial
-    records (uninitialised) and the arrival counters (zero-initialised; the
-    kernel leaves them at zero, so they are reused across calls of any
-    shape).  Grows on demand."""
-
-    def __init__(self):
-        self.records = None
-        self.counters = None
-
-    def get(self, record_bytes: int, num_counters: int, device):
-        device = torch.device(device)
-        if self.records is None or self.records.numel() < record_bytes or self.records.device != device:
-            self.records = torch.empty(max(record_bytes, 16), dtype=torch.uint8, device=device)
-        if self.counters is None or self.counters.numel() < num_counters or self.counters.device != device:
-            self.counters = torch.zeros(max(num_counters, 4), dtype=torch.int32, device=device)
-        return self.records, self.counters
-
-
-_default_streamk_ws: dict = {}
-
-
-def pa_decode_streamk(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
-                      workspace=None, stream=None):
-    """Work-balanced paged decode: equal contiguous ranges of (sequence, kv
-    head, block) tiles per warp of a persistent grid, with log-sum-exp merges
-    of the sequences cut by range boundaries.  `workspace` is a
-    StreamKWorkspace (a per-device default is used if None)."""
-    lib = load()
-    n, hkv, d, b = _pool_dims(k_cache)
-    S, Hq, D = q.shape
-    need = pa_decode_streamk_workspace_size(S, Hq, hkv, D, b, q.dtype)
-    if workspace is None:
-        workspace = _default_streamk_ws.setdefault(q.device.index, StreamKWorkspace())
-    records, counters = workspace.get(need, S * hkv, q.device)
-    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
-    _check(lib.pa_decode_streamk(*args, _dev_ptr(records, "workspace"), records.numel(),
-                                 _dev_ptr(counters, "counters"), counters.numel(), _stream(stream)),
-           "pa_decode_streamk")
 
 
 SPLITK_STATIC_SCRATCH_BYTES = 16 << 20

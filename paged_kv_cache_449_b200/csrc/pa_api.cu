@@ -16,7 +16,6 @@
 #include "pa.h"
 #include "pa_decode.cuh"
 #include "pa_reshape.cuh"
-#include "pa_streamk.cuh"
 
 // Warps per CTA and per-warp shared-memory ring bytes of each decode entry
 // point (measured on B200 over the benchmark workloads): the one-pass kernel
@@ -34,36 +33,28 @@
 #ifndef PA_SPLIT_RING
 #define PA_SPLIT_RING 12288
 #endif
-#ifndef PA_STREAM_WARPS
-#define PA_STREAM_WARPS 4
-#endif
-#ifndef PA_STREAM_RING
-#define PA_STREAM_RING 16384
-#endif
 
 namespace {
 
-enum class Kind { kSingle, kSplit, kStream };
+enum class Kind { kSingle, kSplit };
 
 template <Kind K>
 struct KindTuning;
+// kRingCap bounds the K/V ring of a CTA.
 template <>
 struct KindTuning<Kind::kSingle> {
-    static constexpr int kWarps = PA_SINGLE_WARPS, kRing = PA_SINGLE_RING;
+    static constexpr int kWarps = PA_SINGLE_WARPS, kRing = PA_SINGLE_RING, kRingCap = 200 * 1024;
 };
 template <>
 struct KindTuning<Kind::kSplit> {
-    static constexpr int kWarps = PA_SPLIT_WARPS, kRing = PA_SPLIT_RING;
+    static constexpr int kWarps = PA_SPLIT_WARPS, kRing = PA_SPLIT_RING, kRingCap = 200 * 1024;
 };
-template <>
-struct KindTuning<Kind::kStream> {
-    static constexpr int kWarps = PA_STREAM_WARPS, kRing = PA_STREAM_RING;
-};
+
 
 template <typename T, int D, int B, Kind K>
 struct DecodeConfig {
     static constexpr int kStageBytes = 2 * B * D * static_cast<int>(sizeof(T));  // K + V tile
-    static constexpr int kRingCap = 200 * 1024;                                   // ring bytes per CTA at most
+    static constexpr int kRingCap = KindTuning<K>::kRingCap;                      // ring bytes per CTA at most
     static constexpr int kMaxWarps = kRingCap / kStageBytes;
     static constexpr int kWarps = KindTuning<K>::kWarps < kMaxWarps ? KindTuning<K>::kWarps : kMaxWarps;
     static constexpr int kRaw = KindTuning<K>::kRing / kStageBytes;
@@ -159,63 +150,6 @@ cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p
     });
 }
 
-// ---- stream-K: persistent grid sized to one full wave
-
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return n;
-}
-
-// CTAs per SM of `kernel` at `smem` bytes, cached per (kernel, device, smem).
-template <typename Kernel>
-int resident_ctas(Kernel kernel, int threads, int smem) {
-    static std::mutex mu;
-    static std::map<std::tuple<const void*, int, int>, int> cache;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    const auto key = std::make_tuple(reinterpret_cast<const void*>(kernel), dev, smem);
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        auto it = cache.find(key);
-        if (it != cache.end()) return it->second;
-    }
-    if (ensure_smem(reinterpret_cast<const void*>(kernel)) != cudaSuccess) return 0;
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess) return 0;
-    std::lock_guard<std::mutex> lock(mu);
-    cache[key] = n;
-    return n;
-}
-
-struct StreamPlan {
-    int grid = 0, threads = 0, smem = 0, workers = 0;
-};
-
-template <typename T, int D, int B>
-StreamPlan streamk_plan(int num_seqs) {
-    using C = DecodeConfig<T, D, B, Kind::kStream>;
-    using Smem = pa::StreamSmem<T, D, B, C::kWarps, C::kStages>;
-    auto kernel = pa::pa_decode_streamk_kernel<T, D, B, C::kWarps, C::kStages>;
-    StreamPlan plan;
-    plan.threads = C::kWarps * 32;
-    plan.smem = Smem::total(num_seqs);
-    const int per_sm = resident_ctas(kernel, plan.threads, plan.smem);
-    plan.grid = per_sm * sm_count();
-    plan.workers = plan.grid * C::kWarps;
-    return plan;
-}
-
-template <typename T, int D, int B>
-cudaError_t launch_streamk(pa::StreamParams p, const StreamPlan& plan, cudaStream_t stream) {
-    using C = DecodeConfig<T, D, B, Kind::kStream>;
-    auto kernel = pa::pa_decode_streamk_kernel<T, D, B, C::kWarps, C::kStages>;
-    p.workers = plan.workers;
-    kernel<<<plan.grid, plan.threads, plan.smem, stream>>>(p);
-    return cudaGetLastError();
-}
-
 template <typename T, int D>
 cudaError_t launch_merge(const pa::MergeParams& p, cudaStream_t st) {
     constexpr bool kLog2 = !pa::IsF32<T>::value;
@@ -296,22 +230,6 @@ size_t splitk_bytes(long long seqs, long long heads, long long parts, long long 
     return static_cast<size_t>(seqs * heads * parts * (head_dim + 2) * 4);
 }
 
-constexpr int kStreamMaxSeqs = 16384;  // per-CTA length prefix lives in shared memory
-
-// Stream-K workspace: partial records [workers][2][record_floats(g, D)] fp32.
-size_t streamk_bytes(long long workers, int group, int head_dim) {
-    return static_cast<size_t>(workers * 2 * pa::record_floats(group, head_dim) * 4);
-}
-
-bool streamk_plan_for(pa_dtype dt, int D, int B, int num_seqs, StreamPlan* plan) {
-    const cudaError_t e = with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) {
-        using T = typename decltype(tt)::type;
-        *plan = streamk_plan<T, decltype(dd)::value, decltype(bb)::value>(num_seqs);
-        return cudaSuccess;
-    });
-    return e == cudaSuccess && plan->grid > 0;
-}
-
 }  // namespace
 
 extern "C" {
@@ -357,6 +275,24 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     if (st != PA_OK || num_seqs == 0) return st;
     const pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    const dim3 grid(1, num_kv_heads, num_seqs);
+    const cudaError_t e = decode_dispatch<false>(dtype, head_dim, block_size, p, grid,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value, void* k_cache, void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, float scale, int block_size,
+                           int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                           int max_context_len, int64_t num_blocks, pa_dtype dtype, void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (st != PA_OK || num_seqs == 0) return st;
+    if (!key || !value || !aligned16(key) || !aligned16(value)) return PA_ERR_INVALID_ARG;
+    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.new_key = key;
+    p.new_value = value;
     const dim3 grid(1, num_kv_heads, num_seqs);
     const cudaError_t e = decode_dispatch<false>(dtype, head_dim, block_size, p, grid,
                                                  static_cast<cudaStream_t>(stream));
@@ -422,68 +358,6 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
     m.partition_blocks = pb;
     m.num_partitions = static_cast<int>(parts);
     return merge_dispatch(dtype, head_dim, m, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-pa_status pa_decode_streamk_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                                           int block_size, pa_dtype dtype, size_t* bytes) {
-    if (!bytes || num_seqs < 0) return PA_ERR_INVALID_ARG;
-    // Shape checks only (an empty batch needs no pointers).
-    const DecodeShape shape_only{block_size, 0, num_q_heads, num_kv_heads, head_dim, 0, 0, 1, static_cast<int>(dtype)};
-    const pa_status st = check_decode(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 1.f, shape_only);
-    if (st != PA_OK) return st;
-    if (num_seqs > kStreamMaxSeqs) return PA_ERR_UNSUPPORTED;
-    if (num_seqs == 0) {
-        *bytes = 0;
-        return PA_OK;
-    }
-    StreamPlan plan;
-    if (!streamk_plan_for(dtype, head_dim, block_size, num_seqs, &plan)) return PA_ERR_CUDA;
-    *bytes = streamk_bytes(plan.workers, num_q_heads / num_kv_heads, head_dim);
-    return PA_OK;
-}
-
-pa_status pa_decode_streamk(void* out, const void* q, const void* k_cache, const void* v_cache,
-                            const int32_t* block_tables, const int32_t* context_lens, float scale, int block_size,
-                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
-                            int max_context_len, int64_t num_blocks, pa_dtype dtype, void* workspace,
-                            size_t workspace_bytes, int32_t* counters, int64_t num_counters, void* stream) {
-    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                         max_context_len, num_blocks, static_cast<int>(dtype)};
-    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
-    if (st != PA_OK) return st;
-    if (num_seqs > kStreamMaxSeqs) return PA_ERR_UNSUPPORTED;
-    if (num_seqs == 0) return PA_OK;
-    if (!counters || !aligned4(counters) || num_counters < static_cast<int64_t>(num_seqs) * num_kv_heads)
-        return PA_ERR_WORKSPACE;
-    StreamPlan plan;
-    if (!streamk_plan_for(dtype, head_dim, block_size, num_seqs, &plan)) return PA_ERR_CUDA;
-    const int group = num_q_heads / num_kv_heads;
-    const size_t need = streamk_bytes(plan.workers, group, head_dim);
-    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PA_ERR_WORKSPACE;
-    const pa::DecodeParams d = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
-    pa::StreamParams p{};
-    p.out = out;
-    p.q = q;
-    p.k_cache = k_cache;
-    p.v_cache = v_cache;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.records = static_cast<float*>(workspace);
-    p.counters = counters;
-    p.score_scale = d.score_scale;
-    p.num_seqs = num_seqs;
-    p.num_q_heads = num_q_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.group = group;
-    p.max_blocks_per_seq = max_blocks_per_seq;
-    p.context_cap = d.context_cap;
-    p.num_blocks = num_blocks;
-    const cudaError_t e = with_variant(dtype, head_dim, block_size, [&](auto tt, auto dd, auto bb) {
-        using T = typename decltype(tt)::type;
-        return launch_streamk<T, decltype(dd)::value, decltype(bb)::value>(p, plan,
-                                                                           static_cast<cudaStream_t>(stream));
-    });
-    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(void* stream, int32_t* code) {

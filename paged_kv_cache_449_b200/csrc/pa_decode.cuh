@@ -55,7 +55,36 @@ struct DecodeParams {
     int partition_blocks;  // split: blocks per partition
     int num_partitions;    // split: P
     int* counters;         // split, fused merge: [S*Hkv] arrival counters (zero between calls); null = merge kernel
+    const void* new_key;   // append: [S][Hkv][D] K/V of each sequence's newest token (position L-1), or null
+    const void* new_value;
 };
+
+// Append: the newest token of sequence s (logical position L-1) is written
+// into the block being computed, both in the staged shared-memory tiles and in
+// the pool, before the block is used (the same bytes pa_reshape_and_cache
+// would write at that token's slot).  One lane per 16-byte vector of D.
+template <typename T, int D, int B>
+__device__ __forceinline__ void append_newest_token(const DecodeParams& p, uint8_t* stage, int id, int s, int kvh,
+                                                    int t, int lane) {
+    constexpr int kTile = B * D * static_cast<int>(sizeof(T));
+    constexpr int kVecs = D * static_cast<int>(sizeof(T)) / 16;
+    const long long row = (static_cast<long long>(s) * p.num_kv_heads + kvh) * kVecs;
+    const uint4* ksrc = reinterpret_cast<const uint4*>(p.new_key) + row;
+    const uint4* vsrc = reinterpret_cast<const uint4*>(p.new_value) + row;
+    char* kpool = reinterpret_cast<char*>(const_cast<void*>(p.k_cache));
+    char* vpool = reinterpret_cast<char*>(const_cast<void*>(p.v_cache));
+    const long long tile = (static_cast<long long>(id) * p.num_kv_heads + kvh) * kTile;
+    for (int v = lane; v < kVecs; v += 32) {
+        const uint4 kv = ksrc[v], vv = vsrc[v];
+        const int off = (v * B + t) * 16;
+        *reinterpret_cast<uint4*>(stage + off) = kv;
+        *reinterpret_cast<uint4*>(stage + kTile + off) = vv;
+        *reinterpret_cast<uint4*>(kpool + tile + off) = kv;
+        *reinterpret_cast<uint4*>(vpool + tile + off) = vv;
+    }
+    fence_proxy_async_smem();  // the stage is refilled by bulk copies later
+    __syncwarp();
+}
 
 // Fused split-K merge, run by the CTA that completes the last partition of
 // (sequence s, kv head kvh): combines the np partial results of each of the
@@ -130,6 +159,20 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int group = p.group;
 
+    // Issued before the context length arrives, so the three loads overlap:
+    // this warp's first 32 block-table entries (any entry of the row is
+    // readable; entries past the context are discarded below) and, for the
+    // tensor-core path, the query fragments.
+    const int b0_first = SPLIT ? part * p.partition_blocks : 0;
+    const int32_t* bt = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq + b0_first + warp;
+    int first_ids = -1;
+    if (b0_first + warp + lane * NW < p.max_blocks_per_seq) first_ids = __ldg(bt + lane * NW);
+    const T* qrows = reinterpret_cast<const T*>(p.q) +
+                     (static_cast<long long>(s) * p.num_q_heads + kvh * group) * D;
+    typename WarpState<T, D, B>::type acc;
+    acc.reset();
+    if constexpr (!kF32) acc.load_q(qrows, group, lane);
+
     int L = p.context_lens[s];
     if (L < 0 || L > p.context_cap) {
         if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
@@ -148,8 +191,6 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         if (b0 >= nblk) return;  // this partition is past the end of the sequence
         b1 = min(nblk, b0 + p.partition_blocks);
     }
-    const T* qrows = reinterpret_cast<const T*>(p.q) +
-                     (static_cast<long long>(s) * p.num_q_heads + kvh * group) * D;
     if constexpr (!SPLIT) {
         if (nblk == 0) {  // empty context: zero output
             T* out = reinterpret_cast<T*>(p.out) + (static_cast<long long>(s) * p.num_q_heads + kvh * group) * D;
@@ -174,12 +215,11 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     }
     __syncwarp();
 
-    const int32_t* bt = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq + b0 + warp;
     auto load_ids = [&](int round) -> int {
         const int i = round * 32 + lane;
         int id = -1;
         if (i < n_w) {
-            id = __ldg(bt + i * NW);
+            id = round == 0 ? first_ids : __ldg(bt + i * NW);
             if (id < 0 || static_cast<long long>(id) >= p.num_blocks) {
                 flag_error(1 /* PA_DEVERR_BLOCK_ID */);
                 id = -1;
@@ -215,13 +255,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         }
     };
 
-    typename WarpState<T, D, B>::type acc;
-    acc.reset();
-    if constexpr (kF32) {
-        acc.qs = qs;
-    } else {
-        acc.load_q(qrows, group, lane);
-    }
+    if constexpr (kF32) acc.qs = qs;
 
     int issued = n_w < STAGES ? n_w : STAGES;
     for (int i = 0; i < issued; ++i) issue(i);
@@ -242,6 +276,8 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         const int j = b0 + warp + i * NW;  // logical block index
         const int valid = id < 0 ? 0 : min(B, L - j * B);
         uint8_t* stage = wring + st * 2 * kTile;
+        if (p.new_key != nullptr && j == nblk - 1 && id >= 0)
+            append_newest_token<T, D, B>(p, stage, id, s, kvh, (L - 1) % B, lane);
         if constexpr (kF32) {
             acc.block(reinterpret_cast<const float*>(stage), reinterpret_cast<const float*>(stage + kTile), valid,
                       group, p.score_scale, lane);

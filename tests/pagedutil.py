@@ -198,9 +198,6 @@ def gpu_decode(batch, mode="single", partition_size=512, dev=None, max_context_l
     if mode == "single":
         pa.pa_decode(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"], dev["context_lens"],
                      batch.scale, max_context_len=mcl)
-    elif mode == "streamk":
-        pa.pa_decode_streamk(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"],
-                             dev["context_lens"], batch.scale, max_context_len=mcl)
     else:  # "splitk" (merge fused into the partition kernel) or "splitk2" (separate merge kernel)
         pa.pa_decode_splitk(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"],
                             dev["context_lens"], batch.scale, mcl, partition_size=partition_size,

@@ -33,8 +33,8 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size", "pa_decode_streamk",
-        "pa_decode_streamk_workspace_size", "pa_decode_splitk_static", "pa_get_device_error",
+        "pa_decode", "pa_decode_append", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
+        "pa_decode_splitk_static", "pa_get_device_error",
         "pa_reshape_and_cache", "pa_status_string"])
 
 
@@ -98,7 +98,6 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_decode_splitk(*args, 512, 16, 100, None, 0, None) == 3       # workspace too small
     assert lib.pa_decode_splitk(*args, 512, 0, 1 << 20, None, 0, None) == 3    # no workspace
     assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, 16, 3, None) == 3     # too few counters
-    assert lib.pa_decode_streamk(*args, 16, 1 << 30, 16, 3, None) == 3         # too few counters
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

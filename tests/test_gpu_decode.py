@@ -31,7 +31,7 @@ def no_device_errors():
     assert pa.pa_get_device_error() == 0
 
 
-def _full_check(orc, b, modes=("single", "splitk", "splitk2", "streamk"), parts=(512, 16)):
+def _full_check(orc, b, modes=("single", "splitk", "splitk2"), parts=(512, 16)):
     ref = oracle_decode_sampled(orc, b, range(b.num_seqs))
     for mode in modes:
         # a partition is a whole number of blocks
@@ -84,7 +84,7 @@ def test_llama3_8b_decode_sampled(orc):
     rng = np.random.default_rng(0)
     lens = b.context_lens.numpy()
     seqs = list(rng.choice(b.num_seqs, 6, replace=False)) + [int(lens.argmax()), int(lens.argmin())]
-    _sampled(orc, b, seqs, ("single", "splitk", "splitk2", "streamk"))
+    _sampled(orc, b, seqs, ("single", "splitk", "splitk2"))
 
 
 @pytest.mark.parametrize("block_size", [8, 16, 32])
@@ -95,21 +95,21 @@ def test_continuous_batching_mix_sampled(orc, block_size):
     short = np.nonzero(lens <= 64)[0]
     long = np.nonzero(lens >= 600)[0]
     seqs = list(rng.choice(short, 6, replace=False)) + list(rng.choice(long, 3, replace=False))
-    _sampled(orc, b, seqs, ("single", "splitk", "splitk2", "streamk"))
+    _sampled(orc, b, seqs, ("single", "splitk", "splitk2"))
 
 
 @pytest.mark.parametrize("prefix_len", [1024, 1000])
 def test_prefix_sharing_sampled(orc, prefix_len):
     b = workloads.prefix_sharing(seed=0, device="cuda", prefix_len=prefix_len)
     rng = np.random.default_rng(prefix_len)
-    _sampled(orc, b, rng.choice(b.num_seqs, 6, replace=False), ("single", "splitk", "splitk2", "streamk"))
+    _sampled(orc, b, rng.choice(b.num_seqs, 6, replace=False), ("single", "splitk", "splitk2"))
 
 
 def test_llama3_70b_long_sampled(orc):
     b = workloads.llama3_70b_long(seed=0, device="cuda")
     lens = b.context_lens.numpy()
     seqs = [int(lens.argmax()), int(lens.argmin()), 7]
-    _sampled(orc, b, seqs, ("splitk", "splitk2", "single", "streamk"))
+    _sampled(orc, b, seqs, ("splitk", "splitk2", "single"))
 
 
 def test_splitk_oracle_form_matches(orc):

@@ -11,7 +11,7 @@ import oracle
 import workloads
 import paged_kv_cache_449_b200 as pa
 from pagedutil import (as_f64, check_tolerance, device_batch, gpu_decode, logical_kv, materialize_shared,
-                       permute_physical, relayout_block_size)
+                       oracle_decode_sampled, permute_physical, relayout_block_size)
 
 pytestmark = pytest.mark.gpu
 
@@ -135,7 +135,7 @@ def test_needle_every_position(dtype, B, mode, part):
 def test_permutation_invariance_bit_exact():
     b = workloads.continuous_batching_mix(seed=2, device="cuda", num_seqs=40)
     c = permute_physical(b, seed=9)
-    for mode in ("single", "splitk", "splitk2", "streamk"):
+    for mode in ("single", "splitk", "splitk2"):
         assert torch.equal(_bits(gpu_decode(b, mode)), _bits(gpu_decode(c, mode)))
 
 
@@ -144,7 +144,7 @@ def test_shared_vs_copied_bit_exact(prefix_len):
     b = workloads.prefix_sharing(seed=1, device="cuda", prefix_len=prefix_len, num_seqs=16)
     twin = materialize_shared(b)
     assert twin.num_blocks > b.num_blocks
-    for mode in ("single", "splitk", "splitk2", "streamk"):
+    for mode in ("single", "splitk", "splitk2"):
         assert torch.equal(_bits(gpu_decode(b, mode)), _bits(gpu_decode(twin, mode)))
 
 
@@ -154,14 +154,14 @@ def test_block_size_within_tolerance(orc):
     ref = orc.decode(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.scale, 16, 8)
     for nb in (8, 32):
         c = relayout_block_size(b, nb)
-        for mode in ("single", "splitk", "splitk2", "streamk"):
+        for mode in ("single", "splitk", "splitk2"):
             check_tolerance(as_f64(gpu_decode(c, mode)), ref, b.dtype)
 
 
 def test_run_to_run_deterministic():
     b = workloads.llama3_8b_decode(seed=3, device="cuda", num_seqs=16, num_blocks=4096)
     dev = device_batch(b)
-    for mode in ("single", "splitk", "splitk2", "streamk"):
+    for mode in ("single", "splitk", "splitk2"):
         first = gpu_decode(b, mode, dev=dev)
         for _ in range(3):
             assert torch.equal(_bits(first), _bits(gpu_decode(b, mode, dev=dev)))
@@ -177,7 +177,7 @@ def test_out_of_range_block_id_is_flagged_not_read():
     bad[0, 1] = b.num_blocks + 1000
     bad[1, 0] = -7
     c = b.__class__(**{**b.__dict__, "block_tables": bad})
-    for mode in ("single", "splitk", "splitk2", "streamk"):
+    for mode in ("single", "splitk", "splitk2"):
         out = gpu_decode(c, mode)
         assert torch.isfinite(out.float()).all()
         assert pa.pa_get_device_error() & pa.DEVERR_BLOCK_ID
@@ -217,3 +217,37 @@ def test_host_side_errors_raise():
     with pytest.raises(pa.PagedAttentionError):
         pa.pa_decode(out, dev["q"][:, :3].contiguous(), dev["k_cache"], dev["v_cache"], dev["block_tables"],
                      dev["context_lens"], b.scale)   # 3 q heads over 2 kv heads
+
+
+# ---------------------------------------------------------------------------- append (write + decode in one launch)
+
+@pytest.mark.parametrize("make", [
+    lambda: workloads.tiny_mha_f32(seed=0),
+    lambda: workloads.continuous_batching_mix(seed=4, device="cuda", num_seqs=40, block_size=8),
+    lambda: workloads.llama3_8b_decode(seed=5, device="cuda", num_seqs=24, num_blocks=4096),
+    lambda: workloads.random_small(seed=6, dtype=torch.float16, lens=(0, 1, 16, 17, 300), num_q_heads=8,
+                                   num_kv_heads=2, head_dim=64, block_size=32),
+])
+def test_append_equals_reshape_then_decode(orc, make):
+    b = make()
+    # separate pools for the two routes
+    d1, d2 = device_batch(b), device_batch(b)
+    d2["k_cache"], d2["v_cache"] = d2["k_cache"].clone(), d2["v_cache"].clone()
+    nk, nv = b.new_key.cuda().contiguous(), b.new_value.cuda().contiguous()
+    pa.pa_reshape_and_cache(nk, nv, d1["k_cache"], d1["v_cache"], b.slot_mapping.cuda())
+    ref_gpu = gpu_decode(b, "single", dev=d1)
+    out = torch.full_like(d2["q"], float("nan"))
+    pa.pa_decode_append(out, d2["q"], nk, nv, d2["k_cache"], d2["v_cache"], d2["block_tables"], d2["context_lens"],
+                        b.scale, max_context_len=b.max_context_len)
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(out), _bits(ref_gpu))
+    assert torch.equal(_bits(d2["k_cache"]), _bits(d1["k_cache"]))
+    assert torch.equal(_bits(d2["v_cache"]), _bits(d1["v_cache"]))
+    # and the oracle's write + decode
+    seqs = list(range(0, b.num_seqs, max(1, b.num_seqs // 8)))
+    kc, vc = b.k_cache.cpu().contiguous(), b.v_cache.cpu().contiguous()
+    orc.reshape_and_cache(b.new_key.cpu().contiguous(), b.new_value.cpu().contiguous(), kc, vc, b.slot_mapping,
+                          b.block_size)
+    c = b.__class__(**{**b.__dict__, "k_cache": kc, "v_cache": vc})
+    check_tolerance(as_f64(out[seqs]), oracle_decode_sampled(orc, c, seqs), b.dtype)
+    assert pa.pa_get_device_error() == 0

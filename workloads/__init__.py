@@ -22,7 +22,7 @@ Conventions of the generated batch:
   * pools are shaped [num_blocks, Hkv, D // x, B, x] with x = 16 bytes / element
     size (the library's pool layout; only the shape is used here);
   * block_tables rows list the physical ids of logical blocks 0..ceil(L/B)-1;
-    the remaining entries hold -1 and are never read;
+    the remaining entries hold -1 (ignored by the kernels);
   * a slot is physical_block * B + offset (the library's slot format); the
     "decode-consistent" slot of sequence s is the position of its newest token,
     context_lens[s] - 1, so a step writes that token and then attends over it.
