@@ -62,21 +62,32 @@ struct DecodeParams {
 // Append: the newest token of sequence s (logical position L-1) is written
 // into the block being computed, both in the staged shared-memory tiles and in
 // the pool, before the block is used (the same bytes pa_reshape_and_cache
-// would write at that token's slot).  One lane per 16-byte vector of D.
+// would write at that token's slot).  Lane v holds 16-byte vector v of the
+// new K and V rows (D * sizeof(T) <= 512 bytes), loaded early by load_row.
+template <typename T, int D>
+struct NewRow {
+    static constexpr int kVecs = D * static_cast<int>(sizeof(T)) / 16;
+    static_assert(kVecs <= 32, "one 16-byte vector per lane");
+    uint4 k, v;
+    __device__ __forceinline__ void load_row(const DecodeParams& p, int s, int kvh, int lane) {
+        if (lane < kVecs) {
+            const long long row = (static_cast<long long>(s) * p.num_kv_heads + kvh) * kVecs;
+            k = reinterpret_cast<const uint4*>(p.new_key)[row + lane];
+            v = reinterpret_cast<const uint4*>(p.new_value)[row + lane];
+        }
+    }
+};
+
 template <typename T, int D, int B>
-__device__ __forceinline__ void append_newest_token(const DecodeParams& p, uint8_t* stage, int id, int s, int kvh,
-                                                    int t, int lane) {
+__device__ __forceinline__ void append_newest_token(const DecodeParams& p, const NewRow<T, D>& nr, uint8_t* stage,
+                                                    int id, int kvh, int t, int lane) {
     constexpr int kTile = B * D * static_cast<int>(sizeof(T));
-    constexpr int kVecs = D * static_cast<int>(sizeof(T)) / 16;
-    const long long row = (static_cast<long long>(s) * p.num_kv_heads + kvh) * kVecs;
-    const uint4* ksrc = reinterpret_cast<const uint4*>(p.new_key) + row;
-    const uint4* vsrc = reinterpret_cast<const uint4*>(p.new_value) + row;
     char* kpool = reinterpret_cast<char*>(const_cast<void*>(p.k_cache));
     char* vpool = reinterpret_cast<char*>(const_cast<void*>(p.v_cache));
     const long long tile = (static_cast<long long>(id) * p.num_kv_heads + kvh) * kTile;
-    for (int v = lane; v < kVecs; v += 32) {
-        const uint4 kv = ksrc[v], vv = vsrc[v];
-        const int off = (v * B + t) * 16;
+    if (lane < NewRow<T, D>::kVecs) {
+        const uint4 kv = nr.k, vv = nr.v;
+        const int off = (lane * B + t) * 16;
         *reinterpret_cast<uint4*>(stage + off) = kv;
         *reinterpret_cast<uint4*>(stage + kTile + off) = vv;
         *reinterpret_cast<uint4*>(kpool + tile + off) = kv;
@@ -207,6 +218,12 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     // ---- per-warp block stream
     const int nb = b1 - b0;
     const int n_w = nb > warp ? (nb - warp + NW - 1) / NW : 0;
+    // Append: the warp that will compute the last block loads the new row now.
+    const int last_block = nblk - 1;
+    const bool owns_last = p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
+                           (last_block - b0) % NW == warp;
+    NewRow<T, D> new_row;
+    if (owns_last) new_row.load_row(p, s, kvh, lane);
     uint64_t* wbar = bars + warp * STAGES;
     uint8_t* wring = ring + warp * STAGES * 2 * kTile;
     if (lane == 0) {
@@ -276,8 +293,8 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         const int j = b0 + warp + i * NW;  // logical block index
         const int valid = id < 0 ? 0 : min(B, L - j * B);
         uint8_t* stage = wring + st * 2 * kTile;
-        if (p.new_key != nullptr && j == nblk - 1 && id >= 0)
-            append_newest_token<T, D, B>(p, stage, id, s, kvh, (L - 1) % B, lane);
+        if (owns_last && j == last_block && id >= 0)
+            append_newest_token<T, D, B>(p, new_row, stage, id, kvh, (L - 1) % B, lane);
         if constexpr (kF32) {
             acc.block(reinterpret_cast<const float*>(stage), reinterpret_cast<const float*>(stage + kTile), valid,
                       group, p.score_scale, lane);
