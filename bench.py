@@ -10,8 +10,12 @@ Default workload: Llama-3-8B-shaped single-layer decode, bf16 — 64 sequences,
 Prints one JSON line (rank 0).  `value` is KV GB/s over the whole step:
 algorithmic bytes (sum_s L_s*Hkv*D*2*e + Q + out + block-table entries +
 context_lens, plus the new tokens' K/V read and written) / step time, summed
-over ranks and divided by the max-over-ranks time.  Timing: CUDA events per
-step on the launching stream, L2 flushed (a 256 MiB write) between steps.
+over ranks and divided by the max-over-ranks time.  Timing: CUDA events on the
+launching stream around the K timed steps.  L2: by default every step's inputs
+are larger than L2 and the steps rotate over enough independent copies of the
+workload (pools, tables, queries) that a step never finds in L2 what an
+earlier step left there; --l2 flush instead writes a 256 MiB buffer between
+steps and times each step with its own events.
 
 Multi-GPU: sequences are independent, so each rank runs its own batch (weak
 scaling, no data-path collective); only the timing reduction crosses ranks.
@@ -46,7 +50,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama3_8b_decode",
@@ -59,7 +63,9 @@ def parse_args(argv=None):
                          "kernel (splitk2) merge")
     ap.add_argument("--partition-size", type=int, default=1024)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between steps")
+    ap.add_argument("--l2", choices=["rotate", "flush"], default="rotate",
+                    help="rotate: inputs larger than L2, rotated over independent copies, K steps timed as one "
+                         "region; flush: a 256 MiB write between steps, per-step events")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
@@ -225,14 +231,18 @@ class Step:
         self.mode = mode
         self.part = partition_size
         dev = "cuda"
-        self.q = batch.q.to(dev).contiguous()
-        self.k = batch.k_cache.to(dev).contiguous()
-        self.v = batch.v_cache.to(dev).contiguous()
-        self.bt = batch.block_tables.to(dev).contiguous()
-        self.cl = batch.context_lens.to(dev).contiguous()
-        self.nk = batch.new_key.to(dev).contiguous()
-        self.nv = batch.new_value.to(dev).contiguous()
-        self.slots = batch.slot_mapping.to(dev).contiguous()
+
+        def own(t):  # an independent device copy (its own memory, never an alias of the batch's)
+            return t.to(dev).contiguous().clone()
+
+        self.q = own(batch.q)
+        self.k = own(batch.k_cache)
+        self.v = own(batch.v_cache)
+        self.bt = own(batch.block_tables)
+        self.cl = own(batch.context_lens)
+        self.nk = own(batch.new_key)
+        self.nv = own(batch.new_value)
+        self.slots = own(batch.slot_mapping)
         self.out = torch.empty_like(self.q)
         self.mcl = batch.max_context_len
         need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
@@ -259,6 +269,23 @@ class Step:
                               max_context_len=self.mcl, stream=stream)
 
 
+def l2_bytes():
+    try:
+        return int(torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size)
+    except (AttributeError, RuntimeError):
+        return 126 << 20
+
+
+def rotation_copies(unique_bytes, l2):
+    """Independent input copies to rotate over so that, between two uses of a
+    copy, at least twice the L2 capacity of other inputs has been streamed;
+    0 when the workload is too small for that (then L2 is flushed instead)."""
+    if unique_bytes <= 0:
+        return 0
+    r = max(2, math.ceil(2 * l2 / unique_bytes) + 1)
+    return r if r <= 16 else 0
+
+
 def run_gpu(args, world, rank, local):
     import paged_kv_cache_449_b200 as pa
     from paged_kv_cache_449_b200 import build as pabuild
@@ -266,51 +293,76 @@ def run_gpu(args, world, rank, local):
     pa.load()
     batch = make_workload(args.workload, args.seed + rank, "cuda", args.block_size)
     mode = args.mode
-    step = Step(batch, mode, args.partition_size)
     stream = torch.cuda.current_stream()
-    flush = None if args.no_flush else torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    l2 = l2_bytes()
+    copies = rotation_copies(batch.unique_kv_bytes(), l2) if args.l2 == "rotate" else 0
+    steps = [Step(batch, mode, args.partition_size) for _ in range(max(1, copies))]
+    step = steps[0]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if copies == 0 else None
     decode_bytes, reshape_bytes = step_bytes(batch)
 
-    def one(timed_events=None):
-        if timed_events is None:
-            step.reshape(stream)
-            step.decode(stream)
-            return
-        e0, e1, e2 = timed_events
-        e0.record(stream)
-        if step.mode != "append":  # append: the whole step is the decode launch
-            step.reshape(stream)
-            e1.record(stream)
-        step.decode(stream)
-        e2.record(stream)
+    def one(i, ev=None):
+        st = steps[i % len(steps)]
+        if ev is not None:
+            ev[0].record(stream)
+        if st.mode != "append":  # append: the whole step is the decode launch
+            st.reshape(stream)
+        if ev is not None:
+            ev[1].record(stream)
+        st.decode(stream)
+        if ev is not None:
+            ev[2].record(stream)
 
-    for _ in range(args.warmup):
+    for i in range(args.warmup):
         if flush is not None:
             flush.zero_()
-        one()
+        one(i)
     torch.cuda.synchronize()
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    region = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        time.sleep(0.3)
-        for i in range(args.steps):
+        # Untimed steps while the sampler starts: the GPU is under load (and
+        # at load clocks) when the timed region begins.
+        t_busy, i = time.perf_counter() + 0.3, 0
+        while time.perf_counter() < t_busy:
             if flush is not None:
                 flush.zero_()
-            one(events[i])
+            one(i)
+            i += 1
+            if i % 16 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        barrier(world)
+        if flush is None:
+            # Rotated inputs: the K steps back to back, one timed region; the
+            # per-step events inside it split reshape from decode.
+            region[0].record(stream)
+            for i in range(args.steps):
+                one(i, events[i] if mode != "append" else None)
+            region[1].record(stream)
+        else:
+            for i in range(args.steps):
+                flush.zero_()
+                one(i, events[i])
         torch.cuda.synchronize()
     barrier(world)
-    step_ms = [e[0].elapsed_time(e[2]) for e in events]
-    if mode == "append":
-        decode_ms = step_ms
-        reshape_ms = [0.0 for _ in events]
+    if flush is None:
+        local_step = region[0].elapsed_time(region[1]) / args.steps
+        if mode == "append":
+            decode_ms, reshape_ms = [local_step], [0.0]
+        else:
+            decode_ms = [e[1].elapsed_time(e[2]) for e in events]
+            reshape_ms = [e[0].elapsed_time(e[1]) for e in events]
     else:
+        step_ms = [e[0].elapsed_time(e[2]) for e in events]
+        local_step = sum(step_ms) / len(step_ms)
         decode_ms = [e[1].elapsed_time(e[2]) for e in events]
         reshape_ms = [e[0].elapsed_time(e[1]) for e in events]
-    local_step = sum(step_ms) / len(step_ms)
     local_decode = sum(decode_ms) / len(decode_ms)
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error word set during the timed steps")
@@ -324,36 +376,43 @@ def run_gpu(args, world, rank, local):
         host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = host_out.numel() * host_out.element_size()
-        e2e_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
 
-        def e2e_step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            step.q.copy_(host["q"], non_blocking=True)
-            step.nk.copy_(host["nk"], non_blocking=True)
-            step.nv.copy_(host["nv"], non_blocking=True)
-            step.slots.copy_(host["slots"], non_blocking=True)
-            step.bt.copy_(host["bt"], non_blocking=True)
-            step.cl.copy_(host["cl"], non_blocking=True)
-            step.reshape(stream)
-            step.decode(stream)
-            host_out.copy_(step.out, non_blocking=True)
-            if ev is not None:
-                ev[1].record(stream)
+        def e2e_step(i):
+            st = steps[i % len(steps)]
+            st.q.copy_(host["q"], non_blocking=True)
+            st.nk.copy_(host["nk"], non_blocking=True)
+            st.nv.copy_(host["nv"], non_blocking=True)
+            st.slots.copy_(host["slots"], non_blocking=True)
+            st.bt.copy_(host["bt"], non_blocking=True)
+            st.cl.copy_(host["cl"], non_blocking=True)
+            st.reshape(stream)
+            st.decode(stream)
+            host_out.copy_(st.out, non_blocking=True)
 
-        for _ in range(args.warmup):
+        for i in range(args.warmup):
             if flush is not None:
                 flush.zero_()
-            e2e_step()
+            e2e_step(i)
         torch.cuda.synchronize()
         barrier(world)
-        for i in range(args.steps):
-            if flush is not None:
+        if flush is None:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+            ev[0].record(stream)
+            for i in range(args.steps):
+                e2e_step(i)
+            ev[1].record(stream)
+            torch.cuda.synchronize()
+            e2e_ms = ev[0].elapsed_time(ev[1]) / args.steps
+        else:
+            e2e_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+            for i in range(args.steps):
                 flush.zero_()
-            e2e_step(e2e_events[i])
-        torch.cuda.synchronize()
+                e2e_events[i][0].record(stream)
+                e2e_step(i)
+                e2e_events[i][1].record(stream)
+            torch.cuda.synchronize()
+            e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_events) / args.steps
         barrier(world)
-        e2e_ms = sum(e[0].elapsed_time(e[1]) for e in e2e_events) / args.steps
         e2e_ms_max = reduce_max(e2e_ms, world)
         e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms_max, "_local_bytes": decode_bytes + reshape_bytes}
@@ -394,8 +453,10 @@ def run_gpu(args, world, rank, local):
                              "append": "pa_decode_append"}.get(mode, "pa_decode"),
             "partition_size": args.partition_size if mode.startswith("splitk") else None,
             "parallelism": f"replicas x{world} (sequence batches, no collective)",
-            "l2": "flushed between steps (256 MiB write), per-step CUDA events" if flush is not None
-            else "not flushed",
+            "l2": (f"inputs larger than L2 ({batch.unique_kv_bytes() / 1e6:.0f} MB of distinct KV per step vs "
+                   f"{l2 / 1e6:.0f} MB L2), rotated over {len(steps)} independent copies; K steps in one "
+                   f"CUDA-event region") if flush is None
+            else "flushed between steps (256 MiB write), per-step CUDA events",
             "step": ("pa_decode_append: newest token of every sequence written + decode, one launch" if mode == "append"
                      else "pa_reshape_and_cache (newest token of every sequence) + decode"),
         },

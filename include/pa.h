@@ -85,6 +85,20 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
 #define PA_DEVERR_CONTEXT_LEN  2  /* a context length < 0 or above the stated maximum */
 #define PA_DEVERR_SLOT         4  /* a slot >= num_blocks * block_size */
 #define PA_DEVERR_TIMEOUT      8  /* an asynchronous copy did not complete in time */
+#define PA_DEVERR_SEQ_ORDER   16  /* a seq_order entry outside [0, num_seqs) */
+
+/*
+ * seq_order (pa_decode, pa_decode_append, pa_decode_splitk) — NULL, or an
+ * int32 [num_seqs] device array holding a permutation of 0..num_seqs-1,
+ * 4-byte aligned.  The pages fix no processing order; this is a scheduling
+ * hint only.  The GPU starts the thread blocks of sequence seq_order[0]
+ * first, then seq_order[1], ...; a host scheduler that knows the context
+ * lengths passes them longest first, so long sequences do not start last and
+ * hold up the end of the launch.  The results are bit-identical for every
+ * order.  An entry outside [0, num_seqs) sets PA_DEVERR_SEQ_ORDER and the
+ * thread blocks it names do nothing; a repeated entry is the caller's error
+ * (the sequences it leaves out are then not computed).
+ */
 
 /*
  * pa_reshape_and_cache — write the K/V of new tokens into the pools.
@@ -123,7 +137,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     const int32_t* block_tables, const int32_t* context_lens, float scale,
                     int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                     int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
-                    void* stream);
+                    const int32_t* seq_order, void* stream);
 
 /*
  * pa_decode_append — one decode step in one launch: for every sequence s with
@@ -146,7 +160,7 @@ pa_status pa_decode_append(void* out, const void* q, const void* key, const void
                            void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
                            float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
                            int head_dim, int max_blocks_per_seq, int max_context_len, int64_t num_blocks,
-                           pa_dtype dtype, void* stream);
+                           pa_dtype dtype, const int32_t* seq_order, void* stream);
 
 /*
  * pa_decode_splitk_workspace_size — bytes of workspace pa_decode_splitk needs:
@@ -192,7 +206,7 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
                            int head_dim, int max_blocks_per_seq, int max_context_len,
                            int64_t num_blocks, pa_dtype dtype, int partition_size, void* workspace,
                            size_t workspace_bytes, int32_t* counters, int64_t num_counters,
-                           void* stream);
+                           const int32_t* seq_order, void* stream);
 
 /*
  * pa_decode_splitk_static — pa_decode_splitk for callers that cannot
@@ -220,7 +234,8 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
  *   Every call on a device shares the one array: calls that may overlap on
  *   the GPU (different streams without ordering between them) race on it and
  *   must not be issued.
- *   Other arguments, results and errors as in pa_decode_splitk.
+ *   Other arguments, results and errors as in pa_decode_splitk with
+ *   seq_order NULL.
  */
 #define PA_SPLITK_STATIC_SCRATCH_BYTES (16u << 20)
 

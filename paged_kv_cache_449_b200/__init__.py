@@ -21,7 +21,8 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "Counters",
            "pa_decode_splitk_static", "SPLITK_STATIC_SCRATCH_BYTES",
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
-           "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT"]
+           "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT",
+           "DEVERR_SEQ_ORDER", "longest_first"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -29,7 +30,7 @@ _LIB_PATH = os.path.join(_HERE, "libpa.so")
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 _DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
 STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE", 4: "PA_ERR_CUDA"}
-DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT = 1, 2, 4, 8
+DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_SEQ_ORDER = 1, 2, 4, 8, 16
 
 
 class PagedAttentionError(RuntimeError):
@@ -59,13 +60,13 @@ def load() -> ctypes.CDLL:
     lib.pa_reshape_and_cache.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I, P]
     decode_args = [P, P, P, P, P, P, F, I, I, I, I, I, I, I, I64, I]
     lib.pa_decode.restype = I
-    lib.pa_decode.argtypes = decode_args + [P]
+    lib.pa_decode.argtypes = decode_args + [P, P]
     lib.pa_decode_append.restype = I
-    lib.pa_decode_append.argtypes = [P, P, P, P] + decode_args[2:] + [P]
+    lib.pa_decode_append.argtypes = [P, P, P, P] + decode_args[2:] + [P, P]
     lib.pa_decode_splitk_workspace_size.restype = I
     lib.pa_decode_splitk_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
     lib.pa_decode_splitk.restype = I
-    lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P, I64, P]
+    lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P, I64, P, P]
     lib.pa_decode_splitk_static.restype = I
     lib.pa_decode_splitk_static.argtypes = decode_args + [I, P]
     lib.pa_get_device_error.restype = I
@@ -134,22 +135,41 @@ def _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, ma
             Hq, hkv, D, int(block_tables.shape[1]), int(max_context_len), n, _DTYPE[q.dtype]]
 
 
-def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None, stream=None):
+def longest_first(context_lens) -> torch.Tensor:
+    """The scheduling hint `seq_order` for a batch whose context lengths the
+    host knows: sequence indices by decreasing length (ties by index), as a
+    CPU int32 tensor to be copied to the device with the other step inputs."""
+    lens = torch.as_tensor(context_lens).detach().to("cpu", torch.int64).reshape(-1)
+    return torch.sort(-lens, stable=True).indices.to(torch.int32)
+
+
+def _order_ptr(seq_order, num_seqs):
+    if seq_order is None:
+        return None
+    if seq_order.dtype != torch.int32 or seq_order.numel() != num_seqs:
+        raise ValueError("seq_order must be an int32 permutation of range(num_seqs)")
+    return _dev_ptr(seq_order, "seq_order")
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None, stream=None,
+              seq_order=None):
     """Paged decode attention, one launch.  out, q: [S, Hq, D]; block_tables
-    int32 [S, max_blocks]; context_lens int32 [S]."""
+    int32 [S, max_blocks]; context_lens int32 [S]; seq_order: None or an int32
+    device permutation of range(S), the order in which sequences are started
+    (see longest_first); the result does not depend on it."""
     lib = load()
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
-    _check(lib.pa_decode(*args, _stream(stream)), "pa_decode")
+    _check(lib.pa_decode(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode")
 
 
 def pa_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
-                     stream=None):
+                     stream=None, seq_order=None):
     """One decode step: write each sequence's newest token (key/value [S, Hkv,
     D]) at position context_lens[s]-1, then attend over the whole context."""
     lib = load()
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_append(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
-                                _stream(stream)), "pa_decode_append")
+                                _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_append")
 
 
 def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size=512) -> int:
@@ -182,7 +202,7 @@ _splitk_ws_cache: dict = {}
 
 
 def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
-                     partition_size=512, workspace=None, fused=True, counters=None, stream=None):
+                     partition_size=512, workspace=None, fused=True, counters=None, stream=None, seq_order=None):
     """Split-K paged decode (partitions of partition_size tokens + log-sum-exp
     merge).  `workspace` is a CUDA uint8 tensor of at least
     pa_decode_splitk_workspace_size(...) bytes (allocated here if None).
@@ -207,7 +227,8 @@ def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale
         cptr, ncount = _dev_ptr(buf, "counters"), buf.numel()
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_splitk(*args, int(partition_size), _dev_ptr(workspace, "workspace"),
-                                workspace.numel() * workspace.element_size(), cptr, ncount, _stream(stream)),
+                                workspace.numel() * workspace.element_size(), cptr, ncount,
+                                _order_ptr(seq_order, S), _stream(stream)),
            "pa_decode_splitk")
 
 

@@ -17,37 +17,46 @@
 #include "pa_decode.cuh"
 #include "pa_reshape.cuh"
 
-// Warps per CTA and per-warp shared-memory ring bytes of each decode entry
-// point (measured on B200 over the benchmark workloads): the one-pass kernel
-// streams a whole sequence per CTA and wants more warps in flight per CTA; the
-// split-K kernel runs many short CTAs and wants more CTAs per SM.
-#ifndef PA_SINGLE_WARPS
-#define PA_SINGLE_WARPS 8
+// Two CTA shapes for the decode kernels, measured on B200 over the benchmark
+// workloads (warps per CTA, shared-memory ring bytes per warp):
+//  * deep: one large CTA per SM with a two-stage ring per warp; best when the
+//    grid is at most PA_DEEP_MAX_CTAS_PER_SM CTAs per SM (few, long
+//    sequences per SM), where each CTA streams long enough to amortise its
+//    start-up;
+//  * wide: small CTAs, several resident per SM, so one CTA's start-up
+//    (block-table read, first copies) and final merge overlap other CTAs'
+//    streaming; best for grids of many short CTAs (split-K partitions,
+//    batches of short sequences).
+#ifndef PA_DEEP_WARPS
+#define PA_DEEP_WARPS 8
 #endif
-#ifndef PA_SINGLE_RING
-#define PA_SINGLE_RING 16384
+#ifndef PA_DEEP_RING
+#define PA_DEEP_RING 16384
 #endif
-#ifndef PA_SPLIT_WARPS
-#define PA_SPLIT_WARPS 4
+#ifndef PA_WIDE_WARPS
+#define PA_WIDE_WARPS 4
 #endif
-#ifndef PA_SPLIT_RING
-#define PA_SPLIT_RING 12288
+#ifndef PA_WIDE_RING
+#define PA_WIDE_RING 12288
+#endif
+#ifndef PA_DEEP_MAX_CTAS_PER_SM
+#define PA_DEEP_MAX_CTAS_PER_SM 4
 #endif
 
 namespace {
 
-enum class Kind { kSingle, kSplit };
+enum class Kind { kDeep, kWide };
 
 template <Kind K>
 struct KindTuning;
 // kRingCap bounds the K/V ring of a CTA.
 template <>
-struct KindTuning<Kind::kSingle> {
-    static constexpr int kWarps = PA_SINGLE_WARPS, kRing = PA_SINGLE_RING, kRingCap = 200 * 1024;
+struct KindTuning<Kind::kDeep> {
+    static constexpr int kWarps = PA_DEEP_WARPS, kRing = PA_DEEP_RING, kRingCap = 200 * 1024;
 };
 template <>
-struct KindTuning<Kind::kSplit> {
-    static constexpr int kWarps = PA_SPLIT_WARPS, kRing = PA_SPLIT_RING, kRingCap = 200 * 1024;
+struct KindTuning<Kind::kWide> {
+    static constexpr int kWarps = PA_WIDE_WARPS, kRing = PA_WIDE_RING, kRingCap = 200 * 1024;
 };
 
 
@@ -132,9 +141,9 @@ cudaError_t with_variant(pa_dtype dt, int D, int B, F&& f) {
     }
 }
 
-template <typename T, int D, int B, bool SPLIT>
+template <typename T, int D, int B, bool SPLIT, Kind K>
 cudaError_t launch_decode(const pa::DecodeParams& p, dim3 grid, cudaStream_t stream) {
-    using C = DecodeConfig<T, D, B, SPLIT ? Kind::kSplit : Kind::kSingle>;
+    using C = DecodeConfig<T, D, B, K>;
     auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
@@ -142,11 +151,35 @@ cudaError_t launch_decode(const pa::DecodeParams& p, dim3 grid, cudaStream_t str
     return cudaGetLastError();
 }
 
+// Streaming multiprocessors of the current device, once per device.
+int sm_count() {
+    static std::mutex mu;
+    static std::map<int, int> counts;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = counts.find(dev);
+    if (it != counts.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return counts[dev] = n;
+}
+
+// The split kernel always runs wide CTAs; the one-pass kernel runs deep CTAs
+// unless its grid holds more than PA_DEEP_MAX_CTAS_PER_SM CTAs per SM.
 template <bool SPLIT>
 cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p, dim3 grid, cudaStream_t st) {
+    const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
+    const bool deep = !SPLIT && ctas <= static_cast<long long>(PA_DEEP_MAX_CTAS_PER_SM) * sm_count();
     return with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) {
         using T = typename decltype(tt)::type;
-        return launch_decode<T, decltype(dd)::value, decltype(bb)::value, SPLIT>(p, grid, st);
+        constexpr int kD = decltype(dd)::value, kB = decltype(bb)::value;
+        if constexpr (SPLIT) {
+            return launch_decode<T, kD, kB, true, Kind::kWide>(p, grid, st);
+        } else {
+            return deep ? launch_decode<T, kD, kB, false, Kind::kDeep>(p, grid, st)
+                        : launch_decode<T, kD, kB, false, Kind::kWide>(p, grid, st);
+        }
     });
 }
 
@@ -269,12 +302,15 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache
 pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* block_tables, const int32_t* context_lens, float scale, int block_size,
                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
-                    int max_context_len, int64_t num_blocks, pa_dtype dtype, void* stream) {
+                    int max_context_len, int64_t num_blocks, pa_dtype dtype, const int32_t* seq_order,
+                    void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     if (st != PA_OK || num_seqs == 0) return st;
-    const pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
+    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.seq_order = seq_order;
     const dim3 grid(1, num_kv_heads, num_seqs);
     const cudaError_t e = decode_dispatch<false>(dtype, head_dim, block_size, p, grid,
                                                  static_cast<cudaStream_t>(stream));
@@ -284,13 +320,16 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
 pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value, void* k_cache, void* v_cache,
                            const int32_t* block_tables, const int32_t* context_lens, float scale, int block_size,
                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
-                           int max_context_len, int64_t num_blocks, pa_dtype dtype, void* stream) {
+                           int max_context_len, int64_t num_blocks, pa_dtype dtype, const int32_t* seq_order,
+                           void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     if (st != PA_OK || num_seqs == 0) return st;
     if (!key || !value || !aligned16(key) || !aligned16(value)) return PA_ERR_INVALID_ARG;
+    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
     pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.seq_order = seq_order;
     p.new_key = key;
     p.new_value = value;
     const dim3 grid(1, num_kv_heads, num_seqs);
@@ -314,7 +353,7 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
                            int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                            int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
                            int partition_size, void* workspace, size_t workspace_bytes, int32_t* counters,
-                           int64_t num_counters, void* stream) {
+                           int64_t num_counters, const int32_t* seq_order, void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
@@ -322,7 +361,9 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
     if (partition_size <= 0 || partition_size % 16 != 0 || partition_size % block_size != 0)
         return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
+    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
     pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.seq_order = seq_order;
     const int pb = partition_size / block_size;
     const long long cap_blocks = (static_cast<long long>(p.context_cap) + block_size - 1) / block_size;
     const long long parts = (cap_blocks + pb - 1) / pb;
@@ -440,5 +481,5 @@ extern "C" pa_status pa_decode_splitk_static(void* out, const void* q, const voi
     // start at zero, and the previous call's leftovers are never read.
     return pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size, num_seqs,
                             num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, max_context_len, num_blocks,
-                            dtype, partition_size, scratch, kStaticScratchBytes, nullptr, 0, stream);
+                            dtype, partition_size, scratch, kStaticScratchBytes, nullptr, 0, nullptr, stream);
 }

@@ -57,6 +57,7 @@ struct DecodeParams {
     int* counters;         // split, fused merge: [S*Hkv] arrival counters (zero between calls); null = merge kernel
     const void* new_key;   // append: [S][Hkv][D] K/V of each sequence's newest token (position L-1), or null
     const void* new_value;
+    const int32_t* seq_order;  // optional [S] permutation: CTA z works on sequence seq_order[z]; null = z
 };
 
 // Append: the newest token of sequence s (logical position L-1) is written
@@ -167,8 +168,28 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     float* qs = reinterpret_cast<float*>(smem + Smem::kArea + Smem::kBars);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int part = blockIdx.x, kvh = blockIdx.y;
+    int s = blockIdx.z;
+    if (p.seq_order != nullptr) {
+        // CTAs start roughly in blockIdx order, so a longest-first order
+        // starts the long sequences early and leaves the short ones to fill
+        // the SMs at the end of the launch.
+        s = __ldg(p.seq_order + blockIdx.z);
+        if (static_cast<unsigned>(s) >= static_cast<unsigned>(p.num_seqs)) {
+            if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(16 /* PA_DEVERR_SEQ_ORDER */);
+            return;
+        }
+    }
     const int group = p.group;
+
+    // The warp's ring barriers are set up before any global load is issued.
+    uint64_t* wbar = bars + warp * STAGES;
+    uint8_t* wring = ring + warp * STAGES * 2 * kTile;
+    if (lane == 0) {
+        for (int i = 0; i < STAGES; ++i) mbar_init(&wbar[i], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
 
     // Issued before the context length arrives, so the three loads overlap:
     // this warp's first 32 block-table entries (any entry of the row is
@@ -224,13 +245,6 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
                            (last_block - b0) % NW == warp;
     NewRow<T, D> new_row;
     if (owns_last) new_row.load_row(p, s, kvh, lane);
-    uint64_t* wbar = bars + warp * STAGES;
-    uint8_t* wring = ring + warp * STAGES * 2 * kTile;
-    if (lane == 0) {
-        for (int i = 0; i < STAGES; ++i) mbar_init(&wbar[i], 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
 
     auto load_ids = [&](int round) -> int {
         const int i = round * 32 + lane;

@@ -44,7 +44,6 @@ struct WarpMma {
     static constexpr int kMt = D / 16;  // 16-row tiles of head_dim in O^T
     float o[kMt][4];                    // O^T: (d=16mt+r, h=2c), (d, 2c+1), (d+8, 2c), (d+8, 2c+1)
     uint32_t qa[D / 16][2];             // Q as the B operand: head r, d = 16ks+2c.., 16ks+8+2c..
-    uint32_t qn[D / 16][2];             // prefetched Q of the next pair
     float m_run[2];                     // heads 2c, 2c+1 (score domain, base 2)
     float l_run[2];                     // this thread's share of the sums of heads 2c, 2c+1
 
@@ -70,16 +69,6 @@ struct WarpMma {
         }
     }
     __device__ __forceinline__ void load_q(const T* q_rows, int group, int lane) { fetch_q(qa, q_rows, group, lane); }
-    __device__ __forceinline__ void prefetch_q(const T* q_rows, int group, int lane) {
-        fetch_q(qn, q_rows, group, lane);
-    }
-    __device__ __forceinline__ void use_prefetched_q() {
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            qa[ks][0] = qn[ks][0];
-            qa[ks][1] = qn[ks][1];
-        }
-    }
 
     // Zero the 16-bit halves of a V fragment register that belong to tokens
     // >= valid (token `tok` in the low half, tok+1 in the high half).

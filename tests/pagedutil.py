@@ -190,18 +190,18 @@ def device_batch(batch, device="cuda"):
     }
 
 
-def gpu_decode(batch, mode="single", partition_size=512, dev=None, max_context_len=None):
+def gpu_decode(batch, mode="single", partition_size=512, dev=None, max_context_len=None, seq_order=None):
     import paged_kv_cache_449_b200 as pa
     dev = dev or device_batch(batch)
     out = torch.full_like(dev["q"], float("nan"))
     mcl = batch.max_context_len if max_context_len is None else max_context_len
     if mode == "single":
         pa.pa_decode(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"], dev["context_lens"],
-                     batch.scale, max_context_len=mcl)
+                     batch.scale, max_context_len=mcl, seq_order=seq_order)
     else:  # "splitk" (merge fused into the partition kernel) or "splitk2" (separate merge kernel)
         pa.pa_decode_splitk(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"],
                             dev["context_lens"], batch.scale, mcl, partition_size=partition_size,
-                            fused=(mode == "splitk"))
+                            fused=(mode == "splitk"), seq_order=seq_order)
     torch.cuda.synchronize()
     return out
 

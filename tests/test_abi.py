@@ -72,10 +72,10 @@ P = ctypes.c_void_p
 
 def _decode(lib, **kw):
     a = dict(out=16, q=16, k=16, v=16, bt=16, cl=16, scale=0.125, B=16, S=4, Hq=4, Hkv=4, D=64, mb=7, mcl=100,
-             N=64, dt=0)
+             N=64, dt=0, order=None)
     a.update(kw)
     return lib.pa_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["cl"], a["scale"], a["B"], a["S"], a["Hq"],
-                         a["Hkv"], a["D"], a["mb"], a["mcl"], a["N"], a["dt"], None)
+                         a["Hkv"], a["D"], a["mb"], a["mcl"], a["N"], a["dt"], a["order"], None)
 
 
 def test_host_validation_rejects_before_launch(lib):
@@ -90,14 +90,17 @@ def test_host_validation_rejects_before_launch(lib):
     assert _decode(lib, N=0) == 1                  # empty pool
     assert _decode(lib, scale=float("nan")) == 1
     assert _decode(lib, S=0) == 0                  # empty batch: a no-op
+    assert _decode(lib, order=18) == 1             # misaligned seq_order
     assert lib.pa_reshape_and_cache(16, 16, 16, 16, 16, 4, 8, 100, 16, 10, 2, None) == 2   # 200 B rows
     assert lib.pa_reshape_and_cache(16, 16, 16, 16, 12, 4, 8, 128, 16, 10, 2, None) == 1   # slots misaligned
     assert lib.pa_reshape_and_cache(0, 0, 0, 0, 0, 0, 8, 128, 16, 10, 2, None) == 0        # no tokens
     args = [16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 64, 0]
-    assert lib.pa_decode_splitk(*args, 500, 16, 1 << 20, None, 0, None) == 1   # partition not a multiple of 16
-    assert lib.pa_decode_splitk(*args, 512, 16, 100, None, 0, None) == 3       # workspace too small
-    assert lib.pa_decode_splitk(*args, 512, 0, 1 << 20, None, 0, None) == 3    # no workspace
-    assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, 16, 3, None) == 3     # too few counters
+    assert lib.pa_decode_splitk(*args, 500, 16, 1 << 20, None, 0, None, None) == 1   # partition not a multiple of 16
+    assert lib.pa_decode_splitk(*args, 512, 16, 100, None, 0, None, None) == 3       # workspace too small
+    assert lib.pa_decode_splitk(*args, 512, 0, 1 << 20, None, 0, None, None) == 3    # no workspace
+    assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, 16, 3, None, None) == 3     # too few counters
+    assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, None, 0, 6, None) == 1      # misaligned seq_order
+    assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], 2, None) == 1            # misaligned seq_order
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
@@ -105,3 +108,12 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(pa, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         pa.load()
+
+
+def test_longest_first_is_a_stable_descending_permutation():
+    import torch
+    lens = torch.tensor([5, 300, 17, 300, 0, 64], dtype=torch.int32)
+    order = pa.longest_first(lens)
+    assert order.dtype == torch.int32
+    assert order.tolist() == [1, 3, 5, 2, 0, 4]
+    assert pa.longest_first([]).numel() == 0

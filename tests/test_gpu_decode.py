@@ -64,6 +64,20 @@ def test_small_cases_every_element(orc, case):
     _full_check(orc, b)
 
 
+@pytest.mark.parametrize("case", range(len(SMALL)))
+def test_many_short_sequences_every_element(orc, case):
+    # More than 4 CTAs per SM: the one-pass kernel runs its small-CTA shape
+    # (several CTAs per SM) instead of one large CTA per SM.
+    dt, D, B, Hq, Hkv, _ = SMALL[case]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    S = (4 * sms + 1 + Hkv - 1) // Hkv + 3
+    rng = np.random.default_rng(300 + case)
+    lens = tuple(int(x) for x in rng.integers(0, 4 * B + 3, size=S))
+    b = workloads.random_small(seed=200 + case, dtype=dt, lens=lens, num_q_heads=Hq, num_kv_heads=Hkv,
+                               head_dim=D, block_size=B)
+    _full_check(orc, b, modes=("single",))
+
+
 def test_tiny_mha_f32(orc):
     b = workloads.tiny_mha_f32(seed=0)
     _full_check(orc, b, parts=(512, 16, 32))

@@ -167,6 +167,70 @@ def test_run_to_run_deterministic():
             assert torch.equal(_bits(first), _bits(gpu_decode(b, mode, dev=dev)))
 
 
+# ---------------------------------------------------------------------------- processing order
+
+def _orders(b):
+    S = b.num_seqs
+    g = torch.Generator().manual_seed(17)
+    return [pa.longest_first(b.context_lens), torch.arange(S - 1, -1, -1, dtype=torch.int32),
+            torch.randperm(S, generator=g).to(torch.int32)]
+
+
+@pytest.mark.parametrize("make", [
+    # 48 x 8 and 200 x 8 CTAs: more than one wave of resident CTAs, so the
+    # L2 warm-up of later CTAs runs as well.
+    lambda: workloads.llama3_8b_decode(seed=21, device="cuda", num_seqs=48, num_blocks=4096),
+    lambda: workloads.continuous_batching_mix(seed=22, device="cuda", num_seqs=200, block_size=32),
+    lambda: workloads.random_small(seed=23, dtype=torch.float32, lens=(0, 5, 16, 300, 33, 1), num_q_heads=4,
+                                   num_kv_heads=4, head_dim=64, block_size=8),
+])
+def test_seq_order_is_bit_identical(make):
+    b = make()
+    dev = device_batch(b)
+    for mode in ("single", "splitk", "splitk2"):
+        ref = gpu_decode(b, mode, partition_size=256, dev=dev)
+        for order in _orders(b):
+            got = gpu_decode(b, mode, partition_size=256, dev=dev, seq_order=order.cuda())
+            assert torch.equal(_bits(got), _bits(ref)), mode
+    assert pa.pa_get_device_error() == 0
+
+
+def test_seq_order_append_is_bit_identical():
+    b = workloads.continuous_batching_mix(seed=24, device="cuda", num_seqs=64, block_size=16)
+    nk, nv = b.new_key.cuda().contiguous(), b.new_value.cuda().contiguous()
+    outs, pools = [], []
+    for order in [None] + _orders(b):
+        d = device_batch(b)
+        d["k_cache"], d["v_cache"] = d["k_cache"].clone(), d["v_cache"].clone()
+        out = torch.full_like(d["q"], float("nan"))
+        pa.pa_decode_append(out, d["q"], nk, nv, d["k_cache"], d["v_cache"], d["block_tables"], d["context_lens"],
+                            b.scale, max_context_len=b.max_context_len,
+                            seq_order=None if order is None else order.cuda())
+        torch.cuda.synchronize()
+        outs.append(out)
+        pools.append((d["k_cache"], d["v_cache"]))
+    for out, (k, v) in zip(outs[1:], pools[1:]):
+        assert torch.equal(_bits(out), _bits(outs[0]))
+        assert torch.equal(_bits(k), _bits(pools[0][0])) and torch.equal(_bits(v), _bits(pools[0][1]))
+
+
+def test_seq_order_out_of_range_is_flagged_and_skipped():
+    b = workloads.random_small(seed=25, dtype=torch.bfloat16, lens=(40, 20, 70), num_q_heads=4, num_kv_heads=2,
+                               head_dim=128, block_size=16)
+    dev = device_batch(b)
+    ref = gpu_decode(b, "single", dev=dev)
+    pa.pa_get_device_error()
+    order = torch.tensor([2, 99, 0], dtype=torch.int32, device="cuda")   # sequence 1 left out
+    for mode in ("single", "splitk", "splitk2"):
+        got = gpu_decode(b, mode, dev=dev, seq_order=order)
+        assert pa.pa_get_device_error() & pa.DEVERR_SEQ_ORDER
+        for s in (0, 2):
+            check_tolerance(as_f64(got[s]), as_f64(ref[s]), b.dtype)
+        if mode == "single":
+            assert torch.isnan(got[1].float()).all()   # never written
+    assert pa.pa_get_device_error() == 0
+
+
 # ---------------------------------------------------------------------------- error word
 
 def test_out_of_range_block_id_is_flagged_not_read():
