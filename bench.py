@@ -401,31 +401,39 @@ def run_gpu(args, world, rank, local):
             download(st, i, stream)
 
         def pipelined(n, ev0, ev1):
-            """n steps; step i+1's inputs go up on a copy stream while step i
-            computes, and step i's output comes down once its kernels end.
-            A copy of the inputs is reused only after its previous step ended."""
-            side = torch.cuda.Stream()
+            """n steps; step i+1's inputs go up on one copy stream while step i
+            computes, and step i's output comes down on another (opposite
+            directions: separate copy engines) once its kernels end.  A rotated
+            copy's inputs are overwritten only after its previous step ended, and
+            its output only after that output was read back."""
+            up_s, down_s = torch.cuda.Stream(), torch.cuda.Stream()
             R = len(steps)
             up = [torch.cuda.Event() for _ in range(n)]
             done = [torch.cuda.Event() for _ in range(n)]
-            side.wait_stream(stream)
-            ev0.record(side)
-            upload(steps[0], side)
-            up[0].record(side)
+            down = [torch.cuda.Event() for _ in range(n)]
+            up_s.wait_stream(stream)
+            down_s.wait_stream(stream)
+            ev0.record(up_s)
+            upload(steps[0], up_s)
+            up[0].record(up_s)
             for i in range(n):
                 st = steps[i % R]
                 stream.wait_event(up[i])
+                if i - R >= 0:
+                    stream.wait_event(down[i - R])
                 st.reshape(stream)
                 st.decode(stream)
                 done[i].record(stream)
                 if i + 1 < n:
                     if i + 1 - R >= 0:
-                        side.wait_event(done[i + 1 - R])
-                    upload(steps[(i + 1) % R], side)
-                    up[i + 1].record(side)
-                side.wait_event(done[i])
-                download(st, i, side)
-            stream.wait_stream(side)
+                        up_s.wait_event(done[i + 1 - R])
+                    upload(steps[(i + 1) % R], up_s)
+                    up[i + 1].record(up_s)
+                down_s.wait_event(done[i])
+                download(st, i, down_s)
+                down[i].record(down_s)
+            stream.wait_stream(up_s)
+            stream.wait_stream(down_s)
             ev1.record(stream)
 
         e2e_modes = {}
@@ -465,8 +473,8 @@ def run_gpu(args, world, rank, local):
         e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms_max, "_local_bytes": decode_bytes + reshape_bytes,
                "pipelined": "pipelined" in e2e_modes,
-               "how": ("step i+1's inputs uploaded on a second stream while step i computes; step i's output "
-                       "read back when its kernels end" if "pipelined" in e2e_modes
+               "how": ("step i+1's inputs uploaded on a copy stream while step i computes; step i's output "
+                       "read back on another copy stream when its kernels end" if "pipelined" in e2e_modes
                        else "upload, step, read-back serialised on one stream"),
                "serial_ms_per_step": e2e_serial_ms_max}
 

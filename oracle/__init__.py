@@ -66,6 +66,10 @@ class Oracle:
         lib.oracle_decode.argtypes = decode_args
         lib.oracle_decode_partitioned.restype = c.c_int
         lib.oracle_decode_partitioned.argtypes = decode_args + [c.c_int]
+        lib.oracle_copy_blocks.restype = c.c_int
+        lib.oracle_copy_blocks.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64,
+            c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int64, c.c_int]
         lib.oracle_pool_index.restype = c.c_int64
         lib.oracle_pool_index.argtypes = [c.c_int64, c.c_int, c.c_int, c.c_int, c.c_int,
                                           c.c_int, c.c_int, c.c_int]
@@ -107,6 +111,19 @@ class Oracle:
         else:
             self._check(self.lib.oracle_decode_partitioned(*args, int(partition_size)))
         return out
+
+    def copy_blocks(self, dst_k, dst_v, src_k, src_v, block_mapping, block_size):
+        """In place: copy whole blocks (src, dst) = block_mapping[i] ([n, 2]
+        int64) from the source pools to the destination pools (CPU tensors,
+        pool layout; the same tensors on both sides for a copy-on-write)."""
+        for t in (dst_k, dst_v, src_k, src_v):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        m = block_mapping.to(torch.int64).contiguous()
+        Hkv = src_k.shape[1]
+        D = src_k.shape[2] * src_k.shape[4]
+        self._check(self.lib.oracle_copy_blocks(
+            dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(), src_v.data_ptr(), m.data_ptr(),
+            m.shape[0], Hkv, D, block_size, src_k.shape[0], dst_k.shape[0], DTYPE_CODE[src_k.dtype]))
 
     def pool_index(self, block, head, token, dim, num_kv_heads, block_size, head_dim, dtype):
         return int(self.lib.oracle_pool_index(block, head, token, dim, num_kv_heads,

@@ -21,6 +21,8 @@
 //   [P4] "vLLM框架解析：PagedAttention技术如何实现LLM推理20倍加速"
 //        (intelliparadigm.com), §2.3 zero-copy sharing of prefix blocks by
 //        reference count, copy-on-write for isolation.
+//   [P1] §4.2 preemption: a preempted sequence's KV blocks are swapped out to
+//        CPU memory (or dropped and recomputed) and swapped back in later.
 //
 // Readings where the pages are silent (each is listed in the design notes):
 //   * pool layout: an element (block b, kv head h, token t, dim d) lives at
@@ -325,6 +327,44 @@ int oracle_decode_partitioned(double* out, const void* q, const void* k_cache, c
 
 // Position of element (block, head, token, dim) in a pool of the given shape,
 // exported so the layout itself can be pinned against hand-derived offsets.
+// Copies whole physical blocks (every kv head, token and dimension of the K
+// and of the V pool) from a source pool pair to a destination pool pair:
+// block_mapping holds num_pairs (src, dst) block-id pairs.  The same pool as
+// source and destination is the copy-on-write duplicate of a shared block
+// ([P4] §2.3); a host-memory pool on one side is a swap-out or swap-in of a
+// preempted sequence's blocks ([P1] §4.2).  Element by element through the
+// pool layout, pairs in order.  A block id outside its pool is refused.
+int oracle_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                       const int64_t* block_mapping, int64_t num_pairs, int num_kv_heads,
+                       int head_dim, int block_size, int64_t src_num_blocks,
+                       int64_t dst_num_blocks, int dtype) {
+    if (!dst_k || !dst_v || !src_k || !src_v || (!block_mapping && num_pairs > 0)) return kBadArg;
+    if (!dtype_ok(dtype) || num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        src_num_blocks <= 0 || dst_num_blocks <= 0)
+        return kBadArg;
+    const int es = elem_size(dtype);
+    const int vec = 16 / es;
+    if (head_dim % vec != 0) return kBadArg;
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        const int64_t src = block_mapping[2 * i];
+        const int64_t dst = block_mapping[2 * i + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return kBadBlockId;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            for (int t = 0; t < block_size; ++t) {
+                for (int d = 0; d < head_dim; ++d) {
+                    const int64_t from = pool_index(src, h, t, d, num_kv_heads, block_size, head_dim, vec);
+                    const int64_t to = pool_index(dst, h, t, d, num_kv_heads, block_size, head_dim, vec);
+                    std::memcpy(static_cast<uint8_t*>(dst_k) + to * es,
+                                static_cast<const uint8_t*>(src_k) + from * es, es);
+                    std::memcpy(static_cast<uint8_t*>(dst_v) + to * es,
+                                static_cast<const uint8_t*>(src_v) + from * es, es);
+                }
+            }
+        }
+    }
+    return kOk;
+}
+
 int64_t oracle_pool_index(int64_t block, int head, int token, int dim, int num_kv_heads,
                           int block_size, int head_dim, int dtype) {
     return pool_index(block, head, token, dim, num_kv_heads, block_size, head_dim,

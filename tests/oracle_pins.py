@@ -277,6 +277,96 @@ def pin_reshape_scatter(orc):
             v0.view(-1).view(kb.dtype), b.v_cache.view(-1).view(kb.dtype))
 
 
+# ---------------------------------------------------------------------------- block copies (CoW, swap)
+
+def _bits_rows(pool):
+    """A pool as [num_blocks, bytes-per-block / 2] 16-bit words: each block
+    (all its heads, tokens and dimensions) is one contiguous row."""
+    return pool.contiguous().view(pool.shape[0], -1).view(torch.int16)
+
+
+def pin_copy_blocks_rows(orc):
+    """Whole-block copies vs row copies of the pools viewed as [blocks, bytes]
+    (no layout arithmetic): each destination row equals its source row, every
+    other row keeps its bytes, K and V pools independently."""
+    for dt, B, D, Hkv in ((torch.bfloat16, 16, 128, 2), (torch.float32, 8, 64, 3), (torch.float16, 32, 64, 1)):
+        src = workloads.random_small(seed=71, dtype=dt, lens=(40, 9), num_q_heads=Hkv, num_kv_heads=Hkv,
+                                     head_dim=D, block_size=B, extra_blocks=6)
+        dst = workloads.random_small(seed=72, dtype=dt, lens=(17,), num_q_heads=Hkv, num_kv_heads=Hkv,
+                                     head_dim=D, block_size=B, extra_blocks=9)
+        n_src, n_dst = src.num_blocks, dst.num_blocks
+        pairs = torch.tensor([[0, n_dst - 1], [n_src - 1, 0], [2, 3], [2, 5]], dtype=torch.int64)
+        for same in (False, True):   # another pool pair (swap) / the same pool pair (copy-on-write)
+            if same:
+                dk, dv = src.k_cache.clone(), src.v_cache.clone()
+                sk, sv = dk, dv
+                pairs_s = torch.tensor([[0, n_src - 1], [1, 4]], dtype=torch.int64)
+            else:
+                dk, dv = dst.k_cache.clone(), dst.v_cache.clone()
+                sk, sv = src.k_cache.clone(), src.v_cache.clone()
+                pairs_s = pairs
+            want_k, want_v = _bits_rows(dk).clone(), _bits_rows(dv).clone()
+            src_k_rows, src_v_rows = _bits_rows(sk).clone(), _bits_rows(sv).clone()
+            for a, b_ in pairs_s.tolist():
+                want_k[b_] = src_k_rows[a]
+                want_v[b_] = src_v_rows[a]
+            orc.copy_blocks(dk, dv, sk, sv, pairs_s, B)
+            assert torch.equal(_bits_rows(dk), want_k) and torch.equal(_bits_rows(dv), want_v), (dt, same)
+
+
+def pin_copy_on_write_keeps_attention(orc):
+    """Copy-on-write ([P4] §2.3): duplicating a shared block into a free block
+    and pointing one sequence at the duplicate leaves every sequence's
+    attention output bit-identical in fp64."""
+    b = workloads.prefix_sharing(seed=73, prefix_len=40, num_seqs=3, block_size=8, suffix_range=(3, 12))
+    before = _decode(orc, b)
+    used = set(int(x) for x in b.block_tables[b.block_tables >= 0].tolist())
+    free = [i for i in range(b.num_blocks) if i not in used]
+    extra = 3 - len(free)
+    if extra > 0:   # make room for the copies
+        pad = torch.zeros((extra,) + tuple(b.k_cache.shape[1:]), dtype=b.k_cache.dtype)
+        k = torch.cat([b.k_cache, pad]).contiguous()
+        v = torch.cat([b.v_cache, pad]).contiguous()
+        free += list(range(b.num_blocks, b.num_blocks + extra))
+    else:
+        k, v = b.k_cache.clone(), b.v_cache.clone()
+    tables = b.block_tables.clone()
+    pairs = []
+    for s, dst in zip(range(b.num_seqs), free):
+        src = int(tables[s, 0])
+        pairs.append([src, dst])
+        tables[s, 0] = dst
+    orc.copy_blocks(k, v, k, v, torch.tensor(pairs, dtype=torch.int64), b.block_size)
+    after = orc.decode(b.q, k, v, tables, b.context_lens, b.scale, b.block_size, b.num_kv_heads)
+    np.testing.assert_array_equal(after, before)
+
+
+def pin_swap_round_trip(orc):
+    """Preemption by swapping ([P1] §4.2): a sequence's blocks copied out to a
+    second (host) pool and back into other free blocks of the device pool,
+    with its table rewritten, attend exactly as before."""
+    b = workloads.random_small(seed=74, dtype=torch.bfloat16, lens=(37, 20, 5), num_q_heads=4, num_kv_heads=2,
+                               head_dim=64, block_size=8, extra_blocks=8)
+    before = _decode(orc, b)
+    s = 0
+    nblk = (int(b.context_lens[s]) + b.block_size - 1) // b.block_size
+    ids = [int(x) for x in b.block_tables[s, :nblk]]
+    host_k = torch.zeros((nblk,) + tuple(b.k_cache.shape[1:]), dtype=b.k_cache.dtype)
+    host_v = torch.zeros_like(host_k)
+    k, v = b.k_cache.clone(), b.v_cache.clone()
+    orc.copy_blocks(host_k, host_v, k, v, torch.tensor([[i, j] for j, i in enumerate(ids)]), b.block_size)
+    used = set(int(x) for x in b.block_tables[b.block_tables >= 0].tolist())
+    free = [i for i in range(b.num_blocks) if i not in used][:nblk]
+    assert len(free) == nblk
+    k[ids] = 0   # the swapped-out blocks are reused by someone else
+    v[ids] = 0
+    orc.copy_blocks(k, v, host_k, host_v, torch.tensor([[j, f] for j, f in enumerate(free)]), b.block_size)
+    tables = b.block_tables.clone()
+    tables[s, :nblk] = torch.tensor(free, dtype=torch.int32)
+    after = orc.decode(b.q, k, v, tables, b.context_lens, b.scale, b.block_size, b.num_kv_heads)
+    np.testing.assert_array_equal(after, before)
+
+
 def pin_errors(orc):
     from oracle import OracleError
     b = workloads.random_small(seed=61, dtype=torch.float16, lens=(9, 3), num_q_heads=2,
@@ -298,6 +388,13 @@ def pin_errors(orc):
         assert "slot" in str(e)
     else:
         raise AssertionError("oracle accepted a slot past the pool")
+    try:
+        orc.copy_blocks(b.k_cache.clone(), b.v_cache.clone(), b.k_cache, b.v_cache,
+                        torch.tensor([[0, b.num_blocks]]), 8)
+    except OracleError as e:
+        assert "block id" in str(e)
+    else:
+        raise AssertionError("oracle accepted a block copy past the pool")
 
 
 def pin_number_formats(orc):
@@ -333,4 +430,4 @@ def pin_number_formats(orc):
 PINS = [pin_layout_golden, pin_slot_golden, pin_brute_force, pin_dense_equality,
         pin_permutation_invariance, pin_block_size_invariance, pin_shared_vs_copied,
         pin_closed_forms, pin_needle, pin_partitioned, pin_reshape_scatter, pin_errors,
-        pin_number_formats]
+        pin_number_formats, pin_copy_blocks_rows, pin_copy_on_write_keeps_attention, pin_swap_round_trip]

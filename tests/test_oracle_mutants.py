@@ -39,6 +39,14 @@ MUTANTS = {
     "bf16_wrong_half": ("static_cast<uint32_t>(bits) << 16);", "static_cast<uint32_t>(bits) << 15);"),
     "context_len_short": ("attend_plain(qrow.data(), keys, values, len, D, scale_d, dst);",
                           "attend_plain(qrow.data(), keys, values, len > 1 ? len - 1 : len, D, scale_d, dst);"),
+    "copy_v_from_k_pool": ("static_cast<const uint8_t*>(src_v) + from * es, es);",
+                           "static_cast<const uint8_t*>(src_k) + from * es, es);"),
+    "copy_last_token_skipped": ("for (int t = 0; t < block_size; ++t) {\n                for (int d = 0; d < head_dim; ++d) {\n                    const int64_t from",
+                                "for (int t = 0; t < block_size - 1; ++t) {\n                for (int d = 0; d < head_dim; ++d) {\n                    const int64_t from"),
+    "copy_direction_reversed": ("const int64_t src = block_mapping[2 * i];\n        const int64_t dst = block_mapping[2 * i + 1];",
+                                "const int64_t dst = block_mapping[2 * i];\n        const int64_t src = block_mapping[2 * i + 1];"),
+    "copy_head_dropped": ("for (int h = 0; h < num_kv_heads; ++h) {\n            for (int t = 0; t < block_size; ++t) {",
+                          "for (int h = 1; h < num_kv_heads; ++h) {\n            for (int t = 0; t < block_size; ++t) {"),
     "q_from_wrong_head": ("(static_cast<int64_t>(s) * sh.num_q_heads + h) * D + d",
                           "(static_cast<int64_t>(s) * sh.num_q_heads + kvh) * D + d"),
 }
