@@ -45,6 +45,7 @@ import torch
 METRIC = "paged decode KV GB/s & tokens/s (Llama-3-8B shape) as % of B200 HBM peak"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+PCIE_GEN5_X16_GBS = 64.0
 
 
 def parse_args(argv=None):
@@ -57,6 +58,10 @@ def parse_args(argv=None):
                     choices=["tiny_mha_f32", "llama3_8b_decode", "continuous_batching_mix", "prefix_sharing",
                              "llama3_70b_long"])
     ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap_out", "swap_in"], default="decode",
+                    help="decode: the hot-path step (default); copy_blocks: every block of the batch duplicated "
+                         "into free blocks of the same pools (copy-on-write / fork); swap_out / swap_in: every "
+                         "block of the batch copied to / from a pinned host pool (preemption by swapping)")
     ap.add_argument("--mode", choices=["append", "single", "splitk", "splitk2"], default="append",
                     help="append: one pa_decode_append launch per step (write + decode); the others launch "
                          "pa_reshape_and_cache then pa_decode (single) or pa_decode_splitk with fused (splitk) or "
@@ -622,6 +627,91 @@ def run_reference(args, world, rank):
     }
 
 
+def run_blocks(args, world, rank, local):
+    """Block copies through pa_copy_blocks: every block of the batch's
+    sequences, K and V pools, per step."""
+    import paged_kv_cache_449_b200 as pa
+    from paged_kv_cache_449_b200 import build as pabuild
+    pabuild.build()
+    pa.load()
+    batch = make_workload(args.workload, args.seed + rank, "cuda", args.block_size)
+    B = batch.block_size
+    k = batch.k_cache.contiguous()
+    v = batch.v_cache.contiguous()
+    ids = []
+    for s in range(batch.num_seqs):
+        n = (int(batch.context_lens[s]) + B - 1) // B
+        ids += [int(x) for x in batch.block_tables[s, :n].tolist()]
+    ids = sorted(set(ids))
+    n = len(ids)
+    block_bytes = batch.num_kv_heads * B * batch.head_dim * batch.elem_bytes
+    stream = torch.cuda.current_stream()
+    if args.op == "copy_blocks":
+        used = set(ids)
+        free = [i for i in range(batch.num_blocks) if i not in used][:n]
+        n = len(free)
+        mapping = torch.tensor([[a, b] for a, b in zip(ids, free)], dtype=torch.int64, device="cuda")
+        dst_k, dst_v, src_k, src_v = k, v, k, v
+        moved = 2 * n * block_bytes * 2          # K and V pools, read + write
+        bound, peak, peak_kind = "hbm", *measured_peaks()
+        peak_kind = f"{peak_kind} copy bandwidth (burst)"
+    else:
+        host_k = torch.empty((n,) + tuple(k.shape[1:]), dtype=k.dtype).pin_memory()
+        host_v = torch.empty_like(host_k).pin_memory()
+        if args.op == "swap_out":
+            mapping = torch.tensor([[a, j] for j, a in enumerate(ids)], dtype=torch.int64, device="cuda")
+            dst_k, dst_v, src_k, src_v = host_k, host_v, k, v
+        else:
+            mapping = torch.tensor([[j, a] for j, a in enumerate(ids)], dtype=torch.int64, device="cuda")
+            dst_k, dst_v, src_k, src_v = k, v, host_k, host_v
+        moved = 2 * n * block_bytes              # bytes across PCIe
+        bound, peak, peak_kind = "pcie", PCIE_GEN5_X16_GBS, "nominal PCIe Gen5 x16, one direction"
+
+    def one():
+        pa.pa_copy_blocks(dst_k, dst_v, src_k, src_v, mapping, stream=stream)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    pa.pa_get_device_error()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        t_busy = time.perf_counter() + 0.3
+        while time.perf_counter() < t_busy:
+            one()
+            torch.cuda.synchronize()
+        barrier(world)
+        ev[0].record(stream)
+        for _ in range(args.steps):
+            one()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    ms = reduce_max(ev[0].elapsed_time(ev[1]) / args.steps, world)
+    total = reduce_sum(moved, world)
+    achieved = moved / (ev[0].elapsed_time(ev[1]) / args.steps * 1e-3) / 1e9
+    return {
+        "metric": {"copy_blocks": "paged KV block copy (copy-on-write duplicate) GB/s",
+                   "swap_out": "paged KV block swap-out to host GB/s",
+                   "swap_in": "paged KV block swap-in from host GB/s"}[args.op],
+        "value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[batch.dtype],
+        "data": "synthetic (the decode workload's pools and block tables)",
+        "config": {"workload": batch.name, "op": args.op, "blocks": n, "block_bytes_per_pool": block_bytes,
+                   "bytes_counted": "K and V read + written" if bound == "hbm" else "K and V moved across PCIe",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     world, rank, local = dist_setup(args)
@@ -629,6 +719,11 @@ def main(argv=None):
         if args.impl == "reference":
             res = run_reference(args, world, rank)
             if res is not None:
+                print(json.dumps(res), flush=True)
+            return
+        if args.op != "decode":
+            res = run_blocks(args, world, rank, local)
+            if rank == 0:
                 print(json.dumps(res), flush=True)
             return
         res, batch = run_gpu(args, world, rank, local)

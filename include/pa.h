@@ -246,6 +246,34 @@ pa_status pa_decode_splitk_static(void* out, const void* q, const void* k_cache,
                                   int64_t num_blocks, pa_dtype dtype, int partition_size, void* stream);
 
 /*
+ * pa_copy_blocks — copy whole physical blocks (every kv head, token and
+ * dimension, K pool and V pool) from a source pool pair to a destination pool
+ * pair.  The same pools on both sides duplicate a shared block before a
+ * sequence writes into it (copy-on-write, [P4] §2.3); a page-locked host pool
+ * on one side swaps a preempted sequence's blocks out to host memory or back
+ * in ([P1] §4.2 preemption by swapping).
+ *
+ *   dst_k_cache,
+ *   dst_v_cache    destination pools of dst_num_blocks blocks (layout above),
+ *                  written at the destination blocks only
+ *   src_k_cache,
+ *   src_v_cache    source pools of src_num_blocks blocks, read only
+ *   block_mapping  int64 [num_pairs][2]: (source block, destination block),
+ *                  8-byte aligned
+ *   Every pool and block_mapping is device memory or page-locked host memory
+ *   that the device can address (cudaHostAlloc / cudaMallocHost, or
+ *   cudaHostRegister'd and mapped); anything else is PA_ERR_INVALID_ARG.  The
+ *   copy is bit-exact.  A pair naming a block outside its pool sets
+ *   PA_DEVERR_BLOCK_ID and is skipped.  Destinations must be distinct, and no
+ *   block may be both a source and a destination in one call (the result is
+ *   then undefined).  num_pairs == 0 is a no-op.
+ */
+pa_status pa_copy_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache,
+                         const void* src_v_cache, const int64_t* block_mapping, int64_t num_pairs,
+                         int num_kv_heads, int head_dim, int block_size, int64_t src_num_blocks,
+                         int64_t dst_num_blocks, pa_dtype dtype, void* stream);
+
+/*
  * pa_get_device_error — read and clear the device error word of the current
  * GPU.  Synchronises `stream` first, so it reports every launch enqueued on it
  * before the call.  *code receives an OR of PA_DEVERR_* bits (0 = no error).

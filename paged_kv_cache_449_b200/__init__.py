@@ -22,7 +22,7 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "pa_decode_splitk_static", "SPLITK_STATIC_SCRATCH_BYTES",
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT",
-           "DEVERR_SEQ_ORDER", "longest_first"]
+           "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -69,6 +69,8 @@ def load() -> ctypes.CDLL:
     lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P, I64, P, P]
     lib.pa_decode_splitk_static.restype = I
     lib.pa_decode_splitk_static.argtypes = decode_args + [I, P]
+    lib.pa_copy_blocks.restype = I
+    lib.pa_copy_blocks.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I64, I, P]
     lib.pa_get_device_error.restype = I
     lib.pa_get_device_error.argtypes = [P, c.POINTER(c.c_int32)]
     lib.pa_status_string.restype = c.c_char_p
@@ -249,6 +251,35 @@ def pa_decode_splitk_static(out, q, k_cache, v_cache, block_tables, context_lens
     lib = load()
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_splitk_static(*args, int(partition_size), _stream(stream)), "pa_decode_splitk_static")
+
+
+def _accessible_ptr(t: torch.Tensor, name: str) -> int:
+    """A CUDA tensor, or a page-locked CPU tensor (the device reaches it
+    through the unified address space)."""
+    if not (t.is_cuda or (t.device.type == "cpu" and t.is_pinned())):
+        raise ValueError(f"{name} must be a CUDA tensor or a pinned CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def pa_copy_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_mapping, stream=None):
+    """Copy whole blocks (src, dst) = block_mapping[i] (int64 [n, 2], on the
+    device or pinned) from the source pools to the destination pools.  Same
+    pools on both sides: copy-on-write duplicates; a pinned CPU pool on one
+    side: swap-out / swap-in.  Pools are [num_blocks, Hkv, D // X, B, X]."""
+    lib = load()
+    n_src, hkv, d, b = _pool_dims(src_k_cache)
+    n_dst, hkv2, d2, b2 = _pool_dims(dst_k_cache)
+    if (hkv, d, b) != (hkv2, d2, b2) or src_k_cache.dtype != dst_k_cache.dtype:
+        raise ValueError("source and destination pools differ in shape or dtype")
+    if block_mapping.dtype != torch.int64 or block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be int64 [n, 2]")
+    _check(lib.pa_copy_blocks(
+        _accessible_ptr(dst_k_cache, "dst_k_cache"), _accessible_ptr(dst_v_cache, "dst_v_cache"),
+        _accessible_ptr(src_k_cache, "src_k_cache"), _accessible_ptr(src_v_cache, "src_v_cache"),
+        _accessible_ptr(block_mapping, "block_mapping"), int(block_mapping.shape[0]), hkv, d, b, n_src, n_dst,
+        _DTYPE[src_k_cache.dtype], _stream(stream)), "pa_copy_blocks")
 
 
 def pa_get_device_error(stream=None) -> int:

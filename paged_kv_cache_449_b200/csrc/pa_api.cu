@@ -14,6 +14,7 @@
 #include <tuple>
 
 #include "pa.h"
+#include "pa_copy.cuh"
 #include "pa_decode.cuh"
 #include "pa_reshape.cuh"
 
@@ -399,6 +400,55 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
     m.partition_blocks = pb;
     m.num_partitions = static_cast<int>(parts);
     return merge_dispatch(dtype, head_dim, m, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Device memory, or page-locked host memory mapped into the device's address
+// space (what the copy kernel can dereference).
+bool device_accessible(const void* p) {
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();  // the failed query leaves an error behind; clear it
+        return false;
+    }
+    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return true;
+    return attr.type == cudaMemoryTypeHost && attr.devicePointer == p;
+}
+
+pa_status pa_copy_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache, const void* src_v_cache,
+                         const int64_t* block_mapping, int64_t num_pairs, int num_kv_heads, int head_dim,
+                         int block_size, int64_t src_num_blocks, int64_t dst_num_blocks, pa_dtype dtype,
+                         void* stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || src_num_blocks <= 0 ||
+        dst_num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return PA_ERR_UNSUPPORTED;
+    const long long block_bytes =
+        static_cast<long long>(num_kv_heads) * block_size * head_dim * elem_size(dtype);
+    if ((static_cast<long long>(head_dim) * elem_size(dtype)) % 16 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !block_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(dst_k_cache) || !aligned16(dst_v_cache) || !aligned16(src_k_cache) ||
+        !aligned16(src_v_cache) || (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+        return PA_ERR_INVALID_ARG;
+    if (!device_accessible(dst_k_cache) || !device_accessible(dst_v_cache) || !device_accessible(src_k_cache) ||
+        !device_accessible(src_v_cache) || !device_accessible(block_mapping))
+        return PA_ERR_INVALID_ARG;
+    pa::CopyParams p{};
+    p.dst[0] = static_cast<uint4*>(dst_k_cache);
+    p.dst[1] = static_cast<uint4*>(dst_v_cache);
+    p.src[0] = static_cast<const uint4*>(src_k_cache);
+    p.src[1] = static_cast<const uint4*>(src_v_cache);
+    p.mapping = block_mapping;
+    p.num_pairs = num_pairs;
+    p.vecs_per_block = block_bytes / 16;
+    p.src_blocks = src_num_blocks;
+    p.dst_blocks = dst_num_blocks;
+    p.chunks = static_cast<int>((p.vecs_per_block + pa::kChunkVecs - 1) / pa::kChunkVecs);
+    const long long ctas = num_pairs * 2 * p.chunks;
+    if (ctas > INT_MAX) return PA_ERR_UNSUPPORTED;
+    pa::pa_copy_blocks_kernel<<<static_cast<unsigned>(ctas), pa::kCopyThreads, 0,
+                                static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(void* stream, int32_t* code) {

@@ -33,7 +33,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "pa_decode", "pa_decode_append", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
+        "pa_copy_blocks", "pa_decode", "pa_decode_append", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
         "pa_decode_splitk_static", "pa_get_device_error",
         "pa_reshape_and_cache", "pa_status_string"])
 
@@ -101,6 +101,14 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, 16, 3, None, None) == 3     # too few counters
     assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, None, 0, 6, None) == 1      # misaligned seq_order
     assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], 2, None) == 1            # misaligned seq_order
+    cp = [16, 16, 16, 16, 16, 4, 8, 128, 16, 10, 10, 2, None]
+    assert lib.pa_copy_blocks(*cp[:5], 0, *cp[6:]) == 0                             # no pairs: a no-op
+    assert lib.pa_copy_blocks(*cp[:5], -1, *cp[6:]) == 1                            # negative count
+    assert lib.pa_copy_blocks(0, *cp[1:]) == 1                                      # null pool
+    assert lib.pa_copy_blocks(*cp[:4], 12, *cp[5:]) == 1                            # mapping not 8-byte aligned
+    assert lib.pa_copy_blocks(*cp[:2], 24, *cp[3:]) == 1                            # pool not 16-byte aligned
+    assert lib.pa_copy_blocks(*cp[:7], 100, *cp[8:]) == 2                           # 200-byte rows
+    assert lib.pa_copy_blocks(*cp[:9], 0, *cp[10:]) == 1                            # empty source pool
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
