@@ -70,6 +70,19 @@ class Oracle:
         lib.oracle_copy_blocks.argtypes = [
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64,
             c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int64, c.c_int]
+        lib.oracle_reshape_and_cache_e4m3.restype = c.c_int
+        lib.oracle_reshape_and_cache_e4m3.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64,
+            c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int]
+        lib.oracle_decode_e4m3.restype = c.c_int
+        lib.oracle_decode_e4m3.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+            c.c_float, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int, c.c_void_p,
+            c.c_int, c.c_int]
+        lib.oracle_e4m3_value.restype = c.c_double
+        lib.oracle_e4m3_value.argtypes = [c.c_int]
+        lib.oracle_e4m3_encode.restype = c.c_int
+        lib.oracle_e4m3_encode.argtypes = [c.c_float]
         lib.oracle_pool_index.restype = c.c_int64
         lib.oracle_pool_index.argtypes = [c.c_int64, c.c_int, c.c_int, c.c_int, c.c_int,
                                           c.c_int, c.c_int, c.c_int]
@@ -124,6 +137,44 @@ class Oracle:
         self._check(self.lib.oracle_copy_blocks(
             dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(), src_v.data_ptr(), m.data_ptr(),
             m.shape[0], Hkv, D, block_size, src_k.shape[0], dst_k.shape[0], DTYPE_CODE[src_k.dtype]))
+
+    # ---- 8-bit (e4m3) pools: uint8 tensors [N, Hkv, D // 16, B, 16]; fp32 scales [Hkv]
+
+    def reshape_and_cache_e4m3(self, key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, block_size):
+        """In-place quantising write of key/value [T, Hkv, D] into e4m3 pools."""
+        for t in (key, value, k_cache, v_cache, k_scale, v_scale):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        assert k_cache.dtype == torch.uint8 and k_scale.dtype == torch.float32
+        slots = slot_mapping.to(torch.int64).contiguous()
+        T, Hkv, D = key.shape
+        self._check(self.lib.oracle_reshape_and_cache_e4m3(
+            key.data_ptr(), value.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), slots.data_ptr(),
+            k_scale.data_ptr(), v_scale.data_ptr(), T, Hkv, D, block_size, k_cache.shape[0],
+            DTYPE_CODE[key.dtype]))
+
+    def decode_e4m3(self, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, block_size,
+                    num_kv_heads, seqs=None, partition_size=None) -> np.ndarray:
+        """fp64 attention output over e4m3 pools [len(seqs) or S, Hq, D]."""
+        for t in (q, k_cache, v_cache, k_scale, v_scale):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        bt = block_tables.to(torch.int32).contiguous()
+        cl = context_lens.to(torch.int32).contiguous()
+        S, Hq, D = q.shape
+        n = S if seqs is None else len(seqs)
+        out = np.zeros((n, Hq, D), dtype=np.float64)
+        sel = None if seqs is None else np.ascontiguousarray(np.asarray(seqs, dtype=np.int32))
+        self._check(self.lib.oracle_decode_e4m3(
+            out.ctypes.data, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(),
+            v_scale.data_ptr(), bt.data_ptr(), cl.data_ptr(), float(scale), block_size, S, Hq, num_kv_heads, D,
+            bt.shape[1], k_cache.shape[0], DTYPE_CODE[q.dtype], None if sel is None else sel.ctypes.data, n,
+            int(partition_size or 0)))
+        return out
+
+    def e4m3_value(self, bits: int) -> float:
+        return float(self.lib.oracle_e4m3_value(int(bits)))
+
+    def e4m3_encode(self, v: float) -> int:
+        return int(self.lib.oracle_e4m3_encode(float(v)))
 
     def pool_index(self, block, head, token, dim, num_kv_heads, block_size, head_dim, dtype):
         return int(self.lib.oracle_pool_index(block, head, token, dim, num_kv_heads,

@@ -23,6 +23,14 @@
 //        reference count, copy-on-write for isolation.
 //   [P1] §4.2 preemption: a preempted sequence's KV blocks are swapped out to
 //        CPU memory (or dropped and recomputed) and swapped back in later.
+//   [P4] §7 FP8 attention (the rest in FP16) as the next optimisation: here an
+//        8-bit KV pool.  Readings (the pages fix no format): e4m3 codes (OCP
+//        8-bit float, E4M3 "fn": 1 sign, 4 exponent bits with bias 7, 3
+//        mantissa bits, no infinities, S.1111.111 = NaN, largest finite 448);
+//        one fp32 scale per kv head for K and one for V; a stored value x
+//        becomes code = e4m3(x / scale) with the division in fp32 (IEEE,
+//        round to nearest) and the conversion rounding to nearest-even and
+//        saturating to +-448; a code stands for e4m3_value(code) * scale.
 //
 // Readings where the pages are silent (each is listed in the design notes):
 //   * pool layout: an element (block b, kv head h, token t, dim d) lives at
@@ -90,6 +98,45 @@ double from_f16_bits(uint16_t bits) {
     return sign ? -v : v;
 }
 
+// e4m3 bits -> double, field by field (exact).
+double from_e4m3_bits(uint8_t bits) {
+    const int sign = bits >> 7;
+    const int exponent = (bits >> 3) & 0xf;
+    const int mantissa = bits & 0x7;
+    double v;
+    if (exponent == 0xf && mantissa == 0x7) {
+        v = std::numeric_limits<double>::quiet_NaN();
+    } else if (exponent == 0) {
+        v = std::ldexp(static_cast<double>(mantissa), -9);  // subnormal or zero: m * 2^-6 / 8
+    } else {
+        v = std::ldexp(static_cast<double>(mantissa + 8), exponent - 10);  // (1 + m/8) * 2^(e-7)
+    }
+    return sign ? -v : v;
+}
+
+// fp32 -> e4m3 bits: round to nearest, ties to even, at the precision of the
+// binade of |v| (subnormal step 2^-9 below 2^-6), then saturate to 448.
+uint8_t to_e4m3_bits(float v) {
+    const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+    if (std::isnan(v)) return static_cast<uint8_t>(sign | 0x7f);
+    const double a = std::fabs(static_cast<double>(v));
+    if (a == 0.0) return sign;
+    int e2 = 0;
+    std::frexp(a, &e2);                        // a = f * 2^e2, f in [0.5, 1): floor(log2 a) = e2 - 1
+    const int binade = std::max(e2 - 1, -6);   // normal binades start at 2^-6
+    const double quantum = std::ldexp(1.0, binade - 3);
+    double r = std::nearbyint(a / quantum) * quantum;  // default rounding mode: ties to even
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return sign;
+    std::frexp(r, &e2);
+    const int er = e2 - 1;
+    if (er < -6) {
+        return static_cast<uint8_t>(sign | static_cast<int>(std::ldexp(r, 9)));  // m * 2^-9
+    }
+    const int mant = static_cast<int>(std::ldexp(r, -er) * 8.0) - 8;
+    return static_cast<uint8_t>(sign | ((er + 7) << 3) | mant);
+}
+
 // Element `index` of an array of `dtype`, widened to double.
 double element(const void* base, int64_t index, int dtype) {
     if (dtype == kF32) {
@@ -113,7 +160,9 @@ int64_t pool_index(int64_t block, int64_t head, int64_t token, int64_t dim,
 struct Shape {
     int block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks;
     int64_t num_blocks;
-    int dtype;
+    int dtype;                       // queries (and K/V unless e4m3)
+    const float* k_scale = nullptr;  // non-null: the pools hold e4m3 codes, one scale per kv head
+    const float* v_scale = nullptr;
 };
 
 bool shape_ok(const Shape& s) {
@@ -121,7 +170,8 @@ bool shape_ok(const Shape& s) {
     if (s.block_size <= 0 || s.num_seqs < 0 || s.num_q_heads <= 0 || s.num_kv_heads <= 0) return false;
     if (s.head_dim <= 0 || s.max_blocks < 0 || s.num_blocks <= 0) return false;
     if (s.num_q_heads % s.num_kv_heads != 0) return false;
-    const int vec = 16 / elem_size(s.dtype);
+    if ((s.k_scale == nullptr) != (s.v_scale == nullptr)) return false;
+    const int vec = s.k_scale ? 16 : 16 / elem_size(s.dtype);
     return s.head_dim % vec == 0;
 }
 
@@ -130,7 +180,8 @@ bool shape_ok(const Shape& s) {
 int gather_sequence(const void* k_cache, const void* v_cache, const int32_t* table_row,
                     int context_len, int kv_head, const Shape& sh,
                     std::vector<double>& keys, std::vector<double>& values) {
-    const int vec = 16 / elem_size(sh.dtype);
+    const bool e4m3 = sh.k_scale != nullptr;
+    const int vec = e4m3 ? 16 : 16 / elem_size(sh.dtype);
     const int D = sh.head_dim;
     keys.assign(static_cast<size_t>(context_len) * D, 0.0);
     values.assign(static_cast<size_t>(context_len) * D, 0.0);
@@ -142,8 +193,15 @@ int gather_sequence(const void* k_cache, const void* v_cache, const int32_t* tab
         for (int d = 0; d < D; ++d) {
             const int64_t at = pool_index(physical, kv_head, offset, d, sh.num_kv_heads,
                                           sh.block_size, D, vec);
-            keys[static_cast<size_t>(t) * D + d] = element(k_cache, at, sh.dtype);
-            values[static_cast<size_t>(t) * D + d] = element(v_cache, at, sh.dtype);
+            if (e4m3) {  // a code stands for its e4m3 value times its kv head's scale
+                keys[static_cast<size_t>(t) * D + d] =
+                    from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[at]) * static_cast<double>(sh.k_scale[kv_head]);
+                values[static_cast<size_t>(t) * D + d] =
+                    from_e4m3_bits(static_cast<const uint8_t*>(v_cache)[at]) * static_cast<double>(sh.v_scale[kv_head]);
+            } else {
+                keys[static_cast<size_t>(t) * D + d] = element(k_cache, at, sh.dtype);
+                values[static_cast<size_t>(t) * D + d] = element(v_cache, at, sh.dtype);
+            }
         }
     }
     return kOk;
@@ -364,6 +422,58 @@ int oracle_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* 
     }
     return kOk;
 }
+
+// The 8-bit pool's write: key/value rows [T][Hkv][D] (dtype) quantised to
+// e4m3 codes with the kv head's scale and stored through slot_mapping like
+// oracle_reshape_and_cache (pools of 1-byte elements, 16 per vector).
+int oracle_reshape_and_cache_e4m3(const void* key, const void* value, void* k_cache, void* v_cache,
+                                  const int64_t* slot_mapping, const float* k_scale, const float* v_scale,
+                                  int64_t num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                  int64_t num_blocks, int dtype) {
+    if (!key || !value || !k_cache || !v_cache || !k_scale || !v_scale || (!slot_mapping && num_tokens > 0))
+        return kBadArg;
+    if (!dtype_ok(dtype) || num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || head_dim % 16 != 0)
+        return kBadArg;
+    for (int64_t i = 0; i < num_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * block_size) return kBadSlot;
+        const int64_t block = slot / block_size;
+        const int64_t offset = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            for (int d = 0; d < head_dim; ++d) {
+                const int64_t src = (i * num_kv_heads + h) * head_dim + d;
+                const int64_t dst = pool_index(block, h, offset, d, num_kv_heads, block_size, head_dim, 16);
+                const float kx = static_cast<float>(element(key, src, dtype));    // exact
+                const float vx = static_cast<float>(element(value, src, dtype));
+                static_cast<uint8_t*>(k_cache)[dst] = to_e4m3_bits(kx / k_scale[h]);
+                static_cast<uint8_t*>(v_cache)[dst] = to_e4m3_bits(vx / v_scale[h]);
+            }
+        }
+    }
+    return kOk;
+}
+
+// Paged decode over e4m3 pools (queries and output in `dtype`), fp64; with
+// partition > 0 the partitioned form with the log-sum-exp merge.
+int oracle_decode_e4m3(double* out, const void* q, const void* k_cache, const void* v_cache,
+                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                       const int32_t* context_lens, float scale, int block_size, int num_seqs,
+                       int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                       int64_t num_blocks, int dtype, const int32_t* seq_ids, int num_selected,
+                       int partition) {
+    if (!k_scale || !v_scale || partition < 0) return kBadArg;
+    Shape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, num_blocks, dtype};
+    sh.k_scale = k_scale;
+    sh.v_scale = v_scale;
+    return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh, seq_ids,
+                         num_selected, partition);
+}
+
+// The format functions on their own, for the pins.
+double oracle_e4m3_value(int bits) { return from_e4m3_bits(static_cast<uint8_t>(bits)); }
+int oracle_e4m3_encode(float v) { return to_e4m3_bits(v); }
 
 int64_t oracle_pool_index(int64_t block, int head, int token, int dim, int num_kv_heads,
                           int block_size, int head_dim, int dtype) {

@@ -367,6 +367,114 @@ def pin_swap_round_trip(orc):
     np.testing.assert_array_equal(after, before)
 
 
+# ---------------------------------------------------------------------------- 8-bit (e4m3) pools
+
+def pin_e4m3_golden(orc):
+    """Hand-worked e4m3 decodes and encodes (ties to even, saturation)."""
+    g = _golden("e4m3.json")
+    for c in g["decode"]:
+        v = orc.e4m3_value(c["bits"])
+        assert v == c["value"] and math.copysign(1, v) == math.copysign(1, c["value"]), c
+    for c in g["encode"]:
+        assert orc.e4m3_encode(c["value"]) == c["bits"], c
+
+
+def pin_e4m3_against_torch(orc):
+    """Every code's value against torch's float8_e4m3fn conversion; every
+    finite value encodes back to its code; random fp32 values below the
+    saturation threshold (464) encode as torch rounds them."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).tolist()
+    for c in range(256):
+        v = orc.e4m3_value(c)
+        if math.isnan(ref[c]):
+            assert math.isnan(v), c
+            continue
+        assert v == ref[c], c
+        assert orc.e4m3_encode(v) == c, c
+    rng = np.random.default_rng(81)
+    xs = np.concatenate([rng.standard_normal(3000) * s for s in (1e-3, 0.1, 3.0, 100.0)]).astype(np.float32)
+    xs = xs[np.abs(xs) < 464]
+    want = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).tolist()
+    for x, w in zip(xs.tolist(), want):
+        assert orc.e4m3_encode(x) == w, (x, w)
+
+
+def _e4m3_batch(orc, seed, dtype, lens, Hq, Hkv, D, B, extra=6, pow2_scales=False):
+    """A random batch whose every token is written into e4m3 pools by the
+    oracle's quantising write, with per-kv-head scales."""
+    b = workloads.random_small(seed=seed, dtype=dtype, lens=lens, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                               block_size=B, extra_blocks=extra)
+    rng = np.random.default_rng(seed)
+    if pow2_scales:
+        ks = torch.tensor(2.0 ** rng.integers(-6, 2, size=Hkv), dtype=torch.float32)
+        vs = torch.tensor(2.0 ** rng.integers(-6, 2, size=Hkv), dtype=torch.float32)
+    else:
+        ks = torch.tensor(rng.uniform(0.002, 0.05, size=Hkv), dtype=torch.float32)
+        vs = torch.tensor(rng.uniform(0.002, 0.05, size=Hkv), dtype=torch.float32)
+    kc = torch.zeros((b.num_blocks, Hkv, D // 16, B, 16), dtype=torch.uint8)
+    vc = torch.zeros_like(kc)
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        if L == 0:
+            continue
+        per_head = [logical_kv(b, s, h) for h in range(Hkv)]
+        keys = torch.from_numpy(np.stack([k for k, _ in per_head], axis=1)).to(dtype).contiguous()
+        vals = torch.from_numpy(np.stack([v for _, v in per_head], axis=1)).to(dtype).contiguous()
+        slots = torch.tensor([int(b.block_tables[s, t // B]) * B + t % B for t in range(L)], dtype=torch.int64)
+        orc.reshape_and_cache_e4m3(keys, vals, kc, vc, slots, ks, vs, B)
+    return b, kc, vc, ks, vs
+
+
+def pin_e4m3_write_then_single_token(orc):
+    """Quantising write then a one-token context: the output is the stored V
+    row, e4m3(x / scale) * scale, computed here with torch's e4m3 conversion
+    (values below the saturation threshold)."""
+    for dt in (torch.bfloat16, torch.float16, torch.float32):
+        Hkv, D, B = 2, 32, 8
+        x = torch.randn((1, Hkv, D), generator=torch.Generator().manual_seed(82), dtype=torch.float32).to(dt)
+        ks = torch.tensor([0.02, 0.5], dtype=torch.float32)
+        vs = torch.tensor([0.01, 0.25], dtype=torch.float32)
+        kc = torch.zeros((3, Hkv, D // 16, B, 16), dtype=torch.uint8)
+        vc = torch.zeros_like(kc)
+        orc.reshape_and_cache_e4m3(x, x, kc, vc, torch.tensor([2 * B]), ks, vs, B)
+        q = torch.randn((1, 2 * Hkv, D), generator=torch.Generator().manual_seed(83)).to(dt)
+        out = orc.decode_e4m3(q, kc, vc, ks, vs, torch.tensor([[2]], dtype=torch.int32),
+                              torch.tensor([1], dtype=torch.int32), 0.5, B, Hkv)
+        xf = x.to(torch.float32)[0]
+        for h in range(Hkv):
+            stored = ((xf[h] / vs[h]).to(torch.float8_e4m3fn).to(torch.float64) * float(vs[h])).numpy()
+            np.testing.assert_array_equal(out[0, 2 * h], stored)
+            np.testing.assert_array_equal(out[0, 2 * h + 1], stored)
+            kstored = (xf[h] / ks[h]).to(torch.float8_e4m3fn).view(torch.uint8)
+            assert torch.equal(kc[2, h, :, 0, :].reshape(D), kstored)
+
+
+def pin_e4m3_decode_is_dense_decode_of_dequantised_pool(orc):
+    """With power-of-two scales every code * scale is exact in fp32, so e4m3
+    decode must equal (bit for bit in fp64) the plain decode over fp32 pools
+    holding those products; the partitioned form equals it to 1e-13."""
+    for dt, B, D, Hq, Hkv, lens in ((torch.bfloat16, 16, 32, 4, 2, (40, 3, 17)),
+                                    (torch.float16, 8, 16, 2, 1, (9, 30))):
+        b, kc, vc, ks, vs = _e4m3_batch(orc, 83, dt, lens, Hq, Hkv, D, B, pow2_scales=True)
+        codes_k = kc.view(torch.float8_e4m3fn).to(torch.float32)
+        codes_v = vc.view(torch.float8_e4m3fn).to(torch.float32)
+        x = workloads.vec_elems(torch.float32)
+        # dequantise, then relayout [N, Hkv, D/16, B, 16] -> [N, Hkv, D/4, B, 4]
+        dk = (codes_k * ks.view(1, Hkv, 1, 1, 1)).permute(0, 1, 3, 2, 4).reshape(b.num_blocks, Hkv, B, D)
+        dv = (codes_v * vs.view(1, Hkv, 1, 1, 1)).permute(0, 1, 3, 2, 4).reshape(b.num_blocks, Hkv, B, D)
+        fk = dk.reshape(b.num_blocks, Hkv, B, D // x, x).permute(0, 1, 3, 2, 4).contiguous()
+        fv = dv.reshape(b.num_blocks, Hkv, B, D // x, x).permute(0, 1, 3, 2, 4).contiguous()
+        q32 = b.q.to(torch.float32).contiguous()
+        plain = orc.decode(q32, fk, fv, b.block_tables, b.context_lens, b.scale, B, Hkv)
+        got = orc.decode_e4m3(b.q.to(torch.float32).contiguous(), kc, vc, ks, vs, b.block_tables,
+                              b.context_lens, b.scale, B, Hkv)
+        np.testing.assert_array_equal(got, plain)
+        part = orc.decode_e4m3(b.q.to(torch.float32).contiguous(), kc, vc, ks, vs, b.block_tables,
+                               b.context_lens, b.scale, B, Hkv, partition_size=16)
+        assert rel_err(part, plain) <= 1e-13
+
+
 def pin_errors(orc):
     from oracle import OracleError
     b = workloads.random_small(seed=61, dtype=torch.float16, lens=(9, 3), num_q_heads=2,
@@ -430,4 +538,6 @@ def pin_number_formats(orc):
 PINS = [pin_layout_golden, pin_slot_golden, pin_brute_force, pin_dense_equality,
         pin_permutation_invariance, pin_block_size_invariance, pin_shared_vs_copied,
         pin_closed_forms, pin_needle, pin_partitioned, pin_reshape_scatter, pin_errors,
-        pin_number_formats, pin_copy_blocks_rows, pin_copy_on_write_keeps_attention, pin_swap_round_trip]
+        pin_number_formats, pin_copy_blocks_rows, pin_copy_on_write_keeps_attention, pin_swap_round_trip,
+        pin_e4m3_golden, pin_e4m3_against_torch, pin_e4m3_write_then_single_token,
+        pin_e4m3_decode_is_dense_decode_of_dequantised_pool]

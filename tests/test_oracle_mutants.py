@@ -47,6 +47,16 @@ MUTANTS = {
                                 "const int64_t dst = block_mapping[2 * i];\n        const int64_t src = block_mapping[2 * i + 1];"),
     "copy_head_dropped": ("for (int h = 0; h < num_kv_heads; ++h) {\n            for (int t = 0; t < block_size; ++t) {",
                           "for (int h = 1; h < num_kv_heads; ++h) {\n            for (int t = 0; t < block_size; ++t) {"),
+    "e4m3_exponent_bias": ("v = std::ldexp(static_cast<double>(mantissa + 8), exponent - 10);",
+                           "v = std::ldexp(static_cast<double>(mantissa + 8), exponent - 9);"),
+    "e4m3_subnormal_step": ("v = std::ldexp(static_cast<double>(mantissa), -9);",
+                            "v = std::ldexp(static_cast<double>(mantissa), -8);"),
+    "e4m3_ties_away": ("double r = std::nearbyint(a / quantum) * quantum;",
+                       "double r = std::round(a / quantum) * quantum;"),
+    "e4m3_no_saturation": ("if (r > 448.0) r = 448.0;", "if (r > 480.0) r = 448.0;"),
+    "e4m3_scale_multiplied": ("to_e4m3_bits(kx / k_scale[h]);", "to_e4m3_bits(kx * k_scale[h]);"),
+    "e4m3_v_scale_for_keys": ("from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[at]) * static_cast<double>(sh.k_scale[kv_head]);",
+                              "from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[at]) * static_cast<double>(sh.v_scale[kv_head]);"),
     "q_from_wrong_head": ("(static_cast<int64_t>(s) * sh.num_q_heads + h) * D + d",
                           "(static_cast<int64_t>(s) * sh.num_q_heads + kvh) * D + d"),
 }
