@@ -30,11 +30,12 @@ MUTANTS = {
                              "const double w = 1.0 / denom;"),
     "partition_end_short": ("const int t1 = std::min(context_len, t0 + part);",
                             "const int t1 = std::min(context_len, t0 + part - 1);"),
-    "reshape_block_shift": ("const int64_t block = slot / block_size;",
-                            "const int64_t block = (slot + 1) / block_size;"),
+    "reshape_block_shift": ("const int64_t dst = pool_index(block, h, offset, d, num_kv_heads, block_size, head_dim, vec);",
+                            "const int64_t dst = pool_index((slot + 1) / block_size, h, offset, d, num_kv_heads, block_size, head_dim, vec);"),
     "reshape_kv_swapped": ("static_cast<const uint8_t*>(value) + src * es, es);",
                            "static_cast<const uint8_t*>(key) + src * es, es);"),
-    "reshape_skips_slot_zero": ("if (slot < 0) continue;", "if (slot <= 0) continue;"),
+    "reshape_skips_slot_zero": ("if (head_dim % vec != 0) return kBadArg;\n    for (int64_t i = 0; i < num_tokens; ++i) {\n        const int64_t slot = slot_mapping[i];\n        if (slot < 0) continue;",
+                                "if (head_dim % vec != 0) return kBadArg;\n    for (int64_t i = 0; i < num_tokens; ++i) {\n        const int64_t slot = slot_mapping[i];\n        if (slot <= 0) continue;"),
     "f16_exponent_bias": ("exponent - 25);", "exponent - 24);"),
     "bf16_wrong_half": ("static_cast<uint32_t>(bits) << 16);", "static_cast<uint32_t>(bits) << 15);"),
     "context_len_short": ("attend_plain(qrow.data(), keys, values, len, D, scale_d, dst);",
