@@ -67,6 +67,9 @@ def parse_args(argv=None):
                          "pa_reshape_and_cache then pa_decode (single) or pa_decode_splitk with fused (splitk) or "
                          "kernel (splitk2) merge")
     ap.add_argument("--partition-size", type=int, default=1024)
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="KV pool format: the workload's 16-bit/32-bit elements, or 8-bit e4m3 codes with per-kv-head "
+                         "scales (pa_reshape_and_cache_fp8 + pa_decode_fp8 / pa_decode_splitk_fp8)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--l2", choices=["rotate", "flush"], default="rotate",
                     help="rotate: inputs larger than L2, rotated over independent copies, K steps timed as one "
@@ -120,13 +123,15 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def step_bytes(batch):
+def step_bytes(batch, fp8=None):
     """Algorithmic bytes of one step: the decode's (K/V + Q + out + block-table
-    entries + context_lens) and the reshape's (new K/V read + written, slots)."""
-    decode = batch.algorithmic_bytes()
+    entries + context_lens) and the reshape's (new K/V read + written, slots);
+    with 8-bit pools the K/V codes are one byte each (plus the scales)."""
     T = int(batch.slot_mapping.numel())
-    reshape = 2 * 2 * T * batch.num_kv_heads * batch.head_dim * batch.elem_bytes + 8 * T
-    return decode, reshape
+    row = T * batch.num_kv_heads * batch.head_dim
+    if fp8 is not None:
+        return fp8.algorithmic_bytes(batch), 2 * row * (batch.elem_bytes + 1) + 8 * T + 2 * batch.num_kv_heads * 4
+    return batch.algorithmic_bytes(), 2 * 2 * row * batch.elem_bytes + 8 * T
 
 
 class ClockSampler:
@@ -230,20 +235,25 @@ def barrier(world):
 class Step:
     """One hot-path step through the C ABI on device-resident inputs."""
 
-    def __init__(self, batch, mode, partition_size, independent=True):
+    def __init__(self, batch, mode, partition_size, independent=True, fp8=None):
         import paged_kv_cache_449_b200 as pa
         self.pa = pa
         self.b = batch
         self.mode = mode
         self.part = partition_size
+        self.fp8 = fp8 is not None
         dev = "cuda"
 
         def own(t):  # independent: a device copy with its own memory, never an alias of the batch's
             t = t.to(dev).contiguous()
             return t.clone() if independent else t
 
-        self.k = own(batch.k_cache)
-        self.v = own(batch.v_cache)
+        if self.fp8:   # 8-bit pools (e4m3 codes) with per-kv-head scales
+            self.k, self.v = own(fp8.k_cache), own(fp8.v_cache)
+            self.ks, self.vs = own(fp8.k_scale), own(fp8.v_scale)
+        else:
+            self.k = own(batch.k_cache)
+            self.v = own(batch.v_cache)
         # The per-step inputs live in one device buffer (256-byte aligned
         # views), so a step's upload from the host is a single copy.
         specs = [("q", batch.q), ("nk", batch.new_key), ("nv", batch.new_value), ("slots", batch.slot_mapping),
@@ -268,9 +278,22 @@ class Step:
     def reshape(self, stream):
         if self.mode == "append":
             return  # the newest token is written by the decode launch itself
+        if self.fp8:
+            self.pa.pa_reshape_and_cache_fp8(self.nk, self.nv, self.k, self.v, self.slots, self.ks, self.vs,
+                                             stream=stream)
+            return
         self.pa.pa_reshape_and_cache(self.nk, self.nv, self.k, self.v, self.slots, stream=stream)
 
     def decode(self, stream):
+        if self.fp8:
+            if self.mode in ("splitk", "splitk2"):
+                self.pa.pa_decode_splitk_fp8(self.out, self.q, self.k, self.v, self.ks, self.vs, self.bt, self.cl,
+                                             self.b.scale, self.mcl, partition_size=self.part, workspace=self.ws,
+                                             fused=(self.mode == "splitk"), counters=self.counters, stream=stream)
+            else:
+                self.pa.pa_decode_fp8(self.out, self.q, self.k, self.v, self.ks, self.vs, self.bt, self.cl,
+                                      self.b.scale, max_context_len=self.mcl, stream=stream)
+            return
         if self.mode == "append":
             self.pa.pa_decode_append(self.out, self.q, self.nk, self.nv, self.k, self.v, self.bt, self.cl, self.b.scale,
                                      max_context_len=self.mcl, stream=stream)
@@ -307,14 +330,21 @@ def run_gpu(args, world, rank, local):
     pa.load()
     batch = make_workload(args.workload, args.seed + rank, "cuda", args.block_size)
     mode = args.mode
+    fp8 = None
+    if args.kv == "fp8":
+        import workloads
+        if mode == "append":
+            mode = "single"   # the 8-bit pools' write is its own launch
+        fp8 = workloads.random_fp8_pools(batch, seed=args.seed + rank, device="cuda")
     stream = torch.cuda.current_stream()
     l2 = l2_bytes()
-    copies = rotation_copies(batch.unique_kv_bytes(), l2) if args.l2 == "rotate" else 0
+    unique = batch.unique_kv_bytes() // (2 if fp8 is not None else 1)
+    copies = rotation_copies(unique, l2) if args.l2 == "rotate" else 0
     # the first copy may use the batch's own device tensors; the others are clones
-    steps = [Step(batch, mode, args.partition_size, independent=i > 0) for i in range(max(1, copies))]
+    steps = [Step(batch, mode, args.partition_size, independent=i > 0, fp8=fp8) for i in range(max(1, copies))]
     step = steps[0]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if copies == 0 else None
-    decode_bytes, reshape_bytes = step_bytes(batch)
+    decode_bytes, reshape_bytes = step_bytes(batch, fp8)
 
     def one(i, ev=None):
         st = steps[i % len(steps)]
@@ -507,7 +537,8 @@ def run_gpu(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[batch.dtype],
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[batch.dtype]
+        + ("+e4m3 KV (f16 MMA on widened codes)" if fp8 is not None else ""),
         "data": "synthetic (seeded N(0,1) K/V/Q, seeded lengths and shuffled block ids)",
         "config": {
             "workload": batch.name,
@@ -516,15 +547,22 @@ def run_gpu(args, world, rank, local):
             "head_dim": batch.head_dim, "block_size": batch.block_size, "num_blocks": batch.num_blocks,
             "context_len_mean": float(batch.context_lens.float().mean()),
             "context_len_max": batch.max_context_len,
-            "decode_entry": {"splitk": "pa_decode_splitk (fused merge)", "splitk2": "pa_decode_splitk (merge kernel)",
-                             "append": "pa_decode_append"}.get(mode, "pa_decode"),
+            "decode_entry": ({"splitk": "pa_decode_splitk (fused merge)", "splitk2": "pa_decode_splitk (merge kernel)",
+                              "append": "pa_decode_append"}.get(mode, "pa_decode")
+                             if fp8 is None else
+                             {"splitk": "pa_decode_splitk_fp8 (fused merge)",
+                              "splitk2": "pa_decode_splitk_fp8 (merge kernel)"}.get(mode, "pa_decode_fp8")),
+            "kv_pool": ("e4m3 codes, one fp32 scale per kv head for K and for V (random codes)" if fp8 is not None
+                        else "same type as the queries"),
             "partition_size": args.partition_size if mode.startswith("splitk") else None,
             "parallelism": f"replicas x{world} (sequence batches, no collective)",
-            "l2": (f"inputs larger than L2 ({batch.unique_kv_bytes() / 1e6:.0f} MB of distinct KV per step vs "
+            "l2": (f"inputs larger than L2 ({unique / 1e6:.0f} MB of distinct KV per step vs "
                    f"{l2 / 1e6:.0f} MB L2), rotated over {len(steps)} independent copies; K steps in one "
                    f"CUDA-event region") if flush is None
             else "flushed between steps (256 MiB write), per-step CUDA events",
             "step": ("pa_decode_append: newest token of every sequence written + decode, one launch" if mode == "append"
+                     else "pa_reshape_and_cache_fp8 (newest token of every sequence, quantised) + decode"
+                     if fp8 is not None
                      else "pa_reshape_and_cache (newest token of every sequence) + decode"),
         },
         "tokens_per_s": round(total_seqs / (step_ms_max * 1e-3), 1),
@@ -545,7 +583,8 @@ def run_gpu(args, world, rank, local):
             "frac": round(achieved / peak, 4),
             "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
             "algorithmic_bytes_per_launch": int(decode_bytes),
-            "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get((batch.name, mode)),
+            "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get(
+                (batch.name + ("+e4m3" if fp8 is not None else ""), mode)),
         },
         "gpu_launches": int(step.kernels_per_step * args.steps),
         "clocks": clk,
@@ -728,7 +767,7 @@ def main(argv=None):
             return
         res, batch = run_gpu(args, world, rank, local)
         if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not args.no_cpu_baseline and args.kv == "bf16":
                 gbs, desc, spent, n = oracle_sample(batch, args.cpu_sample_seconds)
                 res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                                        "sample": desc}

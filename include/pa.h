@@ -246,6 +246,51 @@ pa_status pa_decode_splitk_static(void* out, const void* q, const void* k_cache,
                                   int64_t num_blocks, pa_dtype dtype, int partition_size, void* stream);
 
 /*
+ * 8-bit KV pools ([P4] §7 names FP8 attention as the next optimisation).  The
+ * pages fix no format; read as e4m3 codes (1 sign, 4 exponent bits with bias
+ * 7, 3 mantissa bits, no infinities, S.1111.111 = NaN, largest finite 448),
+ * one fp32 scale per kv head for K and one for V:
+ *   code = e4m3(x / scale)   (fp32 IEEE division; round to nearest-even;
+ *                             saturate to +-448; finite x)
+ *   value(code) = e4m3_value(code) * scale.
+ * Pools are byte arrays [num_blocks][Hkv][D/16][B][16] (16 codes per 16-byte
+ * vector, vector index outer, token inner).  k_scale and v_scale are device
+ * float arrays [Hkv], 4-byte aligned.  Queries and outputs are fp16 or bf16
+ * (PA_ERR_UNSUPPORTED for fp32).  The decode widens each staged tile exactly
+ * to fp16 and runs the fp16 tensor-core path, so for bf16 queries the query
+ * group is scaled by a power of two into fp16 range first (exact except for
+ * elements below 2^-24 of the group's largest).  NaN codes in a pool give an
+ * unspecified result.
+ */
+
+/* pa_reshape_and_cache_fp8 — pa_reshape_and_cache into 8-bit pools: each
+ * element of key/value [T][Hkv][D] (dtype: fp32, fp16 or bf16) is quantised
+ * with its kv head's scale.  Bit-exact against the definition above. */
+pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache, void* v_cache,
+                                   const int64_t* slot_mapping, const float* k_scale, const float* v_scale,
+                                   int64_t num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                   int64_t num_blocks, pa_dtype dtype, void* stream);
+
+/* pa_decode_fp8 — pa_decode over 8-bit pools; dtype is the query/output type. */
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                        const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                        const int32_t* context_lens, float scale, int block_size, int num_seqs,
+                        int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                        int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                        const int32_t* seq_order, void* stream);
+
+/* pa_decode_splitk_fp8 — pa_decode_splitk over 8-bit pools (same workspace
+ * size, counters and merge forms). */
+pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               const int32_t* context_lens, float scale, int block_size, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                               int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                               int partition_size, void* workspace, size_t workspace_bytes,
+                               int32_t* counters, int64_t num_counters, const int32_t* seq_order,
+                               void* stream);
+
+/*
  * pa_copy_blocks — copy whole physical blocks (every kv head, token and
  * dimension, K pool and V pool) from a source pool pair to a destination pool
  * pair.  The same pools on both sides duplicate a shared block before a

@@ -22,7 +22,8 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "pa_decode_splitk_static", "SPLITK_STATIC_SCRATCH_BYTES",
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT",
-           "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks"]
+           "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
+           "pa_decode_splitk_fp8", "fp8_pool_shape"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -69,6 +70,13 @@ def load() -> ctypes.CDLL:
     lib.pa_decode_splitk.argtypes = decode_args + [I, P, SZ, P, I64, P, P]
     lib.pa_decode_splitk_static.restype = I
     lib.pa_decode_splitk_static.argtypes = decode_args + [I, P]
+    lib.pa_reshape_and_cache_fp8.restype = I
+    lib.pa_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, P, P, I64, I, I, I, I64, I, P]
+    fp8_args = [P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I64, I]
+    lib.pa_decode_fp8.restype = I
+    lib.pa_decode_fp8.argtypes = fp8_args + [P, P]
+    lib.pa_decode_splitk_fp8.restype = I
+    lib.pa_decode_splitk_fp8.argtypes = fp8_args + [I, P, SZ, P, I64, P, P]
     lib.pa_copy_blocks.restype = I
     lib.pa_copy_blocks.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I64, I, P]
     lib.pa_get_device_error.restype = I
@@ -280,6 +288,68 @@ def pa_copy_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_map
         _accessible_ptr(src_k_cache, "src_k_cache"), _accessible_ptr(src_v_cache, "src_v_cache"),
         _accessible_ptr(block_mapping, "block_mapping"), int(block_mapping.shape[0]), hkv, d, b, n_src, n_dst,
         _DTYPE[src_k_cache.dtype], _stream(stream)), "pa_copy_blocks")
+
+
+# ---- 8-bit (e4m3) pools: uint8 tensors [num_blocks, Hkv, D // 16, B, 16], fp32 scales [Hkv] per pool
+
+def fp8_pool_shape(num_blocks, num_kv_heads, head_dim, block_size):
+    return (num_blocks, num_kv_heads, head_dim // 16, block_size, 16)
+
+
+def _scale_ptr(t, name):
+    if t.dtype != torch.float32:
+        raise ValueError(f"{name} must be float32 [num_kv_heads]")
+    return _dev_ptr(t, name)
+
+
+def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, stream=None):
+    """Quantise key/value [T, Hkv, D] to e4m3 codes (x / scale of the kv head)
+    and write them into the 8-bit pools at slot_mapping (int64 [T])."""
+    lib = load()
+    if k_cache.dtype != torch.uint8:
+        raise ValueError("8-bit pools are uint8 tensors")
+    n, hkv, d, b = _pool_dims(k_cache)
+    _check(lib.pa_reshape_and_cache_fp8(
+        _dev_ptr(key, "key"), _dev_ptr(value, "value"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(slot_mapping, "slot_mapping"), _scale_ptr(k_scale, "k_scale"), _scale_ptr(v_scale, "v_scale"),
+        key.shape[0], hkv, d, b, n, _DTYPE[key.dtype], _stream(stream)), "pa_reshape_and_cache_fp8")
+
+
+def _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len):
+    if k_cache.dtype != torch.uint8:
+        raise ValueError("8-bit pools are uint8 tensors")
+    a = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    return a[:4] + [_scale_ptr(k_scale, "k_scale"), _scale_ptr(v_scale, "v_scale")] + a[4:]
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                  max_context_len=None, stream=None, seq_order=None):
+    """pa_decode over 8-bit pools; q/out fp16 or bf16."""
+    lib = load()
+    args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_fp8(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_fp8")
+
+
+def pa_decode_splitk_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                         max_context_len, partition_size=512, workspace=None, fused=True, counters=None,
+                         stream=None, seq_order=None):
+    """pa_decode_splitk over 8-bit pools (workspace and counters as there)."""
+    lib = load()
+    S, Hq, D = q.shape
+    hkv = k_cache.shape[1]
+    need = pa_decode_splitk_workspace_size(S, Hq, D, int(max_context_len), partition_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    cptr, ncount = None, 0
+    if fused:
+        if counters is None:
+            counters = _default_counters.setdefault(q.device.index, Counters())
+        buf = counters.get(S * hkv, q.device) if isinstance(counters, Counters) else counters
+        cptr, ncount = _dev_ptr(buf, "counters"), buf.numel()
+    args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_splitk_fp8(*args, int(partition_size), _dev_ptr(workspace, "workspace"),
+                                    workspace.numel() * workspace.element_size(), cptr, ncount,
+                                    _order_ptr(seq_order, S), _stream(stream)), "pa_decode_splitk_fp8")
 
 
 def pa_get_device_error(stream=None) -> int:

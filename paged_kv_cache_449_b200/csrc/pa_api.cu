@@ -61,17 +61,22 @@ struct KindTuning<Kind::kWide> {
 };
 
 
-template <typename T, int D, int B, Kind K>
+// FP8: the pools hold 1-byte e4m3 codes (stages are half the size of the
+// 16-bit ones) and every warp also keeps fp16 K and V tiles it widens into.
+template <typename T, int D, int B, Kind K, bool FP8 = false>
 struct DecodeConfig {
-    static constexpr int kStageBytes = 2 * B * D * static_cast<int>(sizeof(T));  // K + V tile
-    static constexpr int kRingCap = KindTuning<K>::kRingCap;                      // ring bytes per CTA at most
-    static constexpr int kMaxWarps = kRingCap / kStageBytes;
+    static constexpr int kElem = FP8 ? 1 : static_cast<int>(sizeof(T));
+    static constexpr int kStageBytes = 2 * B * D * kElem;                       // K + V tile
+    static constexpr int kScratch = FP8 ? 2 * B * D * 2 : 0;                    // per warp
+    static constexpr int kRingCap = KindTuning<K>::kRingCap;                    // ring bytes per CTA at most
+    static constexpr int kMaxWarps = kRingCap / (kStageBytes + kScratch);
     static constexpr int kWarps = KindTuning<K>::kWarps < kMaxWarps ? KindTuning<K>::kWarps : kMaxWarps;
     static constexpr int kRaw = KindTuning<K>::kRing / kStageBytes;
-    static constexpr int kFit = kRingCap / (kWarps * kStageBytes);
+    static constexpr int kFit = (kRingCap - kWarps * kScratch) / (kWarps * kStageBytes);
     static constexpr int kStages0 = kRaw < 1 ? 1 : (kRaw > 16 ? 16 : kRaw);
     static constexpr int kStages = kStages0 < kFit ? kStages0 : kFit;
-    using Smem = pa::DecodeSmem<T, D, B, kWarps, kStages>;
+    using Smem = pa::DecodeSmem<T, D, B, kWarps, kStages, FP8>;
+    static_assert(kStages >= 1, "one stage per warp at least");
     static_assert(Smem::kTotal <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -142,10 +147,10 @@ cudaError_t with_variant(pa_dtype dt, int D, int B, F&& f) {
     }
 }
 
-template <typename T, int D, int B, bool SPLIT, Kind K>
+template <typename T, int D, int B, bool SPLIT, Kind K, bool FP8 = false>
 cudaError_t launch_decode(const pa::DecodeParams& p, dim3 grid, cudaStream_t stream) {
-    using C = DecodeConfig<T, D, B, K>;
-    auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT>;
+    using C = DecodeConfig<T, D, B, K, FP8>;
+    auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT, FP8>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
     kernel<<<grid, C::kWarps * 32, C::Smem::kTotal, stream>>>(p);
@@ -168,18 +173,20 @@ int sm_count() {
 
 // The split kernel always runs wide CTAs; the one-pass kernel runs deep CTAs
 // unless its grid holds more than PA_DEEP_MAX_CTAS_PER_SM CTAs per SM.
-template <bool SPLIT>
+template <bool SPLIT, bool FP8 = false>
 cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p, dim3 grid, cudaStream_t st) {
     const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
     const bool deep = !SPLIT && ctas <= static_cast<long long>(PA_DEEP_MAX_CTAS_PER_SM) * sm_count();
-    return with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) {
+    return with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) -> cudaError_t {
         using T = typename decltype(tt)::type;
         constexpr int kD = decltype(dd)::value, kB = decltype(bb)::value;
-        if constexpr (SPLIT) {
-            return launch_decode<T, kD, kB, true, Kind::kWide>(p, grid, st);
+        if constexpr (FP8 && pa::IsF32<T>::value) {
+            return cudaErrorInvalidValue;  // 8-bit pools take 16-bit queries (refused on the host first)
+        } else if constexpr (SPLIT) {
+            return launch_decode<T, kD, kB, true, Kind::kWide, FP8>(p, grid, st);
         } else {
-            return deep ? launch_decode<T, kD, kB, false, Kind::kDeep>(p, grid, st)
-                        : launch_decode<T, kD, kB, false, Kind::kWide>(p, grid, st);
+            return deep ? launch_decode<T, kD, kB, false, Kind::kDeep, FP8>(p, grid, st)
+                        : launch_decode<T, kD, kB, false, Kind::kWide, FP8>(p, grid, st);
         }
     });
 }
@@ -264,6 +271,104 @@ size_t splitk_bytes(long long seqs, long long heads, long long parts, long long 
     return static_cast<size_t>(seqs * heads * parts * (head_dim + 2) * 4);
 }
 
+// Device memory, or page-locked host memory mapped into the device's address
+// space (what the copy kernel can dereference).
+bool device_accessible(const void* p) {
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();  // the failed query leaves an error behind; clear it
+        return false;
+    }
+    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return true;
+    return attr.type == cudaMemoryTypeHost && attr.devicePointer == p;
+}
+
+// The one-pass and split decode bodies, shared by the 16-bit-pool entries
+// (FP8 = false) and the 8-bit-pool entries (FP8 = true, with K/V scales).
+template <bool FP8>
+pa_status check_scales(const DecodeShape& sh, const float* k_scale, const float* v_scale) {
+    if constexpr (FP8) {
+        if (sh.dtype == PA_F32) return PA_ERR_UNSUPPORTED;  // 8-bit pools take 16-bit queries
+        if (sh.num_seqs > 0 && (!k_scale || !v_scale || !aligned4(k_scale) || !aligned4(v_scale)))
+            return PA_ERR_INVALID_ARG;
+    }
+    return PA_OK;
+}
+
+template <bool FP8>
+pa_status decode_one_pass(void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                          const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
+                          float scale, const DecodeShape& sh, const int32_t* seq_order, void* stream) {
+    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (st == PA_OK) st = check_scales<FP8>(sh, k_scale, v_scale);
+    if (st != PA_OK || sh.num_seqs == 0) return st;
+    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
+    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.seq_order = seq_order;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    const dim3 grid(1, sh.num_kv_heads, sh.num_seqs);
+    const cudaError_t e = decode_dispatch<false, FP8>(static_cast<pa_dtype>(sh.dtype), sh.head_dim, sh.block_size,
+                                                      p, grid, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <bool FP8>
+pa_status decode_split(void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                       const float* v_scale, const int32_t* block_tables, const int32_t* context_lens, float scale,
+                       const DecodeShape& sh, int partition_size, void* workspace, size_t workspace_bytes,
+                       int32_t* counters, int64_t num_counters, const int32_t* seq_order, void* stream) {
+    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (st == PA_OK) st = check_scales<FP8>(sh, k_scale, v_scale);
+    if (st != PA_OK) return st;
+    const int block_size = sh.block_size, num_seqs = sh.num_seqs, num_q_heads = sh.num_q_heads;
+    const int num_kv_heads = sh.num_kv_heads, head_dim = sh.head_dim;
+    const pa_dtype dtype = static_cast<pa_dtype>(sh.dtype);
+    if (partition_size <= 0 || partition_size % 16 != 0 || partition_size % block_size != 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
+    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.seq_order = seq_order;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    const int pb = partition_size / block_size;
+    const long long cap_blocks = (static_cast<long long>(p.context_cap) + block_size - 1) / block_size;
+    const long long parts = (cap_blocks + pb - 1) / pb;
+    if (parts > INT_MAX) return PA_ERR_UNSUPPORTED;
+    const size_t need = splitk_bytes(num_seqs, num_q_heads, parts, head_dim);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
+    float* acc = static_cast<float*>(workspace);
+    p.part_acc = acc;
+    p.part_ml = acc + static_cast<size_t>(num_seqs) * num_q_heads * parts * head_dim;
+    p.partition_blocks = pb;
+    p.num_partitions = static_cast<int>(parts);
+    if (counters != nullptr) {
+        if (!aligned4(counters) || num_counters < static_cast<int64_t>(num_seqs) * num_kv_heads)
+            return PA_ERR_WORKSPACE;
+        p.counters = counters;
+    }
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (parts > 0) {
+        const dim3 grid(static_cast<unsigned>(parts), num_kv_heads, num_seqs);
+        const cudaError_t e = decode_dispatch<true, FP8>(dtype, head_dim, block_size, p, grid, s);
+        if (e != cudaSuccess) return PA_ERR_CUDA;
+        if (counters != nullptr) return PA_OK;  // merged inside the partition kernel
+    }
+    pa::MergeParams m{};
+    m.out = out;
+    m.part_acc = p.part_acc;
+    m.part_ml = p.part_ml;
+    m.context_lens = context_lens;
+    m.num_seqs = num_seqs;
+    m.num_q_heads = num_q_heads;
+    m.context_cap = p.context_cap;
+    m.block_size = block_size;
+    m.partition_blocks = pb;
+    m.num_partitions = static_cast<int>(parts);
+    return merge_dispatch(dtype, head_dim, m, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -307,15 +412,8 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
                     void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
-    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
-    if (st != PA_OK || num_seqs == 0) return st;
-    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
-    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
-    p.seq_order = seq_order;
-    const dim3 grid(1, num_kv_heads, num_seqs);
-    const cudaError_t e = decode_dispatch<false>(dtype, head_dim, block_size, p, grid,
-                                                 static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return decode_one_pass<false>(out, q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens, scale, sh,
+                                  seq_order, stream);
 }
 
 pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value, void* k_cache, void* v_cache,
@@ -357,61 +455,72 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
                            int64_t num_counters, const int32_t* seq_order, void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
-    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
-    if (st != PA_OK) return st;
-    if (partition_size <= 0 || partition_size % 16 != 0 || partition_size % block_size != 0)
-        return PA_ERR_INVALID_ARG;
-    if (num_seqs == 0) return PA_OK;
-    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
-    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
-    p.seq_order = seq_order;
-    const int pb = partition_size / block_size;
-    const long long cap_blocks = (static_cast<long long>(p.context_cap) + block_size - 1) / block_size;
-    const long long parts = (cap_blocks + pb - 1) / pb;
-    if (parts > INT_MAX) return PA_ERR_UNSUPPORTED;
-    const size_t need = splitk_bytes(num_seqs, num_q_heads, parts, head_dim);
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_WORKSPACE;
-    float* acc = static_cast<float*>(workspace);
-    p.part_acc = acc;
-    p.part_ml = acc + static_cast<size_t>(num_seqs) * num_q_heads * parts * head_dim;
-    p.partition_blocks = pb;
-    p.num_partitions = static_cast<int>(parts);
-    if (counters != nullptr) {
-        if (!aligned4(counters) || num_counters < static_cast<int64_t>(num_seqs) * num_kv_heads)
-            return PA_ERR_WORKSPACE;
-        p.counters = counters;
-    }
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (parts > 0) {
-        const dim3 grid(static_cast<unsigned>(parts), num_kv_heads, num_seqs);
-        const cudaError_t e = decode_dispatch<true>(dtype, head_dim, block_size, p, grid, s);
-        if (e != cudaSuccess) return PA_ERR_CUDA;
-        if (counters != nullptr) return PA_OK;  // merged inside the partition kernel
-    }
-    pa::MergeParams m{};
-    m.out = out;
-    m.part_acc = p.part_acc;
-    m.part_ml = p.part_ml;
-    m.context_lens = context_lens;
-    m.num_seqs = num_seqs;
-    m.num_q_heads = num_q_heads;
-    m.context_cap = p.context_cap;
-    m.block_size = block_size;
-    m.partition_blocks = pb;
-    m.num_partitions = static_cast<int>(parts);
-    return merge_dispatch(dtype, head_dim, m, s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return decode_split<false>(out, q, k_cache, v_cache, nullptr, nullptr, block_tables, context_lens, scale, sh,
+                               partition_size, workspace, workspace_bytes, counters, num_counters, seq_order,
+                               stream);
 }
 
-// Device memory, or page-locked host memory mapped into the device's address
-// space (what the copy kernel can dereference).
-bool device_accessible(const void* p) {
-    cudaPointerAttributes attr{};
-    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
-        cudaGetLastError();  // the failed query leaves an error behind; clear it
-        return false;
+pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache, void* v_cache,
+                                   const int64_t* slot_mapping, const float* k_scale, const float* v_scale,
+                                   int64_t num_tokens, int num_kv_heads, int head_dim, int block_size,
+                                   int64_t num_blocks, pa_dtype dtype, void* stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return PA_ERR_UNSUPPORTED;
+    if (head_dim % 16 != 0) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping || !k_scale || !v_scale) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) || !aligned4(k_scale) || !aligned4(v_scale))
+        return PA_ERR_INVALID_ARG;
+    pa::ReshapeE4m3Params p{};
+    p.key = key;
+    p.value = value;
+    p.k_cache = static_cast<uint4*>(k_cache);
+    p.v_cache = static_cast<uint4*>(v_cache);
+    p.slot_mapping = slot_mapping;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.num_slots = num_blocks * static_cast<long long>(block_size);
+    const long long threads = num_tokens * num_kv_heads * static_cast<long long>(head_dim / 16);
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > INT_MAX) return PA_ERR_UNSUPPORTED;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned g = static_cast<unsigned>(blocks);
+    switch (dtype) {
+        case PA_F32: pa::pa_reshape_e4m3_kernel<float><<<g, 256, 0, st>>>(p); break;
+        case PA_F16: pa::pa_reshape_e4m3_kernel<__half><<<g, 256, 0, st>>>(p); break;
+        default: pa::pa_reshape_e4m3_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(p); break;
     }
-    if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) return true;
-    return attr.type == cudaMemoryTypeHost && attr.devicePointer == p;
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                        const float* v_scale, const int32_t* block_tables, const int32_t* context_lens, float scale,
+                        int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                        int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                        const int32_t* seq_order, void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    return decode_one_pass<true>(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, sh,
+                                 seq_order, stream);
+}
+
+pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               const int32_t* context_lens, float scale, int block_size, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                               int max_context_len, int64_t num_blocks, pa_dtype dtype, int partition_size,
+                               void* workspace, size_t workspace_bytes, int32_t* counters, int64_t num_counters,
+                               const int32_t* seq_order, void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    return decode_split<true>(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, sh,
+                              partition_size, workspace, workspace_bytes, counters, num_counters, seq_order, stream);
 }
 
 pa_status pa_copy_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k_cache, const void* src_v_cache,

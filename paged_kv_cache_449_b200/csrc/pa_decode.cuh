@@ -31,6 +31,7 @@
 //    (acc, m, l) to the workspace and pa_merge_kernel combines partitions.
 #pragma once
 
+#include "pa_e4m3.cuh"
 #include "pa_warp.cuh"
 
 namespace pa {
@@ -58,6 +59,8 @@ struct DecodeParams {
     const void* new_key;   // append: [S][Hkv][D] K/V of each sequence's newest token (position L-1), or null
     const void* new_value;
     const int32_t* seq_order;  // optional [S] permutation: CTA z works on sequence seq_order[z]; null = z
+    const float* k_scale;      // 8-bit pools: [Hkv] scales of the K and V codes
+    const float* v_scale;
 };
 
 // Append: the newest token of sequence s (logical position L-1) is written
@@ -138,13 +141,14 @@ __device__ __forceinline__ void merge_partitions_cta(const DecodeParams& p, int 
 }
 
 
-template <typename T, int D, int B, int NW, int STAGES>
+template <typename T, int D, int B, int NW, int STAGES, bool FP8 = false>
 struct DecodeSmem {
-    static constexpr int kElem = sizeof(T);
+    static constexpr int kElem = FP8 ? 1 : sizeof(T);
     static constexpr int kTile = B * D * kElem;                 // one (block, head) tile, bytes
     static constexpr int kRing = NW * STAGES * 2 * kTile;       // K and V slots of all warps
+    static constexpr int kScratch = FP8 ? NW * 2 * B * D * 2 : 0;  // 8-bit pools: per-warp fp16 K and V tiles
     static constexpr int kMerge = NW * kMaxGroup * (D + 2) * 4;  // warp states for the CTA merge
-    static constexpr int kArea = kRing > kMerge ? kRing : kMerge;
+    static constexpr int kArea = kRing + kScratch > kMerge ? kRing + kScratch : kMerge;
     static constexpr int kBars = (NW * STAGES * 8 + 15) / 16 * 16;  // keeps what follows 16-byte aligned
     static constexpr int kQ = IsF32<T>::value ? kMaxGroup * D * 4 : 0;
     static constexpr int kTotal = kArea + kBars + kQ;
@@ -154,10 +158,13 @@ struct DecodeSmem {
 // The decode kernel (SPLIT = false: one pass per (seq, kv head); true: one
 // partition of partition_blocks blocks per CTA, partials to the workspace).
 
-template <typename T, int D, int B, int NW, int STAGES, bool SPLIT>
+template <typename T, int D, int B, int NW, int STAGES, bool SPLIT, bool FP8 = false>
 __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constant__ DecodeParams p) {
-    using Smem = DecodeSmem<T, D, B, NW, STAGES>;
+    using Smem = DecodeSmem<T, D, B, NW, STAGES, FP8>;
     constexpr bool kF32 = IsF32<T>::value;
+    static_assert(!(FP8 && kF32), "8-bit pools take 16-bit queries");
+    // 8-bit pools run the fp16 tensor-core path on widened tiles.
+    using TM = typename std::conditional<FP8, __half, T>::type;
     constexpr int kTile = Smem::kTile;
     static_assert(STAGES >= 1 && STAGES <= 32, "ring depth");
     static_assert((kTile % 16) == 0, "bulk copies move multiples of 16 bytes");
@@ -201,9 +208,16 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     if (b0_first + warp + lane * NW < p.max_blocks_per_seq) first_ids = __ldg(bt + lane * NW);
     const T* qrows = reinterpret_cast<const T*>(p.q) +
                      (static_cast<long long>(s) * p.num_q_heads + kvh * group) * D;
-    typename WarpState<T, D, B>::type acc;
+    typename WarpState<TM, D, B>::type acc;
     acc.reset();
-    if constexpr (!kF32) acc.load_q(qrows, group, lane);
+    float score_scale = p.score_scale, out_scale = 1.f;
+    if constexpr (FP8) {
+        const int q_shift = load_q_half<T, D>(acc.qa, qrows, group, lane);
+        score_scale = ldexpf(p.score_scale * __ldg(p.k_scale + kvh), -q_shift);
+        out_scale = __ldg(p.v_scale + kvh);
+    } else if constexpr (!kF32) {
+        acc.load_q(qrows, group, lane);
+    }
 
     int L = p.context_lens[s];
     if (L < 0 || L > p.context_cap) {
@@ -241,10 +255,12 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const int n_w = nb > warp ? (nb - warp + NW - 1) / NW : 0;
     // Append: the warp that will compute the last block loads the new row now.
     const int last_block = nblk - 1;
-    const bool owns_last = p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
+    const bool owns_last = !FP8 && p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
                            (last_block - b0) % NW == warp;
     NewRow<T, D> new_row;
-    if (owns_last) new_row.load_row(p, s, kvh, lane);
+    if constexpr (!FP8) {
+        if (owns_last) new_row.load_row(p, s, kvh, lane);
+    }
 
     auto load_ids = [&](int round) -> int {
         const int i = round * 32 + lane;
@@ -307,13 +323,23 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         const int j = b0 + warp + i * NW;  // logical block index
         const int valid = id < 0 ? 0 : min(B, L - j * B);
         uint8_t* stage = wring + st * 2 * kTile;
-        if (owns_last && j == last_block && id >= 0)
-            append_newest_token<T, D, B>(p, new_row, stage, id, kvh, (L - 1) % B, lane);
-        if constexpr (kF32) {
-            acc.block(reinterpret_cast<const float*>(stage), reinterpret_cast<const float*>(stage + kTile), valid,
-                      group, p.score_scale, lane);
+        if constexpr (FP8) {
+            // widen the staged codes into this warp's fp16 tiles, then the fp16 path
+            uint8_t* wk = smem + Smem::kRing + warp * 2 * B * D * 2;
+            uint8_t* wv = wk + B * D * 2;
+            widen_tile<D, B>(stage, wk, lane);
+            widen_tile<D, B>(stage + kTile, wv, lane);
+            __syncwarp();
+            acc.block(smem_u32(wk), smem_u32(wv), valid, group, score_scale, lane);
         } else {
-            acc.block(smem_u32(stage), smem_u32(stage + kTile), valid, group, p.score_scale, lane);
+            if (owns_last && j == last_block && id >= 0)
+                append_newest_token<T, D, B>(p, new_row, stage, id, kvh, (L - 1) % B, lane);
+            if constexpr (kF32) {
+                acc.block(reinterpret_cast<const float*>(stage), reinterpret_cast<const float*>(stage + kTile),
+                          valid, group, score_scale, lane);
+            } else {
+                acc.block(smem_u32(stage), smem_u32(stage + kTile), valid, group, score_scale, lane);
+            }
         }
         __syncwarp();
         if (i + STAGES < n_w) {
@@ -354,6 +380,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
                 den = fmaf(wt, mml[(w * kMaxGroup + r) * 2 + 1], den);
             }
         }
+        num *= out_scale;  // 8-bit pools: the V scale
         const int h = kvh * group + r;
         if (to_workspace) {
             const long long slot = (static_cast<long long>(s) * p.num_q_heads + h) * p.num_partitions + part;

@@ -9,6 +9,7 @@
 #pragma once
 
 #include "pa_device.cuh"
+#include "pa_e4m3.cuh"
 
 namespace pa {
 
@@ -46,6 +47,48 @@ __global__ void __launch_bounds__(256) pa_reshape_kernel(const __grid_constant__
     const uint4 v = p.value[idx];
     p.k_cache[dst] = k;
     p.v_cache[dst] = v;
+}
+
+// The 8-bit pools' write: one thread quantises sixteen elements of a K row
+// and of the matching V row with its kv head's scales and stores one 16-byte
+// vector of codes into each pool.
+struct ReshapeE4m3Params {
+    const void* key;         // [T][Hkv][D] elements of the input type
+    const void* value;
+    uint4* k_cache;          // [N][Hkv][D/16][B] vectors of 16 codes
+    uint4* v_cache;
+    const int64_t* slot_mapping;
+    const float* k_scale;    // [Hkv]
+    const float* v_scale;
+    long long num_tokens;
+    int num_kv_heads;
+    int head_dim;
+    int block_size;
+    long long num_slots;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) pa_reshape_e4m3_kernel(const __grid_constant__ ReshapeE4m3Params p) {
+    const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int vecs = p.head_dim / 16;
+    const long long per_token = static_cast<long long>(p.num_kv_heads) * vecs;
+    if (idx >= p.num_tokens * per_token) return;
+    const long long i = idx / per_token;
+    const long long slot = p.slot_mapping[i];
+    if (slot < 0) return;  // padding token
+    if (slot >= p.num_slots) {
+        flag_error(4 /* PA_DEVERR_SLOT */);
+        return;
+    }
+    const int rem = static_cast<int>(idx - i * per_token);
+    const int h = rem / vecs;
+    const int j = rem - h * vecs;
+    const long long src = (i * p.num_kv_heads + h) * p.head_dim + j * 16;
+    const long long block = slot / p.block_size;
+    const int offset = static_cast<int>(slot - block * p.block_size);
+    const long long dst = ((block * p.num_kv_heads + h) * vecs + j) * p.block_size + offset;
+    p.k_cache[dst] = quantise16<T>(reinterpret_cast<const T*>(p.key) + src, p.k_scale[h]);
+    p.v_cache[dst] = quantise16<T>(reinterpret_cast<const T*>(p.value) + src, p.v_scale[h]);
 }
 
 }  // namespace pa

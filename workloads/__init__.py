@@ -104,6 +104,42 @@ class Batch:
         return Batch(**moved)
 
 
+@dataclass
+class Fp8Pools:
+    """8-bit KV pools for a batch's block tables: uint8 codes
+    [N, Hkv, D // 16, B, 16] and fp32 scales [Hkv] for K and for V."""
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+
+    def kv_bytes(self, batch: "Batch") -> int:
+        return int(batch.context_lens.to(torch.int64).sum()) * batch.num_kv_heads * batch.head_dim * 2
+
+    def algorithmic_bytes(self, batch: "Batch") -> int:
+        """K/V codes + the kv heads' scales + Q + out + block-table entries + context_lens."""
+        S, Hq, D, e, B = batch.num_seqs, batch.num_q_heads, batch.head_dim, batch.elem_bytes, batch.block_size
+        used_tables = int(((batch.context_lens.to(torch.int64) + B - 1) // B).sum()) * 4
+        return self.kv_bytes(batch) + 2 * batch.num_kv_heads * 4 + 2 * S * Hq * D * e + used_tables + S * 4
+
+
+def random_fp8_pools(batch: "Batch", seed=0, device=None) -> Fp8Pools:
+    """Uniformly random code bytes (the two NaN patterns 0x7f / 0xff replaced
+    by zero) for every block of the pool, and seeded scales in [0.005, 0.05]
+    per kv head.  Stands in for a pool written by the quantising write, for
+    decode measurements and sampled parity."""
+    device = torch.device(device or batch.q.device)
+    g = torch.Generator(device=device).manual_seed(seed)   # drawn where the pool lives
+    shape = (batch.num_blocks, batch.num_kv_heads, batch.head_dim // 16, batch.block_size, 16)
+    pools = []
+    for _ in range(2):
+        codes = torch.randint(0, 256, shape, generator=g, dtype=torch.uint8, device=device)
+        codes[(codes & 0x7f) == 0x7f] = 0
+        pools.append(codes)
+    scales = [torch.empty(batch.num_kv_heads, device=device).uniform_(0.005, 0.05, generator=g) for _ in range(2)]
+    return Fp8Pools(pools[0], pools[1], scales[0], scales[1])
+
+
 # --------------------------------------------------------------------------
 # value generation
 
