@@ -79,6 +79,9 @@ class Oracle:
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
             c.c_float, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int64, c.c_int, c.c_void_p,
             c.c_int, c.c_int]
+        for name in ("oracle_e4m3_k_index", "oracle_e4m3_v_index"):
+            getattr(lib, name).restype = c.c_int64
+            getattr(lib, name).argtypes = [c.c_int64, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int]
         lib.oracle_e4m3_value.restype = c.c_double
         lib.oracle_e4m3_value.argtypes = [c.c_int]
         lib.oracle_e4m3_encode.restype = c.c_int
@@ -138,7 +141,8 @@ class Oracle:
             dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(), src_v.data_ptr(), m.data_ptr(),
             m.shape[0], Hkv, D, block_size, src_k.shape[0], dst_k.shape[0], DTYPE_CODE[src_k.dtype]))
 
-    # ---- 8-bit (e4m3) pools: uint8 tensors [N, Hkv, D // 16, B, 16]; fp32 scales [Hkv]
+    # ---- 8-bit (e4m3) pools: uint8 tensors of B*D bytes per (block, head) tile — K [N, Hkv, D // 16, B, 16],
+    #      V [N, Hkv, D, B] (byte orders in pa_oracle.cpp); fp32 scales [Hkv]
 
     def reshape_and_cache_e4m3(self, key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, block_size):
         """In-place quantising write of key/value [T, Hkv, D] into e4m3 pools."""
@@ -169,6 +173,12 @@ class Oracle:
             bt.shape[1], k_cache.shape[0], DTYPE_CODE[q.dtype], None if sel is None else sel.ctypes.data, n,
             int(partition_size or 0)))
         return out
+
+    def e4m3_k_index(self, block, head, token, dim, num_kv_heads, block_size, head_dim) -> int:
+        return int(self.lib.oracle_e4m3_k_index(block, head, token, dim, num_kv_heads, block_size, head_dim))
+
+    def e4m3_v_index(self, block, head, token, dim, num_kv_heads, block_size, head_dim) -> int:
+        return int(self.lib.oracle_e4m3_v_index(block, head, token, dim, num_kv_heads, block_size, head_dim))
 
     def e4m3_value(self, bits: int) -> float:
         return float(self.lib.oracle_e4m3_value(int(bits)))

@@ -31,6 +31,11 @@
 //        becomes code = e4m3(x / scale) with the division in fp32 (IEEE,
 //        round to nearest) and the conversion rounding to nearest-even and
 //        saturating to +-448; a code stands for e4m3_value(code) * scale.
+//        Layout of the 8-bit pools (a reading as well; one (block, head) tile
+//        of B*D bytes stays contiguous): K as [D/16][B][16] with the 16 dims
+//        j of a vector at byte 4*((j%8)/2) + 2*(j/8) + j%2; V transposed, as
+//        [D][B] with the tokens of each dim row in groups of 16 (8 when B=8)
+//        and token u of a group of 16 at byte 4*((u%8)/2) + 2*(u/8) + u%2.
 //
 // Readings where the pages are silent (each is listed in the design notes):
 //   * pool layout: an element (block b, kv head h, token t, dim d) lives at
@@ -149,6 +154,27 @@ double element(const void* base, int64_t index, int dtype) {
     return dtype == kBF16 ? from_bf16_bits(b) : from_f16_bits(b);
 }
 
+// The byte order inside a 16-element group of the 8-bit pools: element j
+// sits at 4*((j % 8) / 2) + 2*(j / 8) + j % 2.
+int64_t e4m3_slot16(int64_t j) { return 4 * ((j % 8) / 2) + 2 * (j / 8) + j % 2; }
+
+// Position of the code of (block, head, token, dim) in an 8-bit K pool.
+int64_t e4m3_k_index(int64_t block, int64_t head, int64_t token, int64_t dim, int num_kv_heads, int block_size,
+                     int head_dim) {
+    const int64_t tile = block * num_kv_heads + head;
+    const int64_t vector = tile * (head_dim / 16) + dim / 16;
+    return (vector * block_size + token) * 16 + e4m3_slot16(dim % 16);
+}
+
+// Position of the code of (block, head, token, dim) in an 8-bit V pool.
+int64_t e4m3_v_index(int64_t block, int64_t head, int64_t token, int64_t dim, int num_kv_heads, int block_size,
+                     int head_dim) {
+    const int64_t tile = block * num_kv_heads + head;
+    const int64_t row = tile * head_dim + dim;
+    const int64_t in_row = block_size == 8 ? token : 16 * (token / 16) + e4m3_slot16(token % 16);
+    return row * block_size + in_row;
+}
+
 // Position of element (block, head, token, dim) in a pool array (see header).
 int64_t pool_index(int64_t block, int64_t head, int64_t token, int64_t dim,
                    int num_kv_heads, int block_size, int head_dim, int vec) {
@@ -171,6 +197,7 @@ bool shape_ok(const Shape& s) {
     if (s.head_dim <= 0 || s.max_blocks < 0 || s.num_blocks <= 0) return false;
     if (s.num_q_heads % s.num_kv_heads != 0) return false;
     if ((s.k_scale == nullptr) != (s.v_scale == nullptr)) return false;
+    if (s.k_scale && s.block_size != 8 && s.block_size % 16 != 0) return false;
     const int vec = s.k_scale ? 16 : 16 / elem_size(s.dtype);
     return s.head_dim % vec == 0;
 }
@@ -194,10 +221,12 @@ int gather_sequence(const void* k_cache, const void* v_cache, const int32_t* tab
             const int64_t at = pool_index(physical, kv_head, offset, d, sh.num_kv_heads,
                                           sh.block_size, D, vec);
             if (e4m3) {  // a code stands for its e4m3 value times its kv head's scale
+                const int64_t ka = e4m3_k_index(physical, kv_head, offset, d, sh.num_kv_heads, sh.block_size, D);
+                const int64_t va = e4m3_v_index(physical, kv_head, offset, d, sh.num_kv_heads, sh.block_size, D);
                 keys[static_cast<size_t>(t) * D + d] =
-                    from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[at]) * static_cast<double>(sh.k_scale[kv_head]);
+                    from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[ka]) * static_cast<double>(sh.k_scale[kv_head]);
                 values[static_cast<size_t>(t) * D + d] =
-                    from_e4m3_bits(static_cast<const uint8_t*>(v_cache)[at]) * static_cast<double>(sh.v_scale[kv_head]);
+                    from_e4m3_bits(static_cast<const uint8_t*>(v_cache)[va]) * static_cast<double>(sh.v_scale[kv_head]);
             } else {
                 keys[static_cast<size_t>(t) * D + d] = element(k_cache, at, sh.dtype);
                 values[static_cast<size_t>(t) * D + d] = element(v_cache, at, sh.dtype);
@@ -433,7 +462,7 @@ int oracle_reshape_and_cache_e4m3(const void* key, const void* value, void* k_ca
     if (!key || !value || !k_cache || !v_cache || !k_scale || !v_scale || (!slot_mapping && num_tokens > 0))
         return kBadArg;
     if (!dtype_ok(dtype) || num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-        num_blocks <= 0 || head_dim % 16 != 0)
+        num_blocks <= 0 || head_dim % 16 != 0 || (block_size != 8 && block_size % 16 != 0))
         return kBadArg;
     for (int64_t i = 0; i < num_tokens; ++i) {
         const int64_t slot = slot_mapping[i];
@@ -444,11 +473,12 @@ int oracle_reshape_and_cache_e4m3(const void* key, const void* value, void* k_ca
         for (int h = 0; h < num_kv_heads; ++h) {
             for (int d = 0; d < head_dim; ++d) {
                 const int64_t src = (i * num_kv_heads + h) * head_dim + d;
-                const int64_t dst = pool_index(block, h, offset, d, num_kv_heads, block_size, head_dim, 16);
+                const int64_t kdst = e4m3_k_index(block, h, offset, d, num_kv_heads, block_size, head_dim);
+                const int64_t vdst = e4m3_v_index(block, h, offset, d, num_kv_heads, block_size, head_dim);
                 const float kx = static_cast<float>(element(key, src, dtype));    // exact
                 const float vx = static_cast<float>(element(value, src, dtype));
-                static_cast<uint8_t*>(k_cache)[dst] = to_e4m3_bits(kx / k_scale[h]);
-                static_cast<uint8_t*>(v_cache)[dst] = to_e4m3_bits(vx / v_scale[h]);
+                static_cast<uint8_t*>(k_cache)[kdst] = to_e4m3_bits(kx / k_scale[h]);
+                static_cast<uint8_t*>(v_cache)[vdst] = to_e4m3_bits(vx / v_scale[h]);
             }
         }
     }
@@ -469,6 +499,16 @@ int oracle_decode_e4m3(double* out, const void* q, const void* k_cache, const vo
     sh.v_scale = v_scale;
     return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh, seq_ids,
                          num_selected, partition);
+}
+
+// The 8-bit pools' layout functions, for the pins.
+int64_t oracle_e4m3_k_index(int64_t block, int head, int token, int dim, int num_kv_heads, int block_size,
+                            int head_dim) {
+    return e4m3_k_index(block, head, token, dim, num_kv_heads, block_size, head_dim);
+}
+int64_t oracle_e4m3_v_index(int64_t block, int head, int token, int dim, int num_kv_heads, int block_size,
+                            int head_dim) {
+    return e4m3_v_index(block, head, token, dim, num_kv_heads, block_size, head_dim);
 }
 
 // The format functions on their own, for the pins.

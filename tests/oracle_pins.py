@@ -379,6 +379,15 @@ def pin_e4m3_golden(orc):
         assert orc.e4m3_encode(c["value"]) == c["bits"], c
 
 
+def pin_e4m3_layout_golden(orc):
+    """Hand-worked byte offsets of the 8-bit K and V pool layouts."""
+    g = _golden("e4m3_layout.json")
+    for c in g["k"]:
+        assert orc.e4m3_k_index(c["b"], c["h"], c["t"], c["d"], c["Hkv"], c["B"], c["D"]) == c["index"], c
+    for c in g["v"]:
+        assert orc.e4m3_v_index(c["b"], c["h"], c["t"], c["d"], c["Hkv"], c["B"], c["D"]) == c["index"], c
+
+
 def pin_e4m3_against_torch(orc):
     """Every code's value against torch's float8_e4m3fn conversion; every
     finite value encodes back to its code; random fp32 values below the
@@ -447,31 +456,41 @@ def pin_e4m3_write_then_single_token(orc):
             np.testing.assert_array_equal(out[0, 2 * h], stored)
             np.testing.assert_array_equal(out[0, 2 * h + 1], stored)
             kstored = (xf[h] / ks[h]).to(torch.float8_e4m3fn).view(torch.uint8)
-            assert torch.equal(kc[2, h, :, 0, :].reshape(D), kstored)
+            flat = kc.view(-1)
+            for d in range(D):
+                assert int(flat[orc.e4m3_k_index(2, h, 0, d, Hkv, B, D)]) == int(kstored[d]), (h, d)
 
 
 def pin_e4m3_decode_is_dense_decode_of_dequantised_pool(orc):
-    """With power-of-two scales every code * scale is exact in fp32, so e4m3
-    decode must equal (bit for bit in fp64) the plain decode over fp32 pools
-    holding those products; the partitioned form equals it to 1e-13."""
+    """With power-of-two scales every code * scale is exact in fp32.  The same
+    logical rows are written into 8-bit pools (quantising write) and, after
+    quantising and dequantising them with torch's e4m3 conversion, into fp32
+    pools (plain write): e4m3 decode must equal the plain decode bit for bit
+    in fp64, and the partitioned form must equal it to 1e-13."""
     for dt, B, D, Hq, Hkv, lens in ((torch.bfloat16, 16, 32, 4, 2, (40, 3, 17)),
-                                    (torch.float16, 8, 16, 2, 1, (9, 30))):
+                                    (torch.float16, 8, 16, 2, 1, (9, 30)),
+                                    (torch.bfloat16, 32, 16, 2, 2, (70, 33))):
         b, kc, vc, ks, vs = _e4m3_batch(orc, 83, dt, lens, Hq, Hkv, D, B, pow2_scales=True)
-        codes_k = kc.view(torch.float8_e4m3fn).to(torch.float32)
-        codes_v = vc.view(torch.float8_e4m3fn).to(torch.float32)
         x = workloads.vec_elems(torch.float32)
-        # dequantise, then relayout [N, Hkv, D/16, B, 16] -> [N, Hkv, D/4, B, 4]
-        dk = (codes_k * ks.view(1, Hkv, 1, 1, 1)).permute(0, 1, 3, 2, 4).reshape(b.num_blocks, Hkv, B, D)
-        dv = (codes_v * vs.view(1, Hkv, 1, 1, 1)).permute(0, 1, 3, 2, 4).reshape(b.num_blocks, Hkv, B, D)
-        fk = dk.reshape(b.num_blocks, Hkv, B, D // x, x).permute(0, 1, 3, 2, 4).contiguous()
-        fv = dv.reshape(b.num_blocks, Hkv, B, D // x, x).permute(0, 1, 3, 2, 4).contiguous()
+        fk = torch.zeros((b.num_blocks, Hkv, D // x, B, x), dtype=torch.float32)
+        fv = torch.zeros_like(fk)
+        for s in range(b.num_seqs):
+            L = int(b.context_lens[s])
+            if L == 0:
+                continue
+            per_head = [logical_kv(b, s, h) for h in range(Hkv)]
+            keys = torch.from_numpy(np.stack([k for k, _ in per_head], axis=1)).to(dt).to(torch.float32)
+            vals = torch.from_numpy(np.stack([v for _, v in per_head], axis=1)).to(dt).to(torch.float32)
+            dq_k = (keys / ks.view(1, Hkv, 1)).to(torch.float8_e4m3fn).to(torch.float32) * ks.view(1, Hkv, 1)
+            dq_v = (vals / vs.view(1, Hkv, 1)).to(torch.float8_e4m3fn).to(torch.float32) * vs.view(1, Hkv, 1)
+            slots = torch.tensor([int(b.block_tables[s, t // B]) * B + t % B for t in range(L)], dtype=torch.int64)
+            orc.reshape_and_cache(dq_k.contiguous(), dq_v.contiguous(), fk, fv, slots, B)
         q32 = b.q.to(torch.float32).contiguous()
         plain = orc.decode(q32, fk, fv, b.block_tables, b.context_lens, b.scale, B, Hkv)
-        got = orc.decode_e4m3(b.q.to(torch.float32).contiguous(), kc, vc, ks, vs, b.block_tables,
-                              b.context_lens, b.scale, B, Hkv)
+        got = orc.decode_e4m3(q32, kc, vc, ks, vs, b.block_tables, b.context_lens, b.scale, B, Hkv)
         np.testing.assert_array_equal(got, plain)
-        part = orc.decode_e4m3(b.q.to(torch.float32).contiguous(), kc, vc, ks, vs, b.block_tables,
-                               b.context_lens, b.scale, B, Hkv, partition_size=16)
+        part = orc.decode_e4m3(q32, kc, vc, ks, vs, b.block_tables, b.context_lens, b.scale, B, Hkv,
+                               partition_size=16)
         assert rel_err(part, plain) <= 1e-13
 
 
@@ -539,5 +558,5 @@ PINS = [pin_layout_golden, pin_slot_golden, pin_brute_force, pin_dense_equality,
         pin_permutation_invariance, pin_block_size_invariance, pin_shared_vs_copied,
         pin_closed_forms, pin_needle, pin_partitioned, pin_reshape_scatter, pin_errors,
         pin_number_formats, pin_copy_blocks_rows, pin_copy_on_write_keeps_attention, pin_swap_round_trip,
-        pin_e4m3_golden, pin_e4m3_against_torch, pin_e4m3_write_then_single_token,
+        pin_e4m3_golden, pin_e4m3_layout_golden, pin_e4m3_against_torch, pin_e4m3_write_then_single_token,
         pin_e4m3_decode_is_dense_decode_of_dequantised_pool]

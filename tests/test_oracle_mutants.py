@@ -56,8 +56,12 @@ MUTANTS = {
                        "double r = std::round(a / quantum) * quantum;"),
     "e4m3_no_saturation": ("if (r > 448.0) r = 448.0;", "if (r > 480.0) r = 448.0;"),
     "e4m3_scale_multiplied": ("to_e4m3_bits(kx / k_scale[h]);", "to_e4m3_bits(kx * k_scale[h]);"),
-    "e4m3_v_scale_for_keys": ("from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[at]) * static_cast<double>(sh.k_scale[kv_head]);",
-                              "from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[at]) * static_cast<double>(sh.v_scale[kv_head]);"),
+    "e4m3_v_scale_for_keys": ("from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[ka]) * static_cast<double>(sh.k_scale[kv_head]);",
+                              "from_e4m3_bits(static_cast<const uint8_t*>(k_cache)[ka]) * static_cast<double>(sh.v_scale[kv_head]);"),
+    "e4m3_byte_order_natural": ("int64_t e4m3_slot16(int64_t j) { return 4 * ((j % 8) / 2) + 2 * (j / 8) + j % 2; }",
+                                "int64_t e4m3_slot16(int64_t j) { return j; }"),
+    "e4m3_v_not_transposed": ("const int64_t va = e4m3_v_index(physical, kv_head, offset, d, sh.num_kv_heads, sh.block_size, D);",
+                              "const int64_t va = e4m3_k_index(physical, kv_head, offset, d, sh.num_kv_heads, sh.block_size, D);"),
     "q_from_wrong_head": ("(static_cast<int64_t>(s) * sh.num_q_heads + h) * D + d",
                           "(static_cast<int64_t>(s) * sh.num_q_heads + kvh) * D + d"),
 }
