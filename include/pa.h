@@ -253,14 +253,18 @@ pa_status pa_decode_splitk_static(void* out, const void* q, const void* k_cache,
  *   code = e4m3(x / scale)   (fp32 IEEE division; round to nearest-even;
  *                             saturate to +-448; finite x)
  *   value(code) = e4m3_value(code) * scale.
- * Pools are byte arrays [num_blocks][Hkv][D/16][B][16] (16 codes per 16-byte
- * vector, vector index outer, token inner).  k_scale and v_scale are device
+ * Pools are byte arrays of B*D-byte (block, head) tiles.  K tile:
+ * [D/16][B][16], dim j of a 16-dim vector at byte 4*((j%8)/2) + 2*(j/8) + j%2.
+ * V tile, transposed: [D][B], the tokens of each dim row in groups of 16
+ * with token u of a group at the same byte order (B = 8: natural order).
+ * Block sizes 8, 16 and 32.  k_scale and v_scale are device
  * float arrays [Hkv], 4-byte aligned.  Queries and outputs are fp16 or bf16
  * (PA_ERR_UNSUPPORTED for fp32).  The decode widens each staged tile exactly
  * to fp16 and runs the fp16 tensor-core path, so for bf16 queries the query
  * group is scaled by a power of two into fp16 range first (exact except for
  * elements below 2^-24 of the group's largest).  NaN codes in a pool give an
- * unspecified result.
+ * unspecified result.  (The byte orders let one 32-bit shared-memory load
+ * hold the four codes of a thread's MMA fragment.)
  */
 
 /* pa_reshape_and_cache_fp8 — pa_reshape_and_cache into 8-bit pools: each

@@ -290,7 +290,8 @@ def pa_copy_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_map
         _DTYPE[src_k_cache.dtype], _stream(stream)), "pa_copy_blocks")
 
 
-# ---- 8-bit (e4m3) pools: uint8 tensors [num_blocks, Hkv, D // 16, B, 16], fp32 scales [Hkv] per pool
+# ---- 8-bit (e4m3) pools: uint8 tensors shaped [num_blocks, Hkv, D // 16, B, 16] (one B*D-byte tile per
+#      (block, head); inside a tile K and V keep the byte orders of pa.h), fp32 scales [Hkv] per pool
 
 def fp8_pool_shape(num_blocks, num_kv_heads, head_dim, block_size):
     return (num_blocks, num_kv_heads, head_dim // 16, block_size, 16)

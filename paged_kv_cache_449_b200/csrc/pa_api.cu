@@ -40,6 +40,20 @@
 #ifndef PA_WIDE_RING
 #define PA_WIDE_RING 12288
 #endif
+// The same two shapes for 8-bit pools, whose blocks carry half the bytes
+// for the same tensor-core work per block.
+#ifndef PA_FP8_DEEP_WARPS
+#define PA_FP8_DEEP_WARPS 16
+#endif
+#ifndef PA_FP8_DEEP_RING
+#define PA_FP8_DEEP_RING 12288
+#endif
+#ifndef PA_FP8_WIDE_WARPS
+#define PA_FP8_WIDE_WARPS 4
+#endif
+#ifndef PA_FP8_WIDE_RING
+#define PA_FP8_WIDE_RING 8192
+#endif
 #ifndef PA_DEEP_MAX_CTAS_PER_SM
 #define PA_DEEP_MAX_CTAS_PER_SM 4
 #endif
@@ -48,31 +62,38 @@ namespace {
 
 enum class Kind { kDeep, kWide };
 
-template <Kind K>
+template <Kind K, bool FP8>
 struct KindTuning;
 // kRingCap bounds the K/V ring of a CTA.
 template <>
-struct KindTuning<Kind::kDeep> {
+struct KindTuning<Kind::kDeep, false> {
     static constexpr int kWarps = PA_DEEP_WARPS, kRing = PA_DEEP_RING, kRingCap = 200 * 1024;
 };
 template <>
-struct KindTuning<Kind::kWide> {
+struct KindTuning<Kind::kWide, false> {
     static constexpr int kWarps = PA_WIDE_WARPS, kRing = PA_WIDE_RING, kRingCap = 200 * 1024;
+};
+template <>
+struct KindTuning<Kind::kDeep, true> {
+    static constexpr int kWarps = PA_FP8_DEEP_WARPS, kRing = PA_FP8_DEEP_RING, kRingCap = 200 * 1024;
+};
+template <>
+struct KindTuning<Kind::kWide, true> {
+    static constexpr int kWarps = PA_FP8_WIDE_WARPS, kRing = PA_FP8_WIDE_RING, kRingCap = 200 * 1024;
 };
 
 
-// FP8: the pools hold 1-byte e4m3 codes (stages are half the size of the
-// 16-bit ones) and every warp also keeps fp16 K and V tiles it widens into.
+// FP8: the pools hold 1-byte e4m3 codes, so a stage is half the size of a
+// 16-bit one and the same ring bytes hold twice the stages.
 template <typename T, int D, int B, Kind K, bool FP8 = false>
 struct DecodeConfig {
     static constexpr int kElem = FP8 ? 1 : static_cast<int>(sizeof(T));
     static constexpr int kStageBytes = 2 * B * D * kElem;                       // K + V tile
-    static constexpr int kScratch = FP8 ? 2 * B * D * 2 : 0;                    // per warp
-    static constexpr int kRingCap = KindTuning<K>::kRingCap;                    // ring bytes per CTA at most
-    static constexpr int kMaxWarps = kRingCap / (kStageBytes + kScratch);
-    static constexpr int kWarps = KindTuning<K>::kWarps < kMaxWarps ? KindTuning<K>::kWarps : kMaxWarps;
-    static constexpr int kRaw = KindTuning<K>::kRing / kStageBytes;
-    static constexpr int kFit = (kRingCap - kWarps * kScratch) / (kWarps * kStageBytes);
+    static constexpr int kRingCap = KindTuning<K, FP8>::kRingCap;                    // ring bytes per CTA at most
+    static constexpr int kMaxWarps = kRingCap / kStageBytes;
+    static constexpr int kWarps = KindTuning<K, FP8>::kWarps < kMaxWarps ? KindTuning<K, FP8>::kWarps : kMaxWarps;
+    static constexpr int kRaw = KindTuning<K, FP8>::kRing / kStageBytes;
+    static constexpr int kFit = kRingCap / (kWarps * kStageBytes);
     static constexpr int kStages0 = kRaw < 1 ? 1 : (kRaw > 16 ? 16 : kRaw);
     static constexpr int kStages = kStages0 < kFit ? kStages0 : kFit;
     using Smem = pa::DecodeSmem<T, D, B, kWarps, kStages, FP8>;
@@ -473,11 +494,12 @@ pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_c
     if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u) || !aligned4(k_scale) || !aligned4(v_scale))
         return PA_ERR_INVALID_ARG;
+    if (block_size != 8 && block_size % 16 != 0) return PA_ERR_UNSUPPORTED;
     pa::ReshapeE4m3Params p{};
     p.key = key;
     p.value = value;
-    p.k_cache = static_cast<uint4*>(k_cache);
-    p.v_cache = static_cast<uint4*>(v_cache);
+    p.k_cache = static_cast<uint32_t*>(k_cache);
+    p.v_cache = static_cast<uint8_t*>(v_cache);
     p.slot_mapping = slot_mapping;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
@@ -486,7 +508,7 @@ pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_c
     p.head_dim = head_dim;
     p.block_size = block_size;
     p.num_slots = num_blocks * static_cast<long long>(block_size);
-    const long long threads = num_tokens * num_kv_heads * static_cast<long long>(head_dim / 16);
+    const long long threads = num_tokens * num_kv_heads * static_cast<long long>(head_dim / 4);
     const long long blocks = (threads + 255) / 256;
     if (blocks > INT_MAX) return PA_ERR_UNSUPPORTED;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);

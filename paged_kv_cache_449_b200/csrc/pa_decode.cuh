@@ -146,9 +146,8 @@ struct DecodeSmem {
     static constexpr int kElem = FP8 ? 1 : sizeof(T);
     static constexpr int kTile = B * D * kElem;                 // one (block, head) tile, bytes
     static constexpr int kRing = NW * STAGES * 2 * kTile;       // K and V slots of all warps
-    static constexpr int kScratch = FP8 ? NW * 2 * B * D * 2 : 0;  // 8-bit pools: per-warp fp16 K and V tiles
     static constexpr int kMerge = NW * kMaxGroup * (D + 2) * 4;  // warp states for the CTA merge
-    static constexpr int kArea = kRing + kScratch > kMerge ? kRing + kScratch : kMerge;
+    static constexpr int kArea = kRing > kMerge ? kRing : kMerge;
     static constexpr int kBars = (NW * STAGES * 8 + 15) / 16 * 16;  // keeps what follows 16-byte aligned
     static constexpr int kQ = IsF32<T>::value ? kMaxGroup * D * 4 : 0;
     static constexpr int kTotal = kArea + kBars + kQ;
@@ -213,8 +212,8 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     float score_scale = p.score_scale, out_scale = 1.f;
     if constexpr (FP8) {
         const int q_shift = load_q_half<T, D>(acc.qa, qrows, group, lane);
-        score_scale = ldexpf(p.score_scale * __ldg(p.k_scale + kvh), -q_shift);
-        out_scale = __ldg(p.v_scale + kvh);
+        score_scale = ldexpf(p.score_scale * __ldg(p.k_scale + kvh) * kE4m3Unit, -q_shift);
+        out_scale = __ldg(p.v_scale + kvh) * kE4m3Unit;
     } else if constexpr (!kF32) {
         acc.load_q(qrows, group, lane);
     }
@@ -324,13 +323,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         const int valid = id < 0 ? 0 : min(B, L - j * B);
         uint8_t* stage = wring + st * 2 * kTile;
         if constexpr (FP8) {
-            // widen the staged codes into this warp's fp16 tiles, then the fp16 path
-            uint8_t* wk = smem + Smem::kRing + warp * 2 * B * D * 2;
-            uint8_t* wv = wk + B * D * 2;
-            widen_tile<D, B>(stage, wk, lane);
-            widen_tile<D, B>(stage + kTile, wv, lane);
-            __syncwarp();
-            acc.block(smem_u32(wk), smem_u32(wv), valid, group, score_scale, lane);
+            acc.template block<true>(smem_u32(stage), smem_u32(stage + kTile), valid, group, score_scale, lane);
         } else {
             if (owns_last && j == last_block && id >= 0)
                 append_newest_token<T, D, B>(p, new_row, stage, id, kvh, (L - 1) % B, lane);

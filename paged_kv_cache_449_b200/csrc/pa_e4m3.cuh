@@ -7,12 +7,17 @@
 //    +-448 (CUDA's conversion, checked bit for bit against an independent
 //    encoder in the tests);
 //  * read: a code stands for e4m3_value(code) * scale.  Every e4m3 value is
-//    exactly an fp16 value (3 mantissa bits, exponents 2^-9 .. 2^8), so a
-//    staged tile is widened to fp16 without rounding and runs through the
-//    fp16 tensor-core path; the K scale joins the score scale and the V
-//    scale multiplies the finished output.
-//  * pool layout: [num_blocks][Hkv][D/16][B][16] bytes (16 codes per 16-byte
-//    vector), the same vector-outer / token-inner order as the 16-bit pools.
+//    exactly an fp16 value (3 mantissa bits, exponents 2^-9 .. 2^8), so codes
+//    are widened to fp16 without rounding and run through the fp16
+//    tensor-core path; the K scale joins the score scale and the V scale
+//    multiplies the finished output.
+//  * pool layout (one (block, head) tile = B*D contiguous bytes): K as
+//    [D/16][B][16] with dims 2c, 2c+1, 2c+8, 2c+9 of a 16-dim vector at bytes
+//    4c..4c+3; V transposed, [D][B], with tokens 2c, 2c+1, 2c+8, 2c+9 of each
+//    16-token group at bytes 4c..4c+3 (B = 8: natural order).  One 32-bit
+//    shared-memory load then holds exactly the four codes a thread needs for
+//    its part of an MMA A fragment (rows r, cols 2c.., 2c+8..), so staged
+//    tiles feed the tensor cores without ldmatrix or a widened copy.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -39,48 +44,64 @@ __device__ __forceinline__ uint32_t e4m3x2_to_half2(uint32_t two_codes) {
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
-// Sixteen consecutive elements of a row -> sixteen codes (one 16-byte vector).
-template <typename T>
-__device__ __forceinline__ uint4 quantise16(const T* row, float scale) {
-    uint32_t w[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int i = 4 * k + 2 * e;
-            float2 f;
-            f.x = __fdiv_rn(to_float<T>(row[i]), scale);
-            f.y = __fdiv_rn(to_float<T>(row[i + 1]), scale);
-            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
-            word |= static_cast<uint32_t>(c) << (16 * e);
-        }
-        w[k] = word;
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
+__device__ __forceinline__ uint32_t quantise2(float a, float b, float scale) {
+    float2 f;
+    f.x = __fdiv_rn(a, scale);
+    f.y = __fdiv_rn(b, scale);
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3));
 }
 
-// A staged e4m3 (block, head) tile [D/16][B][16] -> an fp16 tile [D/8][B][8]
-// in the warp's scratch area (the layout the fp16 MMA path reads).
-template <int D, int B>
-__device__ __forceinline__ void widen_tile(const uint8_t* src, uint8_t* dst, int lane) {
-    constexpr int kVecs = D / 16 * B;
-#pragma unroll
-    for (int vi = lane; vi < kVecs; vi += 32) {
-        const uint4 c = *reinterpret_cast<const uint4*>(src + vi * 16);
-        const int v = vi / B, t = vi - v * B;
-        uint4 lo, hi;
-        lo.x = e4m3x2_to_half2(c.x);
-        lo.y = e4m3x2_to_half2(c.x >> 16);
-        lo.z = e4m3x2_to_half2(c.y);
-        lo.w = e4m3x2_to_half2(c.y >> 16);
-        hi.x = e4m3x2_to_half2(c.z);
-        hi.y = e4m3x2_to_half2(c.z >> 16);
-        hi.z = e4m3x2_to_half2(c.w);
-        hi.w = e4m3x2_to_half2(c.w >> 16);
-        *reinterpret_cast<uint4*>(dst + ((2 * v) * B + t) * 16) = lo;
-        *reinterpret_cast<uint4*>(dst + ((2 * v + 1) * B + t) * 16) = hi;
-    }
+// Byte of token t inside a V row of B codes.
+__device__ __forceinline__ int v_row_byte(int t, int B) {
+    if (B == 8) return t;
+    const int u = t & 15;
+    return (t & ~15) + 4 * ((u & 7) >> 1) + 2 * (u >> 3) + (u & 1);
+}
+
+// Four codes (one 32-bit shared-memory word) -> the two fp16x2 fragment
+// registers they form: bytes 0-1 and bytes 2-3.
+//   PA_E4M3_CVT 0: CUDA's conversion intrinsic per pair;
+//               1: the hardware conversion (cvt.rn.f16x2.e4m3x2) on the two
+//                  16-bit halves of the word;
+//               2: bit placement: code s.eeee.mmm becomes the fp16 pattern
+//                  s.0eeee.mmm0000000, which is the code's value times 2^-8
+//                  exactly (normal and subnormal codes alike; the 2^8 is
+//                  folded into the K and V scales: kE4m3Unit).
+#ifndef PA_E4M3_CVT
+#define PA_E4M3_CVT 1
+#endif
+constexpr float kE4m3Unit = PA_E4M3_CVT == 2 ? 256.f : 1.f;
+
+__device__ __forceinline__ void e4m3x4_to_frags(uint32_t w, uint32_t& lo, uint32_t& hi) {
+#if PA_E4M3_CVT == 0
+    lo = e4m3x2_to_half2(w);
+    hi = e4m3x2_to_half2(w >> 16);
+#elif PA_E4M3_CVT == 1
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi) : "r"(w));
+#else
+    // byte k of w to the high byte of a 16-bit lane, then drop the sign's
+    // neighbour bit: (x & 0x8000) | ((x >> 1) & 0x3f80) per lane
+    const uint32_t x0 = __byte_perm(w, 0u, 0x1404);   // [b1:00 | b0:00]
+    const uint32_t x1 = __byte_perm(w, 0u, 0x3424);   // [b3:00 | b2:00]
+    lo = (x0 & 0x80008000u) | ((x0 >> 1) & 0x3f803f80u);
+    hi = (x1 & 0x80008000u) | ((x1 >> 1) & 0x3f803f80u);
+#endif
+}
+
+// Two codes in the low 16 bits -> one fp16x2 register (same scaling as above).
+__device__ __forceinline__ uint32_t e4m3x2_to_frag(uint32_t w) {
+#if PA_E4M3_CVT == 0
+    return e4m3x2_to_half2(w);
+#elif PA_E4M3_CVT == 1
+    uint32_t r;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(r) : "r"(w));
+    return r;
+#else
+    const uint32_t x = __byte_perm(w, 0u, 0x1404);
+    return (x & 0x80008000u) | ((x >> 1) & 0x3f803f80u);
+#endif
 }
 
 // Query fragments for the fp16 MMA from 16-bit query rows.  fp16 rows load

@@ -15,6 +15,7 @@
 #pragma once
 
 #include "pa_device.cuh"
+#include "pa_e4m3.cuh"
 
 namespace pa {
 
@@ -78,7 +79,9 @@ struct WarpMma {
     }
 
     // One block of B tokens: K tile at kbase, V tile at vbase (shared memory,
-    // layout [D/8][B][8]); tokens >= valid are masked out.
+    // layout [D/8][B][8]; E4M3: the 8-bit pools' K and V tile layouts, codes
+    // widened to fp16 in registers); tokens >= valid are masked out.
+    template <bool E4M3 = false>
     __device__ __forceinline__ void block(uint32_t kbase, uint32_t vbase, int valid, int group, float scale_log2,
                                           int lane) {
         const int r = lane >> 2, c = lane & 3;
@@ -92,11 +95,24 @@ struct WarpMma {
             if constexpr (B >= 16) {
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const int tok = tg * 16 + (mtx & 1) * 8 + row;
-                    const int chunk = 2 * ks + (mtx >> 1);
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4(kbase + (chunk * B + tok) * 16, a0, a1, a2, a3);
+                    if constexpr (E4M3) {  // tokens r, r+8 of the group; dims 2c.., 2c+8.. of vector ks
+                        const uint32_t at = kbase + ((ks * B + tg * 16 + r) * 16 + 4 * c);
+                        e4m3x4_to_frags(lds32(at), a0, a2);
+                        e4m3x4_to_frags(lds32(at + 8 * 16), a1, a3);
+                    } else {
+                        const int tok = tg * 16 + (mtx & 1) * 8 + row;
+                        const int chunk = 2 * ks + (mtx >> 1);
+                        ldsm_x4(kbase + (chunk * B + tok) * 16, a0, a1, a2, a3);
+                    }
                     Mma<T>::k16(sc, a0, a1, a2, a3, qa[ks][0], qa[ks][1]);
+                }
+            } else if constexpr (E4M3) {  // 8-token blocks: rows 8..15 of the tile are zero
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    uint32_t a0, a2;
+                    e4m3x4_to_frags(lds32(kbase + ((ks * 8 + r) * 16 + 4 * c)), a0, a2);
+                    Mma<T>::k16(sc, a0, 0u, a2, 0u, qa[ks][0], qa[ks][1]);
                 }
             } else {  // 8-token blocks: rows 8..15 of the tile are zero
 #pragma unroll
@@ -145,10 +161,16 @@ struct WarpMma {
                 const int tlo = tg * 16 + 2 * c, thi = tlo + 8;
 #pragma unroll
                 for (int mt = 0; mt < kMt; ++mt) {
-                    const int tok = tg * 16 + (mtx >> 1) * 8 + row;
-                    const int chunk = 2 * mt + (mtx & 1);
                     uint32_t a0, a1, a2, a3;
-                    ldsm_x4_trans(vbase + (chunk * B + tok) * 16, a0, a1, a2, a3);
+                    if constexpr (E4M3) {  // dim rows r, r+8 of tile mt; tokens 2c.., 2c+8.. of the group
+                        const uint32_t at = vbase + ((16 * mt + r) * B + 16 * tg + 4 * c);
+                        e4m3x4_to_frags(lds32(at), a0, a2);
+                        e4m3x4_to_frags(lds32(at + 8 * B), a1, a3);
+                    } else {
+                        const int tok = tg * 16 + (mtx >> 1) * 8 + row;
+                        const int chunk = 2 * mt + (mtx & 1);
+                        ldsm_x4_trans(vbase + (chunk * B + tok) * 16, a0, a1, a2, a3);
+                    }
                     if (partial) {
                         a0 = mask_pair(a0, tlo, valid);
                         a1 = mask_pair(a1, tlo, valid);
@@ -156,6 +178,17 @@ struct WarpMma {
                         a3 = mask_pair(a3, thi, valid);
                     }
                     Mma<T>::k16(o[mt], a0, a1, a2, a3, b0, b1);
+                }
+            } else if constexpr (E4M3) {
+#pragma unroll
+                for (int mt = 0; mt < kMt; ++mt) {
+                    uint32_t y0 = e4m3x2_to_frag(lds16(vbase + ((16 * mt + r) * 8 + 2 * c)));
+                    uint32_t y1 = e4m3x2_to_frag(lds16(vbase + ((16 * mt + r + 8) * 8 + 2 * c)));
+                    if (partial) {
+                        y0 = mask_pair(y0, 2 * c, valid);
+                        y1 = mask_pair(y1, 2 * c, valid);
+                    }
+                    Mma<T>::k8(o[mt], y0, y1, b0);
                 }
             } else {
 #pragma unroll
