@@ -75,6 +75,8 @@ def parse_args(argv=None):
                     help="rotate: inputs larger than L2, rotated over independent copies, K steps timed as one "
                          "region; flush: a 256 MiB write between steps, per-step events")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture each rotated copy's step into a CUDA graph once and replay it in the timed region")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     return ap.parse_args(argv)
@@ -346,17 +348,18 @@ def run_gpu(args, world, rank, local):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if copies == 0 else None
     decode_bytes, reshape_bytes = step_bytes(batch, fp8)
 
-    def one(i, ev=None):
+    def one(i, ev=None, on=None):
+        s_ = on if on is not None else stream
         st = steps[i % len(steps)]
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(s_)
         if st.mode != "append":  # append: the whole step is the decode launch
-            st.reshape(stream)
+            st.reshape(s_)
         if ev is not None:
-            ev[1].record(stream)
-        st.decode(stream)
+            ev[1].record(s_)
+        st.decode(s_)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(s_)
 
     for i in range(args.warmup):
         if flush is not None:
@@ -365,6 +368,23 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
+    graphs = None
+    if args.graph:   # one graph per rotated copy, captured after the uncaptured warm-up calls
+        graphs = []
+        for i in range(len(steps)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                one(i, on=torch.cuda.current_stream())   # launches on the capturing stream
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+        def one(i, ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+                ev[1].record(stream)
+            graphs[i % len(graphs)].replay()
+            if ev is not None:
+                ev[2].record(stream)
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     region = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -388,7 +408,7 @@ def run_gpu(args, world, rank, local):
             # per-step events inside it split reshape from decode.
             region[0].record(stream)
             for i in range(args.steps):
-                one(i, events[i] if mode != "append" else None)
+                one(i, events[i] if mode != "append" and graphs is None else None)
             region[1].record(stream)
         else:
             for i in range(args.steps):
@@ -398,7 +418,7 @@ def run_gpu(args, world, rank, local):
     barrier(world)
     if flush is None:
         local_step = region[0].elapsed_time(region[1]) / args.steps
-        if mode == "append":
+        if mode == "append" or graphs is not None:   # one launch, or the whole step replayed as one graph
             decode_ms, reshape_ms = [local_step], [0.0]
         else:
             decode_ms = [e[1].elapsed_time(e[2]) for e in events]
@@ -560,6 +580,7 @@ def run_gpu(args, world, rank, local):
                    f"{l2 / 1e6:.0f} MB L2), rotated over {len(steps)} independent copies; K steps in one "
                    f"CUDA-event region") if flush is None
             else "flushed between steps (256 MiB write), per-step CUDA events",
+            "graph": bool(args.graph),
             "step": ("pa_decode_append: newest token of every sequence written + decode, one launch" if mode == "append"
                      else "pa_reshape_and_cache_fp8 (newest token of every sequence, quantised) + decode"
                      if fp8 is not None

@@ -1,0 +1,101 @@
+"""A decode step captured into a CUDA graph (GPU): after one uncaptured call
+(which sets the kernels' shared-memory limit and caches device attributes),
+the write and decode entry points record into a graph, and replaying it gives
+bit-for-bit the eager result, again after the inputs have changed in place."""
+
+import pytest
+import torch
+
+import workloads
+import paged_kv_cache_449_b200 as pa
+from pagedutil import device_batch
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t):
+    return t.contiguous().view(-1).view(torch.int32 if t.element_size() == 4 else torch.int16)
+
+
+def _copies(b, n):
+    out = []
+    for _ in range(n):
+        d = device_batch(b)
+        d["k_cache"], d["v_cache"] = d["k_cache"].clone(), d["v_cache"].clone()
+        d["nk"], d["nv"] = b.new_key.cuda().clone(), b.new_value.cuda().clone()
+        d["slots"] = b.slot_mapping.cuda().clone()
+        d["out"] = torch.full_like(d["q"], float("nan"))
+        out.append(d)
+    return out
+
+
+def _steps(b):
+    ws = torch.empty(pa.pa_decode_splitk_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim,
+                                                        b.max_context_len, 256), dtype=torch.uint8, device="cuda")
+    counters = pa.Counters()
+    counters.get(b.num_seqs * b.num_kv_heads, "cuda")
+
+    def append(d):
+        pa.pa_decode_append(d["out"], d["q"], d["nk"], d["nv"], d["k_cache"], d["v_cache"], d["block_tables"],
+                            d["context_lens"], b.scale, max_context_len=b.max_context_len)
+
+    def reshape_then_split(d):
+        pa.pa_reshape_and_cache(d["nk"], d["nv"], d["k_cache"], d["v_cache"], d["slots"])
+        pa.pa_decode_splitk(d["out"], d["q"], d["k_cache"], d["v_cache"], d["block_tables"], d["context_lens"],
+                            b.scale, b.max_context_len, partition_size=256, workspace=ws, counters=counters)
+
+    def reshape_then_two_kernel_split(d):
+        pa.pa_reshape_and_cache(d["nk"], d["nv"], d["k_cache"], d["v_cache"], d["slots"])
+        pa.pa_decode_splitk(d["out"], d["q"], d["k_cache"], d["v_cache"], d["block_tables"], d["context_lens"],
+                            b.scale, b.max_context_len, partition_size=256, workspace=ws, fused=False)
+
+    return {"append": append, "split_fused": reshape_then_split, "split_merge_kernel": reshape_then_two_kernel_split}
+
+
+@pytest.mark.parametrize("which", ["append", "split_fused", "split_merge_kernel"])
+def test_graph_replay_equals_eager(which):
+    b = workloads.llama3_8b_decode(seed=31, device="cuda", num_seqs=16, num_blocks=2048)
+    eager, graphed = _copies(b, 2)
+    step = _steps(b)[which]
+    pa.pa_get_device_error()
+    step(graphed)                      # the uncaptured first call
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(graphed)
+    for round_ in range(2):
+        if round_ == 1:                # new queries in place: the graph reads them at replay
+            newq = torch.randn(eager["q"].shape, generator=torch.Generator(device="cuda").manual_seed(5),
+                               device="cuda").to(eager["q"].dtype)
+            eager["q"].copy_(newq)
+            graphed["q"].copy_(newq)
+        step(eager)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(_bits(graphed["out"]), _bits(eager["out"])), (which, round_)
+        assert torch.equal(_bits(graphed["k_cache"]), _bits(eager["k_cache"]))
+    assert pa.pa_get_device_error() == 0
+    del g
+
+
+def test_graph_replay_fp8():
+    b = workloads.llama3_8b_decode(seed=32, device="cuda", num_seqs=16, num_blocks=2048)
+    pools = workloads.random_fp8_pools(b, seed=3, device="cuda")
+    q, bt, cl = b.q.cuda(), b.block_tables.cuda(), b.context_lens.cuda()
+    outs = [torch.full_like(q, float("nan")) for _ in range(2)]
+
+    def step(out):
+        pa.pa_decode_fp8(out, q, pools.k_cache, pools.v_cache, pools.k_scale, pools.v_scale, bt, cl, b.scale,
+                         max_context_len=b.max_context_len)
+
+    step(outs[1])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(outs[1])
+    outs[1].fill_(float("nan"))
+    step(outs[0])
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(outs[1]), _bits(outs[0]))
+    del g
