@@ -86,6 +86,9 @@ class Oracle:
         lib.oracle_e4m3_value.argtypes = [c.c_int]
         lib.oracle_e4m3_encode.restype = c.c_int
         lib.oracle_e4m3_encode.argtypes = [c.c_float]
+        lib.oracle_prefill.restype = c.c_int
+        lib.oracle_prefill.argtypes = [c.c_void_p] * 7 + [c.c_float, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int,
+                                                          c.c_int, c.c_int64, c.c_int]
         lib.oracle_pool_index.restype = c.c_int64
         lib.oracle_pool_index.argtypes = [c.c_int64, c.c_int, c.c_int, c.c_int, c.c_int,
                                           c.c_int, c.c_int, c.c_int]
@@ -185,6 +188,23 @@ class Oracle:
 
     def e4m3_encode(self, v: float) -> int:
         return int(self.lib.oracle_e4m3_encode(float(v)))
+
+    def prefill(self, q, k_cache, v_cache, block_tables, context_lens, query_start, scale, block_size,
+                num_kv_heads) -> np.ndarray:
+        """fp64 chunked-prefill output [T, Hq, D]: query rows query_start[s] ..
+        query_start[s+1]-1 are the newest tokens of sequence s, causal."""
+        for t in (q, k_cache, v_cache):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        bt = block_tables.to(torch.int32).contiguous()
+        cl = context_lens.to(torch.int32).contiguous()
+        qs = query_start.to(torch.int32).contiguous()
+        T, Hq, D = q.shape
+        out = np.zeros((T, Hq, D), dtype=np.float64)
+        self._check(self.lib.oracle_prefill(
+            out.ctypes.data, q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), bt.data_ptr(), cl.data_ptr(),
+            qs.data_ptr(), float(scale), block_size, cl.numel(), Hq, num_kv_heads, D, bt.shape[1], k_cache.shape[0],
+            DTYPE_CODE[q.dtype]))
+        return out
 
     def pool_index(self, block, head, token, dim, num_kv_heads, block_size, head_dim, dtype):
         return int(self.lib.oracle_pool_index(block, head, token, dim, num_kv_heads,

@@ -23,6 +23,11 @@
 //        reference count, copy-on-write for isolation.
 //   [P1] §4.2 preemption: a preempted sequence's KV blocks are swapped out to
 //        CPU memory (or dropped and recomputed) and swapped back in later.
+//   [P1] §4.3 chunked prefill: the prompt of a sequence is processed in chunks
+//        that share the batch with decoding sequences.  Reading: a chunk is the
+//        newest Q tokens of a sequence whose K/V (all L tokens, chunk included)
+//        are already in the pool; chunk query i sits at position L - Q + i and
+//        attends causally to the tokens at positions 0 .. L - Q + i.
 //   [P4] §7 FP8 attention (the rest in FP16) as the next optimisation: here an
 //        8-bit KV pool.  Readings (the pages fix no format): e4m3 codes (OCP
 //        8-bit float, E4M3 "fn": 1 sign, 4 exponent bits with bias 7, 3
@@ -410,6 +415,49 @@ int oracle_decode_partitioned(double* out, const void* q, const void* k_cache, c
                    max_blocks_per_seq, num_blocks, dtype};
     return decode_common(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh, seq_ids,
                          num_selected, partition_size);
+}
+
+// Paged prefill of query chunks ([P1] §4.3 chunked prefill): queries
+// [T][Hq][D] with sequence s owning rows query_start[s] .. query_start[s+1]-1
+// (Q_s of them, Q_s <= context_lens[s]); out [T][Hq][D] doubles.  Query i of
+// sequence s attends to its first L_s - Q_s + i + 1 logical tokens.
+int oracle_prefill(double* out, const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+                   float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                   int max_blocks_per_seq, int64_t num_blocks, int dtype) {
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start) return kBadArg;
+    const Shape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, num_blocks, dtype};
+    if (!shape_ok(sh)) return kBadArg;
+    const int group = num_q_heads / num_kv_heads;
+    const int D = head_dim;
+    const double scale_d = static_cast<double>(scale);
+    std::vector<double> keys, values, qrow(D);
+    if (query_start[0] != 0) return kBadArg;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int len = context_lens[s];
+        const int rc = check_context_len(len, sh);
+        if (rc != kOk) return rc;
+        const int first = query_start[s];
+        const int count = query_start[s + 1] - first;
+        if (count < 0 || count > len) return kBadArg;
+        const int32_t* row = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq;
+        for (int kvh = 0; kvh < num_kv_heads; ++kvh) {
+            const int g = gather_sequence(k_cache, v_cache, row, len, kvh, sh, keys, values);
+            if (g != kOk) return g;
+            for (int i = 0; i < count; ++i) {
+                const int visible = len - count + i + 1;  // positions 0 .. L - Q + i
+                for (int j = 0; j < group; ++j) {
+                    const int h = kvh * group + j;
+                    const int64_t t = first + i;
+                    for (int d = 0; d < D; ++d)
+                        qrow[d] = element(q, (t * num_q_heads + h) * D + d, dtype);
+                    attend_plain(qrow.data(), keys, values, visible, D, scale_d,
+                                 out + (t * num_q_heads + h) * D);
+                }
+            }
+        }
+    }
+    return kOk;
 }
 
 // Position of element (block, head, token, dim) in a pool of the given shape,

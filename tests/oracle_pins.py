@@ -554,9 +554,96 @@ def pin_number_formats(orc):
     np.testing.assert_array_equal(_decode(orc, b)[:, 0], f32.reshape(S, D).astype(np.float64))
 
 
+# ---------------------------------------------------------------------------- chunked prefill
+
+def _prefill(orc, b, qs=None, lens=None):
+    qs = b.meta["query_start"] if qs is None else qs
+    return orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens if lens is None else lens, qs,
+                       b.scale, b.block_size, b.num_kv_heads)
+
+
+def pin_prefill_single_token_chunks_are_decode(orc):
+    """Chunks of one token: each query is the newest token of its sequence,
+    which is exactly decode ([P1] §4.3 mixes both in one batch)."""
+    for dt, B, g in ((torch.bfloat16, 16, 4), (torch.float32, 8, 1)):
+        b = workloads.random_small(seed=91, dtype=dt, lens=(1, 17, 40, 5), num_q_heads=2 * g, num_kv_heads=2,
+                                   head_dim=32, block_size=B)
+        qs = torch.arange(b.num_seqs + 1, dtype=torch.int32)
+        np.testing.assert_array_equal(_prefill(orc, b, qs), _decode(orc, b))
+
+
+def pin_prefill_brute_force(orc):
+    """Causal attention by long-double brute force over the logical K/V (a
+    separate loop nest): query i of a chunk of Q sees positions 0 .. L-Q+i."""
+    for dt, B, Hq, Hkv in ((torch.float32, 8, 4, 2), (torch.float16, 16, 2, 2)):
+        b = workloads.chunked_prefill(seed=92, dtype=dt, num_seqs=3, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=16,
+                                      block_size=B, context_range=(3, 40), chunk_range=(1, 40))
+        got = _prefill(orc, b)
+        qs = b.meta["query_start"].tolist()
+        g = Hq // Hkv
+        for s in range(b.num_seqs):
+            L = int(b.context_lens[s])
+            Q = qs[s + 1] - qs[s]
+            for kvh in range(Hkv):
+                K, V = logical_kv(b, s, kvh)
+                K, V = K.astype(np.longdouble), V.astype(np.longdouble)
+                for i in range(Q):
+                    p = L - Q + i
+                    for j in range(g):
+                        h = kvh * g + j
+                        qv = as_f64(b.q[qs[s] + i, h]).astype(np.longdouble)
+                        z = (K[:p + 1] @ qv) * np.longdouble(np.float32(b.scale))
+                        w = np.exp(z - z.max())
+                        ref = (w[:, None] * V[:p + 1]).sum(0) / w.sum()
+                        assert rel_err(got[qs[s] + i, h], ref.astype(np.float64)) <= 1e-12, (s, i, h)
+
+
+def pin_prefill_future_tokens_are_invisible(orc):
+    """Changing the K/V of the chunk's last token leaves every earlier query of
+    the chunk bit-identical, and changes the last query's output."""
+    b = workloads.chunked_prefill(seed=93, dtype=torch.bfloat16, num_seqs=2, num_q_heads=4, num_kv_heads=2,
+                                  head_dim=32, block_size=16, context_range=(30, 50), chunk_range=(8, 12))
+    before = _prefill(orc, b)
+    k, v = b.k_cache.clone(), b.v_cache.clone()
+    qs = b.meta["query_start"].tolist()
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        blk = int(b.block_tables[s, (L - 1) // 16])
+        k[blk, :, :, (L - 1) % 16, :] = 7.0
+        v[blk, :, :, (L - 1) % 16, :] = -9.0
+    c = b.__class__(**{**b.__dict__, "k_cache": k, "v_cache": v})
+    after = _prefill(orc, c)
+    for s in range(b.num_seqs):
+        np.testing.assert_array_equal(after[qs[s]:qs[s + 1] - 1], before[qs[s]:qs[s + 1] - 1])
+        assert np.abs(after[qs[s + 1] - 1] - before[qs[s + 1] - 1]).max() > 1e-3
+
+
+def pin_prefill_chunk_split(orc):
+    """A chunk of Q tokens equals the same chunk run as two chunks (the first
+    Q1 tokens with context L - Q + Q1, then the rest with context L), bit for
+    bit: chunking does not change any query's attention."""
+    b = workloads.chunked_prefill(seed=94, dtype=torch.float16, num_seqs=3, num_q_heads=4, num_kv_heads=1,
+                                  head_dim=16, block_size=8, context_range=(20, 60), chunk_range=(6, 20))
+    whole = _prefill(orc, b)
+    qs = b.meta["query_start"].tolist()
+    for s in range(b.num_seqs):
+        Q = qs[s + 1] - qs[s]
+        L = int(b.context_lens[s])
+        Q1 = Q // 2
+        one = b.__class__(**{**b.__dict__, "num_seqs": 1, "q": b.q[qs[s]:qs[s] + Q1].contiguous(),
+                             "block_tables": b.block_tables[s:s + 1], "context_lens": torch.tensor([L - Q + Q1],
+                                                                                                  dtype=torch.int32)})
+        two = b.__class__(**{**b.__dict__, "num_seqs": 1, "q": b.q[qs[s] + Q1:qs[s + 1]].contiguous(),
+                             "block_tables": b.block_tables[s:s + 1], "context_lens": torch.tensor([L], dtype=torch.int32)})
+        a = _prefill(orc, one, torch.tensor([0, Q1], dtype=torch.int32))
+        c = _prefill(orc, two, torch.tensor([0, Q - Q1], dtype=torch.int32))
+        np.testing.assert_array_equal(np.concatenate([a, c]), whole[qs[s]:qs[s + 1]])
+
+
 PINS = [pin_layout_golden, pin_slot_golden, pin_brute_force, pin_dense_equality,
         pin_permutation_invariance, pin_block_size_invariance, pin_shared_vs_copied,
         pin_closed_forms, pin_needle, pin_partitioned, pin_reshape_scatter, pin_errors,
         pin_number_formats, pin_copy_blocks_rows, pin_copy_on_write_keeps_attention, pin_swap_round_trip,
         pin_e4m3_golden, pin_e4m3_layout_golden, pin_e4m3_against_torch, pin_e4m3_write_then_single_token,
-        pin_e4m3_decode_is_dense_decode_of_dequantised_pool]
+        pin_e4m3_decode_is_dense_decode_of_dequantised_pool, pin_prefill_single_token_chunks_are_decode,
+        pin_prefill_brute_force, pin_prefill_future_tokens_are_invisible, pin_prefill_chunk_split]

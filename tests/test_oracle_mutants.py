@@ -62,6 +62,9 @@ MUTANTS = {
                                 "int64_t e4m3_slot16(int64_t j) { return j; }"),
     "e4m3_v_not_transposed": ("const int64_t va = e4m3_v_index(physical, kv_head, offset, d, sh.num_kv_heads, sh.block_size, D);",
                               "const int64_t va = e4m3_k_index(physical, kv_head, offset, d, sh.num_kv_heads, sh.block_size, D);"),
+    "prefill_causal_off_by_one": ("const int visible = len - count + i + 1;", "const int visible = len - count + i + 2;"),
+    "prefill_not_causal": ("const int visible = len - count + i + 1;", "const int visible = len;"),
+    "prefill_rows_reversed": ("const int64_t t = first + i;", "const int64_t t = first + count - 1 - i;"),
     "q_from_wrong_head": ("(static_cast<int64_t>(s) * sh.num_q_heads + h) * D + d",
                           "(static_cast<int64_t>(s) * sh.num_q_heads + kvh) * D + d"),
 }

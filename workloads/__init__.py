@@ -140,6 +140,32 @@ def random_fp8_pools(batch: "Batch", seed=0, device=None) -> Fp8Pools:
     return Fp8Pools(pools[0], pools[1], scales[0], scales[1])
 
 
+def chunked_prefill(seed=0, device="cpu", dtype=torch.bfloat16, num_seqs=8, num_q_heads=32, num_kv_heads=8,
+                    head_dim=128, block_size=16, context_range=(1024, 4096), chunk_range=(256, 1024),
+                    num_blocks=None) -> Batch:
+    """Chunked prefill: every sequence's K/V (context uniform on
+    `context_range`) is already in the pool with shuffled block ids, and its
+    newest Q tokens (uniform on `chunk_range`, at most the context) are the
+    query chunk.  q is [sum Q, Hq, D]; meta["query_start"] is the int32
+    [S + 1] prefix sum of the chunk lengths."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(context_range[0], context_range[1], size=num_seqs, endpoint=True)
+    chunks = np.minimum(rng.integers(chunk_range[0], chunk_range[1], size=num_seqs, endpoint=True), lens)
+    need = int(sum((int(L) + block_size - 1) // block_size for L in lens))
+    N = num_blocks or need + 16
+    ids = rng.permutation(N)[:need].astype(np.int32)
+    tables, _ = _tables_from_lens(lens, block_size, ids)
+    slots = _decode_slots(tables, lens, block_size)
+    b = make_batch(f"chunked_prefill_{str(dtype).split('.')[-1]}", dtype=dtype, lens=lens, num_q_heads=num_q_heads,
+                   num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size, num_blocks=N, tables=tables,
+                   slots=slots, seed=seed, device=device)
+    T = int(chunks.sum())
+    b.q = _normal((T, num_q_heads, head_dim), dtype, device, seed + 7)
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    b.meta = dict(b.meta, query_start=torch.from_numpy(qs))
+    return b
+
+
 # --------------------------------------------------------------------------
 # value generation
 
