@@ -16,8 +16,10 @@ from oracle_pins import PINS
 SRC = os.path.join(os.path.dirname(oracle.__file__), "pa_oracle.cpp")
 
 MUTANTS = {
-    "gqa_interleaved_heads": ("const int h = kvh * group + j;",
+    "gqa_interleaved_heads": ("const int h = kvh * group + j;  // query head h reads kv head h / group",
                               "const int h = j * sh.num_kv_heads + kvh;"),
+    "prefill_gqa_interleaved": ("const int h = kvh * group + j;\n                    const int64_t t = first + i;",
+                                "const int h = j * num_kv_heads + kvh;\n                    const int64_t t = first + i;"),
     "layout_token_outer": ("return (vector * block_size + token) * vec + dim % vec;",
                            "return ((tile * block_size + token) * (head_dim / vec) + dim / vec) * vec + dim % vec;"),
     "offset_off_by_one": ("const int offset = t % sh.block_size;",
