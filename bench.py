@@ -58,7 +58,7 @@ def parse_args(argv=None):
                     choices=["tiny_mha_f32", "llama3_8b_decode", "continuous_batching_mix", "prefix_sharing",
                              "llama3_70b_long"])
     ap.add_argument("--block-size", type=int, default=None)
-    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap_out", "swap_in"], default="decode",
+    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap_out", "swap_in", "prefill"], default="decode",
                     help="decode: the hot-path step (default); copy_blocks: every block of the batch duplicated "
                          "into free blocks of the same pools (copy-on-write / fork); swap_out / swap_in: every "
                          "block of the batch copied to / from a pinned host pool (preemption by swapping)")
@@ -687,6 +687,83 @@ def run_reference(args, world, rank):
     }
 
 
+def measured_tensor_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 (burst)"
+    return 1590.0, "fallback bf16"
+
+
+def run_prefill(args, world, rank, local):
+    """Chunked prefill through pa_prefill: Llama-3-8B heads, 8 sequences with
+    contexts U[1024, 4096] whose newest U[256, 1024] tokens are the chunk."""
+    import paged_kv_cache_449_b200 as pa
+    import workloads
+    from paged_kv_cache_449_b200 import build as pabuild
+    pabuild.build()
+    pa.load()
+    b = workloads.chunked_prefill(seed=args.seed + rank, device="cuda")
+    qs = b.meta["query_start"]
+    chunks = (qs[1:] - qs[:-1]).to(torch.int64)
+    lens = b.context_lens.to(torch.int64)
+    # every query row sees L - Q + i + 1 keys: QK^T and PV are 2 * D flops per key each
+    visible = int(((lens - chunks) * chunks + chunks * (chunks + 1) // 2).sum())
+    flops = 4 * b.head_dim * b.num_q_heads * visible
+    dev = {k: getattr(b, k).cuda().contiguous() for k in ("q", "k_cache", "v_cache", "block_tables", "context_lens")}
+    qsd = qs.cuda()
+    out = torch.empty_like(dev["q"])
+    maxq = int(chunks.max())
+    stream = torch.cuda.current_stream()
+
+    def one():
+        pa.pa_prefill(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"], dev["context_lens"], qsd,
+                      b.scale, max_context_len=b.max_context_len, max_query_len=maxq, stream=stream)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    pa.pa_get_device_error()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        t_busy = time.perf_counter() + 0.3
+        while time.perf_counter() < t_busy:
+            one()
+            torch.cuda.synchronize()
+        barrier(world)
+        ev[0].record(stream)
+        for _ in range(args.steps):
+            one()
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error word set during the timed steps")
+    local_ms = ev[0].elapsed_time(ev[1]) / args.steps
+    ms = reduce_max(local_ms, world)
+    total = reduce_sum(flops, world)
+    peak, kind = measured_tensor_peak()
+    achieved = flops / (local_ms * 1e-3) / 1e12
+    return {
+        "metric": "paged chunked prefill TFLOP/s (Llama-3-8B attention shape)",
+        "value": round(total / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) Q/K/V, seeded context and chunk lengths, shuffled block ids)",
+        "config": {"workload": b.name, "global_batch": b.num_seqs, "query_tokens": int(chunks.sum()),
+                   "context_len_mean": float(lens.float().mean()), "chunk_len_mean": float(chunks.float().mean()),
+                   "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim,
+                   "block_size": b.block_size, "flops_per_step": flops, "parallelism": f"replicas x{world}",
+                   "l2": "not flushed: compute-bound (the K/V of a sequence is reread by its query tiles)",
+                   "mma": "mma.sync m16n8k16 bf16, fp32 accumulate"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "peak_kind": kind,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+
+
 def run_blocks(args, world, rank, local):
     """Block copies through pa_copy_blocks: every block of the batch's
     sequences, K and V pools, per step."""
@@ -782,7 +859,7 @@ def main(argv=None):
                 print(json.dumps(res), flush=True)
             return
         if args.op != "decode":
-            res = run_blocks(args, world, rank, local)
+            res = (run_prefill if args.op == "prefill" else run_blocks)(args, world, rank, local)
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return

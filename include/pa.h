@@ -295,6 +295,30 @@ pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, co
                                void* stream);
 
 /*
+ * pa_prefill — chunked prefill over the paged pool ([P1] §4.3 chunked
+ * prefill; attention as in [P3] §2.3).  Sequence s brings Q_s = query_start
+ * [s+1] - query_start[s] query tokens: the newest Q_s of its context_lens[s]
+ * = L_s tokens, whose K/V are already in the pool (pa_reshape_and_cache).
+ * Query i of sequence s sits at position L_s - Q_s + i and attends causally:
+ *   out[query_start[s]+i, h, :] = sum_{t <= L_s-Q_s+i} softmax_t(scale *
+ *                                 q.K[s,t]) V[s,t].
+ *
+ *   out, q         [T][num_q_heads][head_dim], T = query_start[num_seqs],
+ *                  fp16 or bf16 (PA_ERR_UNSUPPORTED for fp32), 16-byte aligned
+ *   query_start    int32 [num_seqs + 1], query_start[0] = 0, non-decreasing,
+ *                  with Q_s <= L_s; 4-byte aligned device memory
+ *   max_query_len  an upper bound of every Q_s (sizes the grid)
+ *   Other arguments as in pa_decode.  A sequence whose length or chunk is out
+ *   of range sets PA_DEVERR_CONTEXT_LEN and its rows are not written.
+ *   Tensor cores through warp-level mma.sync (fp32 accumulation).
+ */
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
+                     float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                     int head_dim, int max_blocks_per_seq, int max_context_len, int max_query_len,
+                     int64_t num_blocks, pa_dtype dtype, void* stream);
+
+/*
  * pa_copy_blocks — copy whole physical blocks (every kv head, token and
  * dimension, K pool and V pool) from a source pool pair to a destination pool
  * pair.  The same pools on both sides duplicate a shared block before a

@@ -23,7 +23,7 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT",
            "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
-           "pa_decode_splitk_fp8", "fp8_pool_shape"]
+           "pa_decode_splitk_fp8", "fp8_pool_shape", "pa_prefill"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -77,6 +77,8 @@ def load() -> ctypes.CDLL:
     lib.pa_decode_fp8.argtypes = fp8_args + [P, P]
     lib.pa_decode_splitk_fp8.restype = I
     lib.pa_decode_splitk_fp8.argtypes = fp8_args + [I, P, SZ, P, I64, P, P]
+    lib.pa_prefill.restype = I
+    lib.pa_prefill.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I64, I, P]
     lib.pa_copy_blocks.restype = I
     lib.pa_copy_blocks.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I64, I, P]
     lib.pa_get_device_error.restype = I
@@ -351,6 +353,25 @@ def pa_decode_splitk_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_table
     _check(lib.pa_decode_splitk_fp8(*args, int(partition_size), _dev_ptr(workspace, "workspace"),
                                     workspace.numel() * workspace.element_size(), cptr, ncount,
                                     _order_ptr(seq_order, S), _stream(stream)), "pa_decode_splitk_fp8")
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start, scale, max_context_len=None,
+               max_query_len=None, stream=None):
+    """Causal chunked prefill: q/out [T, Hq, D] (fp16/bf16); query_start int32
+    [S + 1] on the device; sequence s's chunk is its newest Q_s tokens."""
+    lib = load()
+    n, hkv, d, b = _pool_dims(k_cache)
+    T, Hq, D = q.shape
+    S = int(context_lens.numel())
+    if max_context_len is None:
+        max_context_len = int(block_tables.shape[1]) * b
+    if max_query_len is None:
+        max_query_len = T
+    _check(lib.pa_prefill(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+        _dev_ptr(block_tables, "block_tables"), _dev_ptr(context_lens, "context_lens"),
+        _dev_ptr(query_start, "query_start"), float(scale), b, S, Hq, hkv, D, int(block_tables.shape[1]),
+        int(max_context_len), int(max_query_len), n, _DTYPE[q.dtype], _stream(stream)), "pa_prefill")
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -16,6 +16,7 @@
 #include "pa.h"
 #include "pa_copy.cuh"
 #include "pa_decode.cuh"
+#include "pa_prefill.cuh"
 #include "pa_reshape.cuh"
 
 // Two CTA shapes for the decode kernels, measured on B200 over the benchmark
@@ -304,6 +305,20 @@ bool device_accessible(const void* p) {
     return attr.type == cudaMemoryTypeHost && attr.devicePointer == p;
 }
 
+// Chunked prefill: 4 warps (64 MMA rows) per CTA, a 4-stage block ring.
+constexpr int kPrefillWarps = 4;
+constexpr int kPrefillStages = 4;
+
+template <typename T, int D, int B>
+cudaError_t launch_prefill(const pa::PrefillParams& p, dim3 grid, cudaStream_t st) {
+    using Sm = pa::PrefillSmem<T, D, B, kPrefillWarps, kPrefillStages>;
+    auto kernel = pa::pa_prefill_kernel<T, D, B, kPrefillWarps, kPrefillStages>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kPrefillWarps * 32, Sm::kTotal, st>>>(p);
+    return cudaGetLastError();
+}
+
 // The one-pass and split decode bodies, shared by the 16-bit-pool entries
 // (FP8 = false) and the 8-bit-pool entries (FP8 = true, with K/V scales).
 template <bool FP8>
@@ -580,6 +595,50 @@ pa_status pa_copy_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k
     pa::pa_copy_blocks_kernel<<<static_cast<unsigned>(ctas), pa::kCopyThreads, 0,
                                 static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, const int32_t* query_start, float scale, int block_size,
+                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                     int max_context_len, int max_query_len, int64_t num_blocks, pa_dtype dtype, void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (st != PA_OK) return st;
+    if (dtype == PA_F32) return PA_ERR_UNSUPPORTED;  // the tensor-core path takes 16-bit inputs
+    if (max_query_len < 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+    if (!query_start || !aligned4(query_start)) return PA_ERR_INVALID_ARG;
+    pa::PrefillParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start = query_start;
+    p.score_scale = scale * 1.4426950408889634f;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.context_cap = context_cap(sh);
+    p.num_blocks = num_blocks;
+    p.tile_tokens = kPrefillWarps * 16 / p.group;
+    const long long tiles = (static_cast<long long>(max_query_len) + p.tile_tokens - 1) / p.tile_tokens;
+    if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = with_variant(dtype, head_dim, block_size, [&](auto tt, auto dd, auto bb) -> cudaError_t {
+        using T = typename decltype(tt)::type;
+        if constexpr (pa::IsF32<T>::value) {
+            return cudaErrorInvalidValue;
+        } else {
+            return launch_prefill<T, decltype(dd)::value, decltype(bb)::value>(p, grid, s);
+        }
+    });
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_get_device_error(void* stream, int32_t* code) {

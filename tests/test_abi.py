@@ -34,7 +34,7 @@ def lib():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "pa_copy_blocks", "pa_decode", "pa_decode_append", "pa_decode_fp8", "pa_decode_splitk",
-        "pa_decode_splitk_fp8", "pa_decode_splitk_workspace_size", "pa_reshape_and_cache_fp8",
+        "pa_decode_splitk_fp8", "pa_decode_splitk_workspace_size", "pa_reshape_and_cache_fp8", "pa_prefill",
         "pa_decode_splitk_static", "pa_get_device_error",
         "pa_reshape_and_cache", "pa_status_string"])
 
@@ -118,6 +118,11 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_decode_splitk_fp8(*f8, 1, 512, 16, 100, None, 0, None, None) == 3       # workspace too small
     assert lib.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 16, 16, 4, 8, 40, 16, 10, 2, None) == 2  # D % 16
     assert lib.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 0, 16, 4, 8, 64, 16, 10, 2, None) == 1   # no scale
+    pf = [16, 16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 100, 64]
+    assert lib.pa_prefill(*pf, 0, None) == 2                                             # fp32 queries
+    assert lib.pa_prefill(*pf[:6], 0, *pf[7:], 2, None) == 1                             # no query_start
+    assert lib.pa_prefill(*pf[:15], -1, 64, 2, None) == 1                                # negative max query
+    assert lib.pa_prefill(*pf[:15], 0, 64, 2, None) == 0                                 # no queries: no-op
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

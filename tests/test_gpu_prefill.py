@@ -1,0 +1,89 @@
+"""Chunked prefill on the GPU against the oracle's causal prefill (every
+element), across dtypes, head dims, block sizes, GQA groups and chunk shapes
+(single-token chunks, whole-context chunks, ragged chunks); single-token
+chunks against the decode kernel; malformed chunks flagged on the device."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import paged_kv_cache_449_b200 as pa
+from pagedutil import as_f64, check_tolerance, device_batch, gpu_decode
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.default()
+
+
+@pytest.fixture(autouse=True)
+def no_device_errors():
+    pa.pa_get_device_error()
+    yield
+    assert pa.pa_get_device_error() == 0
+
+
+def _gpu_prefill(b, qs=None):
+    qs = b.meta["query_start"] if qs is None else qs
+    dev = device_batch(b)
+    out = torch.full_like(dev["q"], float("nan"))
+    Q = (qs[1:] - qs[:-1]).max().item() if qs.numel() > 1 else 0
+    pa.pa_prefill(out, dev["q"], dev["k_cache"], dev["v_cache"], dev["block_tables"], dev["context_lens"],
+                  qs.cuda(), b.scale, max_context_len=b.max_context_len, max_query_len=int(Q))
+    torch.cuda.synchronize()
+    return out
+
+
+CASES = [
+    # dtype, D, B, Hq, Hkv, context range, chunk range
+    (torch.bfloat16, 128, 16, 32, 8, (1, 90), (1, 90)),
+    (torch.bfloat16, 128, 8, 8, 8, (20, 70), (10, 70)),
+    (torch.float16, 64, 32, 16, 2, (30, 130), (1, 40)),
+    (torch.float16, 128, 16, 8, 1, (40, 80), (33, 80)),
+    (torch.bfloat16, 64, 8, 4, 2, (1, 50), (1, 5)),
+    (torch.bfloat16, 64, 32, 8, 4, (60, 200), (60, 200)),
+]
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_prefill_every_element(orc, case):
+    dt, D, B, Hq, Hkv, ctx, chunk = CASES[case]
+    b = workloads.chunked_prefill(seed=1000 + case, dtype=dt, num_seqs=5, num_q_heads=Hq, num_kv_heads=Hkv,
+                                  head_dim=D, block_size=B, context_range=ctx, chunk_range=chunk)
+    ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.meta["query_start"], b.scale,
+                      B, Hkv)
+    got = _gpu_prefill(b)
+    check_tolerance(as_f64(got), ref, dt)
+
+
+def test_prefill_llama3_8b_shape(orc):
+    b = workloads.chunked_prefill(seed=1010, num_seqs=4, context_range=(512, 1024), chunk_range=(64, 256))
+    ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.meta["query_start"], b.scale,
+                      b.block_size, b.num_kv_heads)
+    got = _gpu_prefill(b)
+    check_tolerance(as_f64(got), ref, b.dtype)
+    assert torch.isfinite(got.float()).all()
+
+
+def test_single_token_chunks_match_decode():
+    b = workloads.llama3_8b_decode(seed=1020, num_seqs=12, num_blocks=2048)
+    qs = torch.arange(b.num_seqs + 1, dtype=torch.int32)
+    pre = _gpu_prefill(b, qs)
+    dec = gpu_decode(b, "single")
+    check_tolerance(as_f64(pre), as_f64(dec), b.dtype)
+
+
+def test_chunk_longer_than_context_is_flagged():
+    b = workloads.random_small(seed=1030, dtype=torch.bfloat16, lens=(10, 20), num_q_heads=4, num_kv_heads=2,
+                               head_dim=64, block_size=16)
+    qs = torch.tensor([0, 12, 14], dtype=torch.int32)   # 12 queries over a 10-token context
+    b.q = torch.randn((14, 4, 64)).to(torch.bfloat16)
+    pa.pa_get_device_error()
+    out = _gpu_prefill(b, qs)
+    assert pa.pa_get_device_error() & pa.DEVERR_CONTEXT_LEN
+    assert torch.isnan(out[:12].float()).all()        # sequence 0 left unwritten
+    assert torch.isfinite(out[12:].float()).all()
