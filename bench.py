@@ -106,10 +106,13 @@ def make_workload(name, seed, device, block_size=None):
 # in profiles/).  Keyed by a hash of the kernel sources: once the kernels change,
 # the figure no longer describes them and the bench reports null.
 NCU_TRAFFIC = {
-    "f600580e5d5cd5e1": {
-        ("llama3_8b_decode_bf16", "append"): 292.742656e6 + 4.359424e6,
-        ("continuous_batching_mix_bf16_B16", "append"): 211.573248e6 + 4.276736e6,
-        ("llama3_70b_long_bf16", "splitk"): 2.519436e9 + 10.189568e6,
+    "c644f2dd4445b1a8": {
+        ("llama3_8b_decode_bf16", "append"): 292.741632e6 + 3.549696e6,
+        ("continuous_batching_mix_bf16_B16", "append"): 211.572992e6 + 4.641024e6,
+        ("llama3_70b_long_bf16", "splitk"): 2.519422e9 + 11.374080e6,
+        ("llama3_8b_decode_bf16+e4m3", "single"): 146.536448e6 + 4.014592e6,
+        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260378e9 + 6.991872e6,
+        ("chunked_prefill_bfloat16", "prefill"): 120.610560e6 + 6.072064e6,
     },
 }
 
@@ -544,7 +547,10 @@ def run_gpu(args, world, rank, local):
         e2e.pop("_local_bytes")
     clk = clocks.summary()
     peak, peak_kind = measured_peaks()
-    achieved = decode_bytes / (local_decode * 1e-3) / 1e9
+    # Shared-prefix blocks are read from HBM once per step however many
+    # sequences name them: the roofline counts them once.
+    roof_bytes = batch.algorithmic_bytes(unique=True) if fp8 is None else decode_bytes
+    achieved = roof_bytes / (local_decode * 1e-3) / 1e9
     value = total_bytes / (step_ms_max * 1e-3) / 1e9
     result = {
         "metric": METRIC,
@@ -603,7 +609,9 @@ def run_gpu(args, world, rank, local):
             "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
-            "algorithmic_bytes_per_launch": int(decode_bytes),
+            "algorithmic_bytes_per_launch": int(roof_bytes),
+            "bytes_basis": ("unique: shared-prefix blocks counted once" if roof_bytes != decode_bytes
+                            else "logical = unique"),
             "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get(
                 (batch.name + ("+e4m3" if fp8 is not None else ""), mode)),
         },
@@ -758,7 +766,8 @@ def run_prefill(args, world, rank, local):
                    "l2": "not flushed: compute-bound (the K/V of a sequence is reread by its query tiles)",
                    "mma": "mma.sync m16n8k16 bf16, fp32 accumulate"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "peak_kind": kind,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None},
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get((b.name, "prefill"))},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }
