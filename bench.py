@@ -291,7 +291,10 @@ class Step:
 
     def decode(self, stream):
         if self.fp8:
-            if self.mode in ("splitk", "splitk2"):
+            if self.mode == "append":
+                self.pa.pa_decode_append_fp8(self.out, self.q, self.nk, self.nv, self.k, self.v, self.ks, self.vs,
+                                             self.bt, self.cl, self.b.scale, max_context_len=self.mcl, stream=stream)
+            elif self.mode in ("splitk", "splitk2"):
                 self.pa.pa_decode_splitk_fp8(self.out, self.q, self.k, self.v, self.ks, self.vs, self.bt, self.cl,
                                              self.b.scale, self.mcl, partition_size=self.part, workspace=self.ws,
                                              fused=(self.mode == "splitk"), counters=self.counters, stream=stream)
@@ -338,8 +341,6 @@ def run_gpu(args, world, rank, local):
     fp8 = None
     if args.kv == "fp8":
         import workloads
-        if mode == "append":
-            mode = "single"   # the 8-bit pools' write is its own launch
         fp8 = workloads.random_fp8_pools(batch, seed=args.seed + rank, device="cuda")
     stream = torch.cuda.current_stream()
     l2 = l2_bytes()
@@ -577,7 +578,8 @@ def run_gpu(args, world, rank, local):
                               "append": "pa_decode_append"}.get(mode, "pa_decode")
                              if fp8 is None else
                              {"splitk": "pa_decode_splitk_fp8 (fused merge)",
-                              "splitk2": "pa_decode_splitk_fp8 (merge kernel)"}.get(mode, "pa_decode_fp8")),
+                              "splitk2": "pa_decode_splitk_fp8 (merge kernel)",
+                              "append": "pa_decode_append_fp8"}.get(mode, "pa_decode_fp8")),
             "kv_pool": ("e4m3 codes, one fp32 scale per kv head for K and for V (random codes)" if fp8 is not None
                         else "same type as the queries"),
             "partition_size": args.partition_size if mode.startswith("splitk") else None,
@@ -587,7 +589,10 @@ def run_gpu(args, world, rank, local):
                    f"CUDA-event region") if flush is None
             else "flushed between steps (256 MiB write), per-step CUDA events",
             "graph": bool(args.graph),
-            "step": ("pa_decode_append: newest token of every sequence written + decode, one launch" if mode == "append"
+            "step": ("pa_decode_append" + ("_fp8: newest token of every sequence quantised and written + decode, one "
+                                           "launch" if fp8 is not None else
+                                           ": newest token of every sequence written + decode, one launch")
+                     if mode == "append"
                      else "pa_reshape_and_cache_fp8 (newest token of every sequence, quantised) + decode"
                      if fp8 is not None
                      else "pa_reshape_and_cache (newest token of every sequence) + decode"),

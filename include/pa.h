@@ -283,6 +283,18 @@ pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const voi
                         int max_context_len, int64_t num_blocks, pa_dtype dtype,
                         const int32_t* seq_order, void* stream);
 
+/* pa_decode_append_fp8 — pa_decode_append over 8-bit pools: every sequence's
+ * newest token (key/value [num_seqs][num_kv_heads][head_dim] in dtype, 16-byte
+ * aligned) is quantised like pa_reshape_and_cache_fp8, written at position
+ * L-1 and attended to, in one launch; the result and every pool byte equal
+ * pa_reshape_and_cache_fp8 followed by pa_decode_fp8. */
+pa_status pa_decode_append_fp8(void* out, const void* q, const void* key, const void* value, void* k_cache,
+                               void* v_cache, const float* k_scale, const float* v_scale,
+                               const int32_t* block_tables, const int32_t* context_lens, float scale,
+                               int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                               const int32_t* seq_order, void* stream);
+
 /* pa_decode_splitk_fp8 — pa_decode_splitk over 8-bit pools (same workspace
  * size, counters and merge forms). */
 pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -23,7 +23,7 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT",
            "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
-           "pa_decode_splitk_fp8", "fp8_pool_shape", "pa_prefill"]
+           "pa_decode_splitk_fp8", "fp8_pool_shape", "pa_prefill", "pa_decode_append_fp8"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
     fp8_args = [P, P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I64, I]
     lib.pa_decode_fp8.restype = I
     lib.pa_decode_fp8.argtypes = fp8_args + [P, P]
+    lib.pa_decode_append_fp8.restype = I
+    lib.pa_decode_append_fp8.argtypes = [P, P, P, P] + fp8_args[2:] + [P, P]
     lib.pa_decode_splitk_fp8.restype = I
     lib.pa_decode_splitk_fp8.argtypes = fp8_args + [I, P, SZ, P, I64, P, P]
     lib.pa_prefill.restype = I
@@ -331,6 +333,17 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, cont
     lib = load()
     args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_fp8(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_fp8")
+
+
+def pa_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                         scale, max_context_len=None, stream=None, seq_order=None):
+    """One decode step over 8-bit pools: quantise and write each sequence's
+    newest token (key/value [S, Hkv, D]) at position context_lens[s]-1, then
+    attend over the whole context (one launch)."""
+    lib = load()
+    args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
+    _check(lib.pa_decode_append_fp8(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
+                                    _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_append_fp8")
 
 
 def pa_decode_splitk_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,

@@ -334,7 +334,8 @@ pa_status check_scales(const DecodeShape& sh, const float* k_scale, const float*
 template <bool FP8>
 pa_status decode_one_pass(void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
                           const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
-                          float scale, const DecodeShape& sh, const int32_t* seq_order, void* stream) {
+                          float scale, const DecodeShape& sh, const int32_t* seq_order, void* stream,
+                          const void* new_key = nullptr, const void* new_value = nullptr) {
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     if (st == PA_OK) st = check_scales<FP8>(sh, k_scale, v_scale);
     if (st != PA_OK || sh.num_seqs == 0) return st;
@@ -343,6 +344,8 @@ pa_status decode_one_pass(void* out, const void* q, const void* k_cache, const v
     p.seq_order = seq_order;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
+    p.new_key = new_key;
+    p.new_value = new_value;
     const dim3 grid(1, sh.num_kv_heads, sh.num_seqs);
     const cudaError_t e = decode_dispatch<false, FP8>(static_cast<pa_dtype>(sh.dtype), sh.head_dim, sh.block_size,
                                                       p, grid, static_cast<cudaStream_t>(stream));
@@ -545,6 +548,19 @@ pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const voi
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     return decode_one_pass<true>(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, sh,
                                  seq_order, stream);
+}
+
+pa_status pa_decode_append_fp8(void* out, const void* q, const void* key, const void* value, void* k_cache,
+                               void* v_cache, const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               const int32_t* context_lens, float scale, int block_size, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                               int max_context_len, int64_t num_blocks, pa_dtype dtype, const int32_t* seq_order,
+                               void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PA_ERR_INVALID_ARG;
+    return decode_one_pass<true>(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, sh,
+                                 seq_order, stream, key, value);
 }
 
 pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -101,6 +101,54 @@ __device__ __forceinline__ void append_newest_token(const DecodeParams& p, const
     __syncwarp();
 }
 
+// The same for 8-bit pools: lane 4j + w owns dims 16j + 2w, +1, +8, +9 of the
+// newest row, i.e. word w of K vector j and four bytes of four V dim rows.
+// The codes are computed when the row is loaded (the quantising write's
+// arithmetic) and stored into the staged tile and the pool like above.
+template <typename T, int D>
+struct NewRowE4m3 {
+    uint32_t kword = 0, vcodes = 0;  // vcodes: bytes of dims d0, d0+1, d0+8, d0+9
+    __device__ __forceinline__ void load_row(const DecodeParams& p, int s, int kvh, int lane) {
+        if (lane < D / 4) {
+            const int d0 = 16 * (lane >> 2) + 2 * (lane & 3);
+            const long long row = (static_cast<long long>(s) * p.num_kv_heads + kvh) * D;
+            const T* k = reinterpret_cast<const T*>(p.new_key) + row;
+            const T* v = reinterpret_cast<const T*>(p.new_value) + row;
+            const float ks = __ldg(p.k_scale + kvh), vs = __ldg(p.v_scale + kvh);
+            kword = quantise2(to_float<T>(k[d0]), to_float<T>(k[d0 + 1]), ks) |
+                    (quantise2(to_float<T>(k[d0 + 8]), to_float<T>(k[d0 + 9]), ks) << 16);
+            vcodes = quantise2(to_float<T>(v[d0]), to_float<T>(v[d0 + 1]), vs) |
+                     (quantise2(to_float<T>(v[d0 + 8]), to_float<T>(v[d0 + 9]), vs) << 16);
+        }
+    }
+};
+
+template <typename T, int D, int B>
+__device__ __forceinline__ void append_newest_token_e4m3(const DecodeParams& p, const NewRowE4m3<T, D>& nr,
+                                                         uint8_t* stage, int id, int kvh, int t, int lane) {
+    constexpr int kTile = B * D;
+    uint8_t* kpool = reinterpret_cast<uint8_t*>(const_cast<void*>(p.k_cache));
+    uint8_t* vpool = reinterpret_cast<uint8_t*>(const_cast<void*>(p.v_cache));
+    const long long tile = (static_cast<long long>(id) * p.num_kv_heads + kvh) * kTile;
+    if (lane < D / 4) {
+        const int j = lane >> 2, w = lane & 3;
+        const int d0 = 16 * j + 2 * w;
+        const int koff = ((j * B + t) * 4 + w) * 4;
+        *reinterpret_cast<uint32_t*>(stage + koff) = nr.kword;
+        *reinterpret_cast<uint32_t*>(kpool + tile + koff) = nr.kword;
+        const int at = v_row_byte(t, B);
+        const int dims[4] = {d0, d0 + 1, d0 + 8, d0 + 9};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint8_t code = static_cast<uint8_t>(nr.vcodes >> (8 * e));
+            stage[kTile + dims[e] * B + at] = code;
+            vpool[tile + dims[e] * B + at] = code;
+        }
+    }
+    fence_proxy_async_smem();  // the stage is refilled by bulk copies later
+    __syncwarp();
+}
+
 // Fused split-K merge, run by the CTA that completes the last partition of
 // (sequence s, kv head kvh): combines the np partial results of each of the
 // group's query heads in partition order with a running maximum (the
@@ -254,10 +302,13 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const int n_w = nb > warp ? (nb - warp + NW - 1) / NW : 0;
     // Append: the warp that will compute the last block loads the new row now.
     const int last_block = nblk - 1;
-    const bool owns_last = !FP8 && p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
+    const bool owns_last = p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
                            (last_block - b0) % NW == warp;
     NewRow<T, D> new_row;
-    if constexpr (!FP8) {
+    NewRowE4m3<T, D> new_row8;
+    if constexpr (FP8) {
+        if (owns_last) new_row8.load_row(p, s, kvh, lane);
+    } else {
         if (owns_last) new_row.load_row(p, s, kvh, lane);
     }
 
@@ -323,6 +374,8 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         const int valid = id < 0 ? 0 : min(B, L - j * B);
         uint8_t* stage = wring + st * 2 * kTile;
         if constexpr (FP8) {
+            if (owns_last && j == last_block && id >= 0)
+                append_newest_token_e4m3<T, D, B>(p, new_row8, stage, id, kvh, (L - 1) % B, lane);
             acc.template block<true>(smem_u32(stage), smem_u32(stage + kTile), valid, group, score_scale, lane);
         } else {
             if (owns_last && j == last_block && id >= 0)

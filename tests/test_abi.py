@@ -33,7 +33,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "pa_copy_blocks", "pa_decode", "pa_decode_append", "pa_decode_fp8", "pa_decode_splitk",
+        "pa_copy_blocks", "pa_decode", "pa_decode_append", "pa_decode_append_fp8", "pa_decode_fp8", "pa_decode_splitk",
         "pa_decode_splitk_fp8", "pa_decode_splitk_workspace_size", "pa_reshape_and_cache_fp8", "pa_prefill",
         "pa_decode_splitk_static", "pa_get_device_error",
         "pa_reshape_and_cache", "pa_status_string"])
@@ -112,6 +112,8 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_copy_blocks(*cp[:9], 0, *cp[10:]) == 1                            # empty source pool
     f8 = [16, 16, 16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 64]
     assert lib.pa_decode_fp8(*f8, 0, None, None) == 2                                # fp32 queries
+    assert lib.pa_decode_append_fp8(16, 16, 0, 16, *f8[2:], 2, None, None) == 1      # no new key
+    assert lib.pa_decode_append_fp8(16, 16, 16, 16, *f8[2:], 0, None, None) == 2     # fp32 queries
     assert lib.pa_decode_fp8(*f8[:4], 0, *f8[5:], 2, None, None) == 1                # no K scale
     assert lib.pa_decode_fp8(*f8[:5], 18, *f8[6:], 2, None, None) == 1               # V scale misaligned
     assert lib.pa_decode_splitk_fp8(*f8, 1, 500, 16, 1 << 20, None, 0, None, None) == 1  # partition not x16

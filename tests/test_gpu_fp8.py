@@ -174,3 +174,30 @@ def test_fp32_queries_are_refused():
     with pytest.raises(pa.PagedAttentionError) as e:
         _gpu_fp8_decode(b, pools, "single")
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("make", [
+    lambda: workloads.llama3_8b_decode(seed=1100, device="cuda", num_seqs=24, num_blocks=4096),
+    lambda: workloads.continuous_batching_mix(seed=1101, device="cuda", num_seqs=40, block_size=8),
+    lambda: workloads.random_small(seed=1102, dtype=torch.float16, lens=(0, 1, 16, 17, 300), num_q_heads=8,
+                                   num_kv_heads=2, head_dim=64, block_size=32),
+    lambda: workloads.random_small(seed=1103, dtype=torch.bfloat16, lens=(5, 33, 64, 2), num_q_heads=8,
+                                   num_kv_heads=8, head_dim=128, block_size=16),
+])
+def test_append_fp8_equals_write_then_decode(make):
+    b = make()
+    pools = workloads.random_fp8_pools(b, seed=1110, device="cuda")
+    q, bt, cl = b.q.cuda().contiguous(), b.block_tables.cuda(), b.context_lens.cuda()
+    nk, nv = b.new_key.cuda().contiguous(), b.new_value.cuda().contiguous()
+    k1, v1 = pools.k_cache.clone(), pools.v_cache.clone()
+    k2, v2 = pools.k_cache.clone(), pools.v_cache.clone()
+    ref = torch.full_like(q, float("nan"))
+    pa.pa_reshape_and_cache_fp8(nk, nv, k1, v1, b.slot_mapping.cuda(), pools.k_scale, pools.v_scale)
+    pa.pa_decode_fp8(ref, q, k1, v1, pools.k_scale, pools.v_scale, bt, cl, b.scale, max_context_len=b.max_context_len)
+    got = torch.full_like(q, float("nan"))
+    pa.pa_decode_append_fp8(got, q, nk, nv, k2, v2, pools.k_scale, pools.v_scale, bt, cl, b.scale,
+                            max_context_len=b.max_context_len)
+    torch.cuda.synchronize()
+    assert torch.equal(k2, k1) and torch.equal(v2, v1)
+    bits = lambda t: t.contiguous().view(-1).view(torch.int16)
+    assert torch.equal(bits(got), bits(ref))
