@@ -17,6 +17,7 @@
 #include "pa_copy.cuh"
 #include "pa_decode.cuh"
 #include "pa_prefill.cuh"
+#include "pa_prefill_tc.cuh"
 #include "pa_reshape.cuh"
 
 // Two CTA shapes for the decode kernels, measured on B200 over the benchmark
@@ -308,6 +309,22 @@ bool device_accessible(const void* p) {
 // Chunked prefill: 4 warps (64 MMA rows) per CTA, a 4-stage block ring.
 constexpr int kPrefillWarps = 4;
 constexpr int kPrefillStages = 4;
+
+// Blocks of 16 or 32 tokens run the 5th-generation tensor-core kernel
+// (128 MMA rows per CTA); 8-token blocks, or PA_PREFILL_TC=0, the warp-level one.
+#ifndef PA_PREFILL_TC
+#define PA_PREFILL_TC 1
+#endif
+
+template <typename T, int D, int B>
+cudaError_t launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t st) {
+    using Sm = pa::PrefillTcSmem<T, D, B>;
+    auto kernel = pa::pa_prefill_tc_kernel<T, D, B>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, 128, Sm::kTotal, st>>>(p);
+    return cudaGetLastError();
+}
 
 template <typename T, int D, int B>
 cudaError_t launch_prefill(const pa::PrefillParams& p, dim3 grid, cudaStream_t st) {
@@ -641,17 +658,21 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.context_cap = context_cap(sh);
     p.num_blocks = num_blocks;
-    p.tile_tokens = kPrefillWarps * 16 / p.group;
+    const bool use_tc = PA_PREFILL_TC && block_size != 8;
+    p.tile_tokens = (use_tc ? 128 : kPrefillWarps * 16) / p.group;
     const long long tiles = (static_cast<long long>(max_query_len) + p.tile_tokens - 1) / p.tile_tokens;
     if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
     const dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = with_variant(dtype, head_dim, block_size, [&](auto tt, auto dd, auto bb) -> cudaError_t {
         using T = typename decltype(tt)::type;
+        constexpr int kD = decltype(dd)::value, kB = decltype(bb)::value;
         if constexpr (pa::IsF32<T>::value) {
             return cudaErrorInvalidValue;
+        } else if constexpr (kB != 8) {
+            return use_tc ? launch_prefill_tc<T, kD, kB>(p, grid, s) : launch_prefill<T, kD, kB>(p, grid, s);
         } else {
-            return launch_prefill<T, decltype(dd)::value, decltype(bb)::value>(p, grid, s);
+            return launch_prefill<T, kD, kB>(p, grid, s);
         }
     });
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
