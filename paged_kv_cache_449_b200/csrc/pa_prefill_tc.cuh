@@ -55,6 +55,15 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uin
         ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
+// Same, with A (128 x 16) read from tensor memory: lane = row, 32-bit column c
+// = elements (2c, 2c+1) of the K step, low half first.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
 __device__ __forceinline__ void commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
@@ -78,6 +87,32 @@ __device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 columns of this warp's 32 lanes, without waiting (tcgen05.wait::ld follows).
+__device__ __forceinline__ void ld32_nowait(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void st32u(uint32_t taddr, const uint32_t (&w)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+          "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15]),
+          "r"(w[16]), "r"(w[17]), "r"(w[18]), "r"(w[19]), "r"(w[20]), "r"(w[21]), "r"(w[22]), "r"(w[23]),
+          "r"(w[24]), "r"(w[25]), "r"(w[26]), "r"(w[27]), "r"(w[28]), "r"(w[29]), "r"(w[30]), "r"(w[31])
+        : "memory");
+}
+
 __device__ __forceinline__ void st32(uint32_t taddr, const float (&v)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -98,44 +133,62 @@ __device__ __forceinline__ void st32(uint32_t taddr, const float (&v)[32]) {
 
 }  // namespace tc
 
-#ifndef PA_PREFILL_TC_KEYS
-#define PA_PREFILL_TC_KEYS 64
-#endif
-
+// One key tile per MMA round: 64 keys (4 blocks of 16 tokens or 2 of 32).
 template <typename T, int D, int B>
 struct PrefillTcSmem {
-    static constexpr int kKeys = PA_PREFILL_TC_KEYS;      // keys per tile
-    static constexpr int kBlocks = kKeys / B;             // blocks per tile
+    static constexpr int kKeys = 64;
+    static constexpr int kBlocks = kKeys / B;             // blocks per key tile
     static constexpr int kTile = B * D * 2;               // one (block, head) K or V tile
-    static constexpr int kStage = kBlocks * 2 * kTile;    // K and V of a key tile
+    static constexpr int kStage = kBlocks * 2 * kTile;    // K tiles, then V tiles
     static constexpr int kStages = 2;
-    static constexpr int kQ = 128 * D * 2;
-    static constexpr int kP = 128 * kKeys * 2;
-    static constexpr int kRingOff = 0;
-    static constexpr int kQOff = kStages * kStage;
-    static constexpr int kPOff = kQOff + kQ;
-    static constexpr int kBarOff = kPOff + kP;
-    static constexpr int kTotal = kBarOff + 8 * 8 + 16;
+    static constexpr int kP = 128 * kKeys * 2;            // one P buffer (16-bit)
+    static constexpr int kPOff = kStages * kStage;
+    static constexpr int kBarOff = kPOff + 2 * kP;
+    static constexpr int kNumBars = 11;
+    static constexpr int kMiscOff = kBarOff + 12 * 8;     // tmem base, blk_ok[2], abort
+    static constexpr int kTotal = kMiscOff + 16;
 };
 
+// Bounded mbarrier wait that also gives up when another role of the CTA has
+// raised `abort` (a timed-out wait raises it and flags PA_DEVERR_TIMEOUT).
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t start = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) return false;
+        if (global_timer_ns() - start > kWaitLimitNs) {
+            *abort = 1u;
+            flag_error(8 /* PA_DEVERR_TIMEOUT */);
+            return false;
+        }
+    }
+    return true;
+}
+
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(128) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
     using Sm = PrefillTcSmem<T, D, B>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
-    // S: kKeys columns, then O: D columns (allocations are powers of two)
-    constexpr uint32_t kTmemCols = kKeys + D <= 128 ? 128 : (kKeys + D <= 256 ? 256 : 512);
+    // tensor memory columns: S [0, 64), O [64, 64 + D), Q (packed pairs) [64 + D, 64 + 3D/2)
+    constexpr uint32_t kTmemCols = 256;
+    constexpr uint32_t kOCol = kKeys, kQCol = kKeys + D;
+    static_assert(kQCol + D / 2 <= kTmemCols, "tensor memory budget");
     static_assert(B == 16 || B == 32, "16- or 32-token blocks");
     static_assert(D == 64 || D == 128, "head dims");
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Sm::kBarOff);   // [2]
-    uint64_t* empty = full + 2;                                         // [2]
-    uint64_t* s_done = full + 4;
-    uint64_t* o_done = full + 5;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 8);
-    uint8_t* qs = smem + Sm::kQOff;
-    uint8_t* ps = smem + Sm::kPOff;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBarOff);
+    uint64_t* kv_full = bars;        // [2] copies of a key tile landed
+    uint64_t* kv_empty = bars + 2;   // [2] its O += P V finished
+    uint64_t* s_full = bars + 4;     // S = Q K^T finished
+    uint64_t* s_free = bars + 5;     // the softmax warps have read S
+    uint64_t* p_full = bars + 6;     // [2] P written (and O rescaled)
+    uint64_t* p_free = bars + 8;     // [2] the O += P V reading that P finished
+    uint64_t* drain = bars + 10;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Sm::kMiscOff);
+    uint32_t* blk_ok = misc + 1;     // [2] bit b: block b of the staged tile was fetched
+    volatile uint32_t* abort = misc + 3;
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
     const int group = p.group;
 
@@ -151,71 +204,50 @@ __global__ void __launch_bounds__(128) pa_prefill_tc_kernel(const __grid_constan
     const int tok1 = min(Q, tok0 + p.tile_tokens);
     const int last_pos = L - Q + tok1 - 1;
     const int nblk = last_pos / B + 1;                   // blocks the tile needs
-    const int ntiles = (nblk + kBlocks - 1) / kBlocks;  // key tiles
+    const int ntiles = (nblk + kBlocks - 1) / kBlocks;  // key tiles (>= 1)
 
-    // ---- this thread's row
-    const int row_tok = tok0 + tid / group;
-    const int row_head = kvh * group + tid % group;
-    const bool row_ok = row_tok < tok1;
-    const int row_pos = row_ok ? L - Q + row_tok : -1;
-
-    // ---- Q row into the K-major core-matrix layout: (8-row group g, 8-dim chunk c) at c*2048 + g*128
-    {
-        const T* qrow = reinterpret_cast<const T*>(p.q) +
-                        (static_cast<long long>(q0 + (row_ok ? row_tok : tok0)) * p.num_q_heads + row_head) * D;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qrow + 8 * c) : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(qs + c * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) = v;
-        }
-    }
-    if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        mbar_init(s_done, 1);
-        mbar_init(o_done, 1);
+    if (tid == 128) {
+        mbar_init(&kv_full[0], 1);
+        mbar_init(&kv_full[1], 1);
+        mbar_init(&kv_empty[0], 1);
+        mbar_init(&kv_empty[1], 1);
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
+        mbar_init(&p_full[0], 128);
+        mbar_init(&p_full[1], 128);
+        mbar_init(&p_free[0], 1);
+        mbar_init(&p_free[1], 1);
+        mbar_init(drain, 1);
+        *abort = 0u;
         fence_barrier_init();
     }
-    fence_proxy_async_smem();  // Q (generic stores) visible to the tensor cores
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+    if (warp == 4) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t s_tmem = tmem;            // columns 0 .. kKeys-1
-    const uint32_t o_tmem = tmem + kKeys;    // columns kKeys .. kKeys+D-1
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    {   // O starts at zero, so every O += P V accumulates
-        float z[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = 0.f;
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) tc::st32(o_tmem + lane_base + c0, z);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-    }
+    const uint32_t tmem = misc[0];
+    const uint32_t s_tmem = tmem, o_tmem = tmem + kOCol, q_tmem = tmem + kQCol;
 
     // ---- producer: key tile j (its blocks) into stage j % 2
     const int32_t* table = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq;
-    const char* kpool = reinterpret_cast<const char*>(p.k_cache);
-    const char* vpool = reinterpret_cast<const char*>(p.v_cache);
-    const uint64_t policy = l2_evict_first_policy();
-    __shared__ uint32_t blk_ok[2];  // bit b: block b of the staged tile was fetched
-    auto issue = [&](int j) {       // thread 0
+    auto issue = [&](int j) {
         const int st = j & 1;
         uint8_t* base = smem + st * Sm::kStage;
+        const char* kpool = reinterpret_cast<const char*>(p.k_cache);
+        const char* vpool = reinterpret_cast<const char*>(p.v_cache);
+        const uint64_t policy = l2_evict_first_policy();
         uint32_t ok = 0;
         int bytes = 0;
+        int ids[kBlocks];
         for (int b = 0; b < kBlocks; ++b) {
             const int jb = j * kBlocks + b;
-            if (jb >= nblk) break;
-            const int id = __ldg(table + jb);
-            if (id >= 0 && static_cast<long long>(id) < p.num_blocks) {
+            ids[b] = jb < nblk ? __ldg(table + jb) : -1;
+            if (jb >= nblk) continue;
+            if (ids[b] >= 0 && static_cast<long long>(ids[b]) < p.num_blocks) {
                 ok |= 1u << b;
                 bytes += 2 * kTile;
             } else {
@@ -223,195 +255,254 @@ __global__ void __launch_bounds__(128) pa_prefill_tc_kernel(const __grid_constan
             }
         }
         blk_ok[st] = ok;
-        mbar_arrive_expect_tx(&full[st], bytes);
+        mbar_arrive_expect_tx(&kv_full[st], bytes);
         for (int b = 0; b < kBlocks; ++b) {
             if (!(ok >> b & 1u)) continue;
-            const int id = __ldg(table + j * kBlocks + b);
-            const long long off = (static_cast<long long>(id) * p.num_kv_heads + kvh) * kTile;
-            bulk_copy_g2s(base + b * kTile, kpool + off, kTile, &full[st], policy);
-            bulk_copy_g2s(base + (kBlocks + b) * kTile, vpool + off, kTile, &full[st], policy);
+            const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
+            bulk_copy_g2s(base + b * kTile, kpool + off, kTile, &kv_full[st], policy);
+            bulk_copy_g2s(base + (kBlocks + b) * kTile, vpool + off, kTile, &kv_full[st], policy);
         }
     };
-    if (tid == 0) {
+    int issued = 0;
+    if (tid == 160) {
         issue(0);
-        if (ntiles > 1) issue(1);
+        issued = 1;
+        if (ntiles > 1) {
+            issue(1);
+            issued = 2;
+        }
     }
 
-    const float scale = p.score_scale;
-    float m_run = kNegInf, l_run = 0.f;
+    // ---- softmax warps: Q row into tensor memory (pairs packed per 32-bit column), O = 0
+    const int row_tok = tok0 + tid / group;
+    const int row_head = kvh * group + tid % group;
+    const bool row_ok = tid < 128 && row_tok < tok1;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    if (tid < 128) {
+        const T* qrow = reinterpret_cast<const T*>(p.q) +
+                        (static_cast<long long>(q0 + (row_ok ? row_tok : tok0)) * p.num_q_heads + row_head) * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qrow + 2 * c0 + 8 * i) : make_uint4(0, 0, 0, 0);
+                w[4 * i] = v.x;
+                w[4 * i + 1] = v.y;
+                w[4 * i + 2] = v.z;
+                w[4 * i + 3] = v.w;
+            }
+            tc::st32u(q_tmem + lane_base + c0, w);
+        }
+        float z[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) tc::st32(o_tmem + lane_base + c0, z);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+
     bool failed = false;
-    int j = 0;
-    for (; j < ntiles; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait_bounded(&full[st], ph, kWaitLimitNs)) failed = true;
-        if (__syncthreads_or(failed ? 1 : 0)) {
-            failed = true;
-            break;
-        }
-        const uint32_t ok = blk_ok[st];
-        uint8_t* kbase = smem + st * Sm::kStage;
-        uint8_t* vbase = kbase + kBlocks * kTile;
-        const int key0 = j * kKeys;
-
-        // zero V rows of tokens at or past the context in the tile's last needed block
-        {
-            const int lb = (L - 1) / B - j * kBlocks;   // block of the last context token, in this tile
-            if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
-                const int t_from = (L - 1) % B + 1;     // first token past the context in that block
-                for (int i = tid; i < (B - t_from) * (D / 8); i += 128) {
-                    const int t = t_from + i / (D / 8), c = i % (D / 8);
-                    *reinterpret_cast<uint4*>(vbase + lb * kTile + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
-                }
-                fence_proxy_async_smem();
+    if (warp == 5) {
+        // ---------------- producer
+        if (lane == 0) {
+            for (int j = 2; j < ntiles; ++j) {
+                if (!tc_wait(&kv_empty[j & 1], ((j >> 1) - 1) & 1, abort)) break;
+                issue(j);
+                issued = j + 1;
             }
+            // no copy may still be landing when the CTA leaves
+            for (int k = issued > 2 ? issued - 2 : 0; k < issued; ++k)
+                mbar_wait_bounded(&kv_full[k & 1], (k >> 1) & 1, kWaitLimitNs);
         }
-        tc::fence_before();
-        __syncthreads();
-
-        // S = Q K^T (one MMA per block and 16-dim step)
-        if (tid == 0) {
-            tc::fence_after();
+    } else if (warp == 4) {
+        // ---------------- MMA issue (one thread)
+        if (lane == 0) {
             const uint32_t idesc_s = tc::instr_desc<T>(B, false);
-            for (int b = 0; b < kBlocks; ++b) {
-                if (!((ok >> b) & 1u)) continue;
-                const uint32_t kb = smem_u32(kbase + b * kTile);
+            const uint32_t idesc_o = tc::instr_desc<T>(D, true);
+            auto mma_s = [&](int j) {   // S = Q K^T: one MMA per block and 16-dim step, A from tensor memory
+                const uint32_t ok = blk_ok[j & 1];
+                const uint32_t kbase = smem_u32(smem + (j & 1) * Sm::kStage);
+                for (int b = 0; b < kBlocks; ++b) {
+                    if (!((ok >> b) & 1u)) continue;
 #pragma unroll
-                for (int kc = 0; kc < D / 16; ++kc) {
-                    const uint64_t a = tc::smem_desc(smem_u32(qs) + 2 * kc * 2048, 2048, 128);
-                    const uint64_t bd = tc::smem_desc(kb + 2 * kc * B * 16, B * 16, 128);
-                    tc::mma(s_tmem + b * B, a, bd, idesc_s, kc > 0);
+                    for (int kc = 0; kc < D / 16; ++kc)
+                        tc::mma_ts(s_tmem + b * B, q_tmem + kc * 8,
+                                   tc::smem_desc(kbase + b * kTile + 2 * kc * B * 16, B * 16, 128), idesc_s, kc > 0);
+                }
+                tc::commit(s_full);
+            };
+            bool ok_run = tc_wait(&kv_full[0], 0, abort);
+            if (ok_run) {
+                tc::fence_after();
+                mma_s(0);
+            }
+            for (int j = 0; ok_run && j < ntiles; ++j) {
+                const int st = j & 1;
+                if (j + 1 < ntiles) {
+                    if (!tc_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort) || !tc_wait(s_free, j & 1, abort))
+                        break;
+                    tc::fence_after();
+                    mma_s(j + 1);
+                }
+                if (!tc_wait(&p_full[st], (j >> 1) & 1, abort)) break;
+                tc::fence_after();
+                // O += P V: one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
+                const uint32_t ok = blk_ok[st];
+                const uint32_t vbase = smem_u32(smem + st * Sm::kStage + kBlocks * kTile);
+                const uint32_t pbase = smem_u32(smem + Sm::kPOff + st * Sm::kP);
+                for (int b = 0; b < kBlocks; ++b) {
+                    if (!((ok >> b) & 1u)) continue;
+#pragma unroll
+                    for (int ks = 0; ks < B / 16; ++ks) {
+                        const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
+                        tc::mma(o_tmem, tc::smem_desc(pbase + kc * 2048, 2048, 128),
+                                tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
+                    }
+                }
+                tc::commit(&p_free[st]);
+                tc::commit(&kv_empty[st]);
+            }
+            // every MMA this thread issued has finished before the CTA tears down
+            tc::commit(drain);
+            mbar_wait_bounded(drain, 0, kWaitLimitNs);
+        }
+    } else {
+        // ---------------- softmax (thread = row = tensor-memory lane)
+        const float scale = p.score_scale;
+        const int row_pos = row_ok ? L - Q + row_tok : -1;
+        const uint32_t all_blocks = (1u << kBlocks) - 1u;
+        float m_run = kNegInf, l_run = 0.f;
+        for (int j = 0; j < ntiles; ++j) {
+            const int st = j & 1;
+            if (!__all_sync(0xffffffffu, tc_wait(s_full, j & 1, abort))) {
+                failed = true;
+                break;
+            }
+            tc::fence_after();
+            float sv[kKeys];
+#pragma unroll
+            for (int c0 = 0; c0 < kKeys; c0 += 32) tc::ld32_nowait(s_tmem + lane_base + c0, sv + c0);
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
+            // the staged tile's block mask (and, below, its V tiles)
+            if (!__all_sync(0xffffffffu, tc_wait(&kv_full[st], (j >> 1) & 1, abort))) {
+                failed = true;
+                break;
+            }
+            const uint32_t ok = blk_ok[st];
+            const int key0 = j * kKeys;
+            float mx = kNegInf;
+            if (ok == all_blocks && key0 + kKeys - 1 <= row_pos) {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, sv[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < kKeys; ++c) {
+                    const bool vis = ((ok >> (c / B)) & 1u) && key0 + c <= row_pos;
+                    sv[c] = vis ? sv[c] : kNegInf;
+                    mx = fmaxf(mx, sv[c]);
                 }
             }
-            tc::commit(s_done);
-        }
-        if (!mbar_wait_bounded(s_done, j & 1, kWaitLimitNs)) failed = true;
-        tc::fence_after();
-
-        // online softmax over this thread's row of S (held in registers)
-        float sv[kKeys];
-        float mx = kNegInf;
-#pragma unroll
-        for (int c0 = 0; c0 < kKeys; c0 += 32) {
-            float v[32];
-            tc::ld32(s_tmem + lane_base + c0, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int col = c0 + i;
-                const bool vis = ((ok >> (col / B)) & 1u) && key0 + col <= row_pos;
-                sv[col] = vis ? v[i] * scale : kNegInf;
-                mx = fmaxf(mx, sv[col]);
+            mx *= scale;   // base-2 domain (scale > 0)
+            // The reference maximum moves only when a score exceeds it by more
+            // than 2^8: P stays <= 256 and O is rescaled far less often (l and
+            // O share the reference, so the result is the same softmax).
+            const float m_old = m_run;
+            m_run = (m_old == kNegInf || mx > m_old + 8.f) ? fmaxf(m_old, mx) : m_old;
+            const float mu = m_run == kNegInf ? 0.f : m_run;
+            const float alpha = exp2_approx(m_old - mu);
+            // P buffer st was last read by the O += P V of tile j - 2
+            if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&p_free[st], ((j >> 1) - 1) & 1, abort))) {
+                failed = true;
+                break;
             }
-        }
-        // The reference maximum moves only when a score exceeds it by more than
-        // 2^8 (base 2): P stays <= 256, exact for the sums, and O is rescaled
-        // far less often (l and O share the reference, so the result is the
-        // same softmax).
-#ifndef PA_PREFILL_TC_SLACK
-#define PA_PREFILL_TC_SLACK 8.f
-#endif
-        const float mn = (m_run == kNegInf || mx > m_run + PA_PREFILL_TC_SLACK) ? fmaxf(m_run, mx) : m_run;
-        const float mu = mn == kNegInf ? 0.f : mn;
-        const float alpha = exp2_approx(m_run - mu);
-        m_run = mn;
-        // the previous O += P V must be done before P is rewritten and O rescaled
-        if (j > 0 && !mbar_wait_bounded(o_done, (j - 1) & 1, kWaitLimitNs)) failed = true;
-        tc::fence_after();
-        float rs = 0.f;
+            uint8_t* ps = smem + Sm::kPOff + st * Sm::kP;
+            float rs = 0.f;
 #pragma unroll
-        for (int k8 = 0; k8 < kKeys / 8; ++k8) {
-            uint32_t w[4];
+            for (int k8 = 0; k8 < kKeys / 8; ++k8) {
+                uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a0 = exp2_approx(sv[8 * k8 + 2 * e] - mu);
-                const float a1 = exp2_approx(sv[8 * k8 + 2 * e + 1] - mu);
-                rs += a0 + a1;
-                w[e] = Mma<T>::pack(a0, a1);
+                for (int e = 0; e < 4; ++e) {
+                    const float a0 = exp2_approx(fmaf(sv[8 * k8 + 2 * e], scale, -mu));
+                    const float a1 = exp2_approx(fmaf(sv[8 * k8 + 2 * e + 1], scale, -mu));
+                    rs += a0 + a1;
+                    w[e] = Mma<T>::pack(a0, a1);
+                }
+                // (8-row group, 8-key chunk k8) core matrix at k8*2048 + g*128
+                *reinterpret_cast<uint4*>(ps + k8 * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
-            // P row, 8 keys per 16-byte core-matrix row: (8-row group, 8-key chunk k8) at k8*2048 + g*128
-            *reinterpret_cast<uint4*>(ps + k8 * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            l_run = l_run * alpha + rs;
+            // tokens at or past the context in the tile's last needed block: zero
+            // their staged V rows (P is 0 there, but 0 times a stale non-finite
+            // value would not be)
+            {
+                const int lb = (L - 1) / B - j * kBlocks;
+                if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
+                    uint8_t* vt = smem + st * Sm::kStage + (kBlocks + lb) * kTile;
+                    const int t_from = (L - 1) % B + 1;
+                    for (int i = tid; i < (B - t_from) * (D / 8); i += 128) {
+                        const int t = t_from + i / (D / 8), c = i % (D / 8);
+                        *reinterpret_cast<uint4*>(vt + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
+            // rescale this row of O (after the previous O += P V), unless no
+            // row of the warp moved its reference
+            if (!__all_sync(0xffffffffu, m_old == kNegInf || alpha == 1.f)) {
+                if (!__all_sync(0xffffffffu, tc_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort))) {
+                    failed = true;
+                    break;
+                }
+                tc::fence_after();
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float v[32];
+                    tc::ld32(o_tmem + lane_base + c0, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= alpha;
+                    tc::st32(o_tmem + lane_base + c0, v);
+                }
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            }
+            fence_proxy_async_smem();   // P and zeroed V rows visible to the tensor cores
+            tc::fence_before();
+            mbar_arrive(&p_full[st]);
         }
-        l_run = l_run * alpha + rs;
-        // rescale this row of O, unless no row of the warp changed its maximum
-        if (!__all_sync(0xffffffffu, alpha == 1.f)) {
+        // ---- the last O += P V, then this row of the output
+        if (!failed && !__all_sync(0xffffffffu, tc_wait(&p_free[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort)))
+            failed = true;
+        if (!failed && !*abort) {
+            tc::fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            T* dst = reinterpret_cast<T*>(p.out) +
+                     (static_cast<long long>(q0 + (row_ok ? row_tok : tok0)) * p.num_q_heads + row_head) * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 float v[32];
-                tc::ld32(o_tmem + lane_base + c0, v);
+                tc::ld32(o_tmem + lane_base + c0, v);   // collective per warp: every row takes part
+                if (row_ok) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                tc::st32(o_tmem + lane_base + c0, v);
-            }
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        }
-        fence_proxy_async_smem();  // P (generic stores) visible to the tensor cores
-        tc::fence_before();
-        if (__syncthreads_or(failed ? 1 : 0)) {
-            failed = true;
-            break;
-        }
-
-        // O += P V (one MMA per block and 16-key step); then the stage is free
-        if (tid == 0) {
-            tc::fence_after();
-            const uint32_t idesc_o = tc::instr_desc<T>(D, true);
-            for (int b = 0; b < kBlocks; ++b) {
-                if (!((ok >> b) & 1u)) continue;
-                const uint32_t vb = smem_u32(vbase + b * kTile);
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        uint32_t w[4];
 #pragma unroll
-                for (int ks = 0; ks < B / 16; ++ks) {
-                    const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
-                    const uint64_t a = tc::smem_desc(smem_u32(ps) + kc * 2048, 2048, 128);
-                    const uint64_t bd = tc::smem_desc(vb + ks * 2 * 128, 128, B * 16);
-                    tc::mma(o_tmem, a, bd, idesc_o, true);
-                }
-            }
-            tc::commit(o_done);
-            tc::commit(&empty[st]);
-            if (j + 2 < ntiles) {
-                if (mbar_wait_bounded(&empty[st], (j >> 1) & 1, kWaitLimitNs)) {
-                    issue(j + 2);
-                } else {
-                    failed = true;
-                }
-            }
-        }
-    }
-
-    // ---- drain, write the rows, release tensor memory
-    if (!failed && ntiles > 0 && !mbar_wait_bounded(o_done, (ntiles - 1) & 1, kWaitLimitNs)) failed = true;
-    if (__syncthreads_or(failed ? 1 : 0)) {
-        if (tid == 0) {
-            flag_error(8 /* PA_DEVERR_TIMEOUT */);
-            // let the tensor-core work and copies already issued finish before the CTA exits
-            mbar_wait_bounded(o_done, (j > 0 ? j - 1 : 0) & 1, kWaitLimitNs);
-            for (int k = j; k < ntiles && k < j + 2; ++k) mbar_wait_bounded(&full[k & 1], (k >> 1) & 1, kWaitLimitNs);
-        }
-    } else {
-        tc::fence_after();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        T* dst = reinterpret_cast<T*>(p.out) +
-                 (static_cast<long long>(q0 + (row_ok ? row_tok : tok0)) * p.num_q_heads + row_head) * D;
-        float v[32];
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            tc::ld32(o_tmem + lane_base + c0, v);   // collective per warp: every row takes part
-            if (row_ok) {
-#pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        w[e] = Mma<T>::pack(v[8 * k8 + 2 * e] * inv, v[8 * k8 + 2 * e + 1] * inv);
-                    *reinterpret_cast<uint4*>(dst + c0 + 8 * k8) = make_uint4(w[0], w[1], w[2], w[3]);
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = Mma<T>::pack(v[8 * k8 + 2 * e] * inv, v[8 * k8 + 2 * e + 1] * inv);
+                        *reinterpret_cast<uint4*>(dst + c0 + 8 * k8) = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
                 }
             }
         }
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 4) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
