@@ -322,7 +322,7 @@ cudaError_t launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_
     auto kernel = pa::pa_prefill_tc_kernel<T, D, B>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, 192, Sm::kTotal, st>>>(p);
+    kernel<<<grid, 224, Sm::kTotal, st>>>(p);
     return cudaGetLastError();
 }
 

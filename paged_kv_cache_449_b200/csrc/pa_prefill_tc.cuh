@@ -134,19 +134,24 @@ __device__ __forceinline__ void st32(uint32_t taddr, const float (&v)[32]) {
 }  // namespace tc
 
 // One key tile per MMA round: 64 keys (4 blocks of 16 tokens or 2 of 32).
+// K and V tiles have rings of their own: a K stage is free once its S MMAs
+// finish, a V stage once its O += P V finishes, so K is fetched further ahead.
 template <typename T, int D, int B>
 struct PrefillTcSmem {
     static constexpr int kKeys = 64;
     static constexpr int kBlocks = kKeys / B;             // blocks per key tile
     static constexpr int kTile = B * D * 2;               // one (block, head) K or V tile
-    static constexpr int kStage = kBlocks * 2 * kTile;    // K tiles, then V tiles
-    static constexpr int kStages = 2;
+    static constexpr int kStage = kBlocks * kTile;        // the K (or V) tiles of one key tile
+    static constexpr int kKStages = D == 128 ? 3 : 4;
+    static constexpr int kVStages = D == 128 ? 2 : 3;
     static constexpr int kP = 128 * kKeys * 2;            // one P buffer (16-bit)
-    static constexpr int kPOff = kStages * kStage;
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKStages * kStage;
+    static constexpr int kPOff = kVOff + kVStages * kStage;
     static constexpr int kBarOff = kPOff + 2 * kP;
-    static constexpr int kNumBars = 11;
-    static constexpr int kMiscOff = kBarOff + 12 * 8;     // tmem base, blk_ok[2], abort
+    static constexpr int kMiscOff = kBarOff + 32 * 8;     // tmem base, abort
     static constexpr int kTotal = kMiscOff + 16;
+    static_assert(2 * (kTotal + 1024) <= 233472, "two CTAs per SM");
 };
 
 // Bounded mbarrier wait that also gives up when another role of the CTA has
@@ -166,9 +171,10 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
     using Sm = PrefillTcSmem<T, D, B>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
+    constexpr int KS = Sm::kKStages, VS = Sm::kVStages;
     // tensor memory columns: S [0, 64), O [64, 64 + D), Q (packed pairs) [64 + D, 64 + 3D/2)
     constexpr uint32_t kTmemCols = 256;
     constexpr uint32_t kOCol = kKeys, kQCol = kKeys + D;
@@ -177,16 +183,17 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
     static_assert(D == 64 || D == 128, "head dims");
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBarOff);
-    uint64_t* kv_full = bars;        // [2] copies of a key tile landed
-    uint64_t* kv_empty = bars + 2;   // [2] its O += P V finished
-    uint64_t* s_full = bars + 4;     // S = Q K^T finished
-    uint64_t* s_free = bars + 5;     // the softmax warps have read S
-    uint64_t* p_full = bars + 6;     // [2] P written (and O rescaled)
-    uint64_t* p_free = bars + 8;     // [2] the O += P V reading that P finished
-    uint64_t* drain = bars + 10;
+    uint64_t* k_full = bars;         // [KS] K tiles of a key tile landed
+    uint64_t* k_empty = bars + 4;    // [KS] their S MMAs finished
+    uint64_t* v_full = bars + 8;     // [VS] V tiles landed
+    uint64_t* v_empty = bars + 12;   // [VS] their O += P V finished
+    uint64_t* s_full = bars + 16;    // S = Q K^T finished
+    uint64_t* s_free = bars + 17;    // the softmax warps have read S
+    uint64_t* p_full = bars + 18;    // [2] P written (and O rescaled)
+    uint64_t* p_free = bars + 20;    // [2] the O += P V reading that P finished
+    uint64_t* drain = bars + 22;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Sm::kMiscOff);
-    uint32_t* blk_ok = misc + 1;     // [2] bit b: block b of the staged tile was fetched
-    volatile uint32_t* abort = misc + 3;
+    volatile uint32_t* abort = misc + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
@@ -207,16 +214,20 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
     const int ntiles = (nblk + kBlocks - 1) / kBlocks;  // key tiles (>= 1)
 
     if (tid == 128) {
-        mbar_init(&kv_full[0], 1);
-        mbar_init(&kv_full[1], 1);
-        mbar_init(&kv_empty[0], 1);
-        mbar_init(&kv_empty[1], 1);
+        for (int i = 0; i < KS; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < VS; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
         mbar_init(s_full, 1);
         mbar_init(s_free, 4);
-        mbar_init(&p_full[0], 128);
-        mbar_init(&p_full[1], 128);
-        mbar_init(&p_free[0], 1);
-        mbar_init(&p_free[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&p_full[i], 128);
+            mbar_init(&p_free[i], 1);
+        }
         mbar_init(drain, 1);
         *abort = 0u;
         fence_barrier_init();
@@ -232,44 +243,59 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
     const uint32_t tmem = misc[0];
     const uint32_t s_tmem = tmem, o_tmem = tmem + kOCol, q_tmem = tmem + kQCol;
 
-    // ---- producer: key tile j (its blocks) into stage j % 2
+    // ---- block ids of key tile j, and which of them may be fetched (every role
+    //      derives the same mask from the table)
     const int32_t* table = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq;
-    auto issue = [&](int j) {
-        const int st = j & 1;
-        uint8_t* base = smem + st * Sm::kStage;
-        const char* kpool = reinterpret_cast<const char*>(p.k_cache);
-        const char* vpool = reinterpret_cast<const char*>(p.v_cache);
-        const uint64_t policy = l2_evict_first_policy();
-        uint32_t ok = 0;
-        int bytes = 0;
-        int ids[kBlocks];
+    auto load_ids = [&](int j, int (&ids)[kBlocks]) {
+#pragma unroll
         for (int b = 0; b < kBlocks; ++b) {
             const int jb = j * kBlocks + b;
-            ids[b] = jb < nblk ? __ldg(table + jb) : -1;
-            if (jb >= nblk) continue;
-            if (ids[b] >= 0 && static_cast<long long>(ids[b]) < p.num_blocks) {
-                ok |= 1u << b;
-                bytes += 2 * kTile;
-            } else {
-                flag_error(1 /* PA_DEVERR_BLOCK_ID */);
-            }
-        }
-        blk_ok[st] = ok;
-        mbar_arrive_expect_tx(&kv_full[st], bytes);
-        for (int b = 0; b < kBlocks; ++b) {
-            if (!(ok >> b & 1u)) continue;
-            const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
-            bulk_copy_g2s(base + b * kTile, kpool + off, kTile, &kv_full[st], policy);
-            bulk_copy_g2s(base + (kBlocks + b) * kTile, vpool + off, kTile, &kv_full[st], policy);
+            ids[b] = (j < ntiles && jb < nblk) ? __ldg(table + jb) : -1;
         }
     };
+    auto ok_of = [&](const int (&ids)[kBlocks]) {
+        uint32_t ok = 0;
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b)
+            if (ids[b] >= 0 && static_cast<long long>(ids[b]) < p.num_blocks) ok |= 1u << b;
+        return ok;
+    };
+
+    // ---- producers: warp 5 lane 0 fetches K tiles, warp 6 lane 0 V tiles
+    const bool is_producer = (warp == 5 || warp == 6) && lane == 0;
+    const bool v_side = warp == 6;
+    const char* pool = reinterpret_cast<const char*>(v_side ? p.v_cache : p.k_cache);
+    uint64_t* full = v_side ? v_full : k_full;
+    uint64_t* empty = v_side ? v_empty : k_empty;
+    const int nst = v_side ? VS : KS;
+    uint8_t* ring = smem + (v_side ? Sm::kVOff : Sm::kKOff);
+    int ids[kBlocks], nxt[kBlocks];
     int issued = 0;
-    if (tid == 160) {
-        issue(0);
-        issued = 1;
-        if (ntiles > 1) {
-            issue(1);
-            issued = 2;
+    auto produce = [&](int j) {   // copies of key tile j (ids in `ids`) into stage j % nst
+        const int st = j % nst;
+        const uint32_t ok = ok_of(ids);
+        if (!v_side) {
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b)
+                if (j * kBlocks + b < nblk && !((ok >> b) & 1u)) flag_error(1 /* PA_DEVERR_BLOCK_ID */);
+        }
+        mbar_arrive_expect_tx(&full[st], __popc(ok) * kTile);
+        const uint64_t policy = l2_evict_first_policy();
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {
+            if (!((ok >> b) & 1u)) continue;
+            const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
+            bulk_copy_g2s(ring + st * Sm::kStage + b * kTile, pool + off, kTile, &full[st], policy);
+        }
+        issued = j + 1;
+    };
+    if (is_producer) {
+        load_ids(0, ids);
+        for (int j = 0; j < nst && j < ntiles; ++j) {
+            load_ids(j + 1, nxt);
+            produce(j);
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) ids[b] = nxt[b];
         }
     }
 
@@ -306,56 +332,81 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
     tc::fence_after();
 
     bool failed = false;
-    if (warp == 5) {
-        // ---------------- producer
-        if (lane == 0) {
-            for (int j = 2; j < ntiles; ++j) {
-                if (!tc_wait(&kv_empty[j & 1], ((j >> 1) - 1) & 1, abort)) break;
-                issue(j);
-                issued = j + 1;
+    if (warp == 5 || warp == 6) {
+        // ---------------- producers
+        if (is_producer) {
+            for (int j = nst; j < ntiles; ++j) {
+                load_ids(j + 1, nxt);   // the next tile's ids load while this one waits for its stage
+                if (!tc_wait(&empty[j % nst], ((j / nst) - 1) & 1, abort)) break;
+                produce(j);
+#pragma unroll
+                for (int b = 0; b < kBlocks; ++b) ids[b] = nxt[b];
             }
             // no copy may still be landing when the CTA leaves
-            for (int k = issued > 2 ? issued - 2 : 0; k < issued; ++k)
-                mbar_wait_bounded(&kv_full[k & 1], (k >> 1) & 1, kWaitLimitNs);
+            for (int k = issued > nst ? issued - nst : 0; k < issued; ++k)
+                mbar_wait_bounded(&full[k % nst], (k / nst) & 1, kWaitLimitNs);
         }
     } else if (warp == 4) {
-        // ---------------- MMA issue (one thread)
-        if (lane == 0) {
-            const uint32_t idesc_s = tc::instr_desc<T>(B, false);
-            const uint32_t idesc_o = tc::instr_desc<T>(D, true);
-            auto mma_s = [&](int j) {   // S = Q K^T: one MMA per block and 16-dim step, A from tensor memory
-                const uint32_t ok = blk_ok[j & 1];
-                const uint32_t kbase = smem_u32(smem + (j & 1) * Sm::kStage);
-                for (int b = 0; b < kBlocks; ++b) {
-                    if (!((ok >> b) & 1u)) continue;
+        // ---------------- MMA warp: lane 0 issues, the warp zeroes V rows past the context
+        const uint32_t idesc_s = tc::instr_desc<T>(B, false);
+        const uint32_t idesc_o = tc::instr_desc<T>(D, true);
+        const uint32_t k_ring = smem_u32(smem + Sm::kKOff), v_ring = smem_u32(smem + Sm::kVOff);
+        int id_a[kBlocks], id_b[kBlocks];
+        load_ids(0, id_a);
+        load_ids(1, id_b);
+        uint32_t ok_cur = ok_of(id_a), ok_next = ok_of(id_b);
+        auto mma_s = [&](int j, uint32_t ok) {   // S = Q K^T: one MMA per block and 16-dim step, A in tensor memory
+            const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
+            for (int b = 0; b < kBlocks; ++b) {
+                if (!((ok >> b) & 1u)) continue;
 #pragma unroll
-                    for (int kc = 0; kc < D / 16; ++kc)
-                        tc::mma_ts(s_tmem + b * B, q_tmem + kc * 8,
-                                   tc::smem_desc(kbase + b * kTile + 2 * kc * B * 16, B * 16, 128), idesc_s, kc > 0);
-                }
-                tc::commit(s_full);
-            };
-            bool ok_run = tc_wait(&kv_full[0], 0, abort);
-            if (ok_run) {
-                tc::fence_after();
-                mma_s(0);
+                for (int kc = 0; kc < D / 16; ++kc)
+                    tc::mma_ts(s_tmem + b * B, q_tmem + kc * 8,
+                               tc::smem_desc(kbase + b * kTile + 2 * kc * B * 16, B * 16, 128), idesc_s, kc > 0);
             }
-            for (int j = 0; ok_run && j < ntiles; ++j) {
-                const int st = j & 1;
-                if (j + 1 < ntiles) {
-                    if (!tc_wait(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort) || !tc_wait(s_free, j & 1, abort))
-                        break;
+            tc::commit(s_full);
+            tc::commit(&k_empty[j % KS]);
+        };
+        bool run = __all_sync(0xffffffffu, tc_wait(&k_full[0], 0, abort));
+        if (run && lane == 0) {
+            tc::fence_after();
+            mma_s(0, ok_cur);
+        }
+        for (int j = 0; run && j < ntiles; ++j) {
+            load_ids(j + 2, id_a);
+            if (j + 1 < ntiles) {
+                if (!__all_sync(0xffffffffu, tc_wait(&k_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort) &&
+                                                 tc_wait(s_free, j & 1, abort)))
+                    break;
+                if (lane == 0) {
                     tc::fence_after();
-                    mma_s(j + 1);
+                    mma_s(j + 1, ok_next);
                 }
-                if (!tc_wait(&p_full[st], (j >> 1) & 1, abort)) break;
+            }
+            const int vst = j % VS;
+            if (!__all_sync(0xffffffffu, tc_wait(&v_full[vst], (j / VS) & 1, abort))) break;
+            // tokens at or past the context in the tile's last needed block: zero their
+            // staged V rows (P is 0 there, but 0 times a stale non-finite value would not be)
+            uint8_t* vring = smem + Sm::kVOff + vst * Sm::kStage;
+            const int lb = (L - 1) / B - j * kBlocks;
+            if (lb >= 0 && lb < kBlocks && ((ok_cur >> lb) & 1u)) {
+                const int t_from = (L - 1) % B + 1;
+                for (int i = lane; i < (B - t_from) * (D / 8); i += 32) {
+                    const int t = t_from + i / (D / 8), c = i % (D / 8);
+                    *reinterpret_cast<uint4*>(vring + lb * kTile + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            const int st = j & 1;
+            if (!__all_sync(0xffffffffu, tc_wait(&p_full[st], (j >> 1) & 1, abort))) break;
+            if (lane == 0) {
                 tc::fence_after();
                 // O += P V: one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
-                const uint32_t ok = blk_ok[st];
-                const uint32_t vbase = smem_u32(smem + st * Sm::kStage + kBlocks * kTile);
+                const uint32_t vbase = v_ring + vst * Sm::kStage;
                 const uint32_t pbase = smem_u32(smem + Sm::kPOff + st * Sm::kP);
                 for (int b = 0; b < kBlocks; ++b) {
-                    if (!((ok >> b) & 1u)) continue;
+                    if (!((ok_cur >> b) & 1u)) continue;
 #pragma unroll
                     for (int ks = 0; ks < B / 16; ++ks) {
                         const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
@@ -364,20 +415,29 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
                     }
                 }
                 tc::commit(&p_free[st]);
-                tc::commit(&kv_empty[st]);
+                tc::commit(&v_empty[vst]);
             }
-            // every MMA this thread issued has finished before the CTA tears down
+            ok_cur = ok_next;
+            ok_next = ok_of(id_a);
+        }
+        // every MMA lane 0 issued has finished before the CTA tears down
+        if (lane == 0) {
             tc::commit(drain);
             mbar_wait_bounded(drain, 0, kWaitLimitNs);
         }
+        __syncwarp();
     } else {
         // ---------------- softmax (thread = row = tensor-memory lane)
         const float scale = p.score_scale;
         const int row_pos = row_ok ? L - Q + row_tok : -1;
         const uint32_t all_blocks = (1u << kBlocks) - 1u;
+        int id_n[kBlocks];
+        load_ids(0, id_n);
+        uint32_t ok = ok_of(id_n);
         float m_run = kNegInf, l_run = 0.f;
         for (int j = 0; j < ntiles; ++j) {
             const int st = j & 1;
+            load_ids(j + 1, id_n);
             if (!__all_sync(0xffffffffu, tc_wait(s_full, j & 1, abort))) {
                 failed = true;
                 break;
@@ -390,12 +450,6 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
             tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free);
-            // the staged tile's block mask (and, below, its V tiles)
-            if (!__all_sync(0xffffffffu, tc_wait(&kv_full[st], (j >> 1) & 1, abort))) {
-                failed = true;
-                break;
-            }
-            const uint32_t ok = blk_ok[st];
             const int key0 = j * kKeys;
             float mx = kNegInf;
             if (ok == all_blocks && key0 + kKeys - 1 <= row_pos) {
@@ -439,20 +493,6 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
             l_run = l_run * alpha + rs;
-            // tokens at or past the context in the tile's last needed block: zero
-            // their staged V rows (P is 0 there, but 0 times a stale non-finite
-            // value would not be)
-            {
-                const int lb = (L - 1) / B - j * kBlocks;
-                if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
-                    uint8_t* vt = smem + st * Sm::kStage + (kBlocks + lb) * kTile;
-                    const int t_from = (L - 1) % B + 1;
-                    for (int i = tid; i < (B - t_from) * (D / 8); i += 128) {
-                        const int t = t_from + i / (D / 8), c = i % (D / 8);
-                        *reinterpret_cast<uint4*>(vt + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
-                    }
-                }
-            }
             // rescale this row of O (after the previous O += P V), unless no
             // row of the warp moved its reference
             if (!__all_sync(0xffffffffu, m_old == kNegInf || alpha == 1.f)) {
@@ -471,9 +511,10 @@ __global__ void __launch_bounds__(192, 2) pa_prefill_tc_kernel(const __grid_cons
                 }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             }
-            fence_proxy_async_smem();   // P and zeroed V rows visible to the tensor cores
+            fence_proxy_async_smem();   // P visible to the tensor cores
             tc::fence_before();
             mbar_arrive(&p_full[st]);
+            ok = ok_of(id_n);
         }
         // ---- the last O += P V, then this row of the output
         if (!failed && !__all_sync(0xffffffffu, tc_wait(&p_free[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort)))
