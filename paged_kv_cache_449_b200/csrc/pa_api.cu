@@ -3,7 +3,9 @@
 // Nothing here allocates device memory or synchronises, except
 // pa_get_device_error which synchronises the given stream by contract.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <atomic>
 #include <climits>
@@ -316,13 +318,47 @@ constexpr int kPrefillStages = 4;
 #define PA_PREFILL_TC 1
 #endif
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (the library links no driver library); null where there is no driver.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// The K pool viewed as a 2-D tensor of rows (block, kv head, 8-dim chunk), each
+// row the chunk's B tokens x 8 elements (B * 16 bytes), one row per box: the
+// operand of the prefill kernel's gather4 loads.  False when it cannot be
+// described (no driver, or more rows than a 32-bit coordinate reaches).
+bool encode_k_rows(CUtensorMap* map, const void* k_cache, pa_dtype dt, int B, int D, int Hkv, long long num_blocks) {
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) return false;
+    const long long rows = num_blocks * Hkv * (D / 8);
+    if (rows <= 0 || rows > INT_MAX) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(B) * 8, static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(B) * 16};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(B) * 8, 1};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    const CUtensorMapDataType type =
+        dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return encode(map, type, 2, const_cast<void*>(k_cache), dims, strides, box, elem_strides,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int B>
-cudaError_t launch_prefill_tc(const pa::PrefillParams& p, dim3 grid, cudaStream_t st) {
+cudaError_t launch_prefill_tc(const pa::PrefillParams& p, const CUtensorMap& k_rows, dim3 grid, cudaStream_t st) {
     using Sm = pa::PrefillTcSmem<T, D, B>;
     auto kernel = pa::pa_prefill_tc_kernel<T, D, B>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, 224, Sm::kTotal, st>>>(p);
+    kernel<<<grid, 224, Sm::kTotal, st>>>(p, k_rows);
     return cudaGetLastError();
 }
 
@@ -658,7 +694,9 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.context_cap = context_cap(sh);
     p.num_blocks = num_blocks;
-    const bool use_tc = PA_PREFILL_TC && block_size != 8;
+    CUtensorMap k_rows{};
+    const bool use_tc = PA_PREFILL_TC && block_size != 8 &&
+                        encode_k_rows(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks);
     p.tile_tokens = (use_tc ? 128 : kPrefillWarps * 16) / p.group;
     const long long tiles = (static_cast<long long>(max_query_len) + p.tile_tokens - 1) / p.tile_tokens;
     if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
@@ -670,7 +708,7 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
         if constexpr (pa::IsF32<T>::value) {
             return cudaErrorInvalidValue;
         } else if constexpr (kB != 8) {
-            return use_tc ? launch_prefill_tc<T, kD, kB>(p, grid, s) : launch_prefill<T, kD, kB>(p, grid, s);
+            return use_tc ? launch_prefill_tc<T, kD, kB>(p, k_rows, grid, s) : launch_prefill<T, kD, kB>(p, grid, s);
         } else {
             return launch_prefill<T, kD, kB>(p, grid, s);
         }

@@ -25,6 +25,8 @@
 //    path.
 #pragma once
 
+#include <cuda.h>
+
 #include <type_traits>
 
 #include "pa_device.cuh"
@@ -131,11 +133,34 @@ __device__ __forceinline__ void st32(uint32_t taddr, const float (&v)[32]) {
         : "memory");
 }
 
+// Four rows of a 2-D tensor (row coordinates r0..r3, columns from `col`, one
+// box wide) into consecutive shared memory; completion counted on `bar`.
+__device__ __forceinline__ void gather4(void* dst, const CUtensorMap* map, int col, int r0, int r1, int r2, int r3,
+                                        uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Global -> shared bulk copy with the default L2 policy (prefill rereads a
+// sequence's tiles once per query tile, so they should stay in L2).
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 }  // namespace tc
 
 // One key tile per MMA round: 64 keys (4 blocks of 16 tokens or 2 of 32).
 // K and V tiles have rings of their own: a K stage is free once its S MMAs
 // finish, a V stage once its O += P V finishes, so K is fetched further ahead.
+// A K stage holds the tile chunk-major, [D/8][64 keys][8], gathered from the
+// pool's (block, head) tiles by tile::gather4 loads (one 8-dim chunk of four
+// blocks per load), so that one N = 64 MMA covers all of the tile's keys.
 template <typename T, int D, int B>
 struct PrefillTcSmem {
     static constexpr int kKeys = 64;
@@ -171,7 +196,8 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
+                                                                const __grid_constant__ CUtensorMap k_rows) {
     using Sm = PrefillTcSmem<T, D, B>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
     constexpr int KS = Sm::kKStages, VS = Sm::kVStages;
@@ -212,6 +238,11 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
     const int last_pos = L - Q + tok1 - 1;
     const int nblk = last_pos / B + 1;                   // blocks the tile needs
     const int ntiles = (nblk + kBlocks - 1) / kBlocks;  // key tiles (>= 1)
+    // tensor copies land on 128-byte boundaries (the dynamic window starts on one)
+    if (smem_u32(smem) & 127u) {
+        if (tid == 0) flag_error(8 /* PA_DEVERR_TIMEOUT: nothing fetched */);
+        return;
+    }
 
     if (tid == 128) {
         for (int i = 0; i < KS; ++i) {
@@ -264,7 +295,7 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
     // ---- producers: warp 5 lane 0 fetches K tiles, warp 6 lane 0 V tiles
     const bool is_producer = (warp == 5 || warp == 6) && lane == 0;
     const bool v_side = warp == 6;
-    const char* pool = reinterpret_cast<const char*>(v_side ? p.v_cache : p.k_cache);
+    const char* pool = reinterpret_cast<const char*>(p.v_cache);
     uint64_t* full = v_side ? v_full : k_full;
     uint64_t* empty = v_side ? v_empty : k_empty;
     const int nst = v_side ? VS : KS;
@@ -274,18 +305,45 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
     auto produce = [&](int j) {   // copies of key tile j (ids in `ids`) into stage j % nst
         const int st = j % nst;
         const uint32_t ok = ok_of(ids);
+        uint8_t* dst = ring + st * Sm::kStage;
         if (!v_side) {
 #pragma unroll
             for (int b = 0; b < kBlocks; ++b)
                 if (j * kBlocks + b < nblk && !((ok >> b) & 1u)) flag_error(1 /* PA_DEVERR_BLOCK_ID */);
-        }
-        mbar_arrive_expect_tx(&full[st], __popc(ok) * kTile);
-        const uint64_t policy = l2_evict_first_policy();
+            if (ok == 0u) {
+                mbar_arrive_expect_tx(&full[st], 0);   // nothing to fetch: every key is masked
+            } else {
+                // refused ids and blocks past the tile's need read a fetched block instead
+                // (their scores are masked); row (id, head, chunk c) of the 2-D view
+                int rid[kBlocks];
+                int sub = ids[kBlocks - 1];
 #pragma unroll
-        for (int b = 0; b < kBlocks; ++b) {
-            if (!((ok >> b) & 1u)) continue;
-            const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
-            bulk_copy_g2s(ring + st * Sm::kStage + b * kTile, pool + off, kTile, &full[st], policy);
+                for (int b = kBlocks - 1; b >= 0; --b)
+                    if ((ok >> b) & 1u) sub = ids[b];   // the first fetched block
+#pragma unroll
+                for (int b = 0; b < kBlocks; ++b)
+                    rid[b] = ((((ok >> b) & 1u) ? ids[b] : sub) * p.num_kv_heads + kvh) * (D / 8);
+                mbar_arrive_expect_tx(&full[st], Sm::kStage);
+                if constexpr (B == 16) {
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c)
+                        tc::gather4(dst + c * 1024, &k_rows, 0, rid[0] + c, rid[1] + c, rid[2] + c, rid[3] + c,
+                                    &full[st]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < D / 8; c += 2)
+                        tc::gather4(dst + c * 1024, &k_rows, 0, rid[0] + c, rid[1] + c, rid[0] + c + 1,
+                                    rid[1] + c + 1, &full[st]);
+                }
+            }
+        } else {
+            mbar_arrive_expect_tx(&full[st], __popc(ok) * kTile);
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) {
+                if (!((ok >> b) & 1u)) continue;
+                const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
+                tc::bulk_copy(dst + b * kTile, pool + off, kTile, &full[st]);
+            }
         }
         issued = j + 1;
     };
@@ -348,21 +406,20 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
         }
     } else if (warp == 4) {
         // ---------------- MMA warp: lane 0 issues, the warp zeroes V rows past the context
-        const uint32_t idesc_s = tc::instr_desc<T>(B, false);
+        const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
         const uint32_t idesc_o = tc::instr_desc<T>(D, true);
         const uint32_t k_ring = smem_u32(smem + Sm::kKOff), v_ring = smem_u32(smem + Sm::kVOff);
         int id_a[kBlocks], id_b[kBlocks];
         load_ids(0, id_a);
         load_ids(1, id_b);
         uint32_t ok_cur = ok_of(id_a), ok_next = ok_of(id_b);
-        auto mma_s = [&](int j, uint32_t ok) {   // S = Q K^T: one MMA per block and 16-dim step, A in tensor memory
+        auto mma_s = [&](int j, uint32_t ok) {   // S = Q K^T: one N = 64 MMA per 16-dim step, A in tensor memory
             const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
-            for (int b = 0; b < kBlocks; ++b) {
-                if (!((ok >> b) & 1u)) continue;
+            if (ok != 0u) {
 #pragma unroll
                 for (int kc = 0; kc < D / 16; ++kc)
-                    tc::mma_ts(s_tmem + b * B, q_tmem + kc * 8,
-                               tc::smem_desc(kbase + b * kTile + 2 * kc * B * 16, B * 16, 128), idesc_s, kc > 0);
+                    tc::mma_ts(s_tmem, q_tmem + kc * 8, tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128), idesc_s,
+                               kc > 0);
             }
             tc::commit(s_full);
             tc::commit(&k_empty[j % KS]);
