@@ -153,6 +153,27 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
+// Packed pairs of fp32 (one 64-bit register pair): fused multiply-add and add
+// on both halves in one instruction.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 }  // namespace tc
 
 // One key tile per MMA round: 64 keys (4 blocks of 16 tokens or 2 of 32).
@@ -508,18 +529,23 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free);
             const int key0 = j * kKeys;
-            float mx = kNegInf;
+            // row maximum over eight independent partial maxima (no 64-long chain)
+            float m8[8];
             if (ok == all_blocks && key0 + kKeys - 1 <= row_pos) {
 #pragma unroll
-                for (int c = 0; c < kKeys; ++c) mx = fmaxf(mx, sv[c]);
+                for (int c = 0; c < 8; ++c) m8[c] = sv[c];
+#pragma unroll
+                for (int c = 8; c < kKeys; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
             } else {
 #pragma unroll
                 for (int c = 0; c < kKeys; ++c) {
                     const bool vis = ((ok >> (c / B)) & 1u) && key0 + c <= row_pos;
                     sv[c] = vis ? sv[c] : kNegInf;
-                    mx = fmaxf(mx, sv[c]);
+                    m8[c & 7] = c < 8 ? sv[c] : fmaxf(m8[c & 7], sv[c]);
                 }
             }
+            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             mx *= scale;   // base-2 domain (scale > 0)
             // The reference maximum moves only when a score exceeds it by more
             // than 2^8: P stays <= 256 and O is rescaled far less often (l and
@@ -534,20 +560,33 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
                 break;
             }
             uint8_t* ps = smem + Sm::kPOff + st * Sm::kP;
-            float rs = 0.f;
+            // P = 2^(s * scale - mu): arguments and row sums two at a time, the
+            // sums in four independent pairs
+            const uint64_t scale2 = tc::f2(scale, scale), nmu2 = tc::f2(-mu, -mu);
+            uint64_t acc[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[e] = tc::f2(0.f, 0.f);
 #pragma unroll
             for (int k8 = 0; k8 < kKeys / 8; ++k8) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float a0 = exp2_approx(fmaf(sv[8 * k8 + 2 * e], scale, -mu));
-                    const float a1 = exp2_approx(fmaf(sv[8 * k8 + 2 * e + 1], scale, -mu));
-                    rs += a0 + a1;
+                    float x0, x1;
+                    tc::f2_split(tc::fma2(tc::f2(sv[8 * k8 + 2 * e], sv[8 * k8 + 2 * e + 1]), scale2, nmu2), x0, x1);
+                    const float a0 = exp2_approx(x0), a1 = exp2_approx(x1);
+                    acc[e] = tc::add2(acc[e], tc::f2(a0, a1));
                     w[e] = Mma<T>::pack(a0, a1);
                 }
                 // (8-row group, 8-key chunk k8) core matrix at k8*2048 + g*128
                 *reinterpret_cast<uint4*>(ps + k8 * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
                     make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            float rs;
+            {
+                float r[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) tc::f2_split(acc[e], r[2 * e], r[2 * e + 1]);
+                rs = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
             }
             l_run = l_run * alpha + rs;
             // rescale this row of O (after the previous O += P V), unless no
