@@ -188,8 +188,14 @@ struct PrefillTcSmem {
     static constexpr int kBlocks = kKeys / B;             // blocks per key tile
     static constexpr int kTile = B * D * 2;               // one (block, head) K or V tile
     static constexpr int kStage = kBlocks * kTile;        // the K (or V) tiles of one key tile
-    static constexpr int kKStages = D == 128 ? 3 : 4;
-    static constexpr int kVStages = D == 128 ? 2 : 3;
+#ifndef PA_PF_KSTAGES
+#define PA_PF_KSTAGES 2
+#endif
+#ifndef PA_PF_VSTAGES
+#define PA_PF_VSTAGES 3
+#endif
+    static constexpr int kKStages = D == 128 ? PA_PF_KSTAGES : PA_PF_KSTAGES + 1;
+    static constexpr int kVStages = D == 128 ? PA_PF_VSTAGES : PA_PF_VSTAGES + 1;
     static constexpr int kP = 128 * kKeys * 2;            // one P buffer (16-bit)
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKStages * kStage;
@@ -217,7 +223,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
+__global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
                                                                 const __grid_constant__ CUtensorMap k_rows) {
     using Sm = PrefillTcSmem<T, D, B>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
@@ -238,7 +244,7 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
     uint64_t* s_free = bars + 17;    // the softmax warps have read S
     uint64_t* p_full = bars + 18;    // [2] P written (and O rescaled)
     uint64_t* p_free = bars + 20;    // [2] the O += P V reading that P finished
-    uint64_t* drain = bars + 22;
+    uint64_t* drain = bars + 22;     // [2] the S and the O += P V issuers' MMAs finished
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Sm::kMiscOff);
     volatile uint32_t* abort = misc + 1;
 
@@ -280,7 +286,8 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
             mbar_init(&p_full[i], 128);
             mbar_init(&p_free[i], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort = 0u;
         fence_barrier_init();
     }
@@ -426,52 +433,53 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
                 mbar_wait_bounded(&full[k % nst], (k / nst) & 1, kWaitLimitNs);
         }
     } else if (warp == 4) {
-        // ---------------- MMA warp: lane 0 issues, the warp zeroes V rows past the context
-        const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
-        const uint32_t idesc_o = tc::instr_desc<T>(D, true);
-        const uint32_t k_ring = smem_u32(smem + Sm::kKOff), v_ring = smem_u32(smem + Sm::kVOff);
-        int id_a[kBlocks], id_b[kBlocks];
-        load_ids(0, id_a);
-        load_ids(1, id_b);
-        uint32_t ok_cur = ok_of(id_a), ok_next = ok_of(id_b);
-        auto mma_s = [&](int j, uint32_t ok) {   // S = Q K^T: one N = 64 MMA per 16-dim step, A in tensor memory
-            const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
-            if (ok != 0u) {
+        // ---------------- S = Q K^T issue (lane 0): one N = 64 MMA per 16-dim step, A in tensor memory
+        if (lane == 0) {
+            const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
+            const uint32_t k_ring = smem_u32(smem + Sm::kKOff);
+            int id_n[kBlocks];
+            load_ids(0, id_n);
+            for (int j = 0; j < ntiles; ++j) {
+                const uint32_t ok = ok_of(id_n);
+                load_ids(j + 1, id_n);
+                // S(j) overwrites S(j - 1): the softmax warps must have read it
+                if (j > 0 && !tc_wait(s_free, (j - 1) & 1, abort)) break;
+                if (!tc_wait(&k_full[j % KS], (j / KS) & 1, abort)) break;
+                tc::fence_after();
+                const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
+                if (ok != 0u) {
 #pragma unroll
-                for (int kc = 0; kc < D / 16; ++kc)
-                    tc::mma_ts(s_tmem, q_tmem + kc * 8, tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128), idesc_s,
-                               kc > 0);
-            }
-            tc::commit(s_full);
-            tc::commit(&k_empty[j % KS]);
-        };
-        bool run = __all_sync(0xffffffffu, tc_wait(&k_full[0], 0, abort));
-        if (run && lane == 0) {
-            tc::fence_after();
-            mma_s(0, ok_cur);
-        }
-        for (int j = 0; run && j < ntiles; ++j) {
-            load_ids(j + 2, id_a);
-            if (j + 1 < ntiles) {
-                if (!__all_sync(0xffffffffu, tc_wait(&k_full[(j + 1) % KS], ((j + 1) / KS) & 1, abort) &&
-                                                 tc_wait(s_free, j & 1, abort)))
-                    break;
-                if (lane == 0) {
-                    tc::fence_after();
-                    mma_s(j + 1, ok_next);
+                    for (int kc = 0; kc < D / 16; ++kc)
+                        tc::mma_ts(s_tmem, q_tmem + kc * 8, tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128),
+                                   idesc_s, kc > 0);
                 }
+                tc::commit(s_full);
+                tc::commit(&k_empty[j % KS]);
             }
+            // every MMA this thread issued has finished before the CTA tears down
+            tc::commit(&drain[0]);
+            mbar_wait_bounded(&drain[0], 0, kWaitLimitNs);
+        }
+    } else if (warp == 7) {
+        // ---------------- O += P V issue (lane 0); the warp zeroes V rows past the context
+        const uint32_t idesc_o = tc::instr_desc<T>(D, true);
+        const uint32_t v_ring = smem_u32(smem + Sm::kVOff);
+        int id_n[kBlocks];
+        load_ids(0, id_n);
+        for (int j = 0; j < ntiles; ++j) {
+            const uint32_t ok = ok_of(id_n);
+            load_ids(j + 1, id_n);
             const int vst = j % VS;
             if (!__all_sync(0xffffffffu, tc_wait(&v_full[vst], (j / VS) & 1, abort))) break;
             // tokens at or past the context in the tile's last needed block: zero their
             // staged V rows (P is 0 there, but 0 times a stale non-finite value would not be)
-            uint8_t* vring = smem + Sm::kVOff + vst * Sm::kStage;
             const int lb = (L - 1) / B - j * kBlocks;
-            if (lb >= 0 && lb < kBlocks && ((ok_cur >> lb) & 1u)) {
+            if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
+                uint8_t* vt = smem + Sm::kVOff + vst * Sm::kStage + lb * kTile;
                 const int t_from = (L - 1) % B + 1;
                 for (int i = lane; i < (B - t_from) * (D / 8); i += 32) {
                     const int t = t_from + i / (D / 8), c = i % (D / 8);
-                    *reinterpret_cast<uint4*>(vring + lb * kTile + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(vt + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -480,11 +488,11 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
             if (!__all_sync(0xffffffffu, tc_wait(&p_full[st], (j >> 1) & 1, abort))) break;
             if (lane == 0) {
                 tc::fence_after();
-                // O += P V: one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
+                // one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
                 const uint32_t vbase = v_ring + vst * Sm::kStage;
                 const uint32_t pbase = smem_u32(smem + Sm::kPOff + st * Sm::kP);
                 for (int b = 0; b < kBlocks; ++b) {
-                    if (!((ok_cur >> b) & 1u)) continue;
+                    if (!((ok >> b) & 1u)) continue;
 #pragma unroll
                     for (int ks = 0; ks < B / 16; ++ks) {
                         const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
@@ -495,13 +503,10 @@ __global__ void __launch_bounds__(224, 2) pa_prefill_tc_kernel(const __grid_cons
                 tc::commit(&p_free[st]);
                 tc::commit(&v_empty[vst]);
             }
-            ok_cur = ok_next;
-            ok_next = ok_of(id_a);
         }
-        // every MMA lane 0 issued has finished before the CTA tears down
         if (lane == 0) {
-            tc::commit(drain);
-            mbar_wait_bounded(drain, 0, kWaitLimitNs);
+            tc::commit(&drain[1]);
+            mbar_wait_bounded(&drain[1], 0, kWaitLimitNs);
         }
         __syncwarp();
     } else {
