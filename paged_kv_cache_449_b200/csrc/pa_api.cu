@@ -358,7 +358,7 @@ cudaError_t launch_prefill_tc(const pa::PrefillParams& p, const CUtensorMap& k_r
     auto kernel = pa::pa_prefill_tc_kernel<T, D, B>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, 256, Sm::kTotal, st>>>(p, k_rows);
+    kernel<<<grid, 384, Sm::kTotal, st>>>(p, k_rows);
     return cudaGetLastError();
 }
 
@@ -698,7 +698,9 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     const bool use_tc = PA_PREFILL_TC && block_size != 8 &&
                         encode_k_rows(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks);
     p.tile_tokens = (use_tc ? 128 : kPrefillWarps * 16) / p.group;
-    const long long tiles = (static_cast<long long>(max_query_len) + p.tile_tokens - 1) / p.tile_tokens;
+    // the tensor-core kernel takes two query tiles per CTA
+    const long long per_cta = use_tc ? 2LL * p.tile_tokens : p.tile_tokens;
+    const long long tiles = (static_cast<long long>(max_query_len) + per_cta - 1) / per_cta;
     if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
     const dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -176,34 +176,34 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 
 }  // namespace tc
 
+// One CTA per SM holds two tiles of 128 query rows (two consecutive tiles of
+// the same sequence and kv head) that share every K and V tile it fetches.
 // One key tile per MMA round: 64 keys (4 blocks of 16 tokens or 2 of 32).
-// K and V tiles have rings of their own: a K stage is free once its S MMAs
-// finish, a V stage once its O += P V finishes, so K is fetched further ahead.
-// A K stage holds the tile chunk-major, [D/8][64 keys][8], gathered from the
-// pool's (block, head) tiles by tile::gather4 loads (one 8-dim chunk of four
-// blocks per load), so that one N = 64 MMA covers all of the tile's keys.
+// K and V tiles have rings of their own: a K stage is free once the S MMAs
+// of both query tiles finish, a V stage once both O += P V finish.  A K stage
+// holds the tile chunk-major, [D/8][64 keys][8], gathered from the pool's
+// (block, head) tiles by tile::gather4 loads (one 8-dim chunk of four blocks
+// per load), so that one N = 64 MMA covers all of the tile's keys.
 template <typename T, int D, int B>
 struct PrefillTcSmem {
     static constexpr int kKeys = 64;
     static constexpr int kBlocks = kKeys / B;             // blocks per key tile
     static constexpr int kTile = B * D * 2;               // one (block, head) K or V tile
     static constexpr int kStage = kBlocks * kTile;        // the K (or V) tiles of one key tile
-#ifndef PA_PF_KSTAGES
-#define PA_PF_KSTAGES 2
+#ifndef PA_PF_STAGES
+#define PA_PF_STAGES 4
 #endif
-#ifndef PA_PF_VSTAGES
-#define PA_PF_VSTAGES 3
-#endif
-    static constexpr int kKStages = D == 128 ? PA_PF_KSTAGES : PA_PF_KSTAGES + 1;
-    static constexpr int kVStages = D == 128 ? PA_PF_VSTAGES : PA_PF_VSTAGES + 1;
+    static constexpr int kKStages = D == 128 ? PA_PF_STAGES : PA_PF_STAGES + 2;
+    static constexpr int kVStages = kKStages;
     static constexpr int kP = 128 * kKeys * 2;            // one P buffer (16-bit)
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKStages * kStage;
-    static constexpr int kPOff = kVOff + kVStages * kStage;
-    static constexpr int kBarOff = kPOff + 2 * kP;
-    static constexpr int kMiscOff = kBarOff + 32 * 8;     // tmem base, abort
+    static constexpr int kPOff = kVOff + kVStages * kStage;   // [query tile][2 buffers]
+    static constexpr int kBarOff = kPOff + 4 * kP;
+    static constexpr int kMiscOff = kBarOff + 48 * 8;     // tmem base, abort
     static constexpr int kTotal = kMiscOff + 16;
-    static_assert(2 * (kTotal + 1024) <= 233472, "two CTAs per SM");
+    static_assert(kTotal <= 232448, "shared memory per CTA");
+    static_assert(kKStages <= 6, "barrier slots");
 };
 
 // Bounded mbarrier wait that also gives up when another role of the CTA has
@@ -222,76 +222,84 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
     return true;
 }
 
+// Warps 0-3 and 4-7: softmax of query tile 0 and 1 (thread = row = tensor-memory
+// lane); warp 8 issues S = Q K^T, warp 9 O += P V; warps 10 and 11 fetch K and V.
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
+__global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
                                                                 const __grid_constant__ CUtensorMap k_rows) {
     using Sm = PrefillTcSmem<T, D, B>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
     constexpr int KS = Sm::kKStages, VS = Sm::kVStages;
-    // tensor memory columns: S [0, 64), O [64, 64 + D), Q (packed pairs) [64 + D, 64 + 3D/2)
-    constexpr uint32_t kTmemCols = 256;
+    // tensor memory, per query tile q (256 columns at q * 256): S [0, 64),
+    // O [64, 64 + D), Q (packed pairs) [64 + D, 64 + 3D/2)
+    constexpr uint32_t kTmemCols = 512;
     constexpr uint32_t kOCol = kKeys, kQCol = kKeys + D;
-    static_assert(kQCol + D / 2 <= kTmemCols, "tensor memory budget");
+    static_assert(kQCol + D / 2 <= 256, "tensor memory budget");
     static_assert(B == 16 || B == 32, "16- or 32-token blocks");
     static_assert(D == 64 || D == 128, "head dims");
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBarOff);
     uint64_t* k_full = bars;         // [KS] K tiles of a key tile landed
-    uint64_t* k_empty = bars + 4;    // [KS] their S MMAs finished
-    uint64_t* v_full = bars + 8;     // [VS] V tiles landed
-    uint64_t* v_empty = bars + 12;   // [VS] their O += P V finished
-    uint64_t* s_full = bars + 16;    // S = Q K^T finished
-    uint64_t* s_free = bars + 17;    // the softmax warps have read S
-    uint64_t* p_full = bars + 18;    // [2] P written (and O rescaled)
-    uint64_t* p_free = bars + 20;    // [2] the O += P V reading that P finished
-    uint64_t* drain = bars + 22;     // [2] the S and the O += P V issuers' MMAs finished
+    uint64_t* k_empty = bars + 6;    // [KS] the S MMAs reading them finished
+    uint64_t* v_full = bars + 12;    // [VS] V tiles landed
+    uint64_t* v_empty = bars + 18;   // [VS] the O += P V reading them finished
+    uint64_t* s_full = bars + 24;    // [q] S = Q K^T finished
+    uint64_t* s_free = bars + 26;    // [q] the softmax warps have read S
+    uint64_t* p_full = bars + 28;    // [q * 2 + buffer] P written (and O rescaled)
+    uint64_t* p_free = bars + 32;    // [q * 2 + buffer] the O += P V reading that P finished
+    uint64_t* drain = bars + 36;     // [2] the S and the O += P V issuers' MMAs finished
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Sm::kMiscOff);
     volatile uint32_t* abort = misc + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+    const int kvh = blockIdx.y, s = blockIdx.z;
     const int group = p.group;
 
     const int q0 = p.query_start[s];
     const int Q = p.query_start[s + 1] - q0;
     const int L = p.context_lens[s];
     if (L < 0 || L > p.context_cap || Q < 0 || Q > L) {
-        if (tid == 0 && tile == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
+        if (tid == 0 && blockIdx.x == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
         return;
     }
-    const int tok0 = tile * p.tile_tokens;
-    if (tok0 >= Q) return;
-    const int tok1 = min(Q, tok0 + p.tile_tokens);
-    const int last_pos = L - Q + tok1 - 1;
-    const int nblk = last_pos / B + 1;                   // blocks the tile needs
-    const int ntiles = (nblk + kBlocks - 1) / kBlocks;  // key tiles (>= 1)
+    // query tile q covers tokens [tok0[q], tok1[q]) of the chunk; nt[q] key tiles
+    int tok0[2], tok1[2], nt[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        tok0[q] = (2 * blockIdx.x + q) * p.tile_tokens;
+        tok1[q] = min(Q, tok0[q] + p.tile_tokens);
+        nt[q] = tok0[q] < Q ? ((L - Q + tok1[q] - 1) / B + kBlocks) / kBlocks : 0;
+    }
+    if (nt[0] == 0) return;
+    const int ntiles = max(nt[0], nt[1]);                           // key tiles fetched (>= 1)
+    const int nblk = (L - Q + (nt[1] ? tok1[1] : tok1[0]) - 1) / B + 1;   // blocks needed
     // tensor copies land on 128-byte boundaries (the dynamic window starts on one)
     if (smem_u32(smem) & 127u) {
         if (tid == 0) flag_error(8 /* PA_DEVERR_TIMEOUT: nothing fetched */);
         return;
     }
 
-    if (tid == 128) {
+    if (tid == 256) {
         for (int i = 0; i < KS; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
-        }
-        for (int i = 0; i < VS; ++i) {
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(s_free, 4);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&p_full[i], 128);
-            mbar_init(&p_free[i], 1);
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&s_full[q], 1);
+            mbar_init(&s_free[q], 4);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&p_full[q * 2 + b], 128);
+                mbar_init(&p_free[q * 2 + b], 1);
+            }
         }
         mbar_init(&drain[0], 1);
         mbar_init(&drain[1], 1);
         *abort = 0u;
         fence_barrier_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -300,7 +308,6 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = misc[0];
-    const uint32_t s_tmem = tmem, o_tmem = tmem + kOCol, q_tmem = tmem + kQCol;
 
     // ---- block ids of key tile j, and which of them may be fetched (every role
     //      derives the same mask from the table)
@@ -320,13 +327,13 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
         return ok;
     };
 
-    // ---- producers: warp 5 lane 0 fetches K tiles, warp 6 lane 0 V tiles
-    const bool is_producer = (warp == 5 || warp == 6) && lane == 0;
-    const bool v_side = warp == 6;
-    const char* pool = reinterpret_cast<const char*>(p.v_cache);
+    // ---- producers: warp 10 lane 0 fetches K tiles, warp 11 lane 0 V tiles
+    const bool is_producer = (warp == 10 || warp == 11) && lane == 0;
+    const bool v_side = warp == 11;
+    const char* vpool = reinterpret_cast<const char*>(p.v_cache);
     uint64_t* full = v_side ? v_full : k_full;
     uint64_t* empty = v_side ? v_empty : k_empty;
-    const int nst = v_side ? VS : KS;
+    constexpr int nst = KS;
     uint8_t* ring = smem + (v_side ? Sm::kVOff : Sm::kKOff);
     int ids[kBlocks], nxt[kBlocks];
     int issued = 0;
@@ -341,7 +348,7 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             if (ok == 0u) {
                 mbar_arrive_expect_tx(&full[st], 0);   // nothing to fetch: every key is masked
             } else {
-                // refused ids and blocks past the tile's need read a fetched block instead
+                // refused ids and blocks past the need read a fetched block instead
                 // (their scores are masked); row (id, head, chunk c) of the 2-D view
                 int rid[kBlocks];
                 int sub = ids[kBlocks - 1];
@@ -370,7 +377,7 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             for (int b = 0; b < kBlocks; ++b) {
                 if (!((ok >> b) & 1u)) continue;
                 const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
-                tc::bulk_copy(dst + b * kTile, pool + off, kTile, &full[st]);
+                tc::bulk_copy(dst + b * kTile, vpool + off, kTile, &full[st]);
             }
         }
         issued = j + 1;
@@ -386,13 +393,21 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
     }
 
     // ---- softmax warps: Q row into tensor memory (pairs packed per 32-bit column), O = 0
-    const int row_tok = tok0 + tid / group;
-    const int row_head = kvh * group + tid % group;
-    const bool row_ok = tid < 128 && row_tok < tok1;
+    const int qt = warp >> 2;                          // query tile of a softmax warp
+    const int my_tok0 = qt == 1 ? tok0[1] : tok0[0];
+    const int my_tok1 = qt == 1 ? tok1[1] : tok1[0];
+    const int my_nt = qt == 1 ? nt[1] : nt[0];
+    const int row = tid & 127;
+    const bool softmax_warp = warp < 8 && my_nt > 0;
+    const int row_tok = my_tok0 + row / group;
+    const int row_head = kvh * group + row % group;
+    const bool row_ok = warp < 8 && row_tok < my_tok1;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    if (tid < 128) {
+    const uint32_t qbase = tmem + static_cast<uint32_t>(qt & 1) * 256u;
+    const uint32_t s_tmem = qbase, o_tmem = qbase + kOCol, q_tmem = qbase + kQCol;
+    if (softmax_warp) {
         const T* qrow = reinterpret_cast<const T*>(p.q) +
-                        (static_cast<long long>(q0 + (row_ok ? row_tok : tok0)) * p.num_q_heads + row_head) * D;
+                        (static_cast<long long>(q0 + (row_ok ? row_tok : my_tok0)) * p.num_q_heads + row_head) * D;
 #pragma unroll
         for (int c0 = 0; c0 < D / 2; c0 += 32) {
             uint32_t w[32];
@@ -418,7 +433,7 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
     tc::fence_after();
 
     bool failed = false;
-    if (warp == 5 || warp == 6) {
+    if (warp == 10 || warp == 11) {
         // ---------------- producers
         if (is_producer) {
             for (int j = nst; j < ntiles; ++j) {
@@ -432,47 +447,58 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             for (int k = issued > nst ? issued - nst : 0; k < issued; ++k)
                 mbar_wait_bounded(&full[k % nst], (k / nst) & 1, kWaitLimitNs);
         }
-    } else if (warp == 4) {
-        // ---------------- S = Q K^T issue (lane 0): one N = 64 MMA per 16-dim step, A in tensor memory
+    } else if (warp == 8) {
+        // ---------------- S = Q K^T issue (lane 0): per query tile one N = 64 MMA per
+        //                  16-dim step, A (Q) in tensor memory
         if (lane == 0) {
             const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
             const uint32_t k_ring = smem_u32(smem + Sm::kKOff);
             int id_n[kBlocks];
             load_ids(0, id_n);
-            for (int j = 0; j < ntiles; ++j) {
+            bool run = true;
+            for (int j = 0; run && j < ntiles; ++j) {
                 const uint32_t ok = ok_of(id_n);
                 load_ids(j + 1, id_n);
-                // S(j) overwrites S(j - 1): the softmax warps must have read it
-                if (j > 0 && !tc_wait(s_free, (j - 1) & 1, abort)) break;
                 if (!tc_wait(&k_full[j % KS], (j / KS) & 1, abort)) break;
-                tc::fence_after();
                 const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
-                if (ok != 0u) {
 #pragma unroll
-                    for (int kc = 0; kc < D / 16; ++kc)
-                        tc::mma_ts(s_tmem, q_tmem + kc * 8, tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128),
-                                   idesc_s, kc > 0);
+                for (int q = 0; q < 2; ++q) {
+                    if (j >= nt[q]) continue;
+                    // S(j) overwrites S(j - 1): the softmax warps must have read it
+                    if (j > 0 && !tc_wait(&s_free[q], (j - 1) & 1, abort)) {
+                        run = false;
+                        break;
+                    }
+                    tc::fence_after();
+                    const uint32_t qb = tmem + static_cast<uint32_t>(q) * 256u;
+                    if (ok != 0u) {
+#pragma unroll
+                        for (int kc = 0; kc < D / 16; ++kc)
+                            tc::mma_ts(qb, qb + kQCol + kc * 8, tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128),
+                                       idesc_s, kc > 0);
+                    }
+                    tc::commit(&s_full[q]);
                 }
-                tc::commit(s_full);
-                tc::commit(&k_empty[j % KS]);
+                if (run) tc::commit(&k_empty[j % KS]);
             }
             // every MMA this thread issued has finished before the CTA tears down
             tc::commit(&drain[0]);
             mbar_wait_bounded(&drain[0], 0, kWaitLimitNs);
         }
-    } else if (warp == 7) {
+    } else if (warp == 9) {
         // ---------------- O += P V issue (lane 0); the warp zeroes V rows past the context
         const uint32_t idesc_o = tc::instr_desc<T>(D, true);
         const uint32_t v_ring = smem_u32(smem + Sm::kVOff);
         int id_n[kBlocks];
         load_ids(0, id_n);
-        for (int j = 0; j < ntiles; ++j) {
+        bool run = true;
+        for (int j = 0; run && j < ntiles; ++j) {
             const uint32_t ok = ok_of(id_n);
             load_ids(j + 1, id_n);
             const int vst = j % VS;
             if (!__all_sync(0xffffffffu, tc_wait(&v_full[vst], (j / VS) & 1, abort))) break;
-            // tokens at or past the context in the tile's last needed block: zero their
-            // staged V rows (P is 0 there, but 0 times a stale non-finite value would not be)
+            // tokens at or past the context in the last needed block: zero their staged
+            // V rows (P is 0 there, but 0 times a stale non-finite value would not be)
             const int lb = (L - 1) / B - j * kBlocks;
             if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
                 uint8_t* vt = smem + Sm::kVOff + vst * Sm::kStage + lb * kTile;
@@ -484,44 +510,55 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            const int st = j & 1;
-            if (!__all_sync(0xffffffffu, tc_wait(&p_full[st], (j >> 1) & 1, abort))) break;
-            if (lane == 0) {
-                tc::fence_after();
-                // one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
-                const uint32_t vbase = v_ring + vst * Sm::kStage;
-                const uint32_t pbase = smem_u32(smem + Sm::kPOff + st * Sm::kP);
-                for (int b = 0; b < kBlocks; ++b) {
-                    if (!((ok >> b) & 1u)) continue;
+            const uint32_t vbase = v_ring + vst * Sm::kStage;
 #pragma unroll
-                    for (int ks = 0; ks < B / 16; ++ks) {
-                        const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
-                        tc::mma(o_tmem, tc::smem_desc(pbase + kc * 2048, 2048, 128),
-                                tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
-                    }
+            for (int q = 0; q < 2; ++q) {
+                if (j >= nt[q]) continue;
+                const int pb = q * 2 + (j & 1);
+                if (!__all_sync(0xffffffffu, tc_wait(&p_full[pb], (j >> 1) & 1, abort))) {
+                    run = false;
+                    break;
                 }
-                tc::commit(&p_free[st]);
-                tc::commit(&v_empty[vst]);
+                if (lane == 0) {
+                    tc::fence_after();
+                    // one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
+                    const uint32_t pbase = smem_u32(smem + Sm::kPOff + pb * Sm::kP);
+                    const uint32_t ob = tmem + static_cast<uint32_t>(q) * 256u + kOCol;
+                    for (int b = 0; b < kBlocks; ++b) {
+                        if (!((ok >> b) & 1u)) continue;
+#pragma unroll
+                        for (int ks = 0; ks < B / 16; ++ks) {
+                            const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
+                            tc::mma(ob, tc::smem_desc(pbase + kc * 2048, 2048, 128),
+                                    tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
+                        }
+                    }
+                    tc::commit(&p_free[pb]);
+                }
             }
+            if (run && lane == 0) tc::commit(&v_empty[vst]);
         }
         if (lane == 0) {
             tc::commit(&drain[1]);
             mbar_wait_bounded(&drain[1], 0, kWaitLimitNs);
         }
         __syncwarp();
-    } else {
-        // ---------------- softmax (thread = row = tensor-memory lane)
+    } else if (softmax_warp) {
+        // ---------------- softmax of query tile qt (thread = row = tensor-memory lane)
         const float scale = p.score_scale;
         const int row_pos = row_ok ? L - Q + row_tok : -1;
         const uint32_t all_blocks = (1u << kBlocks) - 1u;
+        const int n = my_nt;
+        uint64_t* sfull = &s_full[qt];
+        uint64_t* sfree = &s_free[qt];
         int id_n[kBlocks];
         load_ids(0, id_n);
         uint32_t ok = ok_of(id_n);
         float m_run = kNegInf, l_run = 0.f;
-        for (int j = 0; j < ntiles; ++j) {
-            const int st = j & 1;
+        for (int j = 0; j < n; ++j) {
+            const int pb = qt * 2 + (j & 1);
             load_ids(j + 1, id_n);
-            if (!__all_sync(0xffffffffu, tc_wait(s_full, j & 1, abort))) {
+            if (!__all_sync(0xffffffffu, tc_wait(sfull, j & 1, abort))) {
                 failed = true;
                 break;
             }
@@ -532,7 +569,7 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             tc::fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(s_free);
+            if (lane == 0) mbar_arrive(sfree);
             const int key0 = j * kKeys;
             // row maximum over eight independent partial maxima (no 64-long chain)
             float m8[8];
@@ -559,12 +596,12 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             m_run = (m_old == kNegInf || mx > m_old + 8.f) ? fmaxf(m_old, mx) : m_old;
             const float mu = m_run == kNegInf ? 0.f : m_run;
             const float alpha = exp2_approx(m_old - mu);
-            // P buffer st was last read by the O += P V of tile j - 2
-            if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&p_free[st], ((j >> 1) - 1) & 1, abort))) {
+            // P buffer pb was last read by the O += P V of tile j - 2
+            if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&p_free[pb], ((j >> 1) - 1) & 1, abort))) {
                 failed = true;
                 break;
             }
-            uint8_t* ps = smem + Sm::kPOff + st * Sm::kP;
+            uint8_t* ps = smem + Sm::kPOff + pb * Sm::kP;
             // P = 2^(s * scale - mu): arguments and row sums two at a time, the
             // sums in four independent pairs
             const uint64_t scale2 = tc::f2(scale, scale), nmu2 = tc::f2(-mu, -mu);
@@ -583,7 +620,7 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
                     w[e] = Mma<T>::pack(a0, a1);
                 }
                 // (8-row group, 8-key chunk k8) core matrix at k8*2048 + g*128
-                *reinterpret_cast<uint4*>(ps + k8 * 2048 + (tid >> 3) * 128 + (tid & 7) * 16) =
+                *reinterpret_cast<uint4*>(ps + k8 * 2048 + (row >> 3) * 128 + (row & 7) * 16) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
             float rs;
@@ -597,7 +634,8 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             // rescale this row of O (after the previous O += P V), unless no
             // row of the warp moved its reference
             if (!__all_sync(0xffffffffu, m_old == kNegInf || alpha == 1.f)) {
-                if (!__all_sync(0xffffffffu, tc_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort))) {
+                const int pp = qt * 2 + ((j - 1) & 1);
+                if (!__all_sync(0xffffffffu, tc_wait(&p_free[pp], ((j - 1) >> 1) & 1, abort))) {
                     failed = true;
                     break;
                 }
@@ -614,17 +652,17 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
             }
             fence_proxy_async_smem();   // P visible to the tensor cores
             tc::fence_before();
-            mbar_arrive(&p_full[st]);
+            mbar_arrive(&p_full[pb]);
             ok = ok_of(id_n);
         }
         // ---- the last O += P V, then this row of the output
-        if (!failed && !__all_sync(0xffffffffu, tc_wait(&p_free[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort)))
+        if (!failed && !__all_sync(0xffffffffu, tc_wait(&p_free[qt * 2 + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort)))
             failed = true;
         if (!failed && !*abort) {
             tc::fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             T* dst = reinterpret_cast<T*>(p.out) +
-                     (static_cast<long long>(q0 + (row_ok ? row_tok : tok0)) * p.num_q_heads + row_head) * D;
+                     (static_cast<long long>(q0 + (row_ok ? row_tok : my_tok0)) * p.num_q_heads + row_head) * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 float v[32];
@@ -644,7 +682,7 @@ __global__ void __launch_bounds__(256, 2) pa_prefill_tc_kernel(const __grid_cons
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 8) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
 }
