@@ -195,11 +195,11 @@ struct PrefillTcSmem {
 #endif
     static constexpr int kKStages = D == 128 ? PA_PF_STAGES : PA_PF_STAGES + 2;
     static constexpr int kVStages = kKStages;
-    static constexpr int kP = 128 * kKeys * 2;            // one P buffer (16-bit)
+    static constexpr int kQ = 128 * D * 2;                // one query tile, core-matrix layout
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKStages * kStage;
-    static constexpr int kPOff = kVOff + kVStages * kStage;   // [query tile][2 buffers]
-    static constexpr int kBarOff = kPOff + 4 * kP;
+    static constexpr int kQOff = kVOff + kVStages * kStage;   // [query tile]
+    static constexpr int kBarOff = kQOff + 2 * kQ;
     static constexpr int kMiscOff = kBarOff + 48 * 8;     // tmem base, abort
     static constexpr int kTotal = kMiscOff + 16;
     static_assert(kTotal <= 232448, "shared memory per CTA");
@@ -231,10 +231,10 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
     constexpr int KS = Sm::kKStages, VS = Sm::kVStages;
     // tensor memory, per query tile q (256 columns at q * 256): S [0, 64),
-    // O [64, 64 + D), Q (packed pairs) [64 + D, 64 + 3D/2)
+    // O [64, 64 + D), P (16-bit pairs per column, two buffers of 32 columns)
     constexpr uint32_t kTmemCols = 512;
-    constexpr uint32_t kOCol = kKeys, kQCol = kKeys + D;
-    static_assert(kQCol + D / 2 <= 256, "tensor memory budget");
+    constexpr uint32_t kOCol = kKeys, kPCol = kKeys + D;
+    static_assert(kPCol + kKeys <= 256, "tensor memory budget");
     static_assert(B == 16 || B == 32, "16- or 32-token blocks");
     static_assert(D == 64 || D == 128, "head dims");
     extern __shared__ __align__(128) uint8_t smem[];
@@ -404,23 +404,19 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     const bool row_ok = warp < 8 && row_tok < my_tok1;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t qbase = tmem + static_cast<uint32_t>(qt & 1) * 256u;
-    const uint32_t s_tmem = qbase, o_tmem = qbase + kOCol, q_tmem = qbase + kQCol;
+    const uint32_t s_tmem = qbase, o_tmem = qbase + kOCol, p_tmem = qbase + kPCol;
     if (softmax_warp) {
+        // Q row into shared memory, K-major core-matrix layout: (8-row group g,
+        // 8-dim chunk c) at c * 2048 + g * 128
         const T* qrow = reinterpret_cast<const T*>(p.q) +
                         (static_cast<long long>(q0 + (row_ok ? row_tok : my_tok0)) * p.num_q_heads + row_head) * D;
+        uint8_t* qs = smem + Sm::kQOff + (qt & 1) * Sm::kQ;
 #pragma unroll
-        for (int c0 = 0; c0 < D / 2; c0 += 32) {
-            uint32_t w[32];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qrow + 2 * c0 + 8 * i) : make_uint4(0, 0, 0, 0);
-                w[4 * i] = v.x;
-                w[4 * i + 1] = v.y;
-                w[4 * i + 2] = v.z;
-                w[4 * i + 3] = v.w;
-            }
-            tc::st32u(q_tmem + lane_base + c0, w);
+        for (int c = 0; c < D / 8; ++c) {
+            const uint4 v = row_ok ? *reinterpret_cast<const uint4*>(qrow + 8 * c) : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(qs + c * 2048 + (row >> 3) * 128 + (row & 7) * 16) = v;
         }
+        fence_proxy_async_smem();   // Q (generic stores) visible to the tensor cores
         float z[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) z[i] = 0.f;
@@ -449,7 +445,7 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
         }
     } else if (warp == 8) {
         // ---------------- S = Q K^T issue (lane 0): per query tile one N = 64 MMA per
-        //                  16-dim step, A (Q) in tensor memory
+        //                  16-dim step, Q and K in shared memory
         if (lane == 0) {
             const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
             const uint32_t k_ring = smem_u32(smem + Sm::kKOff);
@@ -471,11 +467,12 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                     }
                     tc::fence_after();
                     const uint32_t qb = tmem + static_cast<uint32_t>(q) * 256u;
+                    const uint32_t qs = smem_u32(smem + Sm::kQOff + q * Sm::kQ);
                     if (ok != 0u) {
 #pragma unroll
                         for (int kc = 0; kc < D / 16; ++kc)
-                            tc::mma_ts(qb, qb + kQCol + kc * 8, tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128),
-                                       idesc_s, kc > 0);
+                            tc::mma(qb, tc::smem_desc(qs + 2 * kc * 2048, 2048, 128),
+                                    tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128), idesc_s, kc > 0);
                     }
                     tc::commit(&s_full[q]);
                 }
@@ -521,17 +518,15 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                 }
                 if (lane == 0) {
                     tc::fence_after();
-                    // one MMA per block and 16-key step, P (K-major) and V (MN-major) in shared memory
-                    const uint32_t pbase = smem_u32(smem + Sm::kPOff + pb * Sm::kP);
-                    const uint32_t ob = tmem + static_cast<uint32_t>(q) * 256u + kOCol;
+                    // one MMA per block and 16-key step: P in tensor memory, V (MN-major) in shared memory
+                    const uint32_t qb = tmem + static_cast<uint32_t>(q) * 256u;
+                    const uint32_t pt = qb + kPCol + static_cast<uint32_t>(j & 1) * (kKeys / 2);
                     for (int b = 0; b < kBlocks; ++b) {
                         if (!((ok >> b) & 1u)) continue;
 #pragma unroll
-                        for (int ks = 0; ks < B / 16; ++ks) {
-                            const int kc = (b * B) / 8 + 2 * ks;   // first 8-key chunk of this step
-                            tc::mma(ob, tc::smem_desc(pbase + kc * 2048, 2048, 128),
-                                    tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
-                        }
+                        for (int ks = 0; ks < B / 16; ++ks)
+                            tc::mma_ts(qb + kOCol, pt + (b * B) / 2 + 8 * ks,
+                                       tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
                     }
                     tc::commit(&p_free[pb]);
                 }
@@ -596,33 +591,31 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
             m_run = (m_old == kNegInf || mx > m_old + 8.f) ? fmaxf(m_old, mx) : m_old;
             const float mu = m_run == kNegInf ? 0.f : m_run;
             const float alpha = exp2_approx(m_old - mu);
-            // P buffer pb was last read by the O += P V of tile j - 2
+            // P buffer j % 2 was last read by the O += P V of tile j - 2
             if (j >= 2 && !__all_sync(0xffffffffu, tc_wait(&p_free[pb], ((j >> 1) - 1) & 1, abort))) {
                 failed = true;
                 break;
             }
-            uint8_t* ps = smem + Sm::kPOff + pb * Sm::kP;
             // P = 2^(s * scale - mu): arguments and row sums two at a time, the
             // sums in four independent pairs
             const uint64_t scale2 = tc::f2(scale, scale), nmu2 = tc::f2(-mu, -mu);
             uint64_t acc[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[e] = tc::f2(0.f, 0.f);
+            uint32_t pw[kKeys / 2];   // P row, 16-bit pairs: the A-operand columns of O += P V
 #pragma unroll
             for (int k8 = 0; k8 < kKeys / 8; ++k8) {
-                uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float x0, x1;
                     tc::f2_split(tc::fma2(tc::f2(sv[8 * k8 + 2 * e], sv[8 * k8 + 2 * e + 1]), scale2, nmu2), x0, x1);
                     const float a0 = exp2_approx(x0), a1 = exp2_approx(x1);
                     acc[e] = tc::add2(acc[e], tc::f2(a0, a1));
-                    w[e] = Mma<T>::pack(a0, a1);
+                    pw[4 * k8 + e] = Mma<T>::pack(a0, a1);
                 }
-                // (8-row group, 8-key chunk k8) core matrix at k8*2048 + g*128
-                *reinterpret_cast<uint4*>(ps + k8 * 2048 + (row >> 3) * 128 + (row & 7) * 16) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
             }
+            static_assert(kKeys / 2 == 32, "one 32-column store");
+            tc::st32u(p_tmem + lane_base + static_cast<uint32_t>(j & 1) * (kKeys / 2), pw);
             float rs;
             {
                 float r[8];
@@ -650,7 +643,7 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                 }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             }
-            fence_proxy_async_smem();   // P visible to the tensor cores
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc::fence_before();
             mbar_arrive(&p_full[pb]);
             ok = ok_of(id_n);
