@@ -264,9 +264,14 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     }
     // query tile q covers tokens [tok0[q], tok1[q]) of the chunk; nt[q] key tiles
     int tok0[2], tok1[2], nt[2];
+#ifndef PA_PF_HEAVY_FIRST
+#define PA_PF_HEAVY_FIRST 1
+#endif
+    // the latest query tiles of a sequence see the most keys: launch them first
+    const int tile = PA_PF_HEAVY_FIRST ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-        tok0[q] = (2 * blockIdx.x + q) * p.tile_tokens;
+        tok0[q] = (2 * tile + q) * p.tile_tokens;
         tok1[q] = min(Q, tok0[q] + p.tile_tokens);
         nt[q] = tok0[q] < Q ? ((L - Q + tok1[q] - 1) / B + kBlocks) / kBlocks : 0;
     }
