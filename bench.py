@@ -811,7 +811,8 @@ def run_prefill(args, world, rank, local):
                    "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim,
                    "block_size": b.block_size, "flops_per_step": flops, "parallelism": f"replicas x{world}",
                    "l2": "not flushed: compute-bound (the K/V of a sequence is reread by its query tiles)",
-                   "mma": "mma.sync m16n8k16 bf16, fp32 accumulate"},
+                   "mma": ("tcgen05.mma kind::f16, M = 128 query rows, Q / S / O in tensor memory, fp32 accumulate"
+                           if b.block_size != 8 else "mma.sync m16n8k16 bf16, fp32 accumulate")},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "peak_kind": kind,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get((b.name, "prefill"))},

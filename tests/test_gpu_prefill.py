@@ -87,3 +87,25 @@ def test_chunk_longer_than_context_is_flagged():
     assert pa.pa_get_device_error() & pa.DEVERR_CONTEXT_LEN
     assert torch.isnan(out[:12].float()).all()        # sequence 0 left unwritten
     assert torch.isfinite(out[12:].float()).all()
+
+
+def test_refused_block_ids_are_flagged_and_masked(orc):
+    """Block ids outside the pool (negative, or past its end) are flagged and
+    never fetched: a whole key tile of them (no block of the tile fetchable),
+    and a single one among fetchable blocks.  Untouched sequences still match
+    the oracle; rows of the damaged sequences stay finite."""
+    b = workloads.chunked_prefill(seed=1040, num_seqs=3, context_range=(200, 400), chunk_range=(40, 150))
+    ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.meta["query_start"], b.scale,
+                      b.block_size, b.num_kv_heads)
+    bad = b.block_tables.clone()
+    per_tile = 64 // b.block_size
+    bad[1, :per_tile] = -7                       # the first 64-key tile of sequence 1: nothing to fetch
+    bad[2, per_tile + 1] = b.num_blocks + 3      # one block of sequence 2's second key tile
+    b.block_tables = bad
+    pa.pa_get_device_error()
+    got = _gpu_prefill(b)
+    assert pa.pa_get_device_error() & pa.DEVERR_BLOCK_ID
+    qs = b.meta["query_start"]
+    s0 = slice(int(qs[0]), int(qs[1]))
+    check_tolerance(as_f64(got[s0]), ref[s0], b.dtype)
+    assert torch.isfinite(got.float()).all()
