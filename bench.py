@@ -106,13 +106,13 @@ def make_workload(name, seed, device, block_size=None):
 # in profiles/).  Keyed by a hash of the kernel sources: once the kernels change,
 # the figure no longer describes them and the bench reports null.
 NCU_TRAFFIC = {
-    "c644f2dd4445b1a8": {
-        ("llama3_8b_decode_bf16", "append"): 292.741632e6 + 3.549696e6,
-        ("continuous_batching_mix_bf16_B16", "append"): 211.572992e6 + 4.641024e6,
-        ("llama3_70b_long_bf16", "splitk"): 2.519422e9 + 11.374080e6,
-        ("llama3_8b_decode_bf16+e4m3", "single"): 146.536448e6 + 4.014592e6,
-        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260378e9 + 6.991872e6,
-        ("chunked_prefill_bfloat16", "prefill"): 120.610560e6 + 6.072064e6,
+    "9afa83d3db90f33c": {
+        ("llama3_8b_decode_bf16", "append"): 292.750e6 + 3.956e6,
+        ("continuous_batching_mix_bf16_B16", "append"): 211.577e6 + 4.173e6,
+        ("llama3_70b_long_bf16", "splitk"): 2.519434e9 + 8.115e6,
+        ("llama3_8b_decode_bf16+e4m3", "single"): 146.561e6 + 3.090e6,
+        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260209e9 + 6.564e6,
+        ("chunked_prefill_bfloat16", "prefill"): 118.550e6 + 20.334e6,
     },
 }
 
