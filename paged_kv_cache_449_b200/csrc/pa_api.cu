@@ -312,8 +312,9 @@ bool device_accessible(const void* p) {
 constexpr int kPrefillWarps = 4;
 constexpr int kPrefillStages = 4;
 
-// Blocks of 16 or 32 tokens run the 5th-generation tensor-core kernel
-// (128 MMA rows per CTA); 8-token blocks, or PA_PREFILL_TC=0, the warp-level one.
+// Blocks of 16 or 32 tokens run the 5th-generation tensor-core kernel (two
+// query tiles of 128 MMA rows per CTA); 8-token blocks, PA_PREFILL_TC=0 or a K
+// pool that no tensor map can describe run the warp-level one.
 #ifndef PA_PREFILL_TC
 #define PA_PREFILL_TC 1
 #endif

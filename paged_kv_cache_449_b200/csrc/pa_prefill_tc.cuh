@@ -2,25 +2,27 @@
 // computation as pa_prefill_kernel ("vLLM核心架构总览" §4.3 chunked prefill,
 // causal attention of each sequence's newest Q tokens over its paged context).
 //
-//  * One CTA of 128 threads per (sequence, kv head, tile of 128 / g query
-//    tokens).  The 128 MMA rows are (query token, head of the GQA group)
-//    pairs; thread t owns row t, which is TMEM lane t.
-//  * Tiles of 128 keys (8 blocks of 16 tokens, or 4 of 32) arrive by bulk
-//    copies into a 2-stage ring.  The paged (block, head) tile layout
-//    [D/8][B][8] is used as the MMA operand directly: K-major B operand of
-//    S = Q K^T (8-token groups 128 bytes apart, the next 8 dims B*16 bytes
-//    apart) and MN-major B operand of O += P V (the same numbers with the
-//    roles of the two offsets exchanged); no copy into another layout.
-//  * S (128 x 128 fp32) and O (128 x D fp32) live in tensor memory.  One
-//    thread issues every MMA; tcgen05.commit arrives on mbarriers that the
-//    other threads wait on (bounded).  Each thread reads its S row with
-//    tcgen05.ld, masks (causal, past the context), runs the online softmax in
-//    base 2, writes its P row (16-bit) into shared memory in the MMA core
-//    matrix layout and rescales its O row in tensor memory before the next
-//    O += P V.
-//  * Tokens past the context in the tile's last block are zeroed in the
-//    staged V tile (P is 0 there, but 0 times a stale non-finite value would
-//    not be); blocks beyond the context or with a refused id get no MMA.
+//  * One CTA (384 threads, one per SM) per (sequence, kv head, pair of query
+//    tiles).  A query tile is 128 MMA rows, (query token, head of the GQA
+//    group) pairs, 128 / g tokens; in a softmax warpgroup thread t owns row t,
+//    which is tensor-memory lane t.  The two tiles share every K/V tile.
+//  * Key tiles of 64 keys.  K arrives chunk-major, [D/8][64][8], by
+//    tile::gather4 loads (one 8-dim chunk of four pool blocks per load), so
+//    S = Q K^T is one N = 64 MMA per 16-dim step; V arrives as whole (block,
+//    head) tiles [D/8][B][8] by 1-D bulk copies, the MN-major B operand of
+//    O += P V as stored.  K and V have four-stage rings of their own.
+//  * Warp roles: 0-3 and 4-7 softmax of query tile 0 and 1; 8 issues S = Q K^T
+//    (Q and K in shared memory); 9 issues O += P V (P in tensor memory, V in
+//    shared memory); 10 and 11 fetch K and V.  tcgen05.commit arrives on the
+//    mbarriers the other roles wait on, every wait bounded.
+//  * Per query tile, S (64 fp32 columns), O (D columns) and two P buffers (32
+//    columns of 16-bit pairs each) live in tensor memory.  The softmax warps
+//    read their S row with tcgen05.ld, mask (causal, refused blocks), run the
+//    online softmax in base 2, write the P row with one tcgen05.st and rescale
+//    their O row in tensor memory when the reference maximum moves.
+//  * Tokens past the context in the last block are zeroed in the staged V tile
+//    (P is 0 there, but 0 times a stale non-finite value would not be); blocks
+//    with a refused id are never fetched and their keys are masked.
 //  * Tensor memory is allocated after every early exit and released on every
 //    path.
 #pragma once
