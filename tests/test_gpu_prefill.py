@@ -46,6 +46,8 @@ CASES = [
     (torch.float16, 128, 16, 8, 1, (40, 80), (33, 80)),
     (torch.bfloat16, 64, 8, 4, 2, (1, 50), (1, 5)),
     (torch.bfloat16, 64, 32, 8, 4, (60, 200), (60, 200)),
+    (torch.bfloat16, 128, 32, 16, 4, (100, 300), (20, 200)),
+    (torch.float16, 128, 32, 32, 8, (64, 64), (64, 64)),
 ]
 
 
@@ -109,3 +111,30 @@ def test_refused_block_ids_are_flagged_and_masked(orc):
     s0 = slice(int(qs[0]), int(qs[1]))
     check_tolerance(as_f64(got[s0]), ref[s0], b.dtype)
     assert torch.isfinite(got.float()).all()
+
+
+def test_empty_chunk_between_sequences(orc):
+    """A sequence with no new tokens (query_start repeats) launches nothing for
+    itself and leaves its neighbours exact."""
+    b = workloads.chunked_prefill(seed=1050, num_seqs=3, context_range=(150, 300), chunk_range=(30, 90))
+    qs = b.meta["query_start"]
+    n0, n2 = int(qs[1] - qs[0]), int(qs[3] - qs[2])
+    b.q = torch.cat([b.q[: n0], b.q[int(qs[2]):]]).contiguous()
+    new_qs = torch.tensor([0, n0, n0, n0 + n2], dtype=torch.int32)
+    ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, new_qs, b.scale, b.block_size,
+                      b.num_kv_heads)
+    got = _gpu_prefill(b, new_qs)
+    check_tolerance(as_f64(got), ref, b.dtype)
+
+
+@pytest.mark.parametrize("qmul", [6.0, 0.01])
+def test_prefill_peaked_and_flat_scores(orc, qmul):
+    """Queries scaled so that scores span many powers of two (the softmax
+    reference moves often, P reaches 2^8 and tiny values) or almost none (a
+    flat softmax over the whole context)."""
+    b = workloads.chunked_prefill(seed=1060, num_seqs=3, context_range=(300, 600), chunk_range=(50, 200))
+    b.q = (b.q.float() * qmul).to(b.dtype).contiguous()
+    ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.meta["query_start"], b.scale,
+                      b.block_size, b.num_kv_heads)
+    got = _gpu_prefill(b)
+    check_tolerance(as_f64(got), ref, b.dtype)
