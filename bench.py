@@ -125,21 +125,25 @@ DECODE_SOURCES = ("pa_api.cu", "pa_decode.cuh", "pa_e4m3.cuh", "pa_warp.cuh", "p
 PREFILL_SOURCES = ("pa_api.cu", "pa_prefill_tc.cuh", "pa_prefill.cuh", "pa_device.cuh")
 
 
+def code_of(text):
+    """A source's code without its comments, tokens joined by single spaces
+    (string literals kept whole, so a "//" inside one is not a comment)."""
+    import re
+    tokens = re.findall(r'"(?:\\.|[^"\\])*"|//[^\n]*|/\*.*?\*/|\S+', text, flags=re.S)
+    return " ".join(t for t in tokens if not (t.startswith("//") or t.startswith("/*")))
+
+
 def kernel_source_hash(names=DECODE_SOURCES):
     """Hash of the named kernel sources' code: comments and whitespace are
     dropped, so that a comment-only edit (which changes no instruction) keeps
     the DRAM traffic taken for the same code."""
     import hashlib
-    import re
     h = hashlib.sha256()
     for name in sorted(names):
         with open(os.path.join(ROOT, "paged_kv_cache_449_b200", "csrc", name), encoding="utf-8") as fh:
             text = fh.read()
-        # string literals are kept whole; comments outside them are dropped
-        tokens = re.findall(r'"(?:\\.|[^"\\])*"|//[^\n]*|/\*.*?\*/|\S+', text, flags=re.S)
-        code = " ".join(t for t in tokens if not (t.startswith("//") or t.startswith("/*")))
         h.update(name.encode())
-        h.update(code.encode())
+        h.update(code_of(text).encode())
     return h.hexdigest()[:16]
 
 
