@@ -84,7 +84,8 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
 #define PA_DEVERR_BLOCK_ID     1  /* a block-table entry outside [0, num_blocks) */
 #define PA_DEVERR_CONTEXT_LEN  2  /* a context length < 0 or above the stated maximum */
 #define PA_DEVERR_SLOT         4  /* a slot >= num_blocks * block_size */
-#define PA_DEVERR_TIMEOUT      8  /* an asynchronous copy did not complete in time */
+#define PA_DEVERR_TIMEOUT      8  /* an asynchronous copy did not complete in time; the
+                                     outputs of the launches concerned are undefined */
 #define PA_DEVERR_SEQ_ORDER   16  /* a seq_order entry outside [0, num_seqs) */
 
 /*
@@ -193,8 +194,9 @@ pa_status pa_decode_splitk_workspace_size(int num_seqs, int num_q_heads, int hea
  *                   num_kv_heads arrival counters (entry s*Hkv + kvh), all
  *                   zero before the first call (allocate it zeroed); every
  *                   completed call leaves the entries it used at zero, so one
- *                   array serves successive calls of any shape.  Zero it again
- *                   after a call that reported PA_DEVERR_TIMEOUT.
+ *                   array serves successive calls of any shape (a partition
+ *                   whose copies timed out still counts as arrived, so this
+ *                   holds after PA_DEVERR_TIMEOUT too).
  *   Other arguments as in pa_decode; here max_context_len also sizes the
  *   partition grid, so every context_lens[s] must be <= max_context_len.
  *   Calls that may run concurrently on the GPU need their own workspace and
@@ -222,15 +224,20 @@ pa_status pa_decode_splitk(void* out, const void* q, const void* k_cache, const 
  * which every GPU that loads the library holds until the process exits.  The
  * library allocates nothing.  The merge runs as the second kernel (the form
  * of pa_decode_splitk without counters), so nothing in the array has to start
- * at zero and the contents left by an earlier call are never read.
+ * at zero and the contents left by an earlier call are never read (a
+ * partition whose copies timed out is written as empty; the outputs of such a
+ * call are not the attention result, see PA_DEVERR_TIMEOUT).
  *
  *   Requests whose partials need more than PA_SPLITK_STATIC_SCRATCH_BYTES
  *   (num_seqs * num_q_heads * ceil(max_context_len / partition_size) *
  *   (head_dim + 2) * 4 bytes) are refused with PA_ERR_WORKSPACE before any
  *   device work; use a larger partition_size or pa_decode_splitk.
  *   The first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture.
+ *   (cudaGetSymbolAddress, with that device current) and caches it for the
+ *   life of the process; make that first call before any stream capture.
+ *   The cached address belongs to the device's primary context: after
+ *   cudaDeviceReset (or anything else that destroys that context) it is no
+ *   longer valid and this entry point must not be called again.
  *   Every call on a device shares the one array: calls that may overlap on
  *   the GPU (different streams without ordering between them) race on it and
  *   must not be issued.

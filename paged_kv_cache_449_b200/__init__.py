@@ -12,6 +12,7 @@ tensor shapes.  Calls run on the current torch CUDA stream unless `stream`
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -116,6 +117,41 @@ def _pool_dims(k_cache: torch.Tensor):
     return n, hkv, dv * x, b
 
 
+def _tensor_device(args, kwargs):
+    """The one CUDA device that every CUDA tensor argument lives on (None if
+    there is none).  The library launches on the current device, so a call
+    whose tensors sit on different GPUs is refused: a kernel would otherwise
+    dereference another GPU's pointers."""
+    found = None
+    for a in list(args) + list(kwargs.values()):
+        dev = None
+        if isinstance(a, torch.Tensor) and a.is_cuda:
+            dev = a.device
+        elif isinstance(a, torch.cuda.Stream):
+            dev = a.device
+        if dev is None:
+            continue
+        if found is None:
+            found = dev
+        elif dev != found:
+            raise ValueError(f"tensors and stream must share one CUDA device (found {found} and {dev})")
+    return found
+
+
+def _on_tensor_device(fn):
+    """Runs fn with the device of its CUDA tensor arguments current, so the
+    launch, the default stream and any per-device state (shared-memory limits,
+    the static split-K array) belong to the GPU that holds the data."""
+    @functools.wraps(fn)
+    def call(*args, **kwargs):
+        dev = _tensor_device(args, kwargs)
+        if dev is None or dev.index == torch.cuda.current_device():
+            return fn(*args, **kwargs)
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+    return call
+
+
 def _dev_ptr(t: torch.Tensor, name: str) -> int:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -128,6 +164,7 @@ def pa_status_string(status: int) -> str:
     return load().pa_status_string(int(status)).decode()
 
 
+@_on_tensor_device
 def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
     """Write key/value [T, Hkv, D] into the pools at slot_mapping (int64 [T])."""
     lib = load()
@@ -165,6 +202,7 @@ def _order_ptr(seq_order, num_seqs):
     return _dev_ptr(seq_order, "seq_order")
 
 
+@_on_tensor_device
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None, stream=None,
               seq_order=None):
     """Paged decode attention, one launch.  out, q: [S, Hq, D]; block_tables
@@ -176,6 +214,7 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_c
     _check(lib.pa_decode(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode")
 
 
+@_on_tensor_device
 def pa_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
                      stream=None, seq_order=None):
     """One decode step: write each sequence's newest token (key/value [S, Hkv,
@@ -215,6 +254,7 @@ _default_counters: dict = {}
 _splitk_ws_cache: dict = {}
 
 
+@_on_tensor_device
 def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                      partition_size=512, workspace=None, fused=True, counters=None, stream=None, seq_order=None):
     """Split-K paged decode (partitions of partition_size tokens + log-sum-exp
@@ -249,6 +289,7 @@ def pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale
 SPLITK_STATIC_SCRATCH_BYTES = 16 << 20
 
 
+@_on_tensor_device
 def pa_decode_splitk_static(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                             partition_size=512, stream=None):
     """Split-K paged decode that allocates nothing: for callers that cannot
@@ -275,6 +316,7 @@ def _accessible_ptr(t: torch.Tensor, name: str) -> int:
     return t.data_ptr()
 
 
+@_on_tensor_device
 def pa_copy_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, block_mapping, stream=None):
     """Copy whole blocks (src, dst) = block_mapping[i] (int64 [n, 2], on the
     device or pinned) from the source pools to the destination pools.  Same
@@ -307,6 +349,7 @@ def _scale_ptr(t, name):
     return _dev_ptr(t, name)
 
 
+@_on_tensor_device
 def pa_reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale, stream=None):
     """Quantise key/value [T, Hkv, D] to e4m3 codes (x / scale of the kv head)
     and write them into the 8-bit pools at slot_mapping (int64 [T])."""
@@ -327,6 +370,7 @@ def _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_
     return a[:4] + [_scale_ptr(k_scale, "k_scale"), _scale_ptr(v_scale, "v_scale")] + a[4:]
 
 
+@_on_tensor_device
 def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
                   max_context_len=None, stream=None, seq_order=None):
     """pa_decode over 8-bit pools; q/out fp16 or bf16."""
@@ -335,6 +379,7 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, cont
     _check(lib.pa_decode_fp8(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_fp8")
 
 
+@_on_tensor_device
 def pa_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                          scale, max_context_len=None, stream=None, seq_order=None):
     """One decode step over 8-bit pools: quantise and write each sequence's
@@ -346,6 +391,7 @@ def pa_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale,
                                     _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_append_fp8")
 
 
+@_on_tensor_device
 def pa_decode_splitk_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
                          max_context_len, partition_size=512, workspace=None, fused=True, counters=None,
                          stream=None, seq_order=None):
@@ -368,6 +414,7 @@ def pa_decode_splitk_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_table
                                     _order_ptr(seq_order, S), _stream(stream)), "pa_decode_splitk_fp8")
 
 
+@_on_tensor_device
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start, scale, max_context_len=None,
                max_query_len=None, stream=None):
     """Causal chunked prefill: q/out [T, Hq, D] (fp16/bf16); query_start int32

@@ -761,18 +761,28 @@ static __device__ __align__(256) float g_splitk_scratch[kStaticScratchBytes / si
 // Device address of g_splitk_scratch on the current device.  In host code
 // the name g_splitk_scratch is only a host-side stand-in, so the address is
 // looked up once per device (with that device current) and cached.
+// A failed runtime call leaves its error as the thread's last error; it is
+// cleared here so that a later launch check does not report it for an
+// unrelated call.
 pa_status static_scratch_address(void** ptr) {
     static std::mutex mu;
-    static void* cached[64] = {};
+    static std::map<int, void*> cached;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(mu);
-    if (cached[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_splitk_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
-        cached[dev] = p;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return PA_ERR_CUDA;
     }
-    *ptr = cached[dev];
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cached.find(dev);
+    if (it == cached.end()) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_splitk_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return PA_ERR_CUDA;
+        }
+        it = cached.emplace(dev, p).first;
+    }
+    *ptr = it->second;
     return PA_OK;
 }
 
@@ -795,8 +805,9 @@ extern "C" pa_status pa_decode_splitk_static(void* out, const void* q, const voi
     const pa_status addr_status = static_scratch_address(&scratch);
     if (addr_status != PA_OK) return addr_status;
     // Two-launch form (no arrival counters): the partition kernel writes every
-    // partial that the merge kernel reads, so no part of the array has to
-    // start at zero, and the previous call's leftovers are never read.
+    // partial that the merge kernel reads (a partition whose copies timed out
+    // is written as empty), so no part of the array has to start at zero and
+    // the previous call's leftovers are never read.
     return pa_decode_splitk(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size, num_seqs,
                             num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, max_context_len, num_blocks,
                             dtype, partition_size, scratch, kStaticScratchBytes, nullptr, 0, nullptr, stream);

@@ -399,20 +399,39 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         for (int k = i; k < issued; ++k) mbar_wait_bounded(&wbar[k % STAGES], (k / STAGES) & 1, kWaitLimitNs);
     }
     const int any_failed = __syncthreads_or(failed ? 1 : 0);
-    if (any_failed) return;
-
-    // ---- merge the warps' states (the ring is free now)
-    float* mo = reinterpret_cast<float*>(smem);
-    float* mml = mo + NW * kMaxGroup * D;
-    acc.store_smem(mo, mml, warp, group, lane);
-    __syncthreads();
 
     constexpr bool kLog2 = !kF32;
     // Split mode writes fp32 partials, except that with the fused merge a
     // sequence with a single partition is finished here.
     const int num_parts = SPLIT ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
     const bool to_workspace = SPLIT && !(p.counters != nullptr && num_parts == 1);
-    for (int idx = threadIdx.x; idx < group * D; idx += NW * 32) {
+    if (any_failed) {
+        // A copy timed out (PA_DEVERR_TIMEOUT is set; the outputs are then not
+        // the attention result).  A partition is recorded as empty (max -inf,
+        // sum 0, zero output) so that no merge reads what an earlier call left
+        // in the workspace, and the fused merge below still counts it, which
+        // brings the arrival counter back to zero.
+        if (!to_workspace) return;
+        for (int idx = threadIdx.x; idx < group * D; idx += NW * 32) {
+            const int r = idx / D, d = idx - r * D;
+            const long long slot =
+                (static_cast<long long>(s) * p.num_q_heads + kvh * group + r) * p.num_partitions + part;
+            p.part_acc[slot * D + d] = 0.f;
+            if (d == 0) {
+                p.part_ml[slot * 2] = kNegInf;
+                p.part_ml[slot * 2 + 1] = 0.f;
+            }
+        }
+    }
+
+    // ---- merge the warps' states (the ring is free now)
+    float* mo = reinterpret_cast<float*>(smem);
+    float* mml = mo + NW * kMaxGroup * D;
+    if (!any_failed) {
+        acc.store_smem(mo, mml, warp, group, lane);
+        __syncthreads();
+    }
+    for (int idx = threadIdx.x; idx < (any_failed ? 0 : group * D); idx += NW * 32) {
         const int r = idx / D, d = idx - r * D;
         float M = kNegInf;
 #pragma unroll

@@ -27,3 +27,24 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """The parity figures of every 16-bit comparison run in this session: the
+    largest per-row rms error ratio and ulp error per output type, with the
+    test that produced each."""
+    try:
+        from pagedutil import DIAGNOSTICS
+    except Exception:  # pragma: no cover
+        return
+    rows = [d for d in DIAGNOSTICS if "rms_row_max" in d]
+    if not rows:
+        return
+    terminalreporter.section("16-bit parity figures (max over checks)")
+    for dt in sorted({d["dtype"] for d in rows}):
+        mine = [d for d in rows if d["dtype"] == dt]
+        r = max(mine, key=lambda d: d["rms_row_max"])
+        u = max(mine, key=lambda d: d["ulp_max"])
+        terminalreporter.write_line(
+            f"{dt}: {len(mine)} checks; per-row rms ratio max {r['rms_row_max']:.3e} ({r['test']}); "
+            f"ulp max {u['ulp_max']:.2f} ({u['test']})")

@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import paged_kv_cache_449_b200 as pa
 from paged_kv_cache_449_b200 import build as pabuild
@@ -141,3 +142,34 @@ def test_longest_first_is_a_stable_descending_permutation():
     assert order.dtype == torch.int32
     assert order.tolist() == [1, 3, 5, 2, 0, 4]
     assert pa.longest_first([]).numel() == 0
+
+
+class _FakeCudaTensor(torch.Tensor):
+    """A CPU tensor that reports a CUDA device: enough for the binding's
+    device check, which runs before anything reaches the library."""
+
+    @staticmethod
+    def make(index):
+        t = torch.Tensor._make_subclass(_FakeCudaTensor, torch.zeros(4))
+        t.fake_device = torch.device("cuda", index)
+        return t
+
+    @property
+    def is_cuda(self):
+        return True
+
+    @property
+    def device(self):
+        return self.fake_device
+
+
+def test_binding_refuses_tensors_on_two_devices():
+    a, b = _FakeCudaTensor.make(0), _FakeCudaTensor.make(1)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.pa_decode(a, b, a, a, a, a, 0.125)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.pa_reshape_and_cache(a, a, a, a, slot_mapping=b)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.pa_decode_splitk_static(a, a, a, a, a, b, 0.125, 64)
+    assert pa._tensor_device((a, 3, None), {"x": a}) == torch.device("cuda", 0)
+    assert pa._tensor_device((torch.zeros(2),), {}) is None

@@ -4,7 +4,7 @@ Every comparison goes through the C ABI (libpa.so via the binding).  Small
 cases compare every output element; the full-size workloads compare seeded
 samples of sequences (the oracle computes each sampled sequence from the same
 pool contents).  Tolerances: fp32 1e-5 relative; fp16/bf16 2e-2 absolute +
-2e-2 relative (check_tolerance)."""
+2e-2 relative, plus the per-row rms and ulp figures (check_tolerance)."""
 
 import numpy as np
 import pytest
@@ -93,12 +93,9 @@ def _sampled(orc, b, seqs, modes, part=512):
         assert torch.isfinite(got.float()).all()
 
 
-def test_llama3_8b_decode_sampled(orc):
+def test_llama3_8b_decode_every_sequence(orc):
     b = workloads.llama3_8b_decode(seed=0, device="cuda")
-    rng = np.random.default_rng(0)
-    lens = b.context_lens.numpy()
-    seqs = list(rng.choice(b.num_seqs, 6, replace=False)) + [int(lens.argmax()), int(lens.argmin())]
-    _sampled(orc, b, seqs, ("single", "splitk", "splitk2"))
+    _sampled(orc, b, range(b.num_seqs), ("single", "splitk", "splitk2"))
 
 
 @pytest.mark.parametrize("block_size", [8, 16, 32])
@@ -122,7 +119,8 @@ def test_prefix_sharing_sampled(orc, prefix_len):
 def test_llama3_70b_long_sampled(orc):
     b = workloads.llama3_70b_long(seed=0, device="cuda")
     lens = b.context_lens.numpy()
-    seqs = [int(lens.argmax()), int(lens.argmin()), 7]
+    rng = np.random.default_rng(70)
+    seqs = [int(lens.argmax()), int(lens.argmin())] + list(rng.choice(b.num_seqs, 8, replace=False))
     _sampled(orc, b, seqs, ("splitk", "splitk2", "single"))
 
 

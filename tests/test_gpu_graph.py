@@ -1,14 +1,17 @@
 """A decode step captured into a CUDA graph (GPU): after one uncaptured call
 (which sets the kernels' shared-memory limit and caches device attributes),
 the write and decode entry points record into a graph, and replaying it gives
-bit-for-bit the eager result, again after the inputs have changed in place."""
+bit-for-bit the eager result, again after the inputs have changed in place.
+Each replayed output is also compared with the oracle (the new tokens written
+by the oracle's own write, then its decode) at the 16-bit tolerance."""
 
 import pytest
 import torch
 
+import oracle
 import workloads
 import paged_kv_cache_449_b200 as pa
-from pagedutil import device_batch
+from pagedutil import as_f64, check_tolerance, device_batch
 
 pytestmark = pytest.mark.gpu
 
@@ -52,6 +55,15 @@ def _steps(b):
     return {"append": append, "split_fused": reshape_then_split, "split_merge_kernel": reshape_then_two_kernel_split}
 
 
+def _oracle_step(b, q):
+    """The oracle's result of one step: the batch's new tokens written at
+    their (decode-consistent) slots, then decode with queries q."""
+    orc = oracle.default()
+    kc, vc = b.k_cache.cpu().clone(), b.v_cache.cpu().clone()
+    orc.reshape_and_cache(b.new_key.cpu(), b.new_value.cpu(), kc, vc, b.slot_mapping, b.block_size)
+    return orc.decode(q.cpu(), kc, vc, b.block_tables, b.context_lens, b.scale, b.block_size, b.num_kv_heads)
+
+
 @pytest.mark.parametrize("which", ["append", "split_fused", "split_merge_kernel"])
 def test_graph_replay_equals_eager(which):
     b = workloads.llama3_8b_decode(seed=31, device="cuda", num_seqs=16, num_blocks=2048)
@@ -74,6 +86,7 @@ def test_graph_replay_equals_eager(which):
         torch.cuda.synchronize()
         assert torch.equal(_bits(graphed["out"]), _bits(eager["out"])), (which, round_)
         assert torch.equal(_bits(graphed["k_cache"]), _bits(eager["k_cache"]))
+        check_tolerance(as_f64(graphed["out"]), _oracle_step(b, graphed["q"]), b.dtype)
     assert pa.pa_get_device_error() == 0
     del g
 
@@ -98,4 +111,8 @@ def test_graph_replay_fp8():
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(_bits(outs[1]), _bits(outs[0]))
+    ref = oracle.default().decode_e4m3(b.q.cpu(), pools.k_cache.cpu(), pools.v_cache.cpu(), pools.k_scale.cpu(),
+                                       pools.v_scale.cpu(), b.block_tables, b.context_lens, b.scale, b.block_size,
+                                       b.num_kv_heads)
+    check_tolerance(as_f64(outs[1]), ref, b.dtype)
     del g
