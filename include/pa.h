@@ -87,6 +87,11 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
 #define PA_DEVERR_TIMEOUT      8  /* an asynchronous copy did not complete in time; the
                                      outputs of the launches concerned are undefined */
 #define PA_DEVERR_SEQ_ORDER   16  /* a seq_order entry outside [0, num_seqs) */
+#define PA_DEVERR_NO_FREE_BLOCK 32  /* pa_blocks_append: the free blocks ran out */
+#define PA_DEVERR_REF_COUNT   64  /* a reference count would drop below zero, a fork into a
+                                     sequence that holds tokens, or a corrupt free ring */
+#define PA_DEVERR_SHARED_BLOCK 128 /* pa_decode_append: the newest token's block is held by
+                                      more than one sequence; its write was skipped */
 
 /*
  * seq_order (pa_decode, pa_decode_append, pa_decode_splitk) — NULL, or an
@@ -155,13 +160,19 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
  *   v_cache        written at the new tokens' rows, read everywhere else
  *   The block holding position L-1 must belong to sequence s alone (a block
  *   shared with other sequences is copied before it is written, as
- *   copy-on-write requires, [P4] §2.3).  Other arguments as in pa_decode.
+ *   copy-on-write requires, [P4] §2.3; pa_blocks_append does that).
+ *   ref_counts     NULL, or int32 [num_blocks] reference counts (those of the
+ *                  pa_blocks_* entry points), 4-byte aligned: a sequence whose
+ *                  newest block's count is not 1 is not written (its output
+ *                  attends over the pool as it is) and PA_DEVERR_SHARED_BLOCK
+ *                  is set.  With NULL the rule above is trusted.
+ *   Other arguments as in pa_decode.
  */
 pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value, void* k_cache,
                            void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
                            float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
                            int head_dim, int max_blocks_per_seq, int max_context_len, int64_t num_blocks,
-                           pa_dtype dtype, const int32_t* seq_order, void* stream);
+                           pa_dtype dtype, const int32_t* ref_counts, const int32_t* seq_order, void* stream);
 
 /*
  * pa_decode_splitk_workspace_size — bytes of workspace pa_decode_splitk needs:
@@ -294,13 +305,14 @@ pa_status pa_decode_fp8(void* out, const void* q, const void* k_cache, const voi
  * newest token (key/value [num_seqs][num_kv_heads][head_dim] in dtype, 16-byte
  * aligned) is quantised like pa_reshape_and_cache_fp8, written at position
  * L-1 and attended to, in one launch; the result and every pool byte equal
- * pa_reshape_and_cache_fp8 followed by pa_decode_fp8. */
+ * pa_reshape_and_cache_fp8 followed by pa_decode_fp8.  ref_counts as in
+ * pa_decode_append. */
 pa_status pa_decode_append_fp8(void* out, const void* q, const void* key, const void* value, void* k_cache,
                                void* v_cache, const float* k_scale, const float* v_scale,
                                const int32_t* block_tables, const int32_t* context_lens, float scale,
                                int block_size, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int max_blocks_per_seq, int max_context_len, int64_t num_blocks, pa_dtype dtype,
-                               const int32_t* seq_order, void* stream);
+                               const int32_t* ref_counts, const int32_t* seq_order, void* stream);
 
 /* pa_decode_splitk_fp8 — pa_decode_splitk over 8-bit pools (same workspace
  * size, counters and merge forms). */
@@ -358,7 +370,9 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
  *   src_k_cache,
  *   src_v_cache    source pools of src_num_blocks blocks, read only
  *   block_mapping  int64 [num_pairs][2]: (source block, destination block),
- *                  8-byte aligned
+ *                  8-byte aligned; a pair with a negative source block is an
+ *                  empty entry and copies nothing (the copy_pairs output of
+ *                  pa_blocks_append can be passed as it is)
  *   Every pool and block_mapping is device memory or page-locked host memory
  *   that the device can address (cudaHostAlloc / cudaMallocHost, or
  *   cudaHostRegister'd and mapped); anything else is PA_ERR_INVALID_ARG.  The
@@ -371,6 +385,94 @@ pa_status pa_copy_blocks(void* dst_k_cache, void* dst_v_cache, const void* src_k
                          const void* src_v_cache, const int64_t* block_mapping, int64_t num_pairs,
                          int num_kv_heads, int head_dim, int block_size, int64_t src_num_blocks,
                          int64_t dst_num_blocks, pa_dtype dtype, void* stream);
+
+/*
+ * Block management on the device ([P3] §2.1 append_token takes a free block
+ * when a sequence's next token starts a new logical block; §2.2 one pool of
+ * equal blocks; [P4] §2.2-2.3 reference counts, prefix blocks shared by
+ * count, copy-on-write, a block whose count reaches zero returns to the free
+ * pool; [P3] §3.2 admission while blocks remain, stopping at the first request
+ * that does not fit).
+ *
+ * State, all caller-owned device memory (num_blocks = N <= 2^31 - 1):
+ *   ref_counts  int32 [N]  references to each block from block-table rows
+ *                          (0 = free)
+ *   free_ids    int32 [N]  the free blocks as a ring: positions head ..
+ *                          tail-1 (mod N) hold them, oldest first
+ *   free_state  int64 [2]  {head, tail}; both only grow; tail - head blocks
+ *                          are free (the host may read it: can_allocate)
+ * together with block_tables (int32 [num_seqs][max_blocks_per_seq]) and
+ * context_lens (int32 [num_seqs]) as the attention entry points read them.
+ * Table entries of unused logical blocks hold -1.  Every operation is one
+ * launch on `stream`, its result is deterministic and equals the plain
+ * sequential bookkeeping: sequences in index (or list) order, blocks in
+ * logical order, the free ring first in first out.  Operations on one state
+ * must not overlap on the GPU.  Errors found on the device set PA_DEVERR_*
+ * bits and skip the offending sequence or pair; nothing faults.
+ */
+
+/* pa_blocks_init — every block free (ring = 0, 1, ..., N-1), counts zero. */
+pa_status pa_blocks_init(int32_t* ref_counts, int32_t* free_ids, int64_t* free_state, int64_t num_blocks,
+                         void* stream);
+
+/*
+ * pa_blocks_append — one step of every sequence: sequence s takes
+ * num_new_tokens[s] >= 0 new token positions L .. L+n-1 (L = its length).
+ *   * A position that starts a logical block gets a block from the ring;
+ *     positions in the sequence's last, partly filled block go there.  If that
+ *     block's count is above one it is first replaced by a private copy
+ *     (copy-on-write): the k-th writer into such a block in this step, in
+ *     sequence order, copies it while k < count - 1; the last holder writes in
+ *     place.  The copy block is taken before new blocks.
+ *   * Sequences are served in index order while free blocks remain; the
+ *     first one whose blocks do not fit, and every later one, are not served
+ *     (PA_DEVERR_NO_FREE_BLOCK): no block, no length change, slots -1.
+ *   * A row that would exceed max_blocks_per_seq * block_size tokens, or a
+ *     negative count, is skipped with PA_DEVERR_CONTEXT_LEN.
+ * Outputs:
+ *   slot_mapping  int64 [num_slots], the step's token slots packed in sequence
+ *                 order (offsets = running sum of num_new_tokens), ready for
+ *                 pa_reshape_and_cache; num_slots must be at least that sum,
+ *                 otherwise nothing is done and PA_DEVERR_SLOT is set
+ *   copy_pairs    int64 [num_seqs][2]: (old block, its copy) for a sequence
+ *                 that copied, (-1, -1) otherwise; pass it to pa_copy_blocks
+ *                 (same pools on both sides) before the new tokens are written
+ *                 (negative entries copy nothing)
+ *   block_tables, context_lens, ref_counts, free_state updated in place.
+ * Also used as scratch while the launch runs: slot_mapping and copy_pairs.
+ * For pa_decode_append (which writes the token at position L-1 itself) call
+ * this with one token per running sequence, then pa_copy_blocks, then
+ * pa_decode_append on the updated tables and lengths.
+ */
+pa_status pa_blocks_append(int32_t* block_tables, int32_t* context_lens, const int32_t* num_new_tokens,
+                           int32_t* ref_counts, const int32_t* free_ids, int64_t* free_state,
+                           int64_t* slot_mapping, int64_t num_slots, int64_t* copy_pairs, int num_seqs,
+                           int max_blocks_per_seq, int block_size, int64_t num_blocks, void* stream);
+
+/*
+ * pa_blocks_fork — for each (parent, child, length) row of forks (int32
+ * [num_forks][3]), in order: the child shares the parent's first `length`
+ * tokens: its row takes the parent's first ceil(length / B) block ids, each
+ * of whose counts goes up by one, and its length becomes `length` (prefix
+ * sharing of a common system prompt, or a parallel sample; [P4] §2.3, §3.1).
+ * The child must hold no tokens and differ from the parent
+ * (PA_DEVERR_REF_COUNT otherwise) and 0 <= length <= the parent's length
+ * (PA_DEVERR_CONTEXT_LEN otherwise); a refused row is skipped.
+ */
+pa_status pa_blocks_fork(int32_t* block_tables, int32_t* context_lens, int32_t* ref_counts, const int32_t* forks,
+                         int num_forks, int num_seqs, int max_blocks_per_seq, int block_size, int64_t num_blocks,
+                         void* stream);
+
+/*
+ * pa_blocks_release — free whole sequences (int32 seqs [num_release], in
+ * order): each block of the sequence, in logical order, loses one reference;
+ * a block whose count reaches zero joins the ring's tail then.  The row is
+ * set to -1 and the length to 0 (a sequence listed twice is freed once).
+ * A count already at zero sets PA_DEVERR_REF_COUNT and is left at zero.
+ */
+pa_status pa_blocks_release(int32_t* block_tables, int32_t* context_lens, int32_t* ref_counts, int32_t* free_ids,
+                            int64_t* free_state, const int32_t* seqs, int num_release, int num_seqs,
+                            int max_blocks_per_seq, int block_size, int64_t num_blocks, void* stream);
 
 /*
  * pa_get_device_error — read and clear the device error word of the current

@@ -468,7 +468,9 @@ int oracle_prefill(double* out, const void* q, const void* k_cache, const void* 
 // source and destination is the copy-on-write duplicate of a shared block
 // ([P4] §2.3); a host-memory pool on one side is a swap-out or swap-in of a
 // preempted sequence's blocks ([P1] §4.2).  Element by element through the
-// pool layout, pairs in order.  A block id outside its pool is refused.
+// pool layout, pairs in order.  A pair whose source id is negative is an empty
+// entry and copies nothing (like a negative slot in the write); any other block
+// id outside its pool is refused.
 int oracle_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
                        const int64_t* block_mapping, int64_t num_pairs, int num_kv_heads,
                        int head_dim, int block_size, int64_t src_num_blocks,
@@ -483,7 +485,8 @@ int oracle_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* 
     for (int64_t i = 0; i < num_pairs; ++i) {
         const int64_t src = block_mapping[2 * i];
         const int64_t dst = block_mapping[2 * i + 1];
-        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return kBadBlockId;
+        if (src < 0) continue;
+        if (src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) return kBadBlockId;
         for (int h = 0; h < num_kv_heads; ++h) {
             for (int t = 0; t < block_size; ++t) {
                 for (int d = 0; d < head_dim; ++d) {

@@ -24,7 +24,9 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "pa_get_device_error", "pa_status_string", "PagedAttentionError", "library_path", "load",
            "pool_shape", "DEVERR_BLOCK_ID", "DEVERR_CONTEXT_LEN", "DEVERR_SLOT", "DEVERR_TIMEOUT",
            "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
-           "pa_decode_splitk_fp8", "fp8_pool_shape", "pa_prefill", "pa_decode_append_fp8"]
+           "pa_decode_splitk_fp8", "fp8_pool_shape", "pa_prefill", "pa_decode_append_fp8",
+           "pa_blocks_init", "pa_blocks_append", "pa_blocks_fork", "pa_blocks_release",
+           "DEVERR_NO_FREE_BLOCK", "DEVERR_REF_COUNT", "DEVERR_SHARED_BLOCK"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -33,6 +35,7 @@ PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 _DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
 STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE", 4: "PA_ERR_CUDA"}
 DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_SEQ_ORDER = 1, 2, 4, 8, 16
+DEVERR_NO_FREE_BLOCK, DEVERR_REF_COUNT, DEVERR_SHARED_BLOCK = 32, 64, 128
 
 
 class PagedAttentionError(RuntimeError):
@@ -55,7 +58,14 @@ def load() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(_LIB_PATH):
         raise RuntimeError(f"libpa.so is not built ({_LIB_PATH}); run paged_kv_cache_449_b200/build.py")
-    lib = ctypes.CDLL(_LIB_PATH)
+    _lib = load_library(_LIB_PATH)
+    return _lib
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Open a build of the library at `path` with the argument types of every
+    entry point declared in include/pa.h."""
+    lib = ctypes.CDLL(path)
     c = ctypes
     P, I, I64, F, SZ = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
     lib.pa_reshape_and_cache.restype = I
@@ -64,7 +74,7 @@ def load() -> ctypes.CDLL:
     lib.pa_decode.restype = I
     lib.pa_decode.argtypes = decode_args + [P, P]
     lib.pa_decode_append.restype = I
-    lib.pa_decode_append.argtypes = [P, P, P, P] + decode_args[2:] + [P, P]
+    lib.pa_decode_append.argtypes = [P, P, P, P] + decode_args[2:] + [P, P, P]
     lib.pa_decode_splitk_workspace_size.restype = I
     lib.pa_decode_splitk_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
     lib.pa_decode_splitk.restype = I
@@ -77,18 +87,25 @@ def load() -> ctypes.CDLL:
     lib.pa_decode_fp8.restype = I
     lib.pa_decode_fp8.argtypes = fp8_args + [P, P]
     lib.pa_decode_append_fp8.restype = I
-    lib.pa_decode_append_fp8.argtypes = [P, P, P, P] + fp8_args[2:] + [P, P]
+    lib.pa_decode_append_fp8.argtypes = [P, P, P, P] + fp8_args[2:] + [P, P, P]
     lib.pa_decode_splitk_fp8.restype = I
     lib.pa_decode_splitk_fp8.argtypes = fp8_args + [I, P, SZ, P, I64, P, P]
     lib.pa_prefill.restype = I
     lib.pa_prefill.argtypes = [P, P, P, P, P, P, P, F, I, I, I, I, I, I, I, I, I64, I, P]
     lib.pa_copy_blocks.restype = I
     lib.pa_copy_blocks.argtypes = [P, P, P, P, P, I64, I, I, I, I64, I64, I, P]
+    lib.pa_blocks_init.restype = I
+    lib.pa_blocks_init.argtypes = [P, P, P, I64, P]
+    lib.pa_blocks_append.restype = I
+    lib.pa_blocks_append.argtypes = [P, P, P, P, P, P, P, I64, P, I, I, I, I64, P]
+    lib.pa_blocks_fork.restype = I
+    lib.pa_blocks_fork.argtypes = [P, P, P, P, I, I, I, I, I64, P]
+    lib.pa_blocks_release.restype = I
+    lib.pa_blocks_release.argtypes = [P, P, P, P, P, P, I, I, I, I, I64, P]
     lib.pa_get_device_error.restype = I
     lib.pa_get_device_error.argtypes = [P, c.POINTER(c.c_int32)]
     lib.pa_status_string.restype = c.c_char_p
     lib.pa_status_string.argtypes = [I]
-    _lib = lib
     return lib
 
 
@@ -215,14 +232,25 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_c
 
 
 @_on_tensor_device
+def _counts_ptr(ref_counts, num_blocks):
+    if ref_counts is None:
+        return None
+    if ref_counts.dtype != torch.int32 or ref_counts.numel() != num_blocks:
+        raise ValueError("ref_counts must be int32 [num_blocks]")
+    return _dev_ptr(ref_counts, "ref_counts")
+
+
 def pa_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
-                     stream=None, seq_order=None):
+                     stream=None, seq_order=None, ref_counts=None):
     """One decode step: write each sequence's newest token (key/value [S, Hkv,
-    D]) at position context_lens[s]-1, then attend over the whole context."""
+    D]) at position context_lens[s]-1, then attend over the whole context.
+    ref_counts (int32 [num_blocks], optional): a sequence whose newest block
+    is held by others is not written (DEVERR_SHARED_BLOCK)."""
     lib = load()
     args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_append(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
-                                _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_append")
+                                _counts_ptr(ref_counts, k_cache.shape[0]), _order_ptr(seq_order, q.shape[0]),
+                                _stream(stream)), "pa_decode_append")
 
 
 def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size=512) -> int:
@@ -381,14 +409,16 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, cont
 
 @_on_tensor_device
 def pa_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
-                         scale, max_context_len=None, stream=None, seq_order=None):
+                         scale, max_context_len=None, stream=None, seq_order=None, ref_counts=None):
     """One decode step over 8-bit pools: quantise and write each sequence's
     newest token (key/value [S, Hkv, D]) at position context_lens[s]-1, then
-    attend over the whole context (one launch)."""
+    attend over the whole context (one launch).  ref_counts as in
+    pa_decode_append."""
     lib = load()
     args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
     _check(lib.pa_decode_append_fp8(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
-                                    _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_append_fp8")
+                                    _counts_ptr(ref_counts, k_cache.shape[0]), _order_ptr(seq_order, q.shape[0]),
+                                    _stream(stream)), "pa_decode_append_fp8")
 
 
 @_on_tensor_device
@@ -432,6 +462,77 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start
         _dev_ptr(block_tables, "block_tables"), _dev_ptr(context_lens, "context_lens"),
         _dev_ptr(query_start, "query_start"), float(scale), b, S, Hq, hkv, D, int(block_tables.shape[1]),
         int(max_context_len), int(max_query_len), n, _DTYPE[q.dtype], _stream(stream)), "pa_prefill")
+
+
+# ---- block management: ref_counts / free_ids int32 [N], free_state int64 [2] (head, tail), block_tables
+#      int32 [S, max_blocks], context_lens int32 [S], all on one device
+
+def _typed(t, dtype, name):
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    return _dev_ptr(t, name)
+
+
+def _state_ptrs(ref_counts, free_ids, free_state):
+    if ref_counts.numel() != free_ids.numel() or free_state.numel() != 2:
+        raise ValueError("ref_counts and free_ids hold num_blocks entries, free_state two")
+    return (_typed(ref_counts, torch.int32, "ref_counts"), _typed(free_ids, torch.int32, "free_ids"),
+            _typed(free_state, torch.int64, "free_state"))
+
+
+def _rows(block_tables, context_lens):
+    if block_tables.dim() != 2 or context_lens.numel() != block_tables.shape[0]:
+        raise ValueError("block_tables is [num_seqs, max_blocks], context_lens [num_seqs]")
+    return (_typed(block_tables, torch.int32, "block_tables"), _typed(context_lens, torch.int32, "context_lens"),
+            int(block_tables.shape[0]), int(block_tables.shape[1]))
+
+
+@_on_tensor_device
+def pa_blocks_init(ref_counts, free_ids, free_state, stream=None):
+    """Every block free (the ring 0..N-1), every count zero."""
+    lib = load()
+    r, f, st = _state_ptrs(ref_counts, free_ids, free_state)
+    _check(lib.pa_blocks_init(r, f, st, ref_counts.numel(), _stream(stream)), "pa_blocks_init")
+
+
+@_on_tensor_device
+def pa_blocks_append(block_tables, context_lens, num_new_tokens, ref_counts, free_ids, free_state, slot_mapping,
+                     copy_pairs, block_size, stream=None):
+    """One step: sequence s takes num_new_tokens[s] (int32 [S]) new positions.
+    Writes the packed slots (int64, at least sum(num_new_tokens) entries) and
+    the copy-on-write pairs (int64 [S, 2]) and updates the tables, lengths,
+    counts and free ring in place."""
+    lib = load()
+    bt, cl, S, mb = _rows(block_tables, context_lens)
+    r, f, st = _state_ptrs(ref_counts, free_ids, free_state)
+    if num_new_tokens.numel() != S or copy_pairs.shape != (S, 2):
+        raise ValueError("num_new_tokens is [num_seqs], copy_pairs [num_seqs, 2]")
+    _check(lib.pa_blocks_append(bt, cl, _typed(num_new_tokens, torch.int32, "num_new_tokens"), r, f, st,
+                                _typed(slot_mapping, torch.int64, "slot_mapping"), slot_mapping.numel(),
+                                _typed(copy_pairs, torch.int64, "copy_pairs"), S, mb, int(block_size),
+                                ref_counts.numel(), _stream(stream)), "pa_blocks_append")
+
+
+@_on_tensor_device
+def pa_blocks_fork(block_tables, context_lens, ref_counts, forks, block_size, stream=None):
+    """forks: int32 [n, 3] rows (parent, child, length), applied in order."""
+    lib = load()
+    bt, cl, S, mb = _rows(block_tables, context_lens)
+    if forks.dim() != 2 or forks.shape[1] != 3:
+        raise ValueError("forks is int32 [n, 3]")
+    _check(lib.pa_blocks_fork(bt, cl, _typed(ref_counts, torch.int32, "ref_counts"),
+                              _typed(forks, torch.int32, "forks"), int(forks.shape[0]), S, mb, int(block_size),
+                              ref_counts.numel(), _stream(stream)), "pa_blocks_fork")
+
+
+@_on_tensor_device
+def pa_blocks_release(block_tables, context_lens, ref_counts, free_ids, free_state, seqs, block_size, stream=None):
+    """Free the sequences seqs (int32 [n]) in order."""
+    lib = load()
+    bt, cl, S, mb = _rows(block_tables, context_lens)
+    r, f, st = _state_ptrs(ref_counts, free_ids, free_state)
+    _check(lib.pa_blocks_release(bt, cl, r, f, st, _typed(seqs, torch.int32, "seqs"), seqs.numel(), S, mb,
+                                 int(block_size), ref_counts.numel(), _stream(stream)), "pa_blocks_release")
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -16,6 +17,7 @@
 #include <tuple>
 
 #include "pa.h"
+#include "pa_blocks.cuh"
 #include "pa_copy.cuh"
 #include "pa_decode.cuh"
 #include "pa_prefill.cuh"
@@ -389,7 +391,8 @@ template <bool FP8>
 pa_status decode_one_pass(void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
                           const float* v_scale, const int32_t* block_tables, const int32_t* context_lens,
                           float scale, const DecodeShape& sh, const int32_t* seq_order, void* stream,
-                          const void* new_key = nullptr, const void* new_value = nullptr) {
+                          const void* new_key = nullptr, const void* new_value = nullptr,
+                          const int32_t* ref_counts = nullptr) {
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     if (st == PA_OK) st = check_scales<FP8>(sh, k_scale, v_scale);
     if (st != PA_OK || sh.num_seqs == 0) return st;
@@ -400,6 +403,7 @@ pa_status decode_one_pass(void* out, const void* q, const void* k_cache, const v
     p.v_scale = v_scale;
     p.new_key = new_key;
     p.new_value = new_value;
+    p.ref_counts = ref_counts;
     const dim3 grid(1, sh.num_kv_heads, sh.num_seqs);
     const cudaError_t e = decode_dispatch<false, FP8>(static_cast<pa_dtype>(sh.dtype), sh.head_dim, sh.block_size,
                                                       p, grid, static_cast<cudaStream_t>(stream));
@@ -512,18 +516,19 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache, const void* v
 pa_status pa_decode_append(void* out, const void* q, const void* key, const void* value, void* k_cache, void* v_cache,
                            const int32_t* block_tables, const int32_t* context_lens, float scale, int block_size,
                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
-                           int max_context_len, int64_t num_blocks, pa_dtype dtype, const int32_t* seq_order,
-                           void* stream) {
+                           int max_context_len, int64_t num_blocks, pa_dtype dtype, const int32_t* ref_counts,
+                           const int32_t* seq_order, void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     if (st != PA_OK || num_seqs == 0) return st;
     if (!key || !value || !aligned16(key) || !aligned16(value)) return PA_ERR_INVALID_ARG;
-    if (!aligned4(seq_order)) return PA_ERR_INVALID_ARG;
+    if (!aligned4(seq_order) || !aligned4(ref_counts)) return PA_ERR_INVALID_ARG;
     pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
     p.seq_order = seq_order;
     p.new_key = key;
     p.new_value = value;
+    p.ref_counts = ref_counts;
     const dim3 grid(1, num_kv_heads, num_seqs);
     const cudaError_t e = decode_dispatch<false>(dtype, head_dim, block_size, p, grid,
                                                  static_cast<cudaStream_t>(stream));
@@ -608,13 +613,14 @@ pa_status pa_decode_append_fp8(void* out, const void* q, const void* key, const 
                                void* v_cache, const float* k_scale, const float* v_scale, const int32_t* block_tables,
                                const int32_t* context_lens, float scale, int block_size, int num_seqs,
                                int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
-                               int max_context_len, int64_t num_blocks, pa_dtype dtype, const int32_t* seq_order,
-                               void* stream) {
+                               int max_context_len, int64_t num_blocks, pa_dtype dtype,
+                               const int32_t* ref_counts, const int32_t* seq_order, void* stream) {
     const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                          max_context_len, num_blocks, static_cast<int>(dtype)};
     if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PA_ERR_INVALID_ARG;
+    if (!aligned4(ref_counts)) return PA_ERR_INVALID_ARG;
     return decode_one_pass<true>(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, sh,
-                                 seq_order, stream, key, value);
+                                 seq_order, stream, key, value, ref_counts);
 }
 
 pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -719,6 +725,124 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+// ---- block management (pa_blocks.cuh)
+
+namespace {
+
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+pa_status check_block_state(const int32_t* ref_counts, const int32_t* free_ids, const int64_t* free_state,
+                            int64_t num_blocks) {
+    if (num_blocks <= 0 || num_blocks > INT_MAX) return PA_ERR_INVALID_ARG;
+    if (!ref_counts || !free_ids || !free_state) return PA_ERR_INVALID_ARG;
+    if (!aligned4(ref_counts) || !aligned4(free_ids) || !aligned8(free_state)) return PA_ERR_INVALID_ARG;
+    return PA_OK;
+}
+
+pa_status check_rows(const int32_t* block_tables, const int32_t* context_lens, int num_seqs, int max_blocks_per_seq,
+                     int block_size) {
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (static_cast<long long>(max_blocks_per_seq) * block_size > INT_MAX) return PA_ERR_UNSUPPORTED;
+    if (num_seqs > 0 && (!block_tables || !context_lens || !aligned4(block_tables) || !aligned4(context_lens)))
+        return PA_ERR_INVALID_ARG;
+    return PA_OK;
+}
+
+pa::BlockState block_state(int32_t* ref_counts, const int32_t* free_ids, int64_t* free_state, int64_t num_blocks) {
+    pa::BlockState st{};
+    st.ref = ref_counts;
+    st.free_ids = const_cast<int32_t*>(free_ids);
+    st.free_state = reinterpret_cast<long long*>(free_state);
+    st.num_blocks = num_blocks;
+    return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_blocks_init(int32_t* ref_counts, int32_t* free_ids, int64_t* free_state, int64_t num_blocks,
+                         void* stream) {
+    const pa_status st = check_block_state(ref_counts, free_ids, free_state, num_blocks);
+    if (st != PA_OK) return st;
+    const long long blocks = std::min<long long>((num_blocks + 255) / 256, 4096);
+    pa::pa_blocks_init_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        block_state(ref_counts, free_ids, free_state, num_blocks));
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_blocks_append(int32_t* block_tables, int32_t* context_lens, const int32_t* num_new_tokens,
+                           int32_t* ref_counts, const int32_t* free_ids, int64_t* free_state, int64_t* slot_mapping,
+                           int64_t num_slots, int64_t* copy_pairs, int num_seqs, int max_blocks_per_seq,
+                           int block_size, int64_t num_blocks, void* stream) {
+    pa_status st = check_block_state(ref_counts, free_ids, free_state, num_blocks);
+    if (st == PA_OK) st = check_rows(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size);
+    if (st != PA_OK) return st;
+    if (num_slots < 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!num_new_tokens || !copy_pairs || !aligned4(num_new_tokens) || !aligned8(copy_pairs)) return PA_ERR_INVALID_ARG;
+    if (num_slots > 0 && (!slot_mapping || !aligned8(slot_mapping))) return PA_ERR_INVALID_ARG;
+    pa::AppendParams p{};
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.num_new = num_new_tokens;
+    p.st = block_state(ref_counts, free_ids, free_state, num_blocks);
+    p.slots = reinterpret_cast<long long*>(slot_mapping);
+    p.num_slots = num_slots;
+    p.pairs = reinterpret_cast<long long*>(copy_pairs);
+    p.num_seqs = num_seqs;
+    p.max_blocks = max_blocks_per_seq;
+    p.block_size = block_size;
+    pa::pa_blocks_append_kernel<<<1, pa::kBlocksThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_blocks_fork(int32_t* block_tables, int32_t* context_lens, int32_t* ref_counts, const int32_t* forks,
+                         int num_forks, int num_seqs, int max_blocks_per_seq, int block_size, int64_t num_blocks,
+                         void* stream) {
+    pa_status st = check_rows(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size);
+    if (st != PA_OK) return st;
+    if (num_forks < 0 || num_blocks <= 0 || num_blocks > INT_MAX) return PA_ERR_INVALID_ARG;
+    if (num_forks == 0 || num_seqs == 0) return PA_OK;
+    if (!ref_counts || !forks || !aligned4(ref_counts) || !aligned4(forks)) return PA_ERR_INVALID_ARG;
+    pa::ForkParams p{};
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.ref = ref_counts;
+    p.forks = forks;
+    p.num_forks = num_forks;
+    p.num_seqs = num_seqs;
+    p.max_blocks = max_blocks_per_seq;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    pa::pa_blocks_fork_kernel<<<1, pa::kBlocksThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_blocks_release(int32_t* block_tables, int32_t* context_lens, int32_t* ref_counts, int32_t* free_ids,
+                            int64_t* free_state, const int32_t* seqs, int num_release, int num_seqs,
+                            int max_blocks_per_seq, int block_size, int64_t num_blocks, void* stream) {
+    pa_status st = check_block_state(ref_counts, free_ids, free_state, num_blocks);
+    if (st == PA_OK) st = check_rows(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size);
+    if (st != PA_OK) return st;
+    if (num_release < 0) return PA_ERR_INVALID_ARG;
+    if (num_release == 0 || num_seqs == 0) return PA_OK;
+    if (!seqs || !aligned4(seqs)) return PA_ERR_INVALID_ARG;
+    pa::ReleaseParams p{};
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.st = block_state(ref_counts, free_ids, free_state, num_blocks);
+    p.seqs = seqs;
+    p.num_release = num_release;
+    p.num_seqs = num_seqs;
+    p.max_blocks = max_blocks_per_seq;
+    p.block_size = block_size;
+    pa::pa_blocks_release_kernel<<<1, pa::kBlocksThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 pa_status pa_get_device_error(void* stream, int32_t* code) {
     if (!code) return PA_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
@@ -812,3 +936,45 @@ extern "C" pa_status pa_decode_splitk_static(void* out, const void* q, const voi
                             num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, max_context_len, num_blocks,
                             dtype, partition_size, scratch, kStaticScratchBytes, nullptr, 0, nullptr, stream);
 }
+
+#ifdef PA_TEST_HOOKS
+// ----------------------------------------------------------------------------
+// Test hooks (libpa_test.so only; declared in pa_test.h).
+
+namespace {
+
+// One warp waits on an mbarrier that no thread or copy ever completes.
+__global__ void pa_test_wait_kernel(unsigned long long limit_ns, long long* elapsed_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        pa::mbar_init(&bar, 1);
+        pa::fence_barrier_init();
+    }
+    __syncwarp();
+    const uint64_t t0 = pa::global_timer_ns();
+    const bool done = pa::mbar_wait_bounded(&bar, 0, limit_ns);
+    const uint64_t t1 = pa::global_timer_ns();
+    if (threadIdx.x == 0) {
+        if (!done) pa::flag_error(PA_DEVERR_TIMEOUT);
+        *elapsed_ns = static_cast<long long>(t1 - t0);
+    }
+}
+
+}  // namespace
+
+extern "C" pa_status pa_test_set_hooks(int64_t wait_limit_ns, int skip_first_copy) {
+    if (wait_limit_ns <= 0) return PA_ERR_INVALID_ARG;
+    const unsigned long long limit = static_cast<unsigned long long>(wait_limit_ns);
+    if (cudaMemcpyToSymbol(pa::g_test_wait_limit_ns, &limit, sizeof(limit)) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(pa::g_test_skip_first_copy, &skip_first_copy, sizeof(int)) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return PA_OK;
+}
+
+extern "C" pa_status pa_test_wait_timeout(int64_t limit_ns, int64_t* elapsed_ns, void* stream) {
+    if (limit_ns <= 0 || !elapsed_ns || (reinterpret_cast<uintptr_t>(elapsed_ns) & 7u)) return PA_ERR_INVALID_ARG;
+    pa_test_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<unsigned long long>(limit_ns),
+                                                                         reinterpret_cast<long long*>(elapsed_ns));
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+#endif  // PA_TEST_HOOKS

@@ -39,7 +39,8 @@ __global__ void __launch_bounds__(kCopyThreads) pa_copy_blocks_kernel(const __gr
     const long long pair = rest >> 1;
     const long long src = p.mapping[2 * pair];
     const long long dst = p.mapping[2 * pair + 1];
-    if (src < 0 || src >= p.src_blocks || dst < 0 || dst >= p.dst_blocks) {
+    if (src < 0) return;  // an empty entry (no copy for this pair)
+    if (src >= p.src_blocks || dst < 0 || dst >= p.dst_blocks) {
         if (threadIdx.x == 0 && pool == 0 && chunk == 0) flag_error(1 /* PA_DEVERR_BLOCK_ID */);
         return;
     }

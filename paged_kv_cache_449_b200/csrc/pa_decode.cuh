@@ -61,6 +61,7 @@ struct DecodeParams {
     const int32_t* seq_order;  // optional [S] permutation: CTA z works on sequence seq_order[z]; null = z
     const float* k_scale;      // 8-bit pools: [Hkv] scales of the K and V codes
     const float* v_scale;
+    const int32_t* ref_counts;  // append: [num_blocks] reference counts, or null (not checked)
 };
 
 // Append: the newest token of sequence s (logical position L-1) is written
@@ -302,8 +303,8 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const int n_w = nb > warp ? (nb - warp + NW - 1) / NW : 0;
     // Append: the warp that will compute the last block loads the new row now.
     const int last_block = nblk - 1;
-    const bool owns_last = p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
-                           (last_block - b0) % NW == warp;
+    bool owns_last = p.new_key != nullptr && last_block >= b0 && last_block < b1 &&
+                     (last_block - b0) % NW == warp;
     NewRow<T, D> new_row;
     NewRowE4m3<T, D> new_row8;
     if constexpr (FP8) {
@@ -338,6 +339,9 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const char* vpool = reinterpret_cast<const char*>(p.v_cache);
     auto issue = [&](int i) {
         const int id = block_id(i);
+#ifdef PA_TEST_HOOKS
+        if (g_test_skip_first_copy && i == 0 && warp == 0 && s == 0 && kvh == 0 && part == 0) return;
+#endif
         if (lane == 0) {
             const int st = i % STAGES;
             uint8_t* dst = wring + st * 2 * kTile;
@@ -356,6 +360,15 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
 
     int issued = n_w < STAGES ? n_w : STAGES;
     for (int i = 0; i < issued; ++i) issue(i);
+    if (owns_last && p.ref_counts != nullptr) {
+        // Copy-on-write guard: the block the newest token goes to must be held
+        // by this sequence alone.  Checked while the first copies are in flight.
+        const int id = __ldg(p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq + last_block);
+        if (id >= 0 && id < p.num_blocks && __ldg(p.ref_counts + id) != 1) {
+            if (lane == 0) flag_error(128 /* PA_DEVERR_SHARED_BLOCK */);
+            owns_last = false;  // no write; the pool is attended as it is
+        }
+    }
     bool failed = false;
     int i = 0;
     for (; i < n_w; ++i) {
@@ -365,7 +378,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
             win1 = load_ids(cur_round + 1);
         }
         const int st = i % STAGES;
-        if (!mbar_wait_bounded(&wbar[st], (i / STAGES) & 1, kWaitLimitNs)) {
+        if (!mbar_wait_bounded(&wbar[st], (i / STAGES) & 1, wait_limit_ns())) {
             failed = true;
             break;
         }
@@ -396,7 +409,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     if (failed) {
         if (lane == 0) flag_error(8 /* PA_DEVERR_TIMEOUT */);
         // Let the copies already in flight land before the CTA may exit.
-        for (int k = i; k < issued; ++k) mbar_wait_bounded(&wbar[k % STAGES], (k / STAGES) & 1, kWaitLimitNs);
+        for (int k = i; k < issued; ++k) mbar_wait_bounded(&wbar[k % STAGES], (k / STAGES) & 1, wait_limit_ns());
     }
     const int any_failed = __syncthreads_or(failed ? 1 : 0);
 
@@ -411,15 +424,19 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         // sum 0, zero output) so that no merge reads what an earlier call left
         // in the workspace, and the fused merge below still counts it, which
         // brings the arrival counter back to zero.
-        if (!to_workspace) return;
-        for (int idx = threadIdx.x; idx < group * D; idx += NW * 32) {
-            const int r = idx / D, d = idx - r * D;
-            const long long slot =
-                (static_cast<long long>(s) * p.num_q_heads + kvh * group + r) * p.num_partitions + part;
-            p.part_acc[slot * D + d] = 0.f;
-            if (d == 0) {
-                p.part_ml[slot * 2] = kNegInf;
-                p.part_ml[slot * 2 + 1] = 0.f;
+        if constexpr (!SPLIT) {
+            return;
+        } else {
+            if (!to_workspace) return;
+            for (int idx = threadIdx.x; idx < group * D; idx += NW * 32) {
+                const int r = idx / D, d = idx - r * D;
+                const long long slot =
+                    (static_cast<long long>(s) * p.num_q_heads + kvh * group + r) * p.num_partitions + part;
+                p.part_acc[slot * D + d] = 0.f;
+                if (d == 0) {
+                    p.part_ml[slot * 2] = kNegInf;
+                    p.part_ml[slot * 2 + 1] = 0.f;
+                }
             }
         }
     }

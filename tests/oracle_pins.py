@@ -522,6 +522,10 @@ def pin_errors(orc):
         assert "block id" in str(e)
     else:
         raise AssertionError("oracle accepted a block copy past the pool")
+    # a negative source id is an empty entry: nothing is copied and nothing is refused
+    k2, v2 = b.k_cache.clone(), b.v_cache.clone()
+    orc.copy_blocks(k2, v2, k2, v2, torch.tensor([[-1, 0], [-1, -1]]), 8)
+    assert torch.equal(k2, b.k_cache) and torch.equal(v2, b.v_cache)
 
 
 def pin_number_formats(orc):

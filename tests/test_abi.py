@@ -16,14 +16,21 @@ from paged_kv_cache_449_b200 import build as pabuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def declared_functions():
+def declared_functions(headers=None):
+    """Entry points declared in include/*.h (all but the test hooks' pa_test.h
+    unless `headers` names the files)."""
     names = []
     for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
-        if h.endswith(".h"):
+        if h.endswith(".h") and (h in headers if headers else h != "pa_test.h"):
             text = open(os.path.join(ROOT, "include", h)).read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
             names += re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
+
+
+def exported(path):
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    return set(re.findall(r"\bT\s+(\w+)$", out, flags=re.M))
 
 
 @pytest.fixture(scope="module")
@@ -37,16 +44,26 @@ def test_header_declares_the_boundary():
         "pa_copy_blocks", "pa_decode", "pa_decode_append", "pa_decode_append_fp8", "pa_decode_fp8", "pa_decode_splitk",
         "pa_decode_splitk_fp8", "pa_decode_splitk_workspace_size", "pa_reshape_and_cache_fp8", "pa_prefill",
         "pa_decode_splitk_static", "pa_get_device_error",
-        "pa_reshape_and_cache", "pa_status_string"])
+        "pa_reshape_and_cache", "pa_status_string",
+        "pa_blocks_init", "pa_blocks_append", "pa_blocks_fork", "pa_blocks_release"])
 
 
 def test_library_exports_every_declared_symbol(lib):
-    out = subprocess.run(["nm", "-D", "--defined-only", pa.library_path()], capture_output=True, text=True,
-                         check=True).stdout
-    exported = set(re.findall(r"\bT\s+(\w+)$", out, flags=re.M))
+    have = exported(pa.library_path())
     for name in declared_functions():
-        assert name in exported, name
+        assert name in have, name
         assert getattr(lib, name) is not None
+    # the test hooks are not in the product library
+    hooks = declared_functions(headers=("pa_test.h",))
+    assert hooks == ["pa_test_set_hooks", "pa_test_wait_timeout"]
+    assert not set(hooks) & have
+
+
+def test_test_library_exports_the_hooks():
+    path = pabuild.build_test()
+    have = exported(path)
+    for name in declared_functions() + declared_functions(headers=("pa_test.h",)):
+        assert name in have, name
 
 
 def test_library_needs_no_cuda_driver_or_shared_cudart(lib):
@@ -102,7 +119,8 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_decode_splitk(*args, 512, 0, 1 << 20, None, 0, None, None) == 3    # no workspace
     assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, 16, 3, None, None) == 3     # too few counters
     assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, None, 0, 6, None) == 1      # misaligned seq_order
-    assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], 2, None) == 1            # misaligned seq_order
+    assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], None, 2, None) == 1      # misaligned seq_order
+    assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], 6, None, None) == 1      # misaligned ref_counts
     cp = [16, 16, 16, 16, 16, 4, 8, 128, 16, 10, 10, 2, None]
     assert lib.pa_copy_blocks(*cp[:5], 0, *cp[6:]) == 0                             # no pairs: a no-op
     assert lib.pa_copy_blocks(*cp[:5], -1, *cp[6:]) == 1                            # negative count
@@ -113,14 +131,29 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_copy_blocks(*cp[:9], 0, *cp[10:]) == 1                            # empty source pool
     f8 = [16, 16, 16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 64]
     assert lib.pa_decode_fp8(*f8, 0, None, None) == 2                                # fp32 queries
-    assert lib.pa_decode_append_fp8(16, 16, 0, 16, *f8[2:], 2, None, None) == 1      # no new key
-    assert lib.pa_decode_append_fp8(16, 16, 16, 16, *f8[2:], 0, None, None) == 2     # fp32 queries
+    assert lib.pa_decode_append_fp8(16, 16, 0, 16, *f8[2:], 2, None, None, None) == 1      # no new key
+    assert lib.pa_decode_append_fp8(16, 16, 16, 16, *f8[2:], 0, None, None, None) == 2     # fp32 queries
+    assert lib.pa_decode_append_fp8(16, 16, 16, 16, *f8[2:], 2, 6, None, None) == 1       # misaligned ref_counts
     assert lib.pa_decode_fp8(*f8[:4], 0, *f8[5:], 2, None, None) == 1                # no K scale
     assert lib.pa_decode_fp8(*f8[:5], 18, *f8[6:], 2, None, None) == 1               # V scale misaligned
     assert lib.pa_decode_splitk_fp8(*f8, 1, 500, 16, 1 << 20, None, 0, None, None) == 1  # partition not x16
     assert lib.pa_decode_splitk_fp8(*f8, 1, 512, 16, 100, None, 0, None, None) == 3       # workspace too small
     assert lib.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 16, 16, 4, 8, 40, 16, 10, 2, None) == 2  # D % 16
     assert lib.pa_reshape_and_cache_fp8(16, 16, 16, 16, 16, 0, 16, 4, 8, 64, 16, 10, 2, None) == 1   # no scale
+    # block management: refused before any launch
+    assert lib.pa_blocks_init(16, 16, 16, 0, None) == 1                                 # no blocks
+    assert lib.pa_blocks_init(16, 16, 12, 8, None) == 1                                 # state not 8-byte aligned
+    assert lib.pa_blocks_init(16, 0, 16, 8, None) == 1                                  # no ring
+    ap = [16, 16, 16, 16, 16, 16, 16, 4, 16, 4, 8, 16, 64, None]
+    assert lib.pa_blocks_append(*ap[:9], 0, *ap[10:]) == 0                              # no sequences: no-op
+    assert lib.pa_blocks_append(*ap[:8], 12, *ap[9:]) == 1                              # pairs not 8-byte aligned
+    assert lib.pa_blocks_append(*ap[:7], -1, *ap[8:]) == 1                              # negative slot capacity
+    assert lib.pa_blocks_append(*ap[:11], 0, *ap[12:]) == 1                             # block size 0
+    assert lib.pa_blocks_append(*ap[:12], 1 << 40, None) == 1                           # more blocks than int32 ids
+    assert lib.pa_blocks_fork(16, 16, 16, 16, 0, 4, 8, 16, 64, None) == 0               # no forks: no-op
+    assert lib.pa_blocks_fork(16, 16, 16, 18, 2, 4, 8, 16, 64, None) == 1               # forks misaligned
+    assert lib.pa_blocks_release(16, 16, 16, 16, 16, 16, -1, 4, 8, 16, 64, None) == 1   # negative count
+    assert lib.pa_blocks_release(16, 16, 16, 16, 16, 0, 2, 4, 8, 16, 64, None) == 1     # no list
     pf = [16, 16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 100, 64]
     assert lib.pa_prefill(*pf, 0, None) == 2                                             # fp32 queries
     assert lib.pa_prefill(*pf[:6], 0, *pf[7:], 2, None) == 1                             # no query_start
