@@ -15,6 +15,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "pa_api.cu")
 LIB = os.path.join(HERE, "libpa.so")
+# The same sources with the test hooks of include/pa_test.h compiled in (for
+# the tests of the kernels' bounded waits); never loaded by the product.
+TEST_LIB = os.path.join(HERE, "libpa_test.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -27,12 +30,13 @@ def nvcc_path() -> str:
 
 def sources() -> list[str]:
     return [SRC] + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + \
-        [os.path.join(ROOT, "include", "pa.h")]
+        sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def build(out: str = LIB, defines: dict | None = None, force: bool = False, verbose: bool = False) -> str:
-    """Compile the library; skipped when `out` is newer than every source."""
-    if not force and not defines and os.path.exists(out):
+    """Compile the library; skipped when `out` is newer than every source
+    (each output file is built with one fixed set of defines)."""
+    if not force and os.path.exists(out):
         if os.path.getmtime(out) >= max(os.path.getmtime(s) for s in sources()):
             return out
     cmd = [nvcc_path(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
@@ -46,6 +50,11 @@ def build(out: str = LIB, defines: dict | None = None, force: bool = False, verb
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
     return out
+
+
+def build_test(force: bool = False) -> str:
+    """libpa_test.so: the library with PA_TEST_HOOKS defined."""
+    return build(TEST_LIB, defines={"PA_TEST_HOOKS": 1}, force=force)
 
 
 if __name__ == "__main__":

@@ -74,6 +74,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait, far above any copy time
 
+#ifdef PA_TEST_HOOKS
+// Test builds only (libpa_test.so): the wait limit, and a switch that makes
+// the first warp of the decode CTA of (sequence 0, kv head 0, partition 0)
+// leave its first ring stage unfilled, so that its wait runs out and the
+// kernel's timeout path runs (no copy is left in flight: the stage is simply
+// never issued).
+__device__ unsigned long long g_test_wait_limit_ns = kWaitLimitNs;
+__device__ int g_test_skip_first_copy = 0;
+__device__ __forceinline__ uint64_t wait_limit_ns() { return g_test_wait_limit_ns; }
+#else
+__device__ __forceinline__ constexpr uint64_t wait_limit_ns() { return kWaitLimitNs; }
+#endif
+
 // Waits for phase `parity` of `bar` to complete, giving up after `limit_ns`
 // of wall time (returns false then).  Never spins without bound.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
