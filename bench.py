@@ -78,6 +78,9 @@ def parse_args(argv=None):
     ap.add_argument("--graph", action="store_true",
                     help="capture each rotated copy's step into a CUDA graph once and replay it in the timed region")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration lines (by default the headline run also times every other "
+                         "configuration and widened row and reports them under `configs`)")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     return ap.parse_args(argv)
 
@@ -647,6 +650,229 @@ def run_gpu(args, world, rank, local):
     return result, batch
 
 
+# ----------------------------------------------------------------------------- every configuration
+
+def time_decode_steps(batch, mode, partition_size, fp8, steps, warmup, world):
+    """Device time of one step (write of the newest tokens + decode) on the
+    batch: rotated independent copies larger than L2 when the workload allows
+    (K steps in one CUDA-event region), else a 256 MiB L2 flush and per-step
+    events.  Returns (ms per step, max over ranks; launches per step; L2
+    note)."""
+    import paged_kv_cache_449_b200 as pa
+    stream = torch.cuda.current_stream()
+    unique = batch.unique_kv_bytes() // (2 if fp8 is not None else 1)
+    copies = rotation_copies(unique, l2_bytes())
+    steps_ = [Step(batch, mode, partition_size, independent=i > 0, fp8=fp8) for i in range(max(1, copies))]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if copies == 0 else None
+
+    def one(i):
+        st = steps_[i % len(steps_)]
+        st.reshape(stream)
+        st.decode(stream)
+
+    for i in range(warmup):
+        if flush is not None:
+            flush.zero_()
+        one(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    if flush is None:
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for i in range(steps):
+            one(i)
+        ev[1].record(stream)
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / steps
+        note = f"rotated over {len(steps_)} independent copies larger than L2, one event region"
+    else:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            one(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+        note = "256 MiB L2 flush between steps, per-step events"
+    barrier(world)
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError(f"device error word set on {batch.name}")
+    return reduce_max(ms, world), steps_[0].kernels_per_step, note
+
+
+def profiled_kernel_ms(fn, n, names):
+    """Average device duration of each named kernel over n calls of fn, from
+    the CUDA activity records of torch.profiler (device timestamps, not a
+    replaying profiler).  None where the records are unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            for i in range(n):
+                fn(i)
+            torch.cuda.synchronize()
+        out = {}
+        for ev in prof.key_averages():
+            for name in names:
+                if name in ev.key:
+                    total = getattr(ev, "device_time_total", None)
+                    if total is None:
+                        total = getattr(ev, "cuda_time_total", 0.0)
+                    cnt = out.get(name, (0.0, 0))
+                    out[name] = (cnt[0] + total, cnt[1] + ev.count)
+        return {k: (t / c / 1e3 if c else None) for k, (t, c) in out.items()}
+    except Exception as err:  # the profiler's CUDA activity records are optional
+        return {"unavailable": str(err)[:200]}
+
+
+def block_manager_step(seed, steps, warmup, world, peak):
+    """A whole decode step with the device block manager, on the Llama-3-8B
+    batch: pa_blocks_append (one token per sequence: a block taken from the
+    free ring when the token starts a block) + pa_copy_blocks (the step's
+    copy-on-write pairs) + pa_decode_append (write + attend, reference counts
+    checked).  The state starts from the batch's tables with each sequence
+    one token short; the lengths grow by one per step (steps + warm-up
+    tokens, negligible next to ~1000-token contexts)."""
+    import paged_kv_cache_449_b200 as pa
+    import workloads
+    b = workloads.llama3_8b_decode(seed=seed, device="cuda")
+    B, N, S = b.block_size, b.num_blocks, b.num_seqs
+    total = steps + warmup + 1
+    mb = b.max_blocks_per_seq + (total + B - 1) // B + 1
+    lens0 = (b.context_lens - 1).to(torch.int64)
+    tables = torch.full((S, mb), -1, dtype=torch.int32)
+    ref = torch.zeros(N, dtype=torch.int32)
+    for s_ in range(S):
+        n = int((lens0[s_] + B - 1) // B)
+        tables[s_, :n] = b.block_tables[s_, :n]
+        ref[b.block_tables[s_, :n].long()] = 1
+    free = torch.nonzero(ref == 0).flatten().to(torch.int32)
+    ring = torch.full((N,), -1, dtype=torch.int32)
+    ring[:free.numel()] = free
+    d = "cuda"
+    tables, lens, ref, ring = tables.to(d), lens0.to(torch.int32).to(d), ref.to(d), ring.to(d)
+    state = torch.tensor([0, free.numel()], dtype=torch.int64, device=d)
+    ones = torch.ones(S, dtype=torch.int32, device=d)
+    slots = torch.empty(S, dtype=torch.int64, device=d)
+    pairs = torch.empty((S, 2), dtype=torch.int64, device=d)
+    k, v, q = b.k_cache, b.v_cache, b.q.to(d)
+    nk, nv = b.new_key.to(d), b.new_value.to(d)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+
+    def one(i):
+        pa.pa_blocks_append(tables, lens, ones, ref, ring, state, slots, pairs, B, stream=stream)
+        pa.pa_copy_blocks(k, v, k, v, pairs, stream=stream)
+        pa.pa_decode_append(out, q, nk, nv, k, v, tables, lens, b.scale, max_context_len=mb * B, stream=stream,
+                            ref_counts=ref)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for i in range(steps):
+        one(i)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms = reduce_max(ev[0].elapsed_time(ev[1]) / steps, world)
+    per_kernel = profiled_kernel_ms(one, 1, ("pa_blocks_append_kernel", "pa_copy_blocks_kernel", "pa_decode_kernel"))
+    if pa.pa_get_device_error() != 0:
+        raise RuntimeError("device error word set in the block-manager step")
+    nbytes = b.algorithmic_bytes()
+    gbs = reduce_sum(nbytes, world) / (ms * 1e-3) / 1e9
+    return {"workload": b.name + " + device block manager",
+            "entry": "pa_blocks_append + pa_copy_blocks + pa_decode_append (ref counts)",
+            "ms_per_step": round(ms, 5), "algorithmic_bytes": int(nbytes), "gb_per_s": round(gbs, 2),
+            "frac_of_measured_hbm": round(gbs / world / peak, 4),
+            "kernel_ms": {k_: (round(v_, 5) if isinstance(v_, float) else v_) for k_, v_ in per_kernel.items()},
+            "kernel_ms_how": "torch.profiler CUDA activity records of one step after the timed ones",
+            "gpu_launches": 3 * steps,
+            "l2": "one copy of the pools (290 MB of KV per step, more than twice the L2), K steps in one event region"}
+
+
+def config_lines(args, world, rank):
+    """One entry per configuration of the hot path (and of the widened rows),
+    each timed on its own seeded workload with the same rules as the
+    headline: device-resident inputs, warm-up, CUDA events, rotated copies
+    larger than L2 (or an L2 flush where the workload is smaller than L2)."""
+    import paged_kv_cache_449_b200 as pa
+    import workloads
+    peak, peak_kind = measured_peaks()
+    K, W = args.steps, max(3, args.warmup)
+    out = {}
+
+    def entry(batch, mode, part=None, fp8=None, note=None):
+        ms, launches, l2 = time_decode_steps(batch, mode, part or args.partition_size, fp8, K, W, world)
+        dec, resh = step_bytes(batch, fp8)
+        logical = dec + resh
+        unique = (batch.algorithmic_bytes(unique=True) if fp8 is None else dec) + resh
+        gbs = reduce_sum(unique, world) / (ms * 1e-3) / 1e9
+        e = {"workload": batch.name + ("+e4m3" if fp8 is not None else ""), "entry": {
+                "append": "pa_decode_append" + ("_fp8" if fp8 is not None else ""),
+                "single": "pa_reshape_and_cache + pa_decode",
+                "splitk": f"pa_reshape_and_cache + pa_decode_splitk (fused merge, partition {part})",
+                "splitk2": f"pa_reshape_and_cache + pa_decode_splitk (merge kernel, partition {part})"}[mode],
+             "seqs": batch.num_seqs, "block_size": batch.block_size, "ms_per_step": round(ms, 5),
+             "algorithmic_bytes": int(unique), "gb_per_s": round(gbs, 2),
+             "frac_of_measured_hbm": round(gbs / world / peak, 4), "frac_of_spec_8tbs": round(gbs / world / SPEC_HBM_GBS, 4),
+             "tokens_per_s": round(reduce_sum(batch.num_seqs, world) / (ms * 1e-3), 1),
+             "gpu_launches": launches * K, "l2": l2}
+        if unique != logical:
+            e["logical_bytes"] = int(logical)
+            e["bytes_basis"] = "unique: shared-prefix blocks counted once (logical bytes beside)"
+        if note:
+            e["note"] = note
+        return e
+
+    seed = args.seed + rank
+    b = workloads.tiny_mha_f32(seed=seed, device="cuda")
+    out["tiny_mha_f32"] = entry(b, "append", note="parity configuration: launch-bound, its GB/s is not a "
+                                                  "bandwidth figure")
+    del b
+    for B in (8, 16, 32):
+        b = workloads.continuous_batching_mix(seed=seed, device="cuda", block_size=B)
+        out[f"continuous_batching_mix_B{B}"] = entry(b, "append")
+        del b
+    b = workloads.prefix_sharing(seed=seed, device="cuda")
+    out["prefix_sharing"] = entry(b, "append")
+    del b
+    b = workloads.llama3_70b_long(seed=seed, device="cuda")
+    out["llama3_70b_long"] = entry(b, "splitk", part=1024)
+    two = entry(b, "splitk2", part=1024)
+    st = Step(b, "splitk2", 1024)
+    stream = torch.cuda.current_stream()
+    per_kernel = profiled_kernel_ms(lambda i: (st.reshape(stream), st.decode(stream)), min(K, 20),
+                                    ("pa_reshape_kernel", "pa_decode_kernel", "pa_merge_kernel"))
+    two["kernel_ms"] = {k: (round(v, 5) if isinstance(v, float) else v) for k, v in per_kernel.items()}
+    two["kernel_ms_how"] = ("torch.profiler CUDA activity records over min(steps, 20) steps on one input copy "
+                            "(L2 not flushed between them)")
+    out["llama3_70b_long_two_kernel"] = two
+    del b, st
+    b = workloads.llama3_8b_decode(seed=seed, device="cuda")
+    f8 = workloads.random_fp8_pools(b, seed=seed, device="cuda")
+    out["llama3_8b_decode_e4m3"] = entry(b, "append", fp8=f8)
+    del b, f8
+    torch.cuda.empty_cache()
+    out["serving_step_with_block_manager"] = block_manager_step(seed, K, W, world, peak)
+    torch.cuda.empty_cache()
+    # the widened rows measured by their own bench modes, trimmed to the figures
+    keep = ("metric", "value", "unit", "ms_per_step", "roofline", "gpu_launches")
+    for name, op, workload, steps in (("chunked_prefill", "prefill", args.workload, K),
+                                      ("copy_blocks_cow", "copy_blocks", "llama3_8b_decode", K),
+                                      ("swap_out", "swap_out", "llama3_8b_decode", min(K, 10)),
+                                      ("swap_in", "swap_in", "llama3_8b_decode", min(K, 10))):
+        sub = argparse.Namespace(**dict(vars(args), op=op, workload=workload, steps=steps, warmup=W,
+                                        block_size=None))
+        res = (run_prefill if op == "prefill" else run_blocks)(sub, world, rank, int(os.environ.get("LOCAL_RANK", "0")))
+        e = {k: res[k] for k in keep if k in res}
+        e["workload"] = res["config"]["workload"]
+        out[name] = e
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------------------- the oracle (CPU)
 
 def oracle_sample(batch, seconds_target, seed=0):
@@ -940,6 +1166,11 @@ def main(argv=None):
                 print(json.dumps(res), flush=True)
             return
         res, batch = run_gpu(args, world, rank, local)
+        headline = (args.workload == "llama3_8b_decode" and args.mode == "append" and args.kv == "bf16"
+                    and args.block_size is None and not args.graph)
+        if headline and not args.no_configs:
+            res["configs"] = config_lines(args, world, rank)
+            res["gpu_launches_configs"] = sum(int(v.get("gpu_launches", 0)) for v in res["configs"].values())
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline and args.kv == "bf16":
                 gbs1, desc1, spent, n = oracle_sample(batch, args.cpu_sample_seconds)
