@@ -250,7 +250,6 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     uint64_t* p_full = bars + 28;    // [q * 2 + buffer] P written (and O rescaled)
     uint64_t* p_free = bars + 32;    // [q * 2 + buffer] the O += P V reading that P finished
     uint64_t* drain = bars + 36;     // [2] the S and the O += P V issuers' MMAs finished
-    uint64_t* turn = bars + 38;      // [q] query tile q's softmax may run its exponentials
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Sm::kMiscOff);
     volatile uint32_t* abort = misc + 1;
 
@@ -304,8 +303,6 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
         }
         mbar_init(&drain[0], 1);
         mbar_init(&drain[1], 1);
-        mbar_init(&turn[0], 4);
-        mbar_init(&turn[1], 4);
         *abort = 0u;
         fence_barrier_init();
     }
@@ -606,18 +603,6 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                 failed = true;
                 break;
             }
-            // The two query tiles take turns at their exponentials (tile 0's of
-            // key tile j, then tile 1's of j, then tile 0's of j + 1, ...): the
-            // exponential unit is the scarcest resource of the loop, and the
-            // tile not at its turn loads, masks and stores meanwhile.
-            const int other_n = qt == 0 ? nt[1] : nt[0];
-            if (qt == 0 ? (j >= 1 && j - 1 < other_n) : (j < other_n)) {
-                const uint32_t par = static_cast<uint32_t>(qt == 0 ? j - 1 : j) & 1u;
-                if (!__all_sync(0xffffffffu, tc_wait(&turn[qt], par, abort))) {
-                    failed = true;
-                    break;
-                }
-            }
             // P = 2^(s * scale - mu): arguments and row sums two at a time, the
             // sums in four independent pairs
             const uint64_t scale2 = tc::f2(scale, scale), nmu2 = tc::f2(-mu, -mu);
@@ -636,8 +621,6 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                     pw[4 * k8 + e] = Mma<T>::pack(a0, a1);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&turn[qt ^ 1]);
             static_assert(kKeys / 2 == 32, "one 32-column store");
             tc::st32u(p_tmem + lane_base + static_cast<uint32_t>(j & 1) * (kKeys / 2), pw);
             float rs;
