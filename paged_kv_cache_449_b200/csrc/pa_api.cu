@@ -795,7 +795,8 @@ pa_status pa_blocks_append(int32_t* block_tables, int32_t* context_lens, const i
     p.num_seqs = num_seqs;
     p.max_blocks = max_blocks_per_seq;
     p.block_size = block_size;
-    pa::pa_blocks_append_kernel<<<1, pa::kBlocksThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    const int threads = std::min(pa::kBlocksThreads, (num_seqs + 31) / 32 * 32);
+    pa::pa_blocks_append_kernel<<<1, threads, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

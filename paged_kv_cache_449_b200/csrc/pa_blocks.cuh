@@ -11,7 +11,7 @@
 //   free_state int64 [2]   head, tail (positions only grow; tail - head free)
 // plus the block tables and context lengths of the attention kernels.
 //
-// Every operation is one launch of one CTA (1024 threads).  The work is a few
+// Every operation is one launch of one CTA (up to 1024 threads).  The work is a few
 // loads and stores per sequence or block, so a launch costs its latency, not
 // bandwidth; one CTA keeps the order of the sequential definition (sequences
 // in index order, blocks in logical order, the ring first in first out)
@@ -121,71 +121,65 @@ __device__ __forceinline__ bool describe_append(const AppendParams& p, int s, in
     return true;
 }
 
+// Free-ring entries staged in shared memory at the start (the blocks a step
+// takes are the ring's first ones); further entries are read from global memory.
+constexpr int kRingWindow = 2048;
+
+// Launched with blockDim.x = a multiple of 32 up to kBlocksThreads (the
+// batch rounded up: a small batch syncs few warps).
 __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const __grid_constant__ AppendParams p) {
     __shared__ long long sh[33];
     __shared__ int shx[kBlocksThreads];
+    __shared__ int32_t window[kRingWindow];
     __shared__ long long taken_sh;
-    __shared__ int abort_sh;
-    const int S = p.num_seqs, B = p.block_size, tid = threadIdx.x;
+    const int S = p.num_seqs, B = p.block_size, tid = threadIdx.x, T = blockDim.x;
     const long long N = p.st.num_blocks;
+    const long long head = p.st.free_state[0], tail = p.st.free_state[1];
+    const long long avail = tail - head;
     long long total;
 
-    // 0. the packed slot array must hold every token of the step
-    long long tokens = 0;
-    for (int base = 0; base < S; base += kBlocksThreads) {
-        const int s = base + tid;
-        const long long n = s < S ? max(p.num_new[s], 0) : 0;
-        cta_exclusive_scan<long long>(n, &total, sh);
-        tokens += total;
+    // 1. per sequence: its token count (the packed slots must hold all of
+    //    them) and whether its first new token falls in a block held by
+    //    others (a copy-on-write candidate).  Counts are read before any
+    //    change.  The candidates are listed in sequence order in slots[]
+    //    (there are at most as many as tokens); pairs[] holds (X, count).
+    //    Meanwhile the first entries of the free ring are staged.
+    const int win = static_cast<int>(min(max(avail, 0ll), static_cast<long long>(kRingWindow)));
+    if (avail >= 0 && avail <= N) {
+        for (int i = tid; i < win; i += T) window[i] = p.st.free_ids[(head + i) % N];
     }
-    const long long head = p.st.free_state[0], tail = p.st.free_state[1];
-    if (tid == 0) {
-        abort_sh = 0;
-        taken_sh = 0;
-        if (tokens > p.num_slots) {
-            flag_error(4 /* PA_DEVERR_SLOT */);
-            abort_sh = 1;
-        } else if (tail - head < 0 || tail - head > N) {
-            flag_error(64 /* PA_DEVERR_REF_COUNT */);
-            abort_sh = 1;
-        }
-    }
-    __syncthreads();
-    if (abort_sh) return;
-    const long long avail = tail - head;
-
-    // 1. copy-on-write candidates: sequences whose first new token falls in
-    //    a block held by others.  The counts are read before any changes;
-    //    pairs[] holds (X, count) for now.
-    for (int base = 0; base < S; base += kBlocksThreads) {
+    long long tokens = 0, W = 0;
+    for (int base = 0; base < S; base += T) {
         const int s = base + tid;
+        long long n_tok = 0, cand = 0;
         if (s < S) {
+            n_tok = max(p.num_new[s], 0);
             int L, n, first_new, new_blocks, X;
             const bool ok = describe_append(p, s, L, n, first_new, new_blocks, X);
             const int r = ok && X >= 0 ? p.st.ref[X] : 0;
-            const bool cand = ok && X >= 0 && r > 1;
+            cand = ok && X >= 0 && r > 1 ? 1 : 0;
             p.pairs[2 * s] = cand ? X : -1;
             p.pairs[2 * s + 1] = cand ? r : 0;
         }
+        const long long at = cta_exclusive_scan<long long>(cand, &total, sh);
+        if (cand && W + at < p.num_slots) p.slots[W + at] = s;   // (a step too big for its slots stops below)
+        W += total;
+        cta_exclusive_scan<long long>(n_tok, &total, sh);
+        tokens += total;
     }
+    if (tokens > p.num_slots || avail < 0 || avail > N) {
+        if (tid == 0) flag_error(tokens > p.num_slots ? 4 /* PA_DEVERR_SLOT */ : 64 /* PA_DEVERR_REF_COUNT */);
+        return;   // uniform: every thread computed the same totals
+    }
+    if (tid == 0) taken_sh = 0;
     __syncthreads();
 
     // 2. the k-th writer (in sequence order) into a block of count r copies
     //    it iff k < r - 1: each earlier writer's copy lowered the count by
-    //    one, and the last holder writes in place.  Candidates are listed in
-    //    sequence order in slots[] (at most one per token of the step), then
-    //    each counts the earlier ones naming its block; pairs[2s+1] becomes
-    //    the copy flag.
-    long long W = 0;
-    for (int base = 0; base < S; base += kBlocksThreads) {
-        const int s = base + tid;
-        const long long c = s < S && p.pairs[2 * s] >= 0 ? 1 : 0;
-        const long long at = cta_exclusive_scan<long long>(c, &total, sh);
-        if (c) p.slots[W + at] = s;
-        W += total;
-    }
-    __syncthreads();
-    for (long long base = 0; base < W; base += kBlocksThreads) {
+    //    one, and the last holder writes in place.  Each candidate counts
+    //    the earlier ones naming its block (tiles of the list staged in
+    //    shared memory); pairs[2s+1] becomes the copy flag.
+    for (long long base = 0; base < W; base += T) {
         const long long i = base + tid;
         int s = -1, X = -1, r = 0, k = 0;
         if (i < W) {
@@ -193,13 +187,13 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
             X = static_cast<int>(p.pairs[2 * s]);
             r = static_cast<int>(p.pairs[2 * s + 1]);
         }
-        for (long long t0 = 0; t0 <= base; t0 += kBlocksThreads) {  // tiles of earlier candidates
+        for (long long t0 = 0; t0 <= base; t0 += T) {  // tiles of earlier candidates
             __syncthreads();
             const long long j = t0 + tid;
             shx[tid] = j < W ? static_cast<int>(p.pairs[2 * p.slots[j]]) : -1;
             __syncthreads();
             if (i < W) {
-                const long long lim = min(static_cast<long long>(kBlocksThreads), i - t0);
+                const long long lim = min(static_cast<long long>(T), i - t0);
                 for (long long u = 0; u < lim; ++u) k += shx[u] == X;
             }
         }
@@ -213,19 +207,17 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
     //    C_s <= free blocks; its blocks are ring positions head + C_s - need_s
     //    onward (the copy first, then new blocks in logical order).
     long long run_need = 0, run_slot = 0;
-    const long long cap_rows = static_cast<long long>(p.max_blocks);
-    for (int base = 0; base < S; base += kBlocksThreads) {
+    const long long cap = static_cast<long long>(p.max_blocks) * B;
+    for (int base = 0; base < S; base += T) {
         const int s = base + tid;
         int L = 0, n = 0, first_new = 0, new_blocks = 0, X = -1;
         bool ok = false, cow = false;
         if (s < S) {
             // the row is unchanged since step 1 (only its own thread writes it, below)
-            const int raw_n = p.num_new[s];
+            n = p.num_new[s];
             L = p.context_lens[s];
-            n = raw_n;
-            if (raw_n > 0) {
-                const long long cap = cap_rows * B;
-                ok = L >= 0 && static_cast<long long>(L) + raw_n <= cap;
+            if (n > 0) {
+                ok = L >= 0 && static_cast<long long>(L) + n <= cap;
                 if (ok) {
                     first_new = (L + B - 1) / B;
                     new_blocks = static_cast<int>((static_cast<long long>(L) + n + B - 1) / B) - first_new;
@@ -252,9 +244,9 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
             for (int i = 0; i < max(n, 0); ++i) p.slots[slot0 + i] = -1;
             continue;
         }
-        long long pos = head + before;
+        long long pos = before;   // offset in the ring from head
         auto take = [&]() -> int {
-            const int id = p.st.free_ids[pos % N];
+            const int id = pos < win ? window[pos] : p.st.free_ids[(head + pos) % N];
             ++pos;
             if (id < 0 || id >= N) {
                 flag_error(64 /* PA_DEVERR_REF_COUNT: the ring holds a bad id */);
