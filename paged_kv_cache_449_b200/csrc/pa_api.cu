@@ -361,7 +361,7 @@ cudaError_t launch_prefill_tc(const pa::PrefillParams& p, const CUtensorMap& k_r
     auto kernel = pa::pa_prefill_tc_kernel<T, D, B>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, 384, Sm::kTotal, st>>>(p, k_rows);
+    kernel<<<grid, 448, Sm::kTotal, st>>>(p, k_rows);
     return cudaGetLastError();
 }
 

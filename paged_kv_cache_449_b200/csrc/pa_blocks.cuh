@@ -144,9 +144,15 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
     //    change.  The candidates are listed in sequence order in slots[]
     //    (there are at most as many as tokens); pairs[] holds (X, count).
     //    Meanwhile the first entries of the free ring are staged.
-    const int win = static_cast<int>(min(max(avail, 0ll), static_cast<long long>(kRingWindow)));
-    if (avail >= 0 && avail <= N) {
-        for (int i = tid; i < win; i += T) window[i] = p.st.free_ids[(head + i) % N];
+    // ring positions are taken modulo N once; later positions wrap by one compare
+    const bool ring_ok = head >= 0 && avail >= 0 && avail <= N;
+    const long long head_at = ring_ok ? head % N : 0;
+    const int win = ring_ok ? static_cast<int>(min(avail, static_cast<long long>(min(kRingWindow, 4 * T)))) : 0;
+    if (ring_ok) {
+        for (int i = tid; i < win; i += T) {
+            const long long at = head_at + i;
+            window[i] = p.st.free_ids[at < N ? at : at - N];
+        }
     }
     long long tokens = 0, W = 0;
     for (int base = 0; base < S; base += T) {
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
         cta_exclusive_scan<long long>(n_tok, &total, sh);
         tokens += total;
     }
-    if (tokens > p.num_slots || avail < 0 || avail > N) {
+    if (tokens > p.num_slots || !ring_ok) {
         if (tid == 0) flag_error(tokens > p.num_slots ? 4 /* PA_DEVERR_SLOT */ : 64 /* PA_DEVERR_REF_COUNT */);
         return;   // uniform: every thread computed the same totals
     }
@@ -246,7 +252,8 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
         }
         long long pos = before;   // offset in the ring from head
         auto take = [&]() -> int {
-            const int id = pos < win ? window[pos] : p.st.free_ids[(head + pos) % N];
+            const long long at = head_at + pos;   // pos < avail <= N
+            const int id = pos < win ? window[pos] : p.st.free_ids[at < N ? at : at - N];
             ++pos;
             if (id < 0 || id >= N) {
                 flag_error(64 /* PA_DEVERR_REF_COUNT: the ring holds a bad id */);
@@ -353,6 +360,11 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_release_kernel(const
     const int tid = threadIdx.x;
     const long long N = p.st.num_blocks;
     const long long head = p.st.free_state[0], tail = p.st.free_state[1];
+    if (head < 0 || tail < head || tail - head > N) {   // not a ring this library wrote
+        if (threadIdx.x == 0) flag_error(64 /* PA_DEVERR_REF_COUNT */);
+        return;
+    }
+    const long long tail_at = tail % N;
     long long pushed = 0, total;
     for (int k = 0; k < p.num_release; ++k) {
         if (tid == 0) {
@@ -398,7 +410,8 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_release_kernel(const
                 if (zero) {
                     const long long pos = tail + pushed + at;
                     if (pos - head < N) {
-                        p.st.free_ids[pos % N] = b;
+                        const long long ring_at = tail_at + pushed + at;   // < 2N
+                        p.st.free_ids[ring_at < N ? ring_at : ring_at - N] = b;
                     } else {
                         flag_error(64 /* PA_DEVERR_REF_COUNT: more free blocks than the pool holds */);
                     }

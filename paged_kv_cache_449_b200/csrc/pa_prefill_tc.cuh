@@ -2,7 +2,7 @@
 // computation as pa_prefill_kernel ("vLLM核心架构总览" §4.3 chunked prefill,
 // causal attention of each sequence's newest Q tokens over its paged context).
 //
-//  * One CTA (384 threads, one per SM) per (sequence, kv head, pair of query
+//  * One CTA (448 threads, one per SM) per (sequence, kv head, pair of query
 //    tiles).  A query tile is 128 MMA rows, (query token, head of the GQA
 //    group) pairs, 128 / g tokens; in a softmax warpgroup thread t owns row t,
 //    which is tensor-memory lane t.  The two tiles share every K/V tile.
@@ -11,10 +11,13 @@
 //    S = Q K^T is one N = 64 MMA per 16-dim step; V arrives as whole (block,
 //    head) tiles [D/8][B][8] by 1-D bulk copies, the MN-major B operand of
 //    O += P V as stored.  K and V have four-stage rings of their own.
-//  * Warp roles: 0-3 and 4-7 softmax of query tile 0 and 1; 8 issues S = Q K^T
-//    (Q and K in shared memory); 9 issues O += P V (P in tensor memory, V in
-//    shared memory); 10 and 11 fetch K and V.  tcgen05.commit arrives on the
-//    mbarriers the other roles wait on, every wait bounded.
+//  * Warp roles: 0-3 and 4-7 softmax of query tile 0 and 1; 8 and 9 issue
+//    S = Q K^T for query tile 0 and 1 (Q and K in shared memory); 10 and 11
+//    issue O += P V for query tile 0 and 1 (P in tensor memory, V in shared
+//    memory); 12 and 13 fetch K and V.  One issuer per query tile keeps each
+//    tile's chain of MMAs from waiting on the other tile's.  tcgen05.commit
+//    arrives on the mbarriers the other roles wait on, every wait bounded; a K
+//    or V stage is free once both tiles' issuers committed it.
 //  * Per query tile, S (64 fp32 columns), O (D columns) and two P buffers (32
 //    columns of 16-bit pairs each) live in tensor memory.  The softmax warps
 //    read their S row with tcgen05.ld, mask (causal, refused blocks), run the
@@ -225,9 +228,10 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 // Warps 0-3 and 4-7: softmax of query tile 0 and 1 (thread = row = tensor-memory
-// lane); warp 8 issues S = Q K^T, warp 9 O += P V; warps 10 and 11 fetch K and V.
+// lane); warps 8 / 9 issue S = Q K^T and 10 / 11 O += P V for query tile 0 / 1;
+// warps 12 and 13 fetch K and V.
 template <typename T, int D, int B>
-__global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
+__global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
                                                                 const __grid_constant__ CUtensorMap k_rows) {
     using Sm = PrefillTcSmem<T, D, B>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     uint64_t* s_free = bars + 26;    // [q] the softmax warps have read S
     uint64_t* p_full = bars + 28;    // [q * 2 + buffer] P written (and O rescaled)
     uint64_t* p_free = bars + 32;    // [q * 2 + buffer] the O += P V reading that P finished
-    uint64_t* drain = bars + 36;     // [2] the S and the O += P V issuers' MMAs finished
+    uint64_t* drain = bars + 36;     // [4] each issuer's MMAs finished
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + Sm::kMiscOff);
     volatile uint32_t* abort = misc + 1;
 
@@ -289,9 +293,9 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     if (tid == 256) {
         for (int i = 0; i < KS; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
+            mbar_init(&k_empty[i], 2);
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            mbar_init(&v_empty[i], 2);
         }
         for (int q = 0; q < 2; ++q) {
             mbar_init(&s_full[q], 1);
@@ -301,8 +305,7 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                 mbar_init(&p_free[q * 2 + b], 1);
             }
         }
-        mbar_init(&drain[0], 1);
-        mbar_init(&drain[1], 1);
+        for (int d = 0; d < 4; ++d) mbar_init(&drain[d], 1);
         *abort = 0u;
         fence_barrier_init();
     }
@@ -335,8 +338,8 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     };
 
     // ---- producers: warp 10 lane 0 fetches K tiles, warp 11 lane 0 V tiles
-    const bool is_producer = (warp == 10 || warp == 11) && lane == 0;
-    const bool v_side = warp == 11;
+    const bool is_producer = (warp == 12 || warp == 13) && lane == 0;
+    const bool v_side = warp == 13;
     const char* vpool = reinterpret_cast<const char*>(p.v_cache);
     uint64_t* full = v_side ? v_full : k_full;
     uint64_t* empty = v_side ? v_empty : k_empty;
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
     tc::fence_after();
 
     bool failed = false;
-    if (warp == 10 || warp == 11) {
+    if (warp == 12 || warp == 13) {
         // ---------------- producers
         if (is_producer) {
             for (int j = nst; j < ntiles; ++j) {
@@ -450,29 +453,23 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
             for (int k = issued > nst ? issued - nst : 0; k < issued; ++k)
                 mbar_wait_bounded(&full[k % nst], (k / nst) & 1, kWaitLimitNs);
         }
-    } else if (warp == 8) {
-        // ---------------- S = Q K^T issue (lane 0): per query tile one N = 64 MMA per
-        //                  16-dim step, Q and K in shared memory
+    } else if (warp == 8 || warp == 9) {
+        // ---------------- S = Q K^T issue (lane 0), one warp per query tile
+        const int q = warp - 8;
         if (lane == 0) {
             const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
             const uint32_t k_ring = smem_u32(smem + Sm::kKOff);
             int id_n[kBlocks];
             load_ids(0, id_n);
-            bool run = true;
-            for (int j = 0; run && j < ntiles; ++j) {
+            for (int j = 0; j < ntiles; ++j) {
                 const uint32_t ok = ok_of(id_n);
                 load_ids(j + 1, id_n);
                 if (!tc_wait(&k_full[j % KS], (j / KS) & 1, abort)) break;
-                const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    if (j >= nt[q]) continue;
+                if (j < nt[q]) {
                     // S(j) overwrites S(j - 1): the softmax warps must have read it
-                    if (j > 0 && !tc_wait(&s_free[q], (j - 1) & 1, abort)) {
-                        run = false;
-                        break;
-                    }
+                    if (j > 0 && !tc_wait(&s_free[q], (j - 1) & 1, abort)) break;
                     tc::fence_after();
+                    const uint32_t kbase = k_ring + (j % KS) * Sm::kStage;
                     const uint32_t qb = tmem + static_cast<uint32_t>(q) * 256u;
                     const uint32_t qs = smem_u32(smem + Sm::kQOff + q * Sm::kQ);
                     if (ok != 0u) {
@@ -483,26 +480,24 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                     }
                     tc::commit(&s_full[q]);
                 }
-                if (run) tc::commit(&k_empty[j % KS]);
+                tc::commit(&k_empty[j % KS]);
             }
-            // every MMA this thread issued has finished before the CTA tears down
-            tc::commit(&drain[0]);
-            mbar_wait_bounded(&drain[0], 0, kWaitLimitNs);
+            tc::commit(&drain[q]);
+            mbar_wait_bounded(&drain[q], 0, kWaitLimitNs);
         }
-    } else if (warp == 9) {
-        // ---------------- O += P V issue (lane 0); the warp zeroes V rows past the context
+    } else if (warp == 10 || warp == 11) {
+        // ---------------- O += P V issue (lane 0), one warp per query tile; each warp
+        //                  zeroes V rows past the context (the same zeros: harmless twice)
+        const int q = warp - 10;
         const uint32_t idesc_o = tc::instr_desc<T>(D, true);
         const uint32_t v_ring = smem_u32(smem + Sm::kVOff);
         int id_n[kBlocks];
         load_ids(0, id_n);
-        bool run = true;
-        for (int j = 0; run && j < ntiles; ++j) {
+        for (int j = 0; j < ntiles; ++j) {
             const uint32_t ok = ok_of(id_n);
             load_ids(j + 1, id_n);
             const int vst = j % VS;
             if (!__all_sync(0xffffffffu, tc_wait(&v_full[vst], (j / VS) & 1, abort))) break;
-            // tokens at or past the context in the last needed block: zero their staged
-            // V rows (P is 0 there, but 0 times a stale non-finite value would not be)
             const int lb = (L - 1) / B - j * kBlocks;
             if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
                 uint8_t* vt = smem + Sm::kVOff + vst * Sm::kStage + lb * kTile;
@@ -514,18 +509,12 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            const uint32_t vbase = v_ring + vst * Sm::kStage;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                if (j >= nt[q]) continue;
+            if (j < nt[q]) {
+                const uint32_t vbase = v_ring + vst * Sm::kStage;
                 const int pb = q * 2 + (j & 1);
-                if (!__all_sync(0xffffffffu, tc_wait(&p_full[pb], (j >> 1) & 1, abort))) {
-                    run = false;
-                    break;
-                }
+                if (!__all_sync(0xffffffffu, tc_wait(&p_full[pb], (j >> 1) & 1, abort))) break;
                 if (lane == 0) {
                     tc::fence_after();
-                    // one MMA per block and 16-key step: P in tensor memory, V (MN-major) in shared memory
                     const uint32_t qb = tmem + static_cast<uint32_t>(q) * 256u;
                     const uint32_t pt = qb + kPCol + static_cast<uint32_t>(j & 1) * (kKeys / 2);
                     for (int b = 0; b < kBlocks; ++b) {
@@ -538,11 +527,11 @@ __global__ void __launch_bounds__(384, 1) pa_prefill_tc_kernel(const __grid_cons
                     tc::commit(&p_free[pb]);
                 }
             }
-            if (run && lane == 0) tc::commit(&v_empty[vst]);
+            if (lane == 0) tc::commit(&v_empty[vst]);
         }
         if (lane == 0) {
-            tc::commit(&drain[1]);
-            mbar_wait_bounded(&drain[1], 0, kWaitLimitNs);
+            tc::commit(&drain[2 + q]);
+            mbar_wait_bounded(&drain[2 + q], 0, kWaitLimitNs);
         }
         __syncwarp();
     } else if (softmax_warp) {
