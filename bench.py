@@ -58,10 +58,13 @@ def parse_args(argv=None):
                     choices=["tiny_mha_f32", "llama3_8b_decode", "continuous_batching_mix", "prefix_sharing",
                              "llama3_70b_long"])
     ap.add_argument("--block-size", type=int, default=None)
-    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap_out", "swap_in", "prefill"], default="decode",
+    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap_out", "swap_in", "prefill", "block_step"],
+                    default="decode",
                     help="decode: the hot-path step (default); copy_blocks: every block of the batch duplicated "
                          "into free blocks of the same pools (copy-on-write / fork); swap_out / swap_in: every "
-                         "block of the batch copied to / from a pinned host pool (preemption by swapping)")
+                         "block of the batch copied to / from a pinned host pool (preemption by swapping); "
+                         "block_step: a decode step through the device block manager (pa_blocks_append + "
+                         "pa_copy_blocks + pa_decode_append)")
     ap.add_argument("--mode", choices=["append", "single", "splitk", "splitk2"], default="append",
                     help="append: one pa_decode_append launch per step (write + decode); the others launch "
                          "pa_reshape_and_cache then pa_decode (single) or pa_decode_splitk with fused (splitk) or "
@@ -262,7 +265,7 @@ def barrier(world):
 class Step:
     """One hot-path step through the C ABI on device-resident inputs."""
 
-    def __init__(self, batch, mode, partition_size, independent=True, fp8=None):
+    def __init__(self, batch, mode, partition_size, independent=True, fp8=None, longest_first=False):
         import paged_kv_cache_449_b200 as pa
         self.pa = pa
         self.b = batch
@@ -285,6 +288,8 @@ class Step:
         # views), so a step's upload from the host is a single copy.
         specs = [("q", batch.q), ("nk", batch.new_key), ("nv", batch.new_value), ("slots", batch.slot_mapping),
                  ("bt", batch.block_tables), ("cl", batch.context_lens)]
+        if longest_first:   # the start order a scheduler that knows the lengths passes (seq_order)
+            specs.append(("order", pa.longest_first(batch.context_lens)))
         offs, total = [], 0
         for _, t in specs:
             offs.append(total)
@@ -294,6 +299,8 @@ class Step:
             view = self.inbuf[off:off + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
             view.copy_(t)
             setattr(self, name, view)
+        if not longest_first:
+            self.order = None
         self.out = torch.empty_like(self.q)
         self.mcl = batch.max_context_len
         need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
@@ -315,7 +322,8 @@ class Step:
         if self.fp8:
             if self.mode == "append":
                 self.pa.pa_decode_append_fp8(self.out, self.q, self.nk, self.nv, self.k, self.v, self.ks, self.vs,
-                                             self.bt, self.cl, self.b.scale, max_context_len=self.mcl, stream=stream)
+                                             self.bt, self.cl, self.b.scale, max_context_len=self.mcl, stream=stream,
+                                             seq_order=self.order)
             elif self.mode in ("splitk", "splitk2"):
                 self.pa.pa_decode_splitk_fp8(self.out, self.q, self.k, self.v, self.ks, self.vs, self.bt, self.cl,
                                              self.b.scale, self.mcl, partition_size=self.part, workspace=self.ws,
@@ -326,7 +334,7 @@ class Step:
             return
         if self.mode == "append":
             self.pa.pa_decode_append(self.out, self.q, self.nk, self.nv, self.k, self.v, self.bt, self.cl, self.b.scale,
-                                     max_context_len=self.mcl, stream=stream)
+                                     max_context_len=self.mcl, stream=stream, seq_order=self.order)
         elif self.mode in ("splitk", "splitk2"):
             self.pa.pa_decode_splitk(self.out, self.q, self.k, self.v, self.bt, self.cl, self.b.scale, self.mcl,
                                      partition_size=self.part, workspace=self.ws, fused=(self.mode == "splitk"),
@@ -652,7 +660,7 @@ def run_gpu(args, world, rank, local):
 
 # ----------------------------------------------------------------------------- every configuration
 
-def time_decode_steps(batch, mode, partition_size, fp8, steps, warmup, world):
+def time_decode_steps(batch, mode, partition_size, fp8, steps, warmup, world, longest_first=False):
     """Device time of one step (write of the newest tokens + decode) on the
     batch: rotated independent copies larger than L2 when the workload allows
     (K steps in one CUDA-event region), else a 256 MiB L2 flush and per-step
@@ -662,7 +670,8 @@ def time_decode_steps(batch, mode, partition_size, fp8, steps, warmup, world):
     stream = torch.cuda.current_stream()
     unique = batch.unique_kv_bytes() // (2 if fp8 is not None else 1)
     copies = rotation_copies(unique, l2_bytes())
-    steps_ = [Step(batch, mode, partition_size, independent=i > 0, fp8=fp8) for i in range(max(1, copies))]
+    steps_ = [Step(batch, mode, partition_size, independent=i > 0, fp8=fp8, longest_first=longest_first)
+              for i in range(max(1, copies))]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if copies == 0 else None
 
     def one(i):
@@ -803,8 +812,9 @@ def config_lines(args, world, rank):
     K, W = args.steps, max(3, args.warmup)
     out = {}
 
-    def entry(batch, mode, part=None, fp8=None, note=None):
-        ms, launches, l2 = time_decode_steps(batch, mode, part or args.partition_size, fp8, K, W, world)
+    def entry(batch, mode, part=None, fp8=None, note=None, longest_first=False):
+        ms, launches, l2 = time_decode_steps(batch, mode, part or args.partition_size, fp8, K, W, world,
+                                             longest_first)
         dec, resh = step_bytes(batch, fp8)
         logical = dec + resh
         unique = (batch.algorithmic_bytes(unique=True) if fp8 is None else dec) + resh
@@ -824,6 +834,8 @@ def config_lines(args, world, rank):
             e["bytes_basis"] = "unique: shared-prefix blocks counted once (logical bytes beside)"
         if note:
             e["note"] = note
+        if longest_first:
+            e["seq_order"] = "longest first (built on the host from the lengths, uploaded with the step's inputs)"
         return e
 
     seed = args.seed + rank
@@ -834,6 +846,7 @@ def config_lines(args, world, rank):
     for B in (8, 16, 32):
         b = workloads.continuous_batching_mix(seed=seed, device="cuda", block_size=B)
         out[f"continuous_batching_mix_B{B}"] = entry(b, "append")
+        out[f"continuous_batching_mix_B{B}_longest_first"] = entry(b, "append", longest_first=True)
         del b
     b = workloads.prefix_sharing(seed=seed, device="cuda")
     out["prefix_sharing"] = entry(b, "append")
@@ -1158,6 +1171,20 @@ def main(argv=None):
         if args.impl == "reference":
             res = run_reference(args, world, rank)
             if res is not None:
+                print(json.dumps(res), flush=True)
+            return
+        if args.op == "block_step":
+            import paged_kv_cache_449_b200 as pa
+            from paged_kv_cache_449_b200 import build as pabuild
+            pabuild.build()
+            pa.load()
+            peak, _ = measured_peaks()
+            with ClockSampler(local) as clocks:
+                res = block_manager_step(args.seed + rank, args.steps, max(3, args.warmup), world, peak)
+            res = dict(res, metric="paged decode step through the device block manager, KV GB/s",
+                       value=res["gb_per_s"], unit="GB/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                       higher_is_better=True, clocks=clocks.summary())
+            if rank == 0:
                 print(json.dumps(res), flush=True)
             return
         if args.op != "decode":
