@@ -789,7 +789,14 @@ def block_manager_step(seed, steps, warmup, world, peak):
     per_kernel = profiled_kernel_ms(one, 1, ("pa_blocks_append_kernel", "pa_copy_blocks_kernel", "pa_decode_kernel"))
     if pa.pa_get_device_error() != 0:
         raise RuntimeError("device error word set in the block-manager step")
-    nbytes = b.algorithmic_bytes()
+    # every step adds a token to every sequence: count the bytes at the mean
+    # length over the timed steps (step i reads lens0 + warmup + i + 1 tokens)
+    grow = warmup + (steps + 1) / 2.0
+    mean_tokens = float(lens0.sum()) + S * grow
+    e = b.elem_bytes
+    tables = sum(math.ceil((float(L) + grow) / B) for L in lens0.tolist()) * 4
+    nbytes = int(mean_tokens * b.num_kv_heads * b.head_dim * 2 * e + 2 * S * b.num_q_heads * b.head_dim * e
+                 + tables + 4 * S + 4 * S * b.num_kv_heads * b.head_dim * e)   # new K/V rows read + written
     gbs = reduce_sum(nbytes, world) / (ms * 1e-3) / 1e9
     return {"workload": b.name + " + device block manager",
             "entry": "pa_blocks_append + pa_copy_blocks + pa_decode_append (ref counts)",
@@ -798,6 +805,8 @@ def block_manager_step(seed, steps, warmup, world, peak):
             "kernel_ms": {k_: (round(v_, 5) if isinstance(v_, float) else v_) for k_, v_ in per_kernel.items()},
             "kernel_ms_how": "torch.profiler CUDA activity records of one step after the timed ones",
             "gpu_launches": 3 * steps,
+            "bytes_basis": ("K/V at the mean context length over the timed steps (each step appends a token to "
+                            "every sequence) + q, out, the new rows, block-table entries and lengths"),
             "l2": "one copy of the pools (290 MB of KV per step, more than twice the L2), K steps in one event region"}
 
 
