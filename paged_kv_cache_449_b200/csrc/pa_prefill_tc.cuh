@@ -196,7 +196,7 @@ struct PrefillTcSmem {
     static constexpr int kTile = B * D * 2;               // one (block, head) K or V tile
     static constexpr int kStage = kBlocks * kTile;        // the K (or V) tiles of one key tile
 #ifndef PA_PF_STAGES
-#define PA_PF_STAGES 4
+#define PA_PF_STAGES 3
 #endif
     static constexpr int kKStages = D == 128 ? PA_PF_STAGES : PA_PF_STAGES + 2;
     static constexpr int kVStages = kKStages;
