@@ -631,7 +631,8 @@ def run_gpu(args, world, rank, local):
         "decode_ms": round(decode_ms_max, 5),
         "reshape_ms": round(sum(reshape_ms) / len(reshape_ms), 5),
         "decode_gbs": round(total_decode_bytes / (decode_ms_max * 1e-3) / 1e9, 2),
-        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "hbm_peak": f"{peak} GB/s, {peak_kind} copy bandwidth",
         "pct_of_spec_8tbs": round(100 * value / world / SPEC_HBM_GBS, 2),
         "roofline": {
             "bound": "hbm",
@@ -801,7 +802,8 @@ def block_manager_step(seed, steps, warmup, world, peak):
     return {"workload": b.name + " + device block manager",
             "entry": "pa_blocks_append + pa_copy_blocks + pa_decode_append (ref counts)",
             "ms_per_step": round(ms, 5), "algorithmic_bytes": int(nbytes), "gb_per_s": round(gbs, 2),
-            "frac_of_measured_hbm": round(gbs / world / peak, 4),
+            "frac_of_hbm_peak": round(gbs / world / peak, 4),
+            "hbm_peak": f"{peak} GB/s, {measured_peaks()[1]} copy bandwidth",
             "kernel_ms": {k_: (round(v_, 5) if isinstance(v_, float) else v_) for k_, v_ in per_kernel.items()},
             "kernel_ms_how": "torch.profiler CUDA activity records of one step after the timed ones",
             "gpu_launches": 3 * steps,
@@ -835,7 +837,7 @@ def config_lines(args, world, rank):
                 "splitk2": f"pa_reshape_and_cache + pa_decode_splitk (merge kernel, partition {part})"}[mode],
              "seqs": batch.num_seqs, "block_size": batch.block_size, "ms_per_step": round(ms, 5),
              "algorithmic_bytes": int(unique), "gb_per_s": round(gbs, 2),
-             "frac_of_measured_hbm": round(gbs / world / peak, 4), "frac_of_spec_8tbs": round(gbs / world / SPEC_HBM_GBS, 4),
+             "frac_of_hbm_peak": round(gbs / world / peak, 4), "frac_of_spec_8tbs": round(gbs / world / SPEC_HBM_GBS, 4),
              "tokens_per_s": round(reduce_sum(batch.num_seqs, world) / (ms * 1e-3), 1),
              "gpu_launches": launches * K, "l2": l2}
         if unique != logical:
