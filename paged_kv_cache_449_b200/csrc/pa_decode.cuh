@@ -371,11 +371,63 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     }
     bool failed = false;
     int i = 0;
+    // Tensor-core path with 16-token blocks and rings of three stages or more:
+    // a warp takes two of its blocks per online-softmax step (one row maximum
+    // and one rescale per 32 tokens) while a third stage stays in flight; a
+    // last odd block goes alone.  (With two stages the pair would leave none
+    // in flight: slower.)
+#ifndef PA_PAIR_MIN_STAGES
+#define PA_PAIR_MIN_STAGES 3
+#endif
+    constexpr bool kPairs = !kF32 && B == 16 && STAGES >= PA_PAIR_MIN_STAGES;
     for (; i < n_w; ++i) {
         if (i > 0 && (i & 31) == 0) {
             win0 = win1;
             ++cur_round;
             win1 = load_ids(cur_round + 1);
+        }
+        if constexpr (kPairs) {
+            if (i + 1 < n_w) {
+                // i is even here, so i + 1 lies in the same 32-entry window round
+                const int st0 = i % STAGES, st1 = (i + 1) % STAGES;
+                if (!mbar_wait_bounded(&wbar[st0], (i / STAGES) & 1, wait_limit_ns()) ||
+                    !mbar_wait_bounded(&wbar[st1], ((i + 1) / STAGES) & 1, wait_limit_ns())) {
+                    failed = true;
+                    break;
+                }
+                const int id0 = block_id(i), id1 = block_id(i + 1);
+                const int j0 = b0 + warp + i * NW, j1 = j0 + NW;
+                const int valid0 = id0 < 0 ? 0 : min(B, L - j0 * B);
+                const int valid1 = id1 < 0 ? 0 : min(B, L - j1 * B);
+                uint8_t* stage0 = wring + st0 * 2 * kTile;
+                uint8_t* stage1 = wring + st1 * 2 * kTile;
+                if (owns_last) {
+                    if constexpr (FP8) {
+                        if (j0 == last_block && id0 >= 0)
+                            append_newest_token_e4m3<T, D, B>(p, new_row8, stage0, id0, kvh, (L - 1) % B, lane);
+                        if (j1 == last_block && id1 >= 0)
+                            append_newest_token_e4m3<T, D, B>(p, new_row8, stage1, id1, kvh, (L - 1) % B, lane);
+                    } else {
+                        if (j0 == last_block && id0 >= 0)
+                            append_newest_token<T, D, B>(p, new_row, stage0, id0, kvh, (L - 1) % B, lane);
+                        if (j1 == last_block && id1 >= 0)
+                            append_newest_token<T, D, B>(p, new_row, stage1, id1, kvh, (L - 1) % B, lane);
+                    }
+                }
+                acc.template block2<FP8>(smem_u32(stage0), smem_u32(stage0 + kTile), valid0, smem_u32(stage1),
+                                         smem_u32(stage1 + kTile), valid1, group, score_scale, lane);
+                __syncwarp();
+                if (i + STAGES < n_w) {
+                    issue(i + STAGES);
+                    ++issued;
+                }
+                if (i + 1 + STAGES < n_w) {
+                    issue(i + 1 + STAGES);
+                    ++issued;
+                }
+                ++i;   // the loop's increment moves past the pair
+                continue;
+            }
         }
         const int st = i % STAGES;
         if (!mbar_wait_bounded(&wbar[st], (i / STAGES) & 1, wait_limit_ns())) {

@@ -208,6 +208,129 @@ struct WarpMma {
         }
     }
 
+    // Two 16-token blocks (a and b) in one online-softmax step: one row
+    // maximum, one rescale of O^T and the running sums for the 32 tokens.
+    // Scores S^T of block a in sa, of block b in sb; returns the P^T operands
+    // of both blocks.
+    __device__ __forceinline__ void softmax_step2(const float (&sa)[4], const float (&sb)[4], int valid_a,
+                                                  int valid_b, int group, float scale_log2, int lane,
+                                                  uint32_t (&pa)[2], uint32_t (&pb)[2]) {
+        const int r = lane >> 2, c = lane & 3;
+        const bool h0ok = 2 * c < group, h1ok = 2 * c + 1 < group;
+        const int t_lo = r, t_hi = r + 8;
+        const float xa0 = (h0ok && t_lo < valid_a) ? sa[0] * scale_log2 : kNegInf;
+        const float xa1 = (h1ok && t_lo < valid_a) ? sa[1] * scale_log2 : kNegInf;
+        const float xa2 = (h0ok && t_hi < valid_a) ? sa[2] * scale_log2 : kNegInf;
+        const float xa3 = (h1ok && t_hi < valid_a) ? sa[3] * scale_log2 : kNegInf;
+        const float xb0 = (h0ok && t_lo < valid_b) ? sb[0] * scale_log2 : kNegInf;
+        const float xb1 = (h1ok && t_lo < valid_b) ? sb[1] * scale_log2 : kNegInf;
+        const float xb2 = (h0ok && t_hi < valid_b) ? sb[2] * scale_log2 : kNegInf;
+        const float xb3 = (h1ok && t_hi < valid_b) ? sb[3] * scale_log2 : kNegInf;
+        float mx0 = fmaxf(fmaxf(xa0, xa2), fmaxf(xb0, xb2));
+        float mx1 = fmaxf(fmaxf(xa1, xa3), fmaxf(xb1, xb3));
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+        const float mu0 = mn0 == kNegInf ? 0.f : mn0, mu1 = mn1 == kNegInf ? 0.f : mn1;
+        const float al0 = exp2_approx(m_run[0] - mu0), al1 = exp2_approx(m_run[1] - mu1);
+        const float pa0 = exp2_approx(xa0 - mu0), pa1 = exp2_approx(xa1 - mu1);
+        const float pa2 = exp2_approx(xa2 - mu0), pa3 = exp2_approx(xa3 - mu1);
+        const float pb0 = exp2_approx(xb0 - mu0), pb1 = exp2_approx(xb1 - mu1);
+        const float pb2 = exp2_approx(xb2 - mu0), pb3 = exp2_approx(xb3 - mu1);
+        l_run[0] = l_run[0] * al0 + ((pa0 + pa2) + (pb0 + pb2));
+        l_run[1] = l_run[1] * al1 + ((pa1 + pa3) + (pb1 + pb3));
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt) {
+            o[mt][0] *= al0;
+            o[mt][1] *= al1;
+            o[mt][2] *= al0;
+            o[mt][3] *= al1;
+        }
+        pa[0] = movmatrix_trans(Mma<T>::pack(pa0, pa1));
+        pa[1] = movmatrix_trans(Mma<T>::pack(pa2, pa3));
+        pb[0] = movmatrix_trans(Mma<T>::pack(pb0, pb1));
+        pb[1] = movmatrix_trans(Mma<T>::pack(pb2, pb3));
+    }
+
+    // Fragments of 16-token blocks (B = 16): K rows (tokens r, r+8; dims of
+    // vector ks) and V^T rows (dims 16mt+r, +8; tokens 2c.., 2c+8..).
+    template <bool E4M3>
+    static __device__ __forceinline__ void k_frag(uint32_t kbase, int ks, int lane, uint32_t& a0, uint32_t& a1,
+                                                  uint32_t& a2, uint32_t& a3) {
+        const int r = lane >> 2, c = lane & 3;
+        if constexpr (E4M3) {
+            const uint32_t at = kbase + ((ks * 16 + r) * 16 + 4 * c);
+            e4m3x4_to_frags(lds32(at), a0, a2);
+            e4m3x4_to_frags(lds32(at + 8 * 16), a1, a3);
+        } else {
+            const int mtx = lane >> 3, row = lane & 7;
+            const int tok = (mtx & 1) * 8 + row;
+            const int chunk = 2 * ks + (mtx >> 1);
+            ldsm_x4(kbase + (chunk * 16 + tok) * 16, a0, a1, a2, a3);
+        }
+    }
+    template <bool E4M3>
+    static __device__ __forceinline__ void v_frag(uint32_t vbase, int mt, int lane, uint32_t& a0, uint32_t& a1,
+                                                  uint32_t& a2, uint32_t& a3) {
+        const int r = lane >> 2, c = lane & 3;
+        if constexpr (E4M3) {
+            const uint32_t at = vbase + ((16 * mt + r) * 16 + 4 * c);
+            e4m3x4_to_frags(lds32(at), a0, a2);
+            e4m3x4_to_frags(lds32(at + 8 * 16), a1, a3);
+        } else {
+            const int mtx = lane >> 3, row = lane & 7;
+            const int tok = (mtx >> 1) * 8 + row;
+            const int chunk = 2 * mt + (mtx & 1);
+            ldsm_x4_trans(vbase + (chunk * 16 + tok) * 16, a0, a1, a2, a3);
+        }
+    }
+
+    // Two blocks of 16 tokens (a, b) in one step: the K and V tiles of each
+    // staged as block() takes them; tokens >= valid_a (valid_b) masked out.
+    template <bool E4M3 = false>
+    __device__ __forceinline__ void block2(uint32_t ka, uint32_t va, int valid_a, uint32_t kb, uint32_t vb,
+                                           int valid_b, int group, float scale_log2, int lane) {
+        static_assert(B == 16, "16-token blocks");
+        const int c = lane & 3;
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            k_frag<E4M3>(ka, ks, lane, a0, a1, a2, a3);
+            k_frag<E4M3>(kb, ks, lane, b0, b1, b2, b3);
+            Mma<T>::k16(sa, a0, a1, a2, a3, qa[ks][0], qa[ks][1]);
+            Mma<T>::k16(sb, b0, b1, b2, b3, qa[ks][0], qa[ks][1]);
+        }
+        uint32_t pa[2], pb[2];
+        softmax_step2(sa, sb, valid_a, valid_b, group, scale_log2, lane, pa, pb);
+        const int tlo = 2 * c, thi = tlo + 8;
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt) {
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            v_frag<E4M3>(va, mt, lane, a0, a1, a2, a3);
+            v_frag<E4M3>(vb, mt, lane, b0, b1, b2, b3);
+            if (valid_a < 16) {
+                a0 = mask_pair(a0, tlo, valid_a);
+                a1 = mask_pair(a1, tlo, valid_a);
+                a2 = mask_pair(a2, thi, valid_a);
+                a3 = mask_pair(a3, thi, valid_a);
+            }
+            if (valid_b < 16) {
+                b0 = mask_pair(b0, tlo, valid_b);
+                b1 = mask_pair(b1, tlo, valid_b);
+                b2 = mask_pair(b2, thi, valid_b);
+                b3 = mask_pair(b3, thi, valid_b);
+            }
+            Mma<T>::k16(o[mt], a0, a1, a2, a3, pa[0], pa[1]);
+            Mma<T>::k16(o[mt], b0, b1, b2, b3, pb[0], pb[1]);
+        }
+    }
+
     __device__ __forceinline__ float head_sum(int e) const {
         float l = l_run[e];
         l += __shfl_xor_sync(0xffffffffu, l, 4);
