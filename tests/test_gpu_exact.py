@@ -99,17 +99,22 @@ def _needle_batch(dtype, B, lens, Hq=8, Hkv=2, D=128, seed=5):
     return b
 
 
-@pytest.mark.parametrize("dtype,B,mode,part", [
-    (torch.bfloat16, 16, "single", None), (torch.bfloat16, 16, "splitk", 32), (torch.float16, 8, "single", None),
-    (torch.float16, 32, "splitk", 64), (torch.bfloat16, 8, "splitk", 16), (torch.float32, 16, "single", None),
-    (torch.float32, 32, "splitk", 32)])
-def test_needle_every_position(dtype, B, mode, part):
+@pytest.mark.parametrize("dtype,B,mode,part,D,lens", [
+    (torch.bfloat16, 16, "single", None, 128, (70, 1, 33)), (torch.bfloat16, 16, "splitk", 32, 128, (70, 1, 33)),
+    (torch.float16, 8, "single", None, 128, (70, 1, 33)), (torch.float16, 32, "splitk", 64, 128, (70, 1, 33)),
+    (torch.bfloat16, 8, "splitk", 16, 128, (70, 1, 33)), (torch.float32, 16, "single", None, 128, (70, 1, 33)),
+    (torch.float32, 32, "splitk", 32, 128, (70, 1, 33)),
+    # deep ring of 4 stages: every warp takes several blocks, two per softmax step
+    (torch.bfloat16, 16, "single", None, 64, (300, 1, 161, 16)),
+    (torch.float16, 16, "splitk2", 128, 64, (300, 17, 161))])
+def test_needle_every_position(dtype, B, mode, part, D, lens):
     """q = 64 e_0 in the query heads of kv head 1; K = 0 except 64 e_0 at one
     logical token t*: that token's score is 4096 and every other weight
     underflows to exactly 0, so the output of those heads is V[t*] bit for
     bit.  Sweeping t* over every position pins the block-table gather, the
-    in-block offset, the GQA head mapping and the partition boundaries."""
-    b = _needle_batch(dtype, B, (70, 1, 33))
+    in-block offset, the GQA head mapping, the pairing of blocks per softmax
+    step and the partition boundaries."""
+    b = _needle_batch(dtype, B, lens, D=D)
     g = b.group
     b.q[:, g:2 * g, 0] = 64.0
     dev = device_batch(b)

@@ -201,3 +201,52 @@ def test_append_fp8_equals_write_then_decode(make):
     assert torch.equal(k2, k1) and torch.equal(v2, v1)
     bits = lambda t: t.contiguous().view(-1).view(torch.int16)
     assert torch.equal(bits(got), bits(ref))
+
+
+# ---------------------------------------------------------------------------- needles
+
+@pytest.mark.parametrize("qdt,D,B,mode,part", [
+    (torch.bfloat16, 128, 16, "single", None),    # deep ring of 3 stages: two blocks per softmax step
+    (torch.float16, 128, 16, "splitk", 64),
+    (torch.bfloat16, 64, 16, "splitk2", 128),
+    (torch.bfloat16, 128, 32, "single", None),
+    (torch.float16, 64, 8, "single", None),
+])
+def test_needle_every_position(orc, qdt, D, B, mode, part):
+    """Scales 1, K codes 0 except e4m3(64) in dim 0 of one logical token t*
+    of kv head 1, q = 64 e_0 in that head's query heads: t*'s score is 4096
+    and every other weight underflows to exactly 0, so those heads' output is
+    the dequantised V row of t* bit for bit.  Sweeping t* over every position
+    of sequences long enough that each warp of a thread block takes several
+    blocks pins the gather, the in-block offsets of both 8-bit tile layouts,
+    the pairing of blocks per softmax step (odd counts, a partial last block)
+    and the partition boundaries."""
+    b = workloads.random_small(seed=1200, dtype=qdt, lens=(600, 1, 290, 529), num_q_heads=8, num_kv_heads=2,
+                               head_dim=D, block_size=B, extra_blocks=3)
+    b.scale = 1.0
+    g = b.group
+    b.q.zero_()
+    b.q[:, g:2 * g, 0] = 64.0
+    shape = pa.fp8_pool_shape(b.num_blocks, b.num_kv_heads, D, B)
+    gen = torch.Generator().manual_seed(1201)
+    vc = torch.randint(0, 256, shape, generator=gen, dtype=torch.int32).to(torch.uint8)
+    vc[(vc & 0x7f) == 0x7f] = 0   # no NaN codes
+    ones = torch.ones(b.num_kv_heads, dtype=torch.float32, device="cuda")
+    pools = workloads.Fp8Pools(torch.zeros(shape, dtype=torch.uint8, device="cuda"), vc.cuda(), ones, ones.clone())
+    kflat = pools.k_cache.view(-1)
+    vflat = vc.view(-1)
+    needle = orc.e4m3_encode(64.0)
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        for t in range(L):
+            blk = int(b.block_tables[s, t // B])
+            at = orc.e4m3_k_index(blk, 1, t % B, 0, b.num_kv_heads, B, D)
+            kflat[at] = needle
+            out = _gpu_fp8_decode(b, pools, mode, part or 512)
+            kflat[at] = 0
+            # + 0.0: a -0 code (0x80) reads as +0, the sum of the other tokens' zero-weighted terms
+            want = (torch.tensor([orc.e4m3_value(int(vflat[orc.e4m3_v_index(blk, 1, t % B, d, b.num_kv_heads, B, D)]))
+                                  for d in range(D)], dtype=torch.float64) + 0.0).to(qdt)
+            for h in range(g, 2 * g):
+                assert torch.equal(out[s, h].cpu().view(torch.int16), want.view(torch.int16)), (s, t, h)
+            assert torch.isfinite(out[s, :g].float()).all()
