@@ -308,6 +308,18 @@ class Step:
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.counters = pa.Counters()
         self.kernels_per_step = {"append": 1, "splitk2": 3}.get(mode, 2)
+        # the one-launch step over these fixed buffers, marshalled once (a
+        # serving loop's form of the call)
+        self.prepared = None
+        if mode == "append":
+            if self.fp8:
+                self.prepared = pa.prepare_decode_append_fp8(
+                    self.out, self.q, self.nk, self.nv, self.k, self.v, self.ks, self.vs, self.bt, self.cl,
+                    batch.scale, max_context_len=self.mcl, seq_order=self.order)
+            else:
+                self.prepared = pa.prepare_decode_append(
+                    self.out, self.q, self.nk, self.nv, self.k, self.v, self.bt, self.cl, batch.scale,
+                    max_context_len=self.mcl, seq_order=self.order)
 
     def reshape(self, stream):
         if self.mode == "append":
@@ -319,6 +331,9 @@ class Step:
         self.pa.pa_reshape_and_cache(self.nk, self.nv, self.k, self.v, self.slots, stream=stream)
 
     def decode(self, stream):
+        if self.prepared is not None:
+            self.prepared(stream)
+            return
         if self.fp8:
             if self.mode == "append":
                 self.pa.pa_decode_append_fp8(self.out, self.q, self.nk, self.nv, self.k, self.v, self.ks, self.vs,

@@ -231,7 +231,6 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_c
     _check(lib.pa_decode(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode")
 
 
-@_on_tensor_device
 def _counts_ptr(ref_counts, num_blocks):
     if ref_counts is None:
         return None
@@ -240,6 +239,14 @@ def _counts_ptr(ref_counts, num_blocks):
     return _dev_ptr(ref_counts, "ref_counts")
 
 
+def _append_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                 seq_order, ref_counts):
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    return [args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
+            _counts_ptr(ref_counts, k_cache.shape[0]), _order_ptr(seq_order, q.shape[0])]
+
+
+@_on_tensor_device
 def pa_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len=None,
                      stream=None, seq_order=None, ref_counts=None):
     """One decode step: write each sequence's newest token (key/value [S, Hkv,
@@ -247,10 +254,44 @@ def pa_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context
     ref_counts (int32 [num_blocks], optional): a sequence whose newest block
     is held by others is not written (DEVERR_SHARED_BLOCK)."""
     lib = load()
-    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
-    _check(lib.pa_decode_append(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
-                                _counts_ptr(ref_counts, k_cache.shape[0]), _order_ptr(seq_order, q.shape[0]),
-                                _stream(stream)), "pa_decode_append")
+    args = _append_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                        seq_order, ref_counts)
+    _check(lib.pa_decode_append(*args, _stream(stream)), "pa_decode_append")
+
+
+class Prepared:
+    """One entry-point call whose arguments were checked and marshalled once:
+    calling it (optionally with a stream; the current stream otherwise) makes
+    the same C-ABI call again, with the same pointers and sizes, on the device
+    that holds its tensors.  For a step repeated over fixed buffers, as a
+    serving loop does, it spares the per-call argument work; the buffers'
+    contents may change between calls, their storage may not (the object keeps
+    a reference to each tensor)."""
+
+    def __init__(self, name, args, device, tensors):
+        self._fn = getattr(load(), name)
+        self._name = name
+        self._args = tuple(args)
+        self._device = device.index
+        self._tensors = tensors
+
+    def __call__(self, stream=None):
+        if torch.cuda.current_device() != self._device:
+            with torch.cuda.device(self._device):
+                return self(stream)
+        _check(self._fn(*self._args, _stream(stream)), self._name)
+
+
+def prepare_decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale,
+                          max_context_len=None, seq_order=None, ref_counts=None) -> Prepared:
+    """pa_decode_append's arguments checked and marshalled once (see Prepared)."""
+    tensors = (out, q, key, value, k_cache, v_cache, block_tables, context_lens, seq_order, ref_counts)
+    dev = _tensor_device(tensors, {})
+    if dev is None:
+        raise ValueError("pa_decode_append takes CUDA tensors")
+    args = _append_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                        seq_order, ref_counts)
+    return Prepared("pa_decode_append", args, dev, tensors)
 
 
 def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size=512) -> int:
@@ -407,6 +448,13 @@ def pa_decode_fp8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, cont
     _check(lib.pa_decode_fp8(*args, _order_ptr(seq_order, q.shape[0]), _stream(stream)), "pa_decode_fp8")
 
 
+def _append_fp8_args(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                     max_context_len, seq_order, ref_counts):
+    args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
+    return [args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
+            _counts_ptr(ref_counts, k_cache.shape[0]), _order_ptr(seq_order, q.shape[0])]
+
+
 @_on_tensor_device
 def pa_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                          scale, max_context_len=None, stream=None, seq_order=None, ref_counts=None):
@@ -415,10 +463,22 @@ def pa_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale,
     attend over the whole context (one launch).  ref_counts as in
     pa_decode_append."""
     lib = load()
-    args = _fp8_args(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale, max_context_len)
-    _check(lib.pa_decode_append_fp8(args[0], args[1], _dev_ptr(key, "key"), _dev_ptr(value, "value"), *args[2:],
-                                    _counts_ptr(ref_counts, k_cache.shape[0]), _order_ptr(seq_order, q.shape[0]),
-                                    _stream(stream)), "pa_decode_append_fp8")
+    args = _append_fp8_args(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                            scale, max_context_len, seq_order, ref_counts)
+    _check(lib.pa_decode_append_fp8(*args, _stream(stream)), "pa_decode_append_fp8")
+
+
+def prepare_decode_append_fp8(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                              scale, max_context_len=None, seq_order=None, ref_counts=None) -> Prepared:
+    """pa_decode_append_fp8's arguments checked and marshalled once (see Prepared)."""
+    tensors = (out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, seq_order,
+               ref_counts)
+    dev = _tensor_device(tensors, {})
+    if dev is None:
+        raise ValueError("pa_decode_append_fp8 takes CUDA tensors")
+    args = _append_fp8_args(out, q, key, value, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                            scale, max_context_len, seq_order, ref_counts)
+    return Prepared("pa_decode_append_fp8", args, dev, tensors)
 
 
 @_on_tensor_device

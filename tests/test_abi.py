@@ -206,3 +206,32 @@ def test_binding_refuses_tensors_on_two_devices():
         pa.pa_decode_splitk_static(a, a, a, a, a, b, 0.125, 64)
     assert pa._tensor_device((a, 3, None), {"x": a}) == torch.device("cuda", 0)
     assert pa._tensor_device((torch.zeros(2),), {}) is None
+
+
+# every entry point that takes tensors, with its number of leading tensor arguments
+TENSOR_ENTRIES = {
+    "pa_reshape_and_cache": 5, "pa_decode": 6, "pa_decode_append": 8, "pa_decode_splitk": 6,
+    "pa_decode_splitk_static": 6, "pa_copy_blocks": 5, "pa_reshape_and_cache_fp8": 7, "pa_decode_fp8": 8,
+    "pa_decode_append_fp8": 10, "pa_decode_splitk_fp8": 8, "pa_prefill": 7, "pa_blocks_init": 3,
+    "pa_blocks_append": 7, "pa_blocks_fork": 4, "pa_blocks_release": 6,
+}
+
+
+def test_every_tensor_entry_checks_the_device():
+    """Each tensor entry point runs under the device guard (a helper may not
+    take its place) and refuses tensors on two devices before any marshalling."""
+    public = {n for n in dir(pa) if n.startswith("pa_") and callable(getattr(pa, n))}
+    takes_tensors = public - {"pa_status_string", "pa_get_device_error", "pa_decode_splitk_workspace_size"}
+    assert takes_tensors == set(TENSOR_ENTRIES)
+    a, b = _FakeCudaTensor.make(0), _FakeCudaTensor.make(1)
+    for name, n in TENSOR_ENTRIES.items():
+        fn = getattr(pa, name)
+        assert getattr(fn, "__wrapped__", None) is not None, name
+        args = [a] * (n - 1) + [b]
+        with pytest.raises(ValueError, match="one CUDA device"):
+            fn(*args, *([0] * 8))
+    for fn, n in ((pa.prepare_decode_append, 8), (pa.prepare_decode_append_fp8, 10)):
+        with pytest.raises(ValueError, match="one CUDA device"):
+            fn(*([a] * (n - 1) + [b]), 0.125)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        pa.prepare_decode_append(*([torch.zeros(2)] * 8), 0.125)

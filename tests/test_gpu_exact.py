@@ -320,3 +320,34 @@ def test_append_equals_reshape_then_decode(orc, make):
     c = b.__class__(**{**b.__dict__, "k_cache": kc, "v_cache": vc})
     check_tolerance(as_f64(out[seqs]), oracle_decode_sampled(orc, c, seqs), b.dtype)
     assert pa.pa_get_device_error() == 0
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_prepared_call_repeats_the_entry(fp8):
+    """A prepared decode step makes the same call as the entry point: outputs
+    and pools bit-identical, also after the buffers' contents change between
+    calls (new queries and new tokens written in place)."""
+    b = workloads.llama3_8b_decode(seed=1300, device="cuda", num_seqs=24, num_blocks=4096)
+    q, nk, nv = b.q.cuda().contiguous(), b.new_key.cuda().contiguous(), b.new_value.cuda().contiguous()
+    bt, cl = b.block_tables.cuda(), b.context_lens.cuda()
+    if fp8:
+        pools = workloads.random_fp8_pools(b, seed=1301, device="cuda")
+        k0, v0, extra = pools.k_cache, pools.v_cache, (pools.k_scale, pools.v_scale)
+        entry, prepare = pa.pa_decode_append_fp8, pa.prepare_decode_append_fp8
+    else:
+        k0, v0, extra = b.k_cache.cuda(), b.v_cache.cuda(), ()
+        entry, prepare = pa.pa_decode_append, pa.prepare_decode_append
+    k1, v1, k2, v2 = k0.clone(), v0.clone(), k0.clone(), v0.clone()
+    ref, got = torch.empty_like(q), torch.empty_like(q)
+    step = prepare(got, q, nk, nv, k2, v2, *extra, bt, cl, b.scale, max_context_len=b.max_context_len)
+    g = torch.Generator(device="cuda").manual_seed(1302)
+    for _ in range(3):
+        entry(ref, q, nk, nv, k1, v1, *extra, bt, cl, b.scale, max_context_len=b.max_context_len)
+        step(torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        assert torch.equal(_bits(got), _bits(ref))
+        assert torch.equal(k1, k2) and torch.equal(v1, v2)
+        q.copy_(torch.randn(q.shape, generator=g, device="cuda").to(q.dtype))
+        nk.copy_(torch.randn(nk.shape, generator=g, device="cuda").to(nk.dtype))
+        nv.copy_(torch.randn(nv.shape, generator=g, device="cuda").to(nv.dtype))
+    assert pa.pa_get_device_error() == 0
