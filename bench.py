@@ -90,6 +90,19 @@ def parse_args(argv=None):
 
 # ----------------------------------------------------------------------------- helpers
 
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -1025,7 +1038,8 @@ def run_reference(args, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (same seeded workload as the GPU arm)",
         "config": {"workload": batch.name, "global_batch": batch.num_seqs},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+                         "cpu": cpu_model(), "host_cores": os.cpu_count()},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -1236,7 +1250,8 @@ def main(argv=None):
                 except (OSError, RuntimeError) as err:   # no worker threads on this host: one core only
                     gbs, desc, cores = gbs1, f"{desc1} (threads unavailable: {err})", 1
                 res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                       "sample": desc, "one_core_value": round(gbs1, 4), "one_core_sample": desc1}
+                                       "sample": desc, "one_core_value": round(gbs1, 4), "one_core_sample": desc1,
+                                       "cpu": cpu_model(), "host_cores": os.cpu_count()}
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:
