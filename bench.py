@@ -125,15 +125,15 @@ def make_workload(name, seed, device, block_size=None):
 # in profiles/).  Keyed by a hash of the kernel sources: once the kernels change,
 # the figure no longer describes them and the bench reports null.
 NCU_TRAFFIC = {
-    "bd65e2259e5daeb1": {
-        ("llama3_8b_decode_bf16", "append"): 292.749e6 + 3.886e6,
-        ("continuous_batching_mix_bf16_B16", "append"): 211.576e6 + 4.036e6,
-        ("llama3_70b_long_bf16", "splitk"): 2.519447e9 + 7.714e6,
-        ("llama3_8b_decode_bf16+e4m3", "append"): 146.828e6 + 3.555e6,
-        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260197e9 + 6.723e6,
+    "2f61bf8a4fbb2a5e": {
+        ("llama3_8b_decode_bf16", "append"): 292.750e6 + 4.040e6,
+        ("continuous_batching_mix_bf16_B16", "append"): 211.607e6 + 4.295e6,
+        ("llama3_70b_long_bf16", "splitk"): 2.519449e9 + 7.665e6,
+        ("llama3_8b_decode_bf16+e4m3", "append"): 146.826e6 + 3.447e6,
+        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260278e9 + 6.659e6,
     },
-    "d46dc2e5cee1688c": {
-        ("chunked_prefill_bfloat16", "prefill"): 118.550e6 + 20.487e6,
+    "80f88590dac967ba": {
+        ("chunked_prefill_bfloat16", "prefill"): 118.550e6 + 20.485e6,
     },
 }
 

@@ -314,9 +314,9 @@ bool device_accessible(const void* p) {
 constexpr int kPrefillWarps = 4;
 constexpr int kPrefillStages = 4;
 
-// Blocks of 16 or 32 tokens run the 5th-generation tensor-core kernel (two
-// query tiles of 128 MMA rows per CTA); 8-token blocks, PA_PREFILL_TC=0 or a K
-// pool that no tensor map can describe run the warp-level one.
+// Blocks of 8, 16 or 32 tokens run the 5th-generation tensor-core kernel (two
+// query tiles of 128 MMA rows per CTA); PA_PREFILL_TC=0 or a K pool that no
+// tensor map can describe run the warp-level one.
 #ifndef PA_PREFILL_TC
 #define PA_PREFILL_TC 1
 #endif
@@ -702,7 +702,7 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     p.context_cap = context_cap(sh);
     p.num_blocks = num_blocks;
     CUtensorMap k_rows{};
-    const bool use_tc = PA_PREFILL_TC && block_size != 8 &&
+    const bool use_tc = PA_PREFILL_TC &&
                         encode_k_rows(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks);
     p.tile_tokens = (use_tc ? 128 : kPrefillWarps * 16) / p.group;
     // the tensor-core kernel takes two query tiles per CTA
@@ -716,10 +716,8 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
         constexpr int kD = decltype(dd)::value, kB = decltype(bb)::value;
         if constexpr (pa::IsF32<T>::value) {
             return cudaErrorInvalidValue;
-        } else if constexpr (kB != 8) {
-            return use_tc ? launch_prefill_tc<T, kD, kB>(p, k_rows, grid, s) : launch_prefill<T, kD, kB>(p, grid, s);
         } else {
-            return launch_prefill<T, kD, kB>(p, grid, s);
+            return use_tc ? launch_prefill_tc<T, kD, kB>(p, k_rows, grid, s) : launch_prefill<T, kD, kB>(p, grid, s);
         }
     });
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -6,11 +6,13 @@
 //    tiles).  A query tile is 128 MMA rows, (query token, head of the GQA
 //    group) pairs, 128 / g tokens; in a softmax warpgroup thread t owns row t,
 //    which is tensor-memory lane t.  The two tiles share every K/V tile.
-//  * Key tiles of 64 keys.  K arrives chunk-major, [D/8][64][8], by
-//    tile::gather4 loads (one 8-dim chunk of four pool blocks per load), so
-//    S = Q K^T is one N = 64 MMA per 16-dim step; V arrives as whole (block,
-//    head) tiles [D/8][B][8] by 1-D bulk copies, the MN-major B operand of
-//    O += P V as stored.  K and V have four-stage rings of their own.
+//  * Key tiles of 64 keys (8, 4 or 2 pool blocks of 8, 16 or 32 tokens).  K
+//    arrives chunk-major, [D/8][64][8], by tile::gather4 loads (one 8-dim chunk
+//    of four pool blocks per load, two chunks of two blocks for 32-token
+//    blocks), so S = Q K^T is one N = 64 MMA per 16-dim step; V arrives as
+//    whole (block, head) tiles [D/8][B][8] by 1-D bulk copies, the MN-major B
+//    operand of O += P V as stored (with 8-token blocks one 16-key step reads
+//    two adjacent tiles).  K and V have three-stage rings of their own.
 //  * Warp roles: 0-3 and 4-7 softmax of query tile 0 and 1; 8 and 9 issue
 //    S = Q K^T for query tile 0 and 1 (Q and K in shared memory); 10 and 11
 //    issue O += P V for query tile 0 and 1 (P in tensor memory, V in shared
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     constexpr uint32_t kTmemCols = 512;
     constexpr uint32_t kOCol = kKeys, kPCol = kKeys + D;
     static_assert(kPCol + kKeys <= 256, "tensor memory budget");
-    static_assert(B == 16 || B == 32, "16- or 32-token blocks");
+    static_assert(B == 8 || B == 16 || B == 32, "8-, 16- or 32-token blocks");
     static_assert(D == 64 || D == 128, "head dims");
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBarOff);
@@ -337,7 +339,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
         return ok;
     };
 
-    // ---- producers: warp 10 lane 0 fetches K tiles, warp 11 lane 0 V tiles
+    // ---- producers: warp 12 lane 0 fetches K tiles, warp 13 lane 0 V tiles
     const bool is_producer = (warp == 12 || warp == 13) && lane == 0;
     const bool v_side = warp == 13;
     const char* vpool = reinterpret_cast<const char*>(p.v_cache);
@@ -369,16 +371,36 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
                 for (int b = 0; b < kBlocks; ++b)
                     rid[b] = ((((ok >> b) & 1u) ? ids[b] : sub) * p.num_kv_heads + kvh) * (D / 8);
                 mbar_arrive_expect_tx(&full[st], Sm::kStage);
-                if constexpr (B == 16) {
+                if constexpr (B <= 16) {   // four blocks' rows of chunk c per load
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c)
-                        tc::gather4(dst + c * 1024, &k_rows, 0, rid[0] + c, rid[1] + c, rid[2] + c, rid[3] + c,
-                                    &full[st]);
+#pragma unroll
+                        for (int g = 0; g < kBlocks / 4; ++g)
+                            tc::gather4(dst + c * 1024 + g * (4 * B * 16), &k_rows, 0, rid[4 * g] + c,
+                                        rid[4 * g + 1] + c, rid[4 * g + 2] + c, rid[4 * g + 3] + c, &full[st]);
                 } else {
 #pragma unroll
                     for (int c = 0; c < D / 8; c += 2)
                         tc::gather4(dst + c * 1024, &k_rows, 0, rid[0] + c, rid[1] + c, rid[0] + c + 1,
                                     rid[1] + c + 1, &full[st]);
+                }
+            }
+        } else if constexpr (B == 8) {
+            // One 16-key MMA step spans two 8-token blocks, so every block of a
+            // tile with any fetchable one is fetched: a refused or unneeded one
+            // as the tile's first fetchable block (P is 0 on its keys), so that
+            // no step reads stale shared memory.
+            int sub = ids[kBlocks - 1];
+#pragma unroll
+            for (int b = kBlocks - 1; b >= 0; --b)
+                if ((ok >> b) & 1u) sub = ids[b];
+            mbar_arrive_expect_tx(&full[st], ok != 0u ? kBlocks * kTile : 0);
+            if (ok != 0u) {
+#pragma unroll
+                for (int b = 0; b < kBlocks; ++b) {
+                    const int id = ((ok >> b) & 1u) ? ids[b] : sub;
+                    const long long off = (static_cast<long long>(id) * p.num_kv_heads + kvh) * kTile;
+                    tc::bulk_copy(dst + b * kTile, vpool + off, kTile, &full[st]);
                 }
             }
         } else {
@@ -517,12 +539,22 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
                     tc::fence_after();
                     const uint32_t qb = tmem + static_cast<uint32_t>(q) * 256u;
                     const uint32_t pt = qb + kPCol + static_cast<uint32_t>(j & 1) * (kKeys / 2);
-                    for (int b = 0; b < kBlocks; ++b) {
-                        if (!((ok >> b) & 1u)) continue;
+                    if constexpr (B == 8) {
+                        // keys 16 pr .. 16 pr + 15: blocks 2 pr and 2 pr + 1, adjacent
+                        // tiles (the next 8 keys one tile further on)
+                        for (int pr = 0; pr < kBlocks / 2; ++pr) {
+                            if (!((ok >> (2 * pr)) & 3u)) continue;
+                            tc::mma_ts(qb + kOCol, pt + 8 * pr, tc::smem_desc(vbase + 2 * pr * kTile, kTile, 128),
+                                       idesc_o, true);
+                        }
+                    } else {
+                        for (int b = 0; b < kBlocks; ++b) {
+                            if (!((ok >> b) & 1u)) continue;
 #pragma unroll
-                        for (int ks = 0; ks < B / 16; ++ks)
-                            tc::mma_ts(qb + kOCol, pt + (b * B) / 2 + 8 * ks,
-                                       tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
+                            for (int ks = 0; ks < B / 16; ++ks)
+                                tc::mma_ts(qb + kOCol, pt + (b * B) / 2 + 8 * ks,
+                                           tc::smem_desc(vbase + b * kTile + ks * 256, 128, B * 16), idesc_o, true);
+                        }
                     }
                     tc::commit(&p_free[pb]);
                 }

@@ -91,12 +91,15 @@ def test_chunk_longer_than_context_is_flagged():
     assert torch.isfinite(out[12:].float()).all()
 
 
-def test_refused_block_ids_are_flagged_and_masked(orc):
+@pytest.mark.parametrize("block_size", [16, 8, 32])
+def test_refused_block_ids_are_flagged_and_masked(orc, block_size):
     """Block ids outside the pool (negative, or past its end) are flagged and
     never fetched: a whole key tile of them (no block of the tile fetchable),
-    and a single one among fetchable blocks.  Untouched sequences still match
-    the oracle; rows of the damaged sequences stay finite."""
-    b = workloads.chunked_prefill(seed=1040, num_seqs=3, context_range=(200, 400), chunk_range=(40, 150))
+    and a single one among fetchable blocks (with 8-token blocks, the partner
+    of a fetchable block in one 16-key MMA step).  Untouched sequences still
+    match the oracle; rows of the damaged sequences stay finite."""
+    b = workloads.chunked_prefill(seed=1040, num_seqs=3, context_range=(200, 400), chunk_range=(40, 150),
+                                  block_size=block_size)
     ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.meta["query_start"], b.scale,
                       b.block_size, b.num_kv_heads)
     bad = b.block_tables.clone()
