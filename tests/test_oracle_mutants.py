@@ -101,13 +101,32 @@ def _pins_failed(lib):
     return [x for x in line[len("FAILED:"):].split(",") if x]
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
-    old, new = MUTANTS[name]
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant built and run against the pins once, several at a time
+    (each is a g++ build and a child process): name -> pins that failed, or
+    None when the mutation's anchor is not in the source exactly once."""
+    from concurrent.futures import ThreadPoolExecutor
+    base = tmp_path_factory.mktemp("mutants")
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation anchor not found exactly once: {old!r}"
-    mutant_src = tmp_path / "pa_oracle_mutant.cpp"
-    mutant_src.write_text(src.replace(old, new))
-    lib = oracle.build(str(mutant_src), str(tmp_path / "liboracle_mutant.so"), force=True)
-    failed = _pins_failed(lib)
+
+    def one(name):
+        old, new = MUTANTS[name]
+        if src.count(old) != 1:
+            return name, None
+        d = base / name
+        d.mkdir()
+        mutant_src = d / "pa_oracle_mutant.cpp"
+        mutant_src.write_text(src.replace(old, new))
+        lib = oracle.build(str(mutant_src), str(d / "liboracle_mutant.so"), force=True)
+        return name, _pins_failed(lib)
+
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        return dict(ex.map(one, sorted(MUTANTS)))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_results):
+    failed = mutant_results[name]
+    assert failed is not None, f"mutation anchor not found exactly once: {MUTANTS[name][0]!r}"
     assert failed, f"no pin caught the planted mistake {name}"
