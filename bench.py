@@ -125,15 +125,17 @@ def make_workload(name, seed, device, block_size=None):
 # in profiles/).  Keyed by a hash of the kernel sources: once the kernels change,
 # the figure no longer describes them and the bench reports null.
 NCU_TRAFFIC = {
-    "2f61bf8a4fbb2a5e": {
-        ("llama3_8b_decode_bf16", "append"): 292.750e6 + 4.040e6,
-        ("continuous_batching_mix_bf16_B16", "append"): 211.607e6 + 4.295e6,
-        ("llama3_70b_long_bf16", "splitk"): 2.519449e9 + 7.665e6,
-        ("llama3_8b_decode_bf16+e4m3", "append"): 146.826e6 + 3.447e6,
-        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260278e9 + 6.659e6,
+    "8d6a4be27dd58bae": {
+        ("llama3_8b_decode_bf16", "append"): 292.753e6 + 3.747e6,
+        ("continuous_batching_mix_bf16_B16", "append"): 211.582e6 + 4.086e6,
+        ("llama3_70b_long_bf16", "splitk"): 2.519437e9 + 7.483e6,
+        ("llama3_8b_decode_bf16+e4m3", "append"): 146.828e6 + 3.282e6,
+        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260203e9 + 6.577e6,
     },
     "80f88590dac967ba": {
         ("chunked_prefill_bfloat16", "prefill"): 118.550e6 + 20.485e6,
+        ("chunked_prefill_bfloat16_B8", "prefill"): 118.375e6 + 20.615e6,
+        ("chunked_prefill_bfloat16_B32", "prefill"): 118.735e6 + 20.586e6,
     },
 }
 
@@ -915,15 +917,19 @@ def config_lines(args, world, rank):
     torch.cuda.empty_cache()
     # the widened rows measured by their own bench modes, trimmed to the figures
     keep = ("metric", "value", "unit", "ms_per_step", "roofline", "gpu_launches")
-    for name, op, workload, steps in (("chunked_prefill", "prefill", args.workload, K),
-                                      ("copy_blocks_cow", "copy_blocks", "llama3_8b_decode", K),
-                                      ("swap_out", "swap_out", "llama3_8b_decode", min(K, 10)),
-                                      ("swap_in", "swap_in", "llama3_8b_decode", min(K, 10))):
+    for name, op, workload, steps, bs in (("chunked_prefill", "prefill", args.workload, K, None),
+                                          ("chunked_prefill_B8", "prefill", args.workload, K, 8),
+                                          ("chunked_prefill_B32", "prefill", args.workload, K, 32),
+                                          ("copy_blocks_cow", "copy_blocks", "llama3_8b_decode", K, None),
+                                          ("swap_out", "swap_out", "llama3_8b_decode", min(K, 10), None),
+                                          ("swap_in", "swap_in", "llama3_8b_decode", min(K, 10), None)):
         sub = argparse.Namespace(**dict(vars(args), op=op, workload=workload, steps=steps, warmup=W,
-                                        block_size=None))
+                                        block_size=bs))
         res = (run_prefill if op == "prefill" else run_blocks)(sub, world, rank, int(os.environ.get("LOCAL_RANK", "0")))
         e = {k: res[k] for k in keep if k in res}
         e["workload"] = res["config"]["workload"]
+        if op == "prefill":
+            e["block_size"] = res["config"]["block_size"]
         out[name] = e
         torch.cuda.empty_cache()
     return out
@@ -1060,7 +1066,7 @@ def run_prefill(args, world, rank, local):
     from paged_kv_cache_449_b200 import build as pabuild
     pabuild.build()
     pa.load()
-    b = workloads.chunked_prefill(seed=args.seed + rank, device="cuda")
+    b = workloads.chunked_prefill(seed=args.seed + rank, device="cuda", block_size=args.block_size or 16)
     qs = b.meta["query_start"]
     chunks = (qs[1:] - qs[:-1]).to(torch.int64)
     lens = b.context_lens.to(torch.int64)
@@ -1113,11 +1119,11 @@ def run_prefill(args, world, rank, local):
                    "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim,
                    "block_size": b.block_size, "flops_per_step": flops, "parallelism": f"replicas x{world}",
                    "l2": "not flushed: compute-bound (the K/V of a sequence is reread by its query tiles)",
-                   "mma": ("tcgen05.mma kind::f16, M = 128 query rows, Q / S / O in tensor memory, fp32 accumulate"
-                           if b.block_size != 8 else "mma.sync m16n8k16 bf16, fp32 accumulate")},
+                   "mma": "tcgen05.mma kind::f16, M = 128 query rows, S / O / P in tensor memory, fp32 accumulate"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "peak_kind": kind,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": NCU_TRAFFIC.get(kernel_source_hash(PREFILL_SOURCES), {}).get((b.name, "prefill"))},
+                     "traffic": NCU_TRAFFIC.get(kernel_source_hash(PREFILL_SOURCES), {}).get(
+                         (b.name if b.block_size == 16 else f"{b.name}_B{b.block_size}", "prefill"))},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }

@@ -195,7 +195,7 @@ struct DecodeSmem {
     static constexpr int kElem = FP8 ? 1 : sizeof(T);
     static constexpr int kTile = B * D * kElem;                 // one (block, head) tile, bytes
     static constexpr int kRing = NW * STAGES * 2 * kTile;       // K and V slots of all warps
-    static constexpr int kMerge = NW * kMaxGroup * (D + 2) * 4;  // warp states for the CTA merge
+    static constexpr int kMerge = NW * kMaxGroup * (kMergeRow<D> + 2) * 4;  // warp states for the CTA merge
     static constexpr int kArea = kRing > kMerge ? kRing : kMerge;
     static constexpr int kBars = (NW * STAGES * 8 + 15) / 16 * 16;  // keeps what follows 16-byte aligned
     static constexpr int kQ = IsF32<T>::value ? kMaxGroup * D * 4 : 0;
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
 
     // ---- merge the warps' states (the ring is free now)
     float* mo = reinterpret_cast<float*>(smem);
-    float* mml = mo + NW * kMaxGroup * D;
+    float* mml = mo + NW * kMaxGroup * kMergeRow<D>;
     if (!any_failed) {
         acc.store_smem(mo, mml, warp, group, lane);
         __syncthreads();
@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
                 const float wt = softmax_exp<kLog2>(mml[(w * kMaxGroup + r) * 2] - M);
-                num = fmaf(wt, mo[(w * kMaxGroup + r) * D + d], num);
+                num = fmaf(wt, mo[(w * kMaxGroup + r) * kMergeRow<D> + d], num);
                 den = fmaf(wt, mml[(w * kMaxGroup + r) * 2 + 1], den);
             }
         }

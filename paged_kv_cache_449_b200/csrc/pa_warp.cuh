@@ -21,6 +21,12 @@ namespace pa {
 
 constexpr int kMaxGroup = 8;
 
+// Row stride (floats) of the accumulator rows in the CTA-merge area of shared
+// memory: four floats of padding put the rows that one store instruction
+// writes (the heads of a thread, two rows apart) in different banks.
+template <int D>
+constexpr int kMergeRow = D + 4;
+
 template <typename T>
 struct IsF32 {
     static constexpr bool value = false;
@@ -361,7 +367,7 @@ struct WarpMma {
     __device__ __forceinline__ void store_smem(float* mo, float* mml, int warp, int group, int lane) {
         const int r = lane >> 2, c = lane & 3;
         const float l0 = head_sum(0), l1 = head_sum(1);
-        for_each(group, lane, [&](int e, int d, float v) { mo[(warp * kMaxGroup + 2 * c + e) * D + d] = v; });
+        for_each(group, lane, [&](int e, int d, float v) { mo[(warp * kMaxGroup + 2 * c + e) * kMergeRow<D> + d] = v; });
         if (r == 0) {
             if (2 * c < group) {
                 mml[(warp * kMaxGroup + 2 * c) * 2] = m_run[0];
@@ -521,7 +527,7 @@ struct WarpF32 {
 #pragma unroll
         for (int h = 0; h < kMaxGroup; ++h) {
             if (h < group && tg == 0) {
-                float* dst = mo + (warp * kMaxGroup + h) * D + cj * 4;
+                float* dst = mo + (warp * kMaxGroup + h) * kMergeRow<D> + cj * 4;
                 dst[0] = o[h][0];
                 dst[1] = o[h][1];
                 dst[2] = o[h][2];
