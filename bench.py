@@ -132,10 +132,10 @@ NCU_TRAFFIC = {
         ("llama3_8b_decode_bf16+e4m3", "append"): 146.828e6 + 3.282e6,
         ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260203e9 + 6.577e6,
     },
-    "80f88590dac967ba": {
-        ("chunked_prefill_bfloat16", "prefill"): 118.550e6 + 20.485e6,
-        ("chunked_prefill_bfloat16_B8", "prefill"): 118.375e6 + 20.615e6,
-        ("chunked_prefill_bfloat16_B32", "prefill"): 118.735e6 + 20.586e6,
+    "32ac9fb6fe993233": {
+        ("chunked_prefill_bfloat16", "prefill"): 118.548e6 + 19.815e6,
+        ("chunked_prefill_bfloat16_B8", "prefill"): 118.374e6 + 19.943e6,
+        ("chunked_prefill_bfloat16_B32", "prefill"): 118.735e6 + 20.086e6,
     },
 }
 

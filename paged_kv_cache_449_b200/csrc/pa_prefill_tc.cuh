@@ -331,6 +331,15 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             ids[b] = (j < ntiles && jb < nblk) ? __ldg(table + jb) : -1;
         }
     };
+    // The same mask computed by a whole warp: lane b loads block b's id (the
+    // id of lane `lane` for tile j; -1 past the need), a ballot gathers them.
+    auto lane_id = [&](int j) -> int {
+        const int jb = j * kBlocks + lane;
+        return (lane < kBlocks && j < ntiles && jb < nblk) ? __ldg(table + jb) : -1;
+    };
+    auto ok_ballot = [&](int id) -> uint32_t {
+        return __ballot_sync(0xffffffffu, id >= 0 && static_cast<long long>(id) < p.num_blocks);
+    };
     auto ok_of = [&](const int (&ids)[kBlocks]) {
         uint32_t ok = 0;
 #pragma unroll
@@ -513,11 +522,10 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
         const int q = warp - 10;
         const uint32_t idesc_o = tc::instr_desc<T>(D, true);
         const uint32_t v_ring = smem_u32(smem + Sm::kVOff);
-        int id_n[kBlocks];
-        load_ids(0, id_n);
+        int id_n = lane_id(0);
         for (int j = 0; j < ntiles; ++j) {
-            const uint32_t ok = ok_of(id_n);
-            load_ids(j + 1, id_n);
+            const uint32_t ok = ok_ballot(id_n);
+            id_n = lane_id(j + 1);
             const int vst = j % VS;
             if (!__all_sync(0xffffffffu, tc_wait(&v_full[vst], (j / VS) & 1, abort))) break;
             const int lb = (L - 1) / B - j * kBlocks;
@@ -574,13 +582,12 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
         const int n = my_nt;
         uint64_t* sfull = &s_full[qt];
         uint64_t* sfree = &s_free[qt];
-        int id_n[kBlocks];
-        load_ids(0, id_n);
-        uint32_t ok = ok_of(id_n);
+        int id_n = lane_id(0);
+        uint32_t ok = ok_ballot(id_n);
         float m_run = kNegInf, l_run = 0.f;
         for (int j = 0; j < n; ++j) {
             const int pb = qt * 2 + (j & 1);
-            load_ids(j + 1, id_n);
+            id_n = lane_id(j + 1);
             if (!__all_sync(0xffffffffu, tc_wait(sfull, j & 1, abort))) {
                 failed = true;
                 break;
@@ -674,7 +681,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc::fence_before();
             mbar_arrive(&p_full[pb]);
-            ok = ok_of(id_n);
+            ok = ok_ballot(id_n);
         }
         // ---- the last O += P V, then this row of the output
         if (!failed && !__all_sync(0xffffffffu, tc_wait(&p_free[qt * 2 + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort)))
