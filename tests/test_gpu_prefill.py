@@ -62,8 +62,12 @@ def test_prefill_every_element(orc, case):
     check_tolerance(as_f64(got), ref, dt)
 
 
-def test_prefill_llama3_8b_shape(orc):
-    b = workloads.chunked_prefill(seed=1010, num_seqs=4, context_range=(512, 1024), chunk_range=(64, 256))
+@pytest.mark.parametrize("block_size", [16, 8, 32])
+def test_prefill_llama3_8b_shape(orc, block_size):
+    """Llama-3-8B heads, every element, at each pool block size (8-token blocks
+    pair two V tiles per MMA step; 32-token blocks gather two chunks per load)."""
+    b = workloads.chunked_prefill(seed=1010, num_seqs=4, context_range=(512, 1024), chunk_range=(64, 256),
+                                  block_size=block_size)
     ref = orc.prefill(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, b.meta["query_start"], b.scale,
                       b.block_size, b.num_kv_heads)
     got = _gpu_prefill(b)
