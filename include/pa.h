@@ -343,12 +343,12 @@ pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, co
  *   of range sets PA_DEVERR_CONTEXT_LEN and its rows are not written; block
  *   ids outside [0, num_blocks) set PA_DEVERR_BLOCK_ID, are never read, and
  *   their keys are left out of the softmax.
- *   Blocks of 16 or 32 tokens run on the 5th-generation tensor cores
- *   (tcgen05, fp32 accumulation in tensor memory); the K pool is then read
- *   through a tensor map built per call, which needs the CUDA driver and at
- *   most 2^31 - 1 rows of (block, kv head, 8 dims).  8-token blocks, or a
- *   pool beyond that, run warp-level mma.sync (fp32 accumulation).  The
- *   result is the same attention either way, within the 16-bit tolerance.
+ *   Every block size runs on the 5th-generation tensor cores (tcgen05, fp32
+ *   accumulation in tensor memory); the K pool is then read through a tensor
+ *   map built per call, which needs the CUDA driver and at most 2^31 - 1 rows
+ *   of (block, kv head, 8 dims).  A pool beyond that runs warp-level mma.sync
+ *   (fp32 accumulation).  The result is the same attention either way, within
+ *   the 16-bit tolerance.
  */
 pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                      const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
