@@ -155,15 +155,27 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
         }
     }
     long long tokens = 0, W = 0;
+    // A batch of at most T sequences takes one pass per phase with one sequence
+    // per thread: step 3 then reuses what step 1 read (kept in registers).
+    const bool one_pass = S <= T;
+    int rL = 0, rn = 0, rfirst = 0, rnew = 0, rX = -1;
+    bool rok = false, rcand = false;
     for (int base = 0; base < S; base += T) {
         const int s = base + tid;
         long long n_tok = 0, cand = 0;
         if (s < S) {
             n_tok = max(p.num_new[s], 0);
-            int L, n, first_new, new_blocks, X;
+            int L = 0, n = 0, first_new = 0, new_blocks = 0, X = -1;
             const bool ok = describe_append(p, s, L, n, first_new, new_blocks, X);
             const int r = ok && X >= 0 ? p.st.ref[X] : 0;
             cand = ok && X >= 0 && r > 1 ? 1 : 0;
+            rL = L;
+            rn = n;
+            rfirst = first_new;
+            rnew = new_blocks;
+            rX = X;
+            rok = ok;
+            rcand = cand != 0;
             p.pairs[2 * s] = cand ? X : -1;
             p.pairs[2 * s + 1] = cand ? r : 0;
         }
@@ -218,7 +230,15 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
         const int s = base + tid;
         int L = 0, n = 0, first_new = 0, new_blocks = 0, X = -1;
         bool ok = false, cow = false;
-        if (s < S) {
+        if (s < S && one_pass) {
+            L = rL;
+            n = rn;
+            first_new = rfirst;
+            new_blocks = rnew;
+            X = rX;
+            ok = rok;
+            cow = ok && rcand && p.pairs[2 * s + 1] == 1;   // the flag step 2 set
+        } else if (s < S) {
             // the row is unchanged since step 1 (only its own thread writes it, below)
             n = p.num_new[s];
             L = p.context_lens[s];
@@ -262,8 +282,9 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
             p.st.ref[id] = 1;
             return id;
         };
+        int c = -1;
         if (cow) {
-            const int c = take();
+            c = take();
             atomicSub(p.st.ref + X, 1);
             row[L / B] = c;
             p.pairs[2 * s] = X;
@@ -272,11 +293,27 @@ __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const 
             p.pairs[2 * s] = -1;
             p.pairs[2 * s + 1] = -1;
         }
-        for (int j = 0; j < new_blocks; ++j) row[first_new + j] = take();
-        for (int i = 0; i < n; ++i) {
-            const int t = L + i;
-            const int blk = row[t / B];
-            p.slots[slot0 + i] = blk < 0 ? -1 : static_cast<long long>(blk) * B + t % B;
+        if (one_pass) {
+            // new blocks taken in logical order as the tokens reach them; each
+            // token's slot from the block it lands in (no read-back of the row)
+            int cur = L % B != 0 ? (cow ? c : X) : -1;
+            int cur_lb = L % B != 0 ? L / B : -1;
+            for (int i = 0; i < n; ++i) {
+                const int t = L + i;
+                if (t / B != cur_lb) {
+                    cur_lb = t / B;
+                    cur = take();
+                    row[cur_lb] = cur;
+                }
+                p.slots[slot0 + i] = cur < 0 ? -1 : static_cast<long long>(cur) * B + t % B;
+            }
+        } else {
+            for (int j = 0; j < new_blocks; ++j) row[first_new + j] = take();
+            for (int i = 0; i < n; ++i) {
+                const int t = L + i;
+                const int blk = row[t / B];
+                p.slots[slot0 + i] = blk < 0 ? -1 : static_cast<long long>(blk) * B + t % B;
+            }
         }
         p.context_lens[s] = L + n;
         atomicAdd(reinterpret_cast<unsigned long long*>(&taken_sh), static_cast<unsigned long long>(need));
