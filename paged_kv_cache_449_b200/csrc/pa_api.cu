@@ -60,6 +60,9 @@
 #ifndef PA_FP8_WIDE_RING
 #define PA_FP8_WIDE_RING 8192
 #endif
+#ifndef PA_TWO_CLASS
+#define PA_TWO_CLASS 1
+#endif
 #ifndef PA_DEEP_MAX_CTAS_PER_SM
 #define PA_DEEP_MAX_CTAS_PER_SM 4
 #endif
@@ -177,7 +180,7 @@ cudaError_t with_variant(pa_dtype dt, int D, int B, F&& f) {
 template <typename T, int D, int B, bool SPLIT, Kind K, bool FP8 = false>
 cudaError_t launch_decode(const pa::DecodeParams& p, dim3 grid, cudaStream_t stream) {
     using C = DecodeConfig<T, D, B, K, FP8>;
-    auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT, FP8>;
+    auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT, FP8, !SPLIT && K == Kind::kWide>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
     kernel<<<grid, C::kWarps * 32, C::Smem::kTotal, stream>>>(p);
@@ -216,6 +219,24 @@ cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p
                         : launch_decode<T, kD, kB, false, Kind::kWide, FP8>(p, grid, st);
         }
     });
+}
+
+// A one-pass launch of many small CTAs (the wide shape) without a start
+// order from the host starts the long sequences first by running the grid
+// twice over: the first half takes the sequences of at least a quarter of
+// max_context_len tokens, the second half the others (CTAs start roughly in
+// blockIdx order; a CTA of the other class leaves at once).  Not for 32-token
+// blocks: there a wide CTA holds one 16 KiB stage per warp and three fit an
+// SM, and starting the long sequences first was measured slower.
+dim3 two_class_grid(pa::DecodeParams& p, dim3 grid, int max_context_len, int block_size) {
+    const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
+    const bool wide = ctas > static_cast<long long>(PA_DEEP_MAX_CTAS_PER_SM) * sm_count();
+    if (!PA_TWO_CLASS || !wide || block_size > 16 || p.seq_order != nullptr || 2LL * grid.z > 65535 ||
+        max_context_len < 4)
+        return grid;
+    p.class_threshold = max_context_len / 4;
+    grid.z *= 2;
+    return grid;
 }
 
 template <typename T, int D>
@@ -404,7 +425,7 @@ pa_status decode_one_pass(void* out, const void* q, const void* k_cache, const v
     p.new_key = new_key;
     p.new_value = new_value;
     p.ref_counts = ref_counts;
-    const dim3 grid(1, sh.num_kv_heads, sh.num_seqs);
+    const dim3 grid = two_class_grid(p, dim3(1, sh.num_kv_heads, sh.num_seqs), sh.max_context_len, sh.block_size);
     const cudaError_t e = decode_dispatch<false, FP8>(static_cast<pa_dtype>(sh.dtype), sh.head_dim, sh.block_size,
                                                       p, grid, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -529,7 +550,7 @@ pa_status pa_decode_append(void* out, const void* q, const void* key, const void
     p.new_key = key;
     p.new_value = value;
     p.ref_counts = ref_counts;
-    const dim3 grid(1, num_kv_heads, num_seqs);
+    const dim3 grid = two_class_grid(p, dim3(1, num_kv_heads, num_seqs), max_context_len, block_size);
     const cudaError_t e = decode_dispatch<false>(dtype, head_dim, block_size, p, grid,
                                                  static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -59,6 +59,8 @@ struct DecodeParams {
     const void* new_key;   // append: [S][Hkv][D] K/V of each sequence's newest token (position L-1), or null
     const void* new_value;
     const int32_t* seq_order;  // optional [S] permutation: CTA z works on sequence seq_order[z]; null = z
+    int class_threshold;       // > 0: grid.z = 2S, CTAs z < S take the sequences of at least this many
+                               // tokens, CTAs z >= S (sequence z - S) the shorter ones
     const float* k_scale;      // 8-bit pools: [Hkv] scales of the K and V codes
     const float* v_scale;
     const int32_t* ref_counts;  // append: [num_blocks] reference counts, or null (not checked)
@@ -206,7 +208,7 @@ struct DecodeSmem {
 // The decode kernel (SPLIT = false: one pass per (seq, kv head); true: one
 // partition of partition_blocks blocks per CTA, partials to the workspace).
 
-template <typename T, int D, int B, int NW, int STAGES, bool SPLIT, bool FP8 = false>
+template <typename T, int D, int B, int NW, int STAGES, bool SPLIT, bool FP8 = false, bool CLASSES = false>
 __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constant__ DecodeParams p) {
     using Smem = DecodeSmem<T, D, B, NW, STAGES, FP8>;
     constexpr bool kF32 = IsF32<T>::value;
@@ -225,6 +227,9 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int part = blockIdx.x, kvh = blockIdx.y;
     int s = blockIdx.z;
+    if constexpr (CLASSES) {   // the wide one-pass shape: the grid may run two classes
+        if (p.class_threshold > 0 && s >= p.num_seqs) s -= p.num_seqs;
+    }
     if (p.seq_order != nullptr) {
         // CTAs start roughly in blockIdx order, so a longest-first order
         // starts the long sequences early and leaves the short ones to fill
@@ -271,6 +276,12 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     if (L < 0 || L > p.context_cap) {
         if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
         L = L < 0 ? 0 : p.context_cap;
+    }
+    // Two classes (no copy is in flight yet): this half of the grid leaves the
+    // sequence to the other half.
+    if constexpr (CLASSES) {
+        if (p.class_threshold > 0 && (L >= p.class_threshold) != (blockIdx.z < static_cast<unsigned>(p.num_seqs)))
+            return;
     }
     const int nblk = (L + B - 1) / B;
     int b0 = 0, b1 = nblk;
