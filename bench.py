@@ -65,7 +65,7 @@ def parse_args(argv=None):
                          "block of the batch copied to / from a pinned host pool (preemption by swapping); "
                          "block_step: a decode step through the device block manager (pa_blocks_append + "
                          "pa_copy_blocks + pa_decode_append)")
-    ap.add_argument("--mode", choices=["append", "single", "splitk", "splitk2"], default="append",
+    ap.add_argument("--mode", choices=["append", "single", "splitk", "splitk2", "shared_prefix"], default="append",
                     help="append: one pa_decode_append launch per step (write + decode); the others launch "
                          "pa_reshape_and_cache then pa_decode (single) or pa_decode_splitk with fused (splitk) or "
                          "kernel (splitk2) merge")
@@ -336,8 +336,12 @@ class Step:
             self.order = None
         self.out = torch.empty_like(self.q)
         self.mcl = batch.max_context_len
-        need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
-                                                  self.part)
+        if mode == "shared_prefix":   # every row begins with the batch's shared blocks
+            need = pa.pa_decode_shared_prefix_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim,
+                                                             batch.meta["shared_blocks"], batch.block_size)
+        else:
+            need = pa.pa_decode_splitk_workspace_size(batch.num_seqs, batch.num_q_heads, batch.head_dim, self.mcl,
+                                                      self.part)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.counters = pa.Counters()
         self.kernels_per_step = {"append": 1, "splitk2": 3}.get(mode, 2)
@@ -353,9 +357,15 @@ class Step:
                 self.prepared = pa.prepare_decode_append(
                     self.out, self.q, self.nk, self.nv, self.k, self.v, self.bt, self.cl, batch.scale,
                     max_context_len=self.mcl, seq_order=self.order)
+        elif mode == "shared_prefix":
+            if self.fp8:
+                raise ValueError("the shared-prefix entry takes 16-bit pools")
+            self.prepared = pa.prepare_decode_shared_prefix(
+                self.out, self.q, self.nk, self.nv, self.k, self.v, self.bt, self.cl, batch.scale,
+                batch.meta["shared_blocks"], max_context_len=self.mcl, workspace=self.ws)
 
     def reshape(self, stream):
-        if self.mode == "append":
+        if self.mode in ("append", "shared_prefix"):
             return  # the newest token is written by the decode launch itself
         if self.fp8:
             self.pa.pa_reshape_and_cache_fp8(self.nk, self.nv, self.k, self.v, self.slots, self.ks, self.vs,
@@ -435,7 +445,7 @@ def run_gpu(args, world, rank, local):
         st = steps[i % len(steps)]
         if ev is not None:
             ev[0].record(s_)
-        if st.mode != "append":  # append: the whole step is the decode launch
+        if st.mode not in ("append", "shared_prefix"):  # there the whole step is the one entry call
             st.reshape(s_)
         if ev is not None:
             ev[1].record(s_)
@@ -490,7 +500,7 @@ def run_gpu(args, world, rank, local):
             # per-step events inside it split reshape from decode.
             region[0].record(stream)
             for i in range(args.steps):
-                one(i, events[i] if mode != "append" and graphs is None else None)
+                one(i, events[i] if mode not in ("append", "shared_prefix") and graphs is None else None)
             region[1].record(stream)
         else:
             for i in range(args.steps):
@@ -500,7 +510,7 @@ def run_gpu(args, world, rank, local):
     barrier(world)
     if flush is None:
         local_step = region[0].elapsed_time(region[1]) / args.steps
-        if mode == "append" or graphs is not None:   # one launch, or the whole step replayed as one graph
+        if mode in ("append", "shared_prefix") or graphs is not None:   # one entry call, or one graph replay
             decode_ms, reshape_ms = [local_step], [0.0]
         else:
             decode_ms = [e[1].elapsed_time(e[2]) for e in events]
@@ -674,7 +684,8 @@ def run_gpu(args, world, rank, local):
             "context_len_mean": float(batch.context_lens.float().mean()),
             "context_len_max": batch.max_context_len,
             "decode_entry": ({"splitk": "pa_decode_splitk (fused merge)", "splitk2": "pa_decode_splitk (merge kernel)",
-                              "append": "pa_decode_append"}.get(mode, "pa_decode")
+                              "append": "pa_decode_append",
+                              "shared_prefix": "pa_decode_shared_prefix (appending)"}.get(mode, "pa_decode")
                              if fp8 is None else
                              {"splitk": "pa_decode_splitk_fp8 (fused merge)",
                               "splitk2": "pa_decode_splitk_fp8 (merge kernel)",
@@ -692,6 +703,10 @@ def run_gpu(args, world, rank, local):
                                            "launch" if fp8 is not None else
                                            ": newest token of every sequence written + decode, one launch")
                      if mode == "append"
+                     else "pa_decode_shared_prefix: the shared prefix once per kv head for all sequences "
+                          "(tcgen05 pass), then each sequence's own blocks with its newest token written, "
+                          "the two merged; two launches"
+                     if mode == "shared_prefix"
                      else "pa_reshape_and_cache_fp8 (newest token of every sequence, quantised) + decode"
                      if fp8 is not None
                      else "pa_reshape_and_cache (newest token of every sequence) + decode"),
@@ -707,6 +722,7 @@ def run_gpu(args, world, rank, local):
             "bound": "hbm",
             "kernel": {"append": "pa_decode_kernel (append)", "splitk": "pa_decode_kernel<split, fused merge>",
                        "splitk2": "pa_decode_kernel<split> + pa_merge_kernel",
+                       "shared_prefix": "pa_prefill_tc_kernel<prefix> + pa_decode_kernel<suffix, append>",
                        }.get(mode, "pa_decode_kernel"),
             "achieved": round(achieved, 2),
             "peak": peak,
@@ -903,7 +919,8 @@ def config_lines(args, world, rank):
                 "append": "pa_decode_append" + ("_fp8" if fp8 is not None else ""),
                 "single": "pa_reshape_and_cache + pa_decode",
                 "splitk": f"pa_reshape_and_cache + pa_decode_splitk (fused merge, partition {part})",
-                "splitk2": f"pa_reshape_and_cache + pa_decode_splitk (merge kernel, partition {part})"}[mode],
+                "splitk2": f"pa_reshape_and_cache + pa_decode_splitk (merge kernel, partition {part})",
+                "shared_prefix": "pa_decode_shared_prefix (appending; prefix pass + own-block pass)"}[mode],
              "seqs": batch.num_seqs, "block_size": batch.block_size, "ms_per_step": round(ms, 5),
              "algorithmic_bytes": int(unique), "gb_per_s": round(gbs, 2),
              "frac_of_hbm_peak": round(gbs / world / peak, 4), "frac_of_spec_8tbs": round(gbs / world / SPEC_HBM_GBS, 4),
@@ -934,6 +951,7 @@ def config_lines(args, world, rank):
         del b
     b = workloads.prefix_sharing(seed=seed, device="cuda")
     out["prefix_sharing"] = entry(b, "append")
+    out["prefix_sharing_shared_prefix"] = entry(b, "shared_prefix")
     del b
     b = workloads.llama3_70b_long(seed=seed, device="cuda")
     out["llama3_70b_long"] = entry(b, "splitk", part=1024)

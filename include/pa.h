@@ -92,6 +92,8 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
                                      sequence that holds tokens, or a corrupt free ring */
 #define PA_DEVERR_SHARED_BLOCK 128 /* pa_decode_append: the newest token's block is held by
                                       more than one sequence; its write was skipped */
+#define PA_DEVERR_PREFIX      256 /* pa_decode_shared_prefix: a row's first prefix_blocks
+                                      entries differ from row 0's */
 
 /*
  * seq_order (pa_decode, pa_decode_append, pa_decode_splitk) — NULL, or an
@@ -357,6 +359,74 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
                      float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
                      int head_dim, int max_blocks_per_seq, int max_context_len, int max_query_len,
                      int64_t num_blocks, pa_dtype dtype, void* stream);
+
+/*
+ * pa_decode_shared_prefix_workspace_size — bytes of workspace
+ * pa_decode_shared_prefix needs at most: per (sequence, query head, partial)
+ * an fp32 partial output of head_dim values plus its running max and sum, for
+ * up to ceil(prefix_blocks * block_size / 64) key partitions of the prefix
+ * and one partial of the sequence's own blocks.
+ */
+pa_status pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int head_dim, int prefix_blocks,
+                                                 int block_size, size_t* bytes);
+
+/*
+ * pa_decode_shared_prefix — pa_decode_append (key != NULL) or pa_decode (key
+ * == value == NULL) for a batch whose sequences all start with the same
+ * prefix_blocks physical blocks: a system prompt shared by every request
+ * ([P1] §4.1, the comparison table: prefix sharing; blocks shared by
+ * reference count, [P4] §2.3).  The result is the same attention over each
+ * sequence's whole context (within the 16-bit tolerance), computed in two
+ * launches on `stream` that may run at the same time:
+ *   1. the prefix, once per kv head for every sequence's query: query rows of
+ *      all sequences against the prefix's K/V tiles on the 5th-generation
+ *      tensor cores (the prefill kernel's form with every prefix key visible),
+ *      key partitions spread over some of the SMs, unnormalised partials
+ *      (output, running max, sum) to `workspace`;
+ *   2. each sequence's own blocks [prefix_blocks, ceil(L/B)) as in pa_decode
+ *      (with the newest token written first when appending), its partial to
+ *      `workspace` too; launched as a programmatic dependent launch, so that
+ *      it fills the SMs the first pass leaves free.
+ * Each (sequence, kv head) counts its partials' arrivals in `counters`; the
+ * CTA that brings the last one, in either launch, merges them with
+ * log-sum-exp weights into `out` (no CTA waits for another).  Both launches
+ * have ended when the second has.  Each prefix K/V byte is read once per kv
+ * head instead of once per sequence.
+ *
+ *   prefix_blocks  the blocks every row of block_tables shares at positions
+ *                  [0, prefix_blocks): row 0's ids are the ones read; a row
+ *                  that differs sets PA_DEVERR_PREFIX (its output then
+ *                  attends over row 0's prefix).  1 <= prefix_blocks <=
+ *                  max_blocks_per_seq and prefix_blocks * block_size <=
+ *                  max_context_len.
+ *   context_lens   every L must cover the prefix: L >= prefix_blocks *
+ *                  block_size, and L > that when appending (the newest token
+ *                  goes to a block of the sequence's own); a sequence that
+ *                  breaks this sets PA_DEVERR_CONTEXT_LEN and gets a zero
+ *                  output row.
+ *   key, value     as in pa_decode_append, or both NULL (no append)
+ *   workspace      device scratch of at least
+ *                  pa_decode_shared_prefix_workspace_size(...) bytes, 16-byte
+ *                  aligned, clobbered; PA_ERR_WORKSPACE if too small
+ *   counters       int32 arrival counters, num_counters >= num_seqs *
+ *                  num_kv_heads, all zero before the first call, and left at
+ *                  zero by every call (as pa_decode_splitk's; one array may
+ *                  serve both entries on one stream); PA_ERR_WORKSPACE if
+ *                  NULL or too short
+ *   ref_counts     as in pa_decode_append
+ *   fp16 or bf16 only (PA_ERR_UNSUPPORTED for fp32).  Where no tensor map can
+ *   describe the K pool (see pa_prefill) the call runs pa_decode_append /
+ *   pa_decode instead, with the same result.  Other arguments as in pa_decode.
+ *   Calls that may run concurrently on the GPU need their own workspace and
+ *   counters.
+ */
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, const void* value, void* k_cache,
+                                  void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                  float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int max_blocks_per_seq, int max_context_len, int64_t num_blocks,
+                                  pa_dtype dtype, int prefix_blocks, void* workspace, size_t workspace_bytes,
+                                  int32_t* counters, int64_t num_counters, const int32_t* ref_counts,
+                                  void* stream);
 
 /*
  * pa_copy_blocks — copy whole physical blocks (every kv head, token and

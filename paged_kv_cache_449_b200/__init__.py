@@ -26,7 +26,8 @@ __all__ = ["pa_reshape_and_cache", "pa_decode", "pa_decode_append", "pa_decode_s
            "DEVERR_SEQ_ORDER", "longest_first", "pa_copy_blocks", "pa_reshape_and_cache_fp8", "pa_decode_fp8",
            "pa_decode_splitk_fp8", "fp8_pool_shape", "pa_prefill", "pa_decode_append_fp8",
            "pa_blocks_init", "pa_blocks_append", "pa_blocks_fork", "pa_blocks_release",
-           "DEVERR_NO_FREE_BLOCK", "DEVERR_REF_COUNT", "DEVERR_SHARED_BLOCK"]
+           "DEVERR_NO_FREE_BLOCK", "DEVERR_REF_COUNT", "DEVERR_SHARED_BLOCK", "DEVERR_PREFIX",
+           "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size", "prepare_decode_shared_prefix"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libpa.so")
@@ -35,7 +36,7 @@ PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 _DTYPE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
 STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE", 4: "PA_ERR_CUDA"}
 DEVERR_BLOCK_ID, DEVERR_CONTEXT_LEN, DEVERR_SLOT, DEVERR_TIMEOUT, DEVERR_SEQ_ORDER = 1, 2, 4, 8, 16
-DEVERR_NO_FREE_BLOCK, DEVERR_REF_COUNT, DEVERR_SHARED_BLOCK = 32, 64, 128
+DEVERR_NO_FREE_BLOCK, DEVERR_REF_COUNT, DEVERR_SHARED_BLOCK, DEVERR_PREFIX = 32, 64, 128, 256
 
 
 class PagedAttentionError(RuntimeError):
@@ -75,6 +76,10 @@ def load_library(path: str) -> ctypes.CDLL:
     lib.pa_decode.argtypes = decode_args + [P, P]
     lib.pa_decode_append.restype = I
     lib.pa_decode_append.argtypes = [P, P, P, P] + decode_args[2:] + [P, P, P]
+    lib.pa_decode_shared_prefix_workspace_size.restype = I
+    lib.pa_decode_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
+    lib.pa_decode_shared_prefix.restype = I
+    lib.pa_decode_shared_prefix.argtypes = [P, P, P, P] + decode_args[2:] + [I, P, SZ, P, I64, P, P]
     lib.pa_decode_splitk_workspace_size.restype = I
     lib.pa_decode_splitk_workspace_size.argtypes = [I, I, I, I, I, c.POINTER(SZ)]
     lib.pa_decode_splitk.restype = I
@@ -292,6 +297,66 @@ def prepare_decode_append(out, q, key, value, k_cache, v_cache, block_tables, co
     args = _append_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                         seq_order, ref_counts)
     return Prepared("pa_decode_append", args, dev, tensors)
+
+
+def pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, prefix_blocks, block_size) -> int:
+    lib = load()
+    size = ctypes.c_size_t(0)
+    _check(lib.pa_decode_shared_prefix_workspace_size(num_seqs, num_q_heads, head_dim, int(prefix_blocks),
+                                                      int(block_size), ctypes.byref(size)),
+           "pa_decode_shared_prefix_workspace_size")
+    return int(size.value)
+
+
+def _shared_prefix_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, prefix_blocks,
+                        max_context_len, workspace, ref_counts, counters):
+    if (key is None) != (value is None):
+        raise ValueError("key and value go together (both None: no append)")
+    S, Hq, D = q.shape
+    b = k_cache.shape[3]
+    if workspace is None:
+        need = pa_decode_shared_prefix_workspace_size(S, Hq, D, prefix_blocks, b)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    args = _decode_args(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len)
+    kp = None if key is None else _dev_ptr(key, "key")
+    vp = None if value is None else _dev_ptr(value, "value")
+    if counters is None:
+        counters = _default_counters.setdefault(q.device.index, Counters())
+    buf = counters.get(S * k_cache.shape[1], q.device) if isinstance(counters, Counters) else counters
+    return [args[0], args[1], kp, vp, *args[2:], int(prefix_blocks), _dev_ptr(workspace, "workspace"),
+            workspace.numel() * workspace.element_size(), _dev_ptr(buf, "counters"), buf.numel(),
+            _counts_ptr(ref_counts, k_cache.shape[0])], workspace, buf
+
+
+@_on_tensor_device
+def pa_decode_shared_prefix(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale, prefix_blocks,
+                            max_context_len=None, workspace=None, stream=None, ref_counts=None, counters=None):
+    """Decode (key = value = None) or decode with append (key/value [S, Hkv,
+    D]) for a batch whose rows all begin with the same prefix_blocks physical
+    blocks: the prefix is attended once per kv head for every sequence on the
+    tensor cores, each sequence's own blocks as in pa_decode, and the two
+    merged.  `workspace`: a CUDA uint8 tensor of at least
+    pa_decode_shared_prefix_workspace_size(...) bytes (allocated here if None);
+    `counters`: a Counters or a zeroed int32 tensor (a per-device default if
+    None)."""
+    lib = load()
+    args, _, _ = _shared_prefix_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale,
+                                     prefix_blocks, max_context_len, workspace, ref_counts, counters)
+    _check(lib.pa_decode_shared_prefix(*args, _stream(stream)), "pa_decode_shared_prefix")
+
+
+def prepare_decode_shared_prefix(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale,
+                                 prefix_blocks, max_context_len=None, workspace=None, ref_counts=None,
+                                 counters=None) -> Prepared:
+    """pa_decode_shared_prefix's arguments checked and marshalled once (see Prepared)."""
+    tensors = (out, q, key, value, k_cache, v_cache, block_tables, context_lens, workspace, ref_counts)
+    dev = _tensor_device(tensors + ((counters,) if isinstance(counters, torch.Tensor) else ()), {})
+    if dev is None:
+        raise ValueError("pa_decode_shared_prefix takes CUDA tensors")
+    args, workspace, buf = _shared_prefix_args(out, q, key, value, k_cache, v_cache, block_tables, context_lens,
+                                               scale, prefix_blocks, max_context_len, workspace, ref_counts,
+                                               counters)
+    return Prepared("pa_decode_shared_prefix", args, dev, tensors + (workspace, buf))
 
 
 def pa_decode_splitk_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size=512) -> int:

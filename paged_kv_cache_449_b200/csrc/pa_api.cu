@@ -60,6 +60,24 @@
 #ifndef PA_FP8_WIDE_RING
 #define PA_FP8_WIDE_RING 8192
 #endif
+// Shared-prefix decode: the decode pass overlaps the prefix pass (1), or
+// starts after it (0).  The prefix pass takes about this many CTAs (0: a
+// quarter of the SMs; the decode pass fills the rest meanwhile): on the
+// 128-sequence, 1024-token-prefix workload 32 of 148 ran 40.3 us, 16 55.5,
+// 64 41.3 and 148 51.3.
+#ifndef PA_PREFIX_OVERLAP
+#define PA_PREFIX_OVERLAP 1
+#endif
+#ifndef PA_PREFIX_CTAS
+#define PA_PREFIX_CTAS 0
+#endif
+// ... and the decode pass's wide grid starts the sequences whose own part is
+// in the upper (8 - N) / 8 of its range first (0: one class; 4 ran 40.3 us
+// there against 47.3 us for one class).
+#ifndef PA_PREFIX_CLASS_EIGHTHS
+#define PA_PREFIX_CLASS_EIGHTHS 4
+#endif
+
 #ifndef PA_TWO_CLASS
 #define PA_TWO_CLASS 1
 #endif
@@ -177,14 +195,34 @@ cudaError_t with_variant(pa_dtype dt, int D, int B, F&& f) {
     }
 }
 
-template <typename T, int D, int B, bool SPLIT, Kind K, bool FP8 = false>
+template <typename T, int D, int B, bool SPLIT, Kind K, bool FP8 = false, bool PREFIX = false>
 cudaError_t launch_decode(const pa::DecodeParams& p, dim3 grid, cudaStream_t stream) {
     using C = DecodeConfig<T, D, B, K, FP8>;
-    auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT, FP8, !SPLIT && K == Kind::kWide>;
+    auto kernel = pa::pa_decode_kernel<T, D, B, C::kWarps, C::kStages, SPLIT, FP8,
+                                       !SPLIT && (!PREFIX || PA_PREFIX_CLASS_EIGHTHS > 0) && K == Kind::kWide,
+                                       PREFIX>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
-    kernel<<<grid, C::kWarps * 32, C::Smem::kTotal, stream>>>(p);
-    return cudaGetLastError();
+    if constexpr (PREFIX) {
+        // Programmatic dependent launch: the CTAs start while the prefix pass
+        // (the launch before, on the same stream) still runs; the two grids
+        // meet only through the arrival counters, and one CTA waits for the
+        // prefix pass to complete (so that this grid ends after it).
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(C::kWarps * 32);
+        cfg.dynamicSmemBytes = C::Smem::kTotal;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = PA_PREFIX_OVERLAP;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kernel, p);
+    } else {
+        kernel<<<grid, C::kWarps * 32, C::Smem::kTotal, stream>>>(p);
+        return cudaGetLastError();
+    }
 }
 
 // Streaming multiprocessors of the current device, once per device.
@@ -203,15 +241,18 @@ int sm_count() {
 
 // The split kernel always runs wide CTAs; the one-pass kernel runs deep CTAs
 // unless its grid holds more than PA_DEEP_MAX_CTAS_PER_SM CTAs per SM.
-template <bool SPLIT, bool FP8 = false>
+template <bool SPLIT, bool FP8 = false, bool PREFIX = false>
 cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p, dim3 grid, cudaStream_t st) {
     const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
     const bool deep = !SPLIT && ctas <= static_cast<long long>(PA_DEEP_MAX_CTAS_PER_SM) * sm_count();
     return with_variant(dt, D, B, [&](auto tt, auto dd, auto bb) -> cudaError_t {
         using T = typename decltype(tt)::type;
         constexpr int kD = decltype(dd)::value, kB = decltype(bb)::value;
-        if constexpr (FP8 && pa::IsF32<T>::value) {
-            return cudaErrorInvalidValue;  // 8-bit pools take 16-bit queries (refused on the host first)
+        if constexpr ((FP8 || PREFIX) && pa::IsF32<T>::value) {
+            return cudaErrorInvalidValue;  // 16-bit only (refused on the host first)
+        } else if constexpr (PREFIX) {
+            return deep ? launch_decode<T, kD, kB, false, Kind::kDeep, false, true>(p, grid, st)
+                        : launch_decode<T, kD, kB, false, Kind::kWide, false, true>(p, grid, st);
         } else if constexpr (SPLIT) {
             return launch_decode<T, kD, kB, true, Kind::kWide, FP8>(p, grid, st);
         } else {
@@ -228,13 +269,13 @@ cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p
 // blockIdx order; a CTA of the other class leaves at once).  Not for 32-token
 // blocks: there a wide CTA holds one 16 KiB stage per warp and three fit an
 // SM, and starting the long sequences first was measured slower.
-dim3 two_class_grid(pa::DecodeParams& p, dim3 grid, int max_context_len, int block_size) {
+dim3 two_class_grid(pa::DecodeParams& p, dim3 grid, int max_context_len, int block_size, int threshold = -1) {
     const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
     const bool wide = ctas > static_cast<long long>(PA_DEEP_MAX_CTAS_PER_SM) * sm_count();
-    if (!PA_TWO_CLASS || !wide || block_size > 16 || p.seq_order != nullptr || 2LL * grid.z > 65535 ||
-        max_context_len < 4)
+    if (threshold < 0) threshold = PA_TWO_CLASS && max_context_len >= 4 ? max_context_len / 4 : 0;
+    if (threshold <= 0 || !wide || block_size > 16 || p.seq_order != nullptr || 2LL * grid.z > 65535)
         return grid;
-    p.class_threshold = max_context_len / 4;
+    p.class_threshold = threshold;
     grid.z *= 2;
     return grid;
 }
@@ -319,6 +360,12 @@ size_t splitk_bytes(long long seqs, long long heads, long long parts, long long 
     return static_cast<size_t>(seqs * heads * parts * (head_dim + 2) * 4);
 }
 
+// 64-key tiles of a shared prefix of prefix_blocks blocks: the most key
+// partitions the prefix pass can take.
+int shared_prefix_tiles(int prefix_blocks, int block_size) {
+    return static_cast<int>((static_cast<long long>(prefix_blocks) * block_size + 63) / 64);
+}
+
 // Device memory, or page-locked host memory mapped into the device's address
 // space (what the copy kernel can dereference).
 bool device_accessible(const void* p) {
@@ -376,10 +423,10 @@ bool encode_k_rows(CUtensorMap* map, const void* k_cache, pa_dtype dt, int B, in
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int D, int B>
+template <typename T, int D, int B, bool PREFIX = false>
 cudaError_t launch_prefill_tc(const pa::PrefillParams& p, const CUtensorMap& k_rows, dim3 grid, cudaStream_t st) {
     using Sm = pa::PrefillTcSmem<T, D, B>;
-    auto kernel = pa::pa_prefill_tc_kernel<T, D, B>;
+    auto kernel = pa::pa_prefill_tc_kernel<T, D, B, PREFIX>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
     kernel<<<grid, 448, Sm::kTotal, st>>>(p, k_rows);
@@ -741,6 +788,120 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
             return use_tc ? launch_prefill_tc<T, kD, kB>(p, k_rows, grid, s) : launch_prefill<T, kD, kB>(p, grid, s);
         }
     });
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int head_dim, int prefix_blocks,
+                                                 int block_size, size_t* bytes) {
+    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || prefix_blocks <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    *bytes = splitk_bytes(num_seqs, num_q_heads, shared_prefix_tiles(prefix_blocks, block_size) + 1, head_dim);
+    return PA_OK;
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, const void* value, void* k_cache,
+                                  void* v_cache, const int32_t* block_tables, const int32_t* context_lens,
+                                  float scale, int block_size, int num_seqs, int num_q_heads, int num_kv_heads,
+                                  int head_dim, int max_blocks_per_seq, int max_context_len, int64_t num_blocks,
+                                  pa_dtype dtype, int prefix_blocks, void* workspace, size_t workspace_bytes,
+                                  int32_t* counters, int64_t num_counters, const int32_t* ref_counts,
+                                  void* stream) {
+    const DecodeShape sh{block_size, num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                         max_context_len, num_blocks, static_cast<int>(dtype)};
+    pa_status st = check_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    if (st != PA_OK) return st;
+    if (dtype == PA_F32) return PA_ERR_UNSUPPORTED;  // the prefix pass runs on the tensor cores
+    if (prefix_blocks <= 0 || prefix_blocks > max_blocks_per_seq ||
+        static_cast<long long>(prefix_blocks) * block_size > max_context_len)
+        return PA_ERR_INVALID_ARG;
+    if ((key == nullptr) != (value == nullptr)) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (key && (!aligned16(key) || !aligned16(value))) return PA_ERR_INVALID_ARG;
+    if (!aligned4(ref_counts)) return PA_ERR_INVALID_ARG;
+    const int tiles = shared_prefix_tiles(prefix_blocks, block_size);
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < splitk_bytes(num_seqs, num_q_heads, tiles + 1, head_dim))
+        return PA_ERR_WORKSPACE;
+    if (!counters || !aligned4(counters) || num_counters < static_cast<int64_t>(num_seqs) * num_kv_heads)
+        return PA_ERR_WORKSPACE;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CUtensorMap k_rows{};
+    if (!PA_PREFILL_TC ||
+        !encode_k_rows(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks)) {
+        // no tensor map for the prefix pass: the plain decode gives the same result
+        pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+        p.new_key = key;
+        p.new_value = value;
+        p.ref_counts = ref_counts;
+        const dim3 grid = two_class_grid(p, dim3(1, num_kv_heads, num_seqs), max_context_len, block_size);
+        return decode_dispatch<false>(dtype, head_dim, block_size, p, grid, s) == cudaSuccess ? PA_OK
+                                                                                               : PA_ERR_CUDA;
+    }
+    // Pass 1 (tensor cores): the prefix once per kv head for all sequences,
+    // key partitions spread over the SMs, unnormalised partials to the workspace.
+    const int group = num_q_heads / num_kv_heads;
+    const int tile_tokens = 128 / group;
+    const long long row_ctas = (static_cast<long long>(num_seqs) + 2 * tile_tokens - 1) / (2 * tile_tokens);
+    const long long per_part = row_ctas * num_kv_heads;
+    long long want = (PA_PREFIX_CTAS > 0 ? PA_PREFIX_CTAS : sm_count() / 4) / per_part;
+    want = want < 1 ? 1 : (want > tiles ? tiles : want);
+    const int tiles_per = static_cast<int>((tiles + want - 1) / want);
+    const int parts = (tiles + tiles_per - 1) / tiles_per;   // every partition holds >= 1 tile (<= tiles)
+    const int slots = parts + 1;                               // + the sequence's own blocks
+    float* acc = static_cast<float*>(workspace);
+    float* ml = acc + static_cast<size_t>(num_seqs) * num_q_heads * slots * head_dim;
+    pa::PrefillParams pp{};
+    pp.out = out;
+    pp.context_lens = context_lens;
+    pp.counters = counters;
+    pp.prefix_append = key != nullptr;
+    pp.q = q;
+    pp.k_cache = k_cache;
+    pp.v_cache = v_cache;
+    pp.block_tables = block_tables;
+    pp.score_scale = scale * 1.4426950408889634f;
+    pp.num_seqs = num_seqs;
+    pp.num_q_heads = num_q_heads;
+    pp.num_kv_heads = num_kv_heads;
+    pp.group = group;
+    pp.max_blocks_per_seq = max_blocks_per_seq;
+    pp.context_cap = context_cap(sh);
+    pp.num_blocks = num_blocks;
+    pp.tile_tokens = tile_tokens;
+    pp.part_acc = acc;
+    pp.part_ml = ml;
+    pp.num_partitions = slots;
+    pp.prefix_len = prefix_blocks * block_size;
+    pp.prefix_tiles = tiles_per;
+    const dim3 pgrid(static_cast<unsigned>(row_ctas), num_kv_heads, parts);
+    cudaError_t e = with_variant(dtype, head_dim, block_size, [&](auto tt, auto dd, auto bb) -> cudaError_t {
+        using T = typename decltype(tt)::type;
+        constexpr int kD = decltype(dd)::value, kB = decltype(bb)::value;
+        if constexpr (pa::IsF32<T>::value) {
+            return cudaErrorInvalidValue;
+        } else {
+            return launch_prefill_tc<T, kD, kB, true>(pp, k_rows, pgrid, s);
+        }
+    });
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    // Pass 2: each sequence's own blocks (and newest token), the prefix
+    // partials folded into the same merge.
+    pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
+    p.new_key = key;
+    p.new_value = value;
+    p.ref_counts = ref_counts;
+    p.part_acc = acc;
+    p.part_ml = ml;
+    p.first_block = prefix_blocks;
+    p.num_partitions = slots;
+    p.counters = counters;
+    const int pre = prefix_blocks * block_size;
+    const dim3 grid = two_class_grid(p, dim3(1, num_kv_heads, num_seqs), max_context_len, block_size,
+                                     PA_PREFIX_CLASS_EIGHTHS > 0
+                                         ? pre + static_cast<int>((static_cast<long long>(max_context_len - pre) *
+                                                                   PA_PREFIX_CLASS_EIGHTHS) / 8)
+                                         : 0);
+    e = decode_dispatch<false, false, true>(dtype, head_dim, block_size, p, grid, s);
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -64,6 +64,13 @@ struct DecodeParams {
     const float* k_scale;      // 8-bit pools: [Hkv] scales of the K and V codes
     const float* v_scale;
     const int32_t* ref_counts;  // append: [num_blocks] reference counts, or null (not checked)
+    // shared-prefix form: every sequence's blocks [0, first_block) are the
+    // prefix that row 0 of block_tables holds, attended by the prefix pass;
+    // this pass attends blocks [first_block, nblk) and writes its partial to
+    // slot num_partitions - 1 of part_acc / part_ml (the prefix pass's key
+    // partitions fill the slots before it); the last of the num_partitions
+    // arrivals on counters[s * Hkv + kvh] merges them
+    int first_block;
 };
 
 // Append: the newest token of sequence s (logical position L-1) is written
@@ -208,7 +215,8 @@ struct DecodeSmem {
 // The decode kernel (SPLIT = false: one pass per (seq, kv head); true: one
 // partition of partition_blocks blocks per CTA, partials to the workspace).
 
-template <typename T, int D, int B, int NW, int STAGES, bool SPLIT, bool FP8 = false, bool CLASSES = false>
+template <typename T, int D, int B, int NW, int STAGES, bool SPLIT, bool FP8 = false, bool CLASSES = false,
+          bool PREFIX = false>
 __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constant__ DecodeParams p) {
     using Smem = DecodeSmem<T, D, B, NW, STAGES, FP8>;
     constexpr bool kF32 = IsF32<T>::value;
@@ -217,6 +225,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     using TM = typename std::conditional<FP8, __half, T>::type;
     constexpr int kTile = Smem::kTile;
     static_assert(STAGES >= 1 && STAGES <= 32, "ring depth");
+    static_assert(!(PREFIX && (SPLIT || FP8 || kF32)), "the shared-prefix form is one pass over 16-bit pools");
     static_assert((kTile % 16) == 0, "bulk copies move multiples of 16 bytes");
 
     extern __shared__ __align__(128) uint8_t smem[];
@@ -227,6 +236,15 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int part = blockIdx.x, kvh = blockIdx.y;
     int s = blockIdx.z;
+    // Shared-prefix form: this grid may start while the prefix pass still runs
+    // (the two meet only through the arrival counters).  CTA 0 waits for that
+    // pass to complete before it leaves, so that this grid, and the work after
+    // it on the stream, end after it.
+    auto prefix_pass_done = [&]() {
+        if constexpr (PREFIX) {
+            if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+        }
+    };
     if constexpr (CLASSES) {   // the wide one-pass shape: the grid may run two classes
         if (p.class_threshold > 0 && s >= p.num_seqs) s -= p.num_seqs;
     }
@@ -255,7 +273,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     // this warp's first 32 block-table entries (any entry of the row is
     // readable; entries past the context are discarded below) and, for the
     // tensor-core path, the query fragments.
-    const int b0_first = SPLIT ? part * p.partition_blocks : 0;
+    const int b0_first = SPLIT ? part * p.partition_blocks : (PREFIX ? p.first_block : 0);
     const int32_t* bt = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq + b0_first + warp;
     int first_ids = -1;
     if (b0_first + warp + lane * NW < p.max_blocks_per_seq) first_ids = __ldg(bt + lane * NW);
@@ -280,8 +298,10 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
     // Two classes (no copy is in flight yet): this half of the grid leaves the
     // sequence to the other half.
     if constexpr (CLASSES) {
-        if (p.class_threshold > 0 && (L >= p.class_threshold) != (blockIdx.z < static_cast<unsigned>(p.num_seqs)))
+        if (p.class_threshold > 0 && (L >= p.class_threshold) != (blockIdx.z < static_cast<unsigned>(p.num_seqs))) {
+            prefix_pass_done();
             return;
+        }
     }
     const int nblk = (L + B - 1) / B;
     int b0 = 0, b1 = nblk;
@@ -296,7 +316,18 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         if (b0 >= nblk) return;  // this partition is past the end of the sequence
         b1 = min(nblk, b0 + p.partition_blocks);
     }
-    if constexpr (!SPLIT) {
+    if constexpr (PREFIX) {
+        // the sequence's own part starts after the shared prefix; a context
+        // that does not reach past it (or, appending, whose newest token would
+        // land in it) is refused: no block is attended, the partial is empty
+        // and the merge writes a zero output
+        b0 = p.first_block;
+        if (shared_prefix_refused(L, b0 * B, p.new_key != nullptr)) {
+            if (threadIdx.x == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
+            b1 = b0;
+        }
+    }
+    if constexpr (!SPLIT && !PREFIX) {
         if (nblk == 0) {  // empty context: zero output
             T* out = reinterpret_cast<T*>(p.out) + (static_cast<long long>(s) * p.num_q_heads + kvh * group) * D;
             for (int i = threadIdx.x; i < group * D; i += NW * 32) out[i] = from_float<T>(0.f);
@@ -378,6 +409,14 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         if (id >= 0 && id < p.num_blocks && __ldg(p.ref_counts + id) != 1) {
             if (lane == 0) flag_error(128 /* PA_DEVERR_SHARED_BLOCK */);
             owns_last = false;  // no write; the pool is attended as it is
+        }
+    }
+    if constexpr (PREFIX) {
+        // the prefix pass read row 0's prefix: every row must hold the same ids there
+        if (kvh == 0 && s != 0) {
+            const int32_t* row = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq;
+            for (int k = threadIdx.x; k < p.first_block; k += NW * 32)
+                if (__ldg(row + k) != __ldg(p.block_tables + k)) flag_error(256 /* PA_DEVERR_PREFIX */);
         }
     }
     bool failed = false;
@@ -478,23 +517,26 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
 
     constexpr bool kLog2 = !kF32;
     // Split mode writes fp32 partials, except that with the fused merge a
-    // sequence with a single partition is finished here.
-    const int num_parts = SPLIT ? (nblk + p.partition_blocks - 1) / p.partition_blocks : 1;
-    const bool to_workspace = SPLIT && !(p.counters != nullptr && num_parts == 1);
+    // sequence with a single partition is finished here; the shared-prefix
+    // form always writes its partial, to the last slot.
+    const int num_parts = SPLIT ? (nblk + p.partition_blocks - 1) / p.partition_blocks
+                                : (PREFIX ? p.num_partitions : 1);
+    const bool to_workspace = (SPLIT && !(p.counters != nullptr && num_parts == 1)) || PREFIX;
+    const int slot_part = PREFIX ? p.num_partitions - 1 : part;
     if (any_failed) {
         // A copy timed out (PA_DEVERR_TIMEOUT is set; the outputs are then not
         // the attention result).  A partition is recorded as empty (max -inf,
         // sum 0, zero output) so that no merge reads what an earlier call left
         // in the workspace, and the fused merge below still counts it, which
         // brings the arrival counter back to zero.
-        if constexpr (!SPLIT) {
+        if constexpr (!SPLIT && !PREFIX) {
             return;
         } else {
             if (!to_workspace) return;
             for (int idx = threadIdx.x; idx < group * D; idx += NW * 32) {
                 const int r = idx / D, d = idx - r * D;
                 const long long slot =
-                    (static_cast<long long>(s) * p.num_q_heads + kvh * group + r) * p.num_partitions + part;
+                    (static_cast<long long>(s) * p.num_q_heads + kvh * group + r) * p.num_partitions + slot_part;
                 p.part_acc[slot * D + d] = 0.f;
                 if (d == 0) {
                     p.part_ml[slot * 2] = kNegInf;
@@ -528,7 +570,7 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
         num *= out_scale;  // 8-bit pools: the V scale
         const int h = kvh * group + r;
         if (to_workspace) {
-            const long long slot = (static_cast<long long>(s) * p.num_q_heads + h) * p.num_partitions + part;
+            const long long slot = (static_cast<long long>(s) * p.num_q_heads + h) * p.num_partitions + slot_part;
             p.part_acc[slot * D + d] = num;
             if (d == 0) {
                 p.part_ml[slot * 2] = M;
@@ -539,9 +581,11 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
             out[d] = from_float<T>(den > 0.f ? num / den : 0.f);
         }
     }
-    if constexpr (SPLIT) {
+    if constexpr (SPLIT || PREFIX) {
         if (p.counters != nullptr && to_workspace) {
-            // Fused merge: the CTA that records the last partition merges them.
+            // Fused merge: the CTA that records the last partition merges them
+            // (shared-prefix form: the last of the prefix pass's partitions
+            // and this pass, whichever kernel it runs in).
             __shared__ int last_arrival;
             __threadfence();
             __syncthreads();
@@ -552,11 +596,22 @@ __global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constan
             __syncthreads();
             if (last_arrival) {
                 __threadfence();
-                merge_partitions_cta<T, D, kLog2, NW * 32>(p, s, kvh, num_parts);
+                if constexpr (PREFIX) {
+                    const bool refused = shared_prefix_refused(L, p.first_block * B, p.new_key != nullptr);
+                    for (int v = threadIdx.x; v < group * D / 4; v += NW * 32) {
+                        const long long row[1] = {static_cast<long long>(s) * p.num_q_heads + kvh * group + (4 * v) / D};
+                        const int c[1] = {v % (D / 4)};
+                        const bool use[1] = {true}, zero[1] = {refused};
+                        merge_shared_prefix<T, D, 1>(p.out, p.part_acc, p.part_ml, num_parts, row, c, use, zero);
+                    }
+                } else {
+                    merge_partitions_cta<T, D, kLog2, NW * 32>(p, s, kvh, num_parts);
+                }
                 if (threadIdx.x == 0) p.counters[static_cast<long long>(s) * p.num_kv_heads + kvh] = 0;
             }
         }
     }
+    prefix_pass_done();
 }
 
 // ----------------------------------------------------------------------------

@@ -244,4 +244,78 @@ __device__ __forceinline__ float softmax_exp(float x) {
 
 constexpr float kNegInf = -INFINITY;
 
+// ---------------------------------------------------------------- shared-prefix decode
+
+// A context of L tokens cannot take the shared-prefix form when it does not
+// reach past the prefix_len shared tokens, or, appending, when its newest
+// token (position L - 1) would land in a shared block.
+__device__ __forceinline__ bool shared_prefix_refused(int L, int prefix_len, bool append) {
+    return L < prefix_len + (append ? 1 : 0);
+}
+
+// The last step of the shared-prefix decode: the np partials of a query head
+// row of (sequence, kv head) -- the prefix pass's key partitions and the
+// sequence's own blocks; unnormalised output, reference maximum (base 2) and
+// sum, [S][Hq][np][D] and [S][Hq][np][2] -- combined with log-sum-exp weights
+// 2^(m_i - max_i m_i) into four output values (16-byte chunk c of the row;
+// zero where `zero`).  U such outputs at once, four partials each step, so
+// that their loads are in flight together; the partials were written by other
+// CTAs, so they are read past L1.
+template <typename T, int D, int U>
+__device__ __forceinline__ void merge_shared_prefix(void* out, const float* part_acc, const float* part_ml, int np,
+                                                    const long long (&row)[U], const int (&c)[U],
+                                                    const bool (&use)[U], const bool (&zero)[U]) {
+    constexpr int kStep = 4;
+    float4 a[U];
+    float M[U], den[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        M[u] = kNegInf;
+        den[u] = 0.f;
+    }
+    for (int q0 = 0; q0 < np; q0 += kStep) {
+        float m[U][kStep], l[U][kStep];
+        float4 x[U][kStep];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int k = 0; k < kStep; ++k) {
+                const bool in = use[u] && q0 + k < np;
+                const long long sl = row[u] * np + q0 + k;
+                m[u][k] = in ? __ldcg(part_ml + sl * 2) : kNegInf;
+                l[u][k] = in ? __ldcg(part_ml + sl * 2 + 1) : 0.f;
+                x[u][k] = in ? __ldcg(reinterpret_cast<const float4*>(part_acc + sl * D) + c[u])
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int k = 0; k < kStep; ++k) {
+                const float mn = fmaxf(M[u], m[u][k]);
+                if (mn != kNegInf) {
+                    const float sa = exp2_approx(M[u] - mn), sb = exp2_approx(m[u][k] - mn);
+                    a[u].x = fmaf(a[u].x, sa, x[u][k].x * sb);
+                    a[u].y = fmaf(a[u].y, sa, x[u][k].y * sb);
+                    a[u].z = fmaf(a[u].z, sa, x[u][k].z * sb);
+                    a[u].w = fmaf(a[u].w, sa, x[u][k].w * sb);
+                    den[u] = fmaf(den[u], sa, l[u][k] * sb);
+                    M[u] = mn;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (!use[u]) continue;
+        const float inv = (!zero[u] && den[u] > 0.f) ? 1.f / den[u] : 0.f;
+        T* dst = reinterpret_cast<T*>(out) + row[u] * D + 4 * c[u];
+        dst[0] = from_float<T>(a[u].x * inv);
+        dst[1] = from_float<T>(a[u].y * inv);
+        dst[2] = from_float<T>(a[u].z * inv);
+        dst[3] = from_float<T>(a[u].w * inv);
+    }
+}
+
 }  // namespace pa

@@ -45,6 +45,23 @@ struct PrefillParams {
     int context_cap;
     long long num_blocks;
     int tile_tokens;                // query tokens per CTA: NW * 16 / group
+    // shared-prefix pass (the tensor-core kernel's PREFIX form): the query rows
+    // are every sequence's decode query, the keys the prefix_len tokens of the
+    // prefix that row 0 of block_tables holds, prefix_tiles 64-key tiles per
+    // CTA (key partition = blockIdx.z); unnormalised partials go to slot
+    // blockIdx.z of part_acc / part_ml ([S][Hq][num_partitions][D], [..][2]),
+    // whose last slot holds the decode pass's partial of the sequence's own
+    // blocks.  Each CTA then arrives on counters[s * Hkv + kvh] for its
+    // sequences; the last of the num_partitions arrivals merges into `out`
+    // (a zero row where context_lens[s] does not reach past the prefix, or,
+    // with prefix_append, its newest token would land in it).
+    float* part_acc;
+    float* part_ml;
+    int32_t* counters;
+    int num_partitions;
+    int prefix_len;
+    int prefix_tiles;
+    int prefix_append;
 };
 
 template <typename T, int D, int B, int NW, int STAGES>

@@ -232,7 +232,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 // Warps 0-3 and 4-7: softmax of query tile 0 and 1 (thread = row = tensor-memory
 // lane); warps 8 / 9 issue S = Q K^T and 10 / 11 O += P V for query tile 0 / 1;
 // warps 12 and 13 fetch K and V.
-template <typename T, int D, int B>
+template <typename T, int D, int B, bool PREFIX = false>
 __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
                                                                 const __grid_constant__ CUtensorMap k_rows) {
     using Sm = PrefillTcSmem<T, D, B>;
@@ -260,15 +260,33 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     volatile uint32_t* abort = misc + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kvh = blockIdx.y, s = blockIdx.z;
+    // PREFIX: the table of row 0 holds the shared prefix; blockIdx.z is the key partition
+    const int kvh = blockIdx.y, s = PREFIX ? 0 : static_cast<int>(blockIdx.z);
     const int group = p.group;
 
-    const int q0 = p.query_start[s];
-    const int Q = p.query_start[s + 1] - q0;
-    const int L = p.context_lens[s];
-    if (L < 0 || L > p.context_cap || Q < 0 || Q > L) {
-        if (tid == 0 && blockIdx.x == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
-        return;
+    int q0, Q, L, tb = 0;   // tb: the first key tile of this CTA
+    if constexpr (PREFIX) {
+        // the decode pass of the sequences' own blocks may start its CTAs now
+        // (it shares nothing with this grid but the arrival counters)
+        asm volatile("griddepcontrol.launch_dependents;");
+        // every sequence's decode query is one "token" of the chunk, and all of
+        // the prefix is visible to it
+        q0 = 0;
+        Q = p.num_seqs;
+        L = p.prefix_len;
+        tb = static_cast<int>(blockIdx.z) * p.prefix_tiles;
+        if (L <= 0 || L > p.context_cap) {   // (the host never launches such a pass)
+            if (tid == 0 && blockIdx.x == 0 && kvh == 0 && blockIdx.z == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
+            return;
+        }
+    } else {
+        q0 = p.query_start[s];
+        Q = p.query_start[s + 1] - q0;
+        L = p.context_lens[s];
+        if (L < 0 || L > p.context_cap || Q < 0 || Q > L) {
+            if (tid == 0 && blockIdx.x == 0 && kvh == 0) flag_error(2 /* PA_DEVERR_CONTEXT_LEN */);
+            return;
+        }
     }
     // query tile q covers tokens [tok0[q], tok1[q]) of the chunk; nt[q] key tiles
     int tok0[2], tok1[2], nt[2];
@@ -281,14 +299,76 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     for (int q = 0; q < 2; ++q) {
         tok0[q] = (2 * tile + q) * p.tile_tokens;
         tok1[q] = min(Q, tok0[q] + p.tile_tokens);
-        nt[q] = tok0[q] < Q ? ((L - Q + tok1[q] - 1) / B + kBlocks) / kBlocks : 0;
+        if constexpr (PREFIX) {
+            nt[q] = tok0[q] < Q ? min(p.prefix_tiles, (L + kKeys - 1) / kKeys - tb) : 0;
+        } else {
+            nt[q] = tok0[q] < Q ? ((L - Q + tok1[q] - 1) / B + kBlocks) / kBlocks : 0;
+        }
     }
-    if (nt[0] == 0) return;
+    // Shared-prefix form, the CTA's last step: its sequences [tok0[0], seq_end)
+    // arrive on their (sequence, kv head) counters once its partials are
+    // written (`empty`: empty partials written here first); the last of the
+    // num_partitions arrivals of a sequence merges its partials into `out`.
+    // The K ring holds the list of sequences this CTA merges.
+    auto prefix_finish = [&](bool empty) {
+        if constexpr (PREFIX) {
+            const int seq_end = min(Q, tok0[0] + 2 * p.tile_tokens);
+            const int rows = (seq_end - tok0[0]) * group;
+            if (empty) {
+                for (int i = tid; i < rows * (D + 2); i += 448) {
+                    const int r = i / (D + 2), e = i % (D + 2);
+                    const long long slot = (static_cast<long long>(tok0[0] + r / group) * p.num_q_heads +
+                                            kvh * group + r % group) * p.num_partitions + blockIdx.z;
+                    if (e < D) p.part_acc[slot * D + e] = 0.f;
+                    else p.part_ml[slot * 2 + (e - D)] = e == D ? kNegInf : 0.f;
+                }
+            }
+            int* merge_list = reinterpret_cast<int*>(smem + Sm::kKOff);
+            volatile uint32_t* n_merge = misc + 2;
+            if (tid == 0) *n_merge = 0u;
+            __threadfence();   // this CTA's partials before its arrivals
+            __syncthreads();
+            for (int t = tok0[0] + tid; t < seq_end; t += 448) {
+                const int old = atomicAdd(p.counters + static_cast<long long>(t) * p.num_kv_heads + kvh, 1);
+                if (old == p.num_partitions - 1) merge_list[atomicAdd(const_cast<uint32_t*>(n_merge), 1u)] = t;
+            }
+            __syncthreads();
+            const int n = static_cast<int>(*n_merge);
+            if (n > 0) {
+                __threadfence();
+                // four outputs per thread and step (sixteen loads in flight)
+                constexpr int kU = 4;
+                const int slices = group * D / 4;
+                for (int w0 = tid; w0 < n * slices; w0 += kU * 448) {
+                    long long row[kU];
+                    int c[kU];
+                    bool use[kU], zero[kU];
+#pragma unroll
+                    for (int u = 0; u < kU; ++u) {
+                        const int w = w0 + u * 448;
+                        use[u] = w < n * slices;
+                        const int t = use[u] ? merge_list[w / slices] : 0, v = w % slices;
+                        int Lt = use[u] ? p.context_lens[t] : 0;
+                        Lt = Lt < 0 ? 0 : (Lt > p.context_cap ? p.context_cap : Lt);   // as the decode pass reads it
+                        zero[u] = shared_prefix_refused(Lt, L, p.prefix_append != 0);
+                        row[u] = static_cast<long long>(t) * p.num_q_heads + kvh * group + (4 * v) / D;
+                        c[u] = v % (D / 4);
+                    }
+                    merge_shared_prefix<T, D, kU>(p.out, p.part_acc, p.part_ml, p.num_partitions, row, c, use, zero);
+                }
+                for (int i = tid; i < n; i += 448)
+                    p.counters[static_cast<long long>(merge_list[i]) * p.num_kv_heads + kvh] = 0;
+            }
+        }
+    };
+    if (nt[0] <= 0) return;   // (no sequence: tok0[0] >= Q; the host gives every key partition a tile)
     const int ntiles = max(nt[0], nt[1]);                           // key tiles fetched (>= 1)
-    const int nblk = (L - Q + (nt[1] ? tok1[1] : tok1[0]) - 1) / B + 1;   // blocks needed
+    // blocks needed (absolute: block index from the start of the table row)
+    const int nblk = PREFIX ? (L + B - 1) / B : (L - Q + (nt[1] ? tok1[1] : tok1[0]) - 1) / B + 1;
     // tensor copies land on 128-byte boundaries (the dynamic window starts on one)
     if (smem_u32(smem) & 127u) {
         if (tid == 0) flag_error(8 /* PA_DEVERR_TIMEOUT: nothing fetched */);
+        prefix_finish(true);
         return;
     }
 
@@ -327,14 +407,14 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     auto load_ids = [&](int j, int (&ids)[kBlocks]) {
 #pragma unroll
         for (int b = 0; b < kBlocks; ++b) {
-            const int jb = j * kBlocks + b;
+            const int jb = (tb + j) * kBlocks + b;
             ids[b] = (j < ntiles && jb < nblk) ? __ldg(table + jb) : -1;
         }
     };
     // The same mask computed by a whole warp: lane b loads block b's id (the
     // id of lane `lane` for tile j; -1 past the need), a ballot gathers them.
     auto lane_id = [&](int j) -> int {
-        const int jb = j * kBlocks + lane;
+        const int jb = (tb + j) * kBlocks + lane;
         return (lane < kBlocks && j < ntiles && jb < nblk) ? __ldg(table + jb) : -1;
     };
     auto ok_ballot = [&](int id) -> uint32_t {
@@ -365,7 +445,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
         if (!v_side) {
 #pragma unroll
             for (int b = 0; b < kBlocks; ++b)
-                if (j * kBlocks + b < nblk && !((ok >> b) & 1u)) flag_error(1 /* PA_DEVERR_BLOCK_ID */);
+                if ((tb + j) * kBlocks + b < nblk && !((ok >> b) & 1u)) flag_error(1 /* PA_DEVERR_BLOCK_ID */);
             if (ok == 0u) {
                 mbar_arrive_expect_tx(&full[st], 0);   // nothing to fetch: every key is masked
             } else {
@@ -528,16 +608,18 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             id_n = lane_id(j + 1);
             const int vst = j % VS;
             if (!__all_sync(0xffffffffu, tc_wait(&v_full[vst], (j / VS) & 1, abort))) break;
-            const int lb = (L - 1) / B - j * kBlocks;
-            if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
-                uint8_t* vt = smem + Sm::kVOff + vst * Sm::kStage + lb * kTile;
-                const int t_from = (L - 1) % B + 1;
-                for (int i = lane; i < (B - t_from) * (D / 8); i += 32) {
-                    const int t = t_from + i / (D / 8), c = i % (D / 8);
-                    *reinterpret_cast<uint4*>(vt + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
+            if constexpr (!PREFIX) {   // (a shared prefix ends on a block boundary: no tail)
+                const int lb = (L - 1) / B - j * kBlocks;
+                if (lb >= 0 && lb < kBlocks && ((ok >> lb) & 1u)) {
+                    uint8_t* vt = smem + Sm::kVOff + vst * Sm::kStage + lb * kTile;
+                    const int t_from = (L - 1) % B + 1;
+                    for (int i = lane; i < (B - t_from) * (D / 8); i += 32) {
+                        const int t = t_from + i / (D / 8), c = i % (D / 8);
+                        *reinterpret_cast<uint4*>(vt + (c * B + t) * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
             }
             if (j < nt[q]) {
                 const uint32_t vbase = v_ring + vst * Sm::kStage;
@@ -577,7 +659,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     } else if (softmax_warp) {
         // ---------------- softmax of query tile qt (thread = row = tensor-memory lane)
         const float scale = p.score_scale;
-        const int row_pos = row_ok ? L - Q + row_tok : -1;
+        const int row_pos = row_ok ? (PREFIX ? INT_MAX : L - Q + row_tok) : -1;
         const uint32_t all_blocks = (1u << kBlocks) - 1u;
         const int n = my_nt;
         uint64_t* sfull = &s_full[qt];
@@ -600,7 +682,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sfree);
-            const int key0 = j * kKeys;
+            const int key0 = (tb + j) * kKeys;
             // row maximum over eight independent partial maxima (no 64-long chain)
             float m8[8];
             if (ok == all_blocks && key0 + kKeys - 1 <= row_pos) {
@@ -686,7 +768,54 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
         // ---- the last O += P V, then this row of the output
         if (!failed && !__all_sync(0xffffffffu, tc_wait(&p_free[qt * 2 + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort)))
             failed = true;
-        if (!failed && !*abort) {
+        if constexpr (PREFIX) {
+            // this key partition's unnormalised partial of the row: O, the
+            // running reference (base 2) and the sum, in the split-K layout;
+            // an empty partial if the pass failed (the error flag is set).
+            // O leaves through shared memory, 32 columns at a time, so that
+            // each store of the warp writes four whole 128-byte row segments:
+            // the warp's 4 KiB slice of its query tile's Q area (no MMA reads
+            // Q any more), 16-byte chunk c of row r at chunk c ^ (r % 8)
+            // (conflict-free both ways).
+            const bool good = __all_sync(0xffffffffu, !failed && !*abort);   // warp-uniform: ld32 is collective
+            const long long slot =
+                (static_cast<long long>(row_ok ? row_tok : 0) * p.num_q_heads + row_head) * p.num_partitions +
+                blockIdx.z;
+            if (good) tc::fence_after();
+            float* stage = reinterpret_cast<float*>(smem + Sm::kQOff + (qt & 1) * Sm::kQ + (warp & 3) * 4096);
+            static_assert(4 * 4096 <= Sm::kQ, "four warps' staging slices fit one query tile's Q area");
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float v[32];
+                if (good) {
+                    tc::ld32(o_tmem + lane_base + c0, v);   // collective per warp: every row takes part
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4*>(stage + lane * 32 + ((c ^ (lane & 7)) * 4)) =
+                        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = 4 * i + (lane >> 3), c = lane & 7;   // row of the warp, chunk
+                    const int trow = (warp & 3) * 32 + rr;               // row of the query tile
+                    const int tok = my_tok0 + trow / group;
+                    if (tok < my_tok1) {
+                        const long long rs = (static_cast<long long>(tok) * p.num_q_heads + kvh * group + trow % group) *
+                                                 p.num_partitions + blockIdx.z;
+                        *reinterpret_cast<float4*>(p.part_acc + rs * D + c0 + 4 * c) =
+                            *reinterpret_cast<const float4*>(stage + rr * 32 + ((c ^ (rr & 7)) * 4));
+                    }
+                }
+                __syncwarp();
+            }
+            if (row_ok)
+                *reinterpret_cast<float2*>(p.part_ml + slot * 2) =
+                    good ? make_float2(m_run, l_run) : make_float2(kNegInf, 0.f);
+        } else if (!failed && !*abort) {
             tc::fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             T* dst = reinterpret_cast<T*>(p.out) +
@@ -713,6 +842,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     if (warp == 8) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
+    prefix_finish(false);
 }
 
 }  // namespace pa

@@ -45,7 +45,8 @@ def test_header_declares_the_boundary():
         "pa_decode_splitk_fp8", "pa_decode_splitk_workspace_size", "pa_reshape_and_cache_fp8", "pa_prefill",
         "pa_decode_splitk_static", "pa_get_device_error",
         "pa_reshape_and_cache", "pa_status_string",
-        "pa_blocks_init", "pa_blocks_append", "pa_blocks_fork", "pa_blocks_release"])
+        "pa_blocks_init", "pa_blocks_append", "pa_blocks_fork", "pa_blocks_release",
+        "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -121,6 +122,23 @@ def test_host_validation_rejects_before_launch(lib):
     assert lib.pa_decode_splitk(*args, 512, 16, 1 << 20, None, 0, 6, None) == 1      # misaligned seq_order
     assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], None, 2, None) == 1      # misaligned seq_order
     assert lib.pa_decode_append(16, 16, 16, 16, *args[2:], 6, None, None) == 1      # misaligned ref_counts
+    # shared prefix: S 4, Hq 4, D 64, prefix 3 blocks of 16 (one 64-key tile + the own-block partial):
+    # 4*4*2*66*4 bytes of workspace; counters for S * Hkv = 16 (sequence, kv head) pairs
+    sp = [16, 16, 16, 16, 16, 16, 16, 16, 0.125, 16, 4, 4, 4, 64, 7, 100, 64, 1]
+    ws = 4 * 4 * 2 * 66 * 4
+    size = ctypes.c_size_t(0)
+    assert lib.pa_decode_shared_prefix_workspace_size(4, 4, 64, 3, 16, ctypes.byref(size)) == 0 and size.value == ws
+    cn = [16, 16]
+    assert lib.pa_decode_shared_prefix(*sp[:17], 0, 3, 16, ws, *cn, None, None) == 2          # fp32
+    assert lib.pa_decode_shared_prefix(*sp, 0, 16, ws, *cn, None, None) == 1                  # no prefix
+    assert lib.pa_decode_shared_prefix(*sp, 8, 16, ws, *cn, None, None) == 1                  # more than a row holds
+    assert lib.pa_decode_shared_prefix(*sp[:3], None, *sp[4:], 3, 16, ws, *cn, None, None) == 1   # key, no value
+    assert lib.pa_decode_shared_prefix(*sp, 3, 16, ws - 1, *cn, None, None) == 3              # workspace too small
+    assert lib.pa_decode_shared_prefix(*sp, 3, 24, ws, *cn, None, None) == 3                  # misaligned workspace
+    assert lib.pa_decode_shared_prefix(*sp, 3, 16, ws, None, 16, None, None) == 3             # no counters
+    assert lib.pa_decode_shared_prefix(*sp, 3, 16, ws, 16, 15, None, None) == 3               # too few counters
+    assert lib.pa_decode_shared_prefix(*sp, 3, 16, ws, 18, 16, None, None) == 3               # misaligned counters
+    assert lib.pa_decode_shared_prefix(*sp, 3, 16, ws, *cn, 6, None) == 1                     # misaligned ref_counts
     cp = [16, 16, 16, 16, 16, 4, 8, 128, 16, 10, 10, 2, None]
     assert lib.pa_copy_blocks(*cp[:5], 0, *cp[6:]) == 0                             # no pairs: a no-op
     assert lib.pa_copy_blocks(*cp[:5], -1, *cp[6:]) == 1                            # negative count
@@ -213,7 +231,7 @@ TENSOR_ENTRIES = {
     "pa_reshape_and_cache": 5, "pa_decode": 6, "pa_decode_append": 8, "pa_decode_splitk": 6,
     "pa_decode_splitk_static": 6, "pa_copy_blocks": 5, "pa_reshape_and_cache_fp8": 7, "pa_decode_fp8": 8,
     "pa_decode_append_fp8": 10, "pa_decode_splitk_fp8": 8, "pa_prefill": 7, "pa_blocks_init": 3,
-    "pa_blocks_append": 7, "pa_blocks_fork": 4, "pa_blocks_release": 6,
+    "pa_blocks_append": 7, "pa_blocks_fork": 4, "pa_blocks_release": 6, "pa_decode_shared_prefix": 8,
 }
 
 
@@ -221,7 +239,8 @@ def test_every_tensor_entry_checks_the_device():
     """Each tensor entry point runs under the device guard (a helper may not
     take its place) and refuses tensors on two devices before any marshalling."""
     public = {n for n in dir(pa) if n.startswith("pa_") and callable(getattr(pa, n))}
-    takes_tensors = public - {"pa_status_string", "pa_get_device_error", "pa_decode_splitk_workspace_size"}
+    takes_tensors = public - {"pa_status_string", "pa_get_device_error", "pa_decode_splitk_workspace_size",
+                              "pa_decode_shared_prefix_workspace_size"}
     assert takes_tensors == set(TENSOR_ENTRIES)
     a, b = _FakeCudaTensor.make(0), _FakeCudaTensor.make(1)
     for name, n in TENSOR_ENTRIES.items():
@@ -233,5 +252,9 @@ def test_every_tensor_entry_checks_the_device():
     for fn, n in ((pa.prepare_decode_append, 8), (pa.prepare_decode_append_fp8, 10)):
         with pytest.raises(ValueError, match="one CUDA device"):
             fn(*([a] * (n - 1) + [b]), 0.125)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.prepare_decode_shared_prefix(*([a] * 7 + [b]), 0.125, 4)
     with pytest.raises(ValueError, match="CUDA tensors"):
         pa.prepare_decode_append(*([torch.zeros(2)] * 8), 0.125)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        pa.prepare_decode_shared_prefix(*([torch.zeros(2)] * 8), 0.125, 4)

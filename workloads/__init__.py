@@ -289,7 +289,8 @@ def continuous_batching_mix(seed=0, device="cpu", block_size=16, num_seqs=256,
 
 
 def prefix_sharing(seed=0, device="cpu", prefix_len=1024, num_seqs=128, block_size=16,
-                   materialize_shared=False, suffix_range=(16, 512)) -> Batch:
+                   materialize_shared=False, suffix_range=(16, 512), dtype=torch.float16, num_q_heads=32,
+                   num_kv_heads=8, head_dim=128, suffix_lens=None) -> Batch:
     """Prefix sharing, fp16: 128 seqs, 32 q / 8 kv heads, D 128, B 16.  Every
     sequence references the same physical blocks for the full blocks of a
     shared `prefix_len`-token prefix (ref count = num_seqs), then a private
@@ -299,10 +300,16 @@ def prefix_sharing(seed=0, device="cpu", prefix_len=1024, num_seqs=128, block_si
 
     materialize_shared=True gives the "copied" twin: every shared block is
     duplicated per sequence instead of referenced, with identical contents, so
-    the logical K/V of every sequence are unchanged."""
+    the logical K/V of every sequence are unchanged.  Test cases may change the
+    element type, the heads and head dim, and give the suffix lengths
+    (`suffix_lens`, one per sequence, 0 allowed) instead of drawing them."""
     rng = np.random.default_rng(seed)
     B = block_size
-    suffix = rng.integers(suffix_range[0], suffix_range[1], size=num_seqs, endpoint=True)
+    if suffix_lens is None:
+        suffix = rng.integers(suffix_range[0], suffix_range[1], size=num_seqs, endpoint=True)
+    else:
+        suffix = np.asarray(suffix_lens, dtype=np.int64)
+        assert suffix.shape == (num_seqs,) and (suffix >= 0).all()
     lens = prefix_len + suffix
     n_full = prefix_len // B
     partial = prefix_len % B != 0
@@ -334,9 +341,10 @@ def prefix_sharing(seed=0, device="cpu", prefix_len=1024, num_seqs=128, block_si
         if partial:
             copies.append((int(priv[0]), original_partial))  # copy-on-write of the partial block
     slots = _decode_slots(tables, lens, B)
-    batch = make_batch(f"prefix_sharing_f16_p{prefix_len}", dtype=torch.float16, lens=lens,
-                       num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=B, num_blocks=N,
-                       tables=tables, slots=slots, seed=seed, device=device)
+    tag = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}[dtype]
+    batch = make_batch(f"prefix_sharing_{tag}_p{prefix_len}", dtype=dtype, lens=lens,
+                       num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B,
+                       num_blocks=N, tables=tables, slots=slots, seed=seed, device=device)
     if copies:
         dst = torch.tensor([d for d, _ in copies], device=batch.k_cache.device)
         src = torch.tensor([s for _, s in copies], device=batch.k_cache.device)
