@@ -143,17 +143,21 @@ def make_workload(name, seed, device, block_size=None):
 # in profiles/).  Keyed by a hash of the kernel sources: once the kernels change,
 # the figure no longer describes them and the bench reports null.
 NCU_TRAFFIC = {
-    "cb15f3334e169811": {
-        ("llama3_8b_decode_bf16", "append"): 292.759e6 + 3.156e6,
-        ("continuous_batching_mix_bf16_B16", "append"): 211.585e6 + 3.571e6,
-        ("llama3_70b_long_bf16", "splitk"): 2.519793e9 + 7.696e6,
-        ("llama3_8b_decode_bf16+e4m3", "append"): 146.832e6 + 3.234e6,
-        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260257e9 + 6.559e6,
+    "cae7ba79f3e870f8": {
+        ("llama3_8b_decode_bf16", "append"): 292.749e6 + 3.424e6,
+        ("continuous_batching_mix_bf16_B16", "append"): 211.576e6 + 3.460e6,
+        ("llama3_70b_long_bf16", "splitk"): 2.519697e9 + 7.579e6,
+        ("llama3_8b_decode_bf16+e4m3", "append"): 146.826e6 + 3.642e6,
+        ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260303e9 + 6.832e6,
     },
-    "1991b0ddd748a96e": {
-        ("chunked_prefill_bfloat16", "prefill"): 118.549e6 + 19.821e6,
-        ("chunked_prefill_bfloat16_B8", "prefill"): 118.422e6 + 19.991e6,
-        ("chunked_prefill_bfloat16_B32", "prefill"): 118.735e6 + 20.112e6,
+    "632e49eccce723ec": {
+        ("chunked_prefill_bfloat16", "prefill"): 118.548e6 + 20.276e6,
+        ("chunked_prefill_bfloat16_B8", "prefill"): 118.411e6 + 20.018e6,
+        ("chunked_prefill_bfloat16_B32", "prefill"): 118.817e6 + 21.134e6,
+    },
+    # the shared-prefix step: its prefix pass plus its decode pass
+    "b5869933e1f2a1b9": {
+        ("prefix_sharing_f16_p1024", "shared_prefix"): 5.318e6 + 0.0 + 151.184e6 + 0.072e6,
     },
 }
 
@@ -162,6 +166,12 @@ NCU_TRAFFIC = {
 # lives in pa_api.cu)
 DECODE_SOURCES = ("pa_api.cu", "pa_decode.cuh", "pa_e4m3.cuh", "pa_warp.cuh", "pa_device.cuh", "pa_reshape.cuh")
 PREFILL_SOURCES = ("pa_api.cu", "pa_prefill_tc.cuh", "pa_prefill.cuh", "pa_device.cuh")
+# the shared-prefix step runs both kernels
+SHARED_PREFIX_SOURCES = tuple(sorted(set(DECODE_SOURCES + PREFILL_SOURCES)))
+
+
+def sources_of(mode):
+    return SHARED_PREFIX_SOURCES if mode == "shared_prefix" else DECODE_SOURCES
 
 
 def code_of(text):
@@ -733,7 +743,7 @@ def run_gpu(args, world, rank, local):
             "algorithmic_bytes_per_launch": int(roof_bytes),
             "bytes_basis": ("unique: shared-prefix blocks counted once" if roof_bytes != decode_bytes
                             else "logical = unique"),
-            "traffic": NCU_TRAFFIC.get(kernel_source_hash(), {}).get(
+            "traffic": NCU_TRAFFIC.get(kernel_source_hash(sources_of(mode)), {}).get(
                 (batch.name + ("+e4m3" if fp8 is not None else ""), mode)),
         },
         "gpu_launches": int(step.kernels_per_step * args.steps),
@@ -933,7 +943,7 @@ def config_lines(args, world, rank):
             e["note"] = note
         if longest_first:
             e["seq_order"] = "longest first (built on the host from the lengths, uploaded with the step's inputs)"
-        traffic = NCU_TRAFFIC.get(kernel_source_hash(), {}).get(
+        traffic = NCU_TRAFFIC.get(kernel_source_hash(sources_of(mode)), {}).get(
             (batch.name + ("+e4m3" if fp8 is not None else ""), mode))
         if traffic is not None and not longest_first:
             e["traffic"] = traffic   # DRAM read + write bytes of the decode launch (profiles/)
