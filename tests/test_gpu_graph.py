@@ -116,3 +116,44 @@ def test_graph_replay_fp8():
                                        b.num_kv_heads)
     check_tolerance(as_f64(outs[1]), ref, b.dtype)
     del g
+
+
+def test_graph_replay_shared_prefix():
+    """The shared-prefix step -- two launches, the second a programmatic
+    dependent launch that meets the first through arrival counters -- captured
+    and replayed: bit-identical to the eager call (outputs and pools), also
+    after new queries are written in place, and the oracle's attention."""
+    b = workloads.prefix_sharing(seed=33, device="cuda", num_seqs=24, prefix_len=256)
+    eager, graphed = _copies(b, 2)
+    P = b.meta["shared_blocks"]
+    need = pa.pa_decode_shared_prefix_workspace_size(b.num_seqs, b.num_q_heads, b.head_dim, P, b.block_size)
+    ws = [torch.empty(need, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    counters = [torch.zeros(b.num_seqs * b.num_kv_heads, dtype=torch.int32, device="cuda") for _ in range(2)]
+
+    def step(d, i):
+        pa.pa_decode_shared_prefix(d["out"], d["q"], d["nk"], d["nv"], d["k_cache"], d["v_cache"], d["block_tables"],
+                                   d["context_lens"], b.scale, P, max_context_len=b.max_context_len,
+                                   workspace=ws[i], counters=counters[i])
+
+    pa.pa_get_device_error()
+    step(graphed, 1)                   # the uncaptured first call
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(graphed, 1)
+    for round_ in range(2):
+        if round_ == 1:
+            newq = torch.randn(eager["q"].shape, generator=torch.Generator(device="cuda").manual_seed(6),
+                               device="cuda").to(eager["q"].dtype)
+            eager["q"].copy_(newq)
+            graphed["q"].copy_(newq)
+        step(eager, 0)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(_bits(graphed["out"]), _bits(eager["out"])), round_
+        assert torch.equal(_bits(graphed["k_cache"]), _bits(eager["k_cache"]))
+        assert torch.equal(_bits(graphed["v_cache"]), _bits(eager["v_cache"]))
+        check_tolerance(as_f64(graphed["out"]), _oracle_step(b, graphed["q"]), b.dtype)
+    assert int(counters[0].abs().sum()) == 0 and int(counters[1].abs().sum()) == 0   # left at zero
+    assert pa.pa_get_device_error() == 0
+    del g
