@@ -62,9 +62,9 @@
 #endif
 // Shared-prefix decode: the decode pass overlaps the prefix pass (1), or
 // starts after it (0).  The prefix pass takes about this many CTAs (0: a
-// quarter of the SMs; the decode pass fills the rest meanwhile): on the
-// 128-sequence, 1024-token-prefix workload 32 of 148 ran 40.3 us, 16 55.5,
-// 64 41.3 and 148 51.3.
+// third of the SMs; the decode pass fills the rest meanwhile): on the
+// 128-sequence, 1024-token-prefix workload 48 of 148 (3 key partitions) ran
+// 38.2 us, 32 39.4, 16 55.5, 64 41.3 and 148 51.3.
 #ifndef PA_PREFIX_OVERLAP
 #define PA_PREFIX_OVERLAP 1
 #endif
@@ -843,7 +843,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, con
     const int tile_tokens = 128 / group;
     const long long row_ctas = (static_cast<long long>(num_seqs) + 2 * tile_tokens - 1) / (2 * tile_tokens);
     const long long per_part = row_ctas * num_kv_heads;
-    long long want = (PA_PREFIX_CTAS > 0 ? PA_PREFIX_CTAS : sm_count() / 4) / per_part;
+    long long want = (PA_PREFIX_CTAS > 0 ? PA_PREFIX_CTAS : sm_count() / 3) / per_part;
     want = want < 1 ? 1 : (want > tiles ? tiles : want);
     const int tiles_per = static_cast<int>((tiles + want - 1) / want);
     const int parts = (tiles + tiles_per - 1) / tiles_per;   // every partition holds >= 1 tile (<= tiles)

@@ -215,9 +215,16 @@ struct DecodeSmem {
 // The decode kernel (SPLIT = false: one pass per (seq, kv head); true: one
 // partition of partition_blocks blocks per CTA, partials to the workspace).
 
+// The shared-prefix form's wide CTAs are held to registers that let five
+// share an SM (112 registers, four per SM, otherwise: 38.2 against 39.1 us on
+// the prefix-sharing workload).
+#ifndef PA_PREFIX_MIN_CTAS
+#define PA_PREFIX_MIN_CTAS 5
+#endif
 template <typename T, int D, int B, int NW, int STAGES, bool SPLIT, bool FP8 = false, bool CLASSES = false,
           bool PREFIX = false>
-__global__ void __launch_bounds__(NW * 32) pa_decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(NW * 32, (PREFIX && NW <= 4) ? PA_PREFIX_MIN_CTAS : 1)
+    pa_decode_kernel(const __grid_constant__ DecodeParams p) {
     using Smem = DecodeSmem<T, D, B, NW, STAGES, FP8>;
     constexpr bool kF32 = IsF32<T>::value;
     static_assert(!(FP8 && kF32), "8-bit pools take 16-bit queries");

@@ -81,6 +81,8 @@ SMALL = [
     (torch.float16, 128, 16, 4, 2, 1, 9, (1, 33)),          # a one-block prefix
     (torch.bfloat16, 64, 16, 8, 4, 64, 130, (1, 200)),      # 16 tiles of keys
     (torch.float16, 128, 8, 32, 8, 13, 33, (1, 70)),        # 8-token blocks, 104-key prefix
+    (torch.bfloat16, 128, 16, 8, 2, 128, 3, (1, 50)),       # few sequences, long prefix: 16 key partitions
+    (torch.float16, 64, 32, 4, 2, 40, 5, (1, 100)),         # 20 key partitions of one tile each
 ]
 
 
