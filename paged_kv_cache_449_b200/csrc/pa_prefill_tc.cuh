@@ -336,8 +336,8 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             const int n = static_cast<int>(*n_merge);
             if (n > 0) {
                 __threadfence();
-                // four outputs per thread and step (sixteen loads in flight)
-                constexpr int kU = 4;
+                // two outputs per thread and step (eight loads in flight)
+                constexpr int kU = 2;
                 const int slices = group * D / 4;
                 for (int w0 = tid; w0 < n * slices; w0 += kU * 448) {
                     long long row[kU];
