@@ -348,11 +348,12 @@ pa_status pa_decode_splitk_fp8(void* out, const void* q, const void* k_cache, co
  *   ids outside [0, num_blocks) set PA_DEVERR_BLOCK_ID, are never read, and
  *   their keys are left out of the softmax.
  *   Every block size runs on the 5th-generation tensor cores (tcgen05, fp32
- *   accumulation in tensor memory); the K pool is then read through a tensor
- *   map built per call, which needs the CUDA driver and at most 2^31 - 1 rows
- *   of (block, kv head, 8 dims).  A pool beyond that runs warp-level mma.sync
- *   (fp32 accumulation).  The result is the same attention either way, within
- *   the 16-bit tolerance.
+ *   accumulation in tensor memory).  With blocks of 16 or 32 tokens the K pool
+ *   is read through a tensor map built per call, which needs the CUDA driver
+ *   and at most 2^31 - 1 rows of (block, kv head, 8 dims); a pool beyond that
+ *   runs warp-level mma.sync (fp32 accumulation).  8-token blocks need no
+ *   tensor map.  The result is the same attention either way, within the
+ *   16-bit tolerance.
  */
 pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                      const int32_t* block_tables, const int32_t* context_lens, const int32_t* query_start,
@@ -414,9 +415,10 @@ pa_status pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, 
  *                  serve both entries on one stream); PA_ERR_WORKSPACE if
  *                  NULL or too short
  *   ref_counts     as in pa_decode_append
- *   fp16 or bf16 only (PA_ERR_UNSUPPORTED for fp32).  Where no tensor map can
- *   describe the K pool (see pa_prefill) the call runs pa_decode_append /
- *   pa_decode instead, with the same result.  Other arguments as in pa_decode.
+ *   fp16 or bf16 only (PA_ERR_UNSUPPORTED for fp32).  Where the prefix pass
+ *   would need a tensor map of the K pool that cannot be built (see
+ *   pa_prefill) the call runs pa_decode_append / pa_decode instead, with the
+ *   same result.  Other arguments as in pa_decode.
  *   Calls that may run concurrently on the GPU need their own workspace and
  *   counters.
  */

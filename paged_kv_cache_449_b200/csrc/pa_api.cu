@@ -423,6 +423,13 @@ bool encode_k_rows(CUtensorMap* map, const void* k_cache, pa_dtype dt, int B, in
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The tensor-core kernel's K operand: blocks of 8 tokens are bulk-copied
+// whole and need no tensor map; larger blocks are gathered through one.
+bool prefill_k_source(CUtensorMap* map, const void* k_cache, pa_dtype dt, int B, int D, int Hkv,
+                      long long num_blocks) {
+    return B == 8 || encode_k_rows(map, k_cache, dt, B, D, Hkv, num_blocks);
+}
+
 template <typename T, int D, int B, bool PREFIX = false>
 cudaError_t launch_prefill_tc(const pa::PrefillParams& p, const CUtensorMap& k_rows, dim3 grid, cudaStream_t st) {
     using Sm = pa::PrefillTcSmem<T, D, B>;
@@ -771,7 +778,7 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     p.num_blocks = num_blocks;
     CUtensorMap k_rows{};
     const bool use_tc = PA_PREFILL_TC &&
-                        encode_k_rows(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks);
+                        prefill_k_source(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks);
     p.tile_tokens = (use_tc ? 128 : kPrefillWarps * 16) / p.group;
     // the tensor-core kernel takes two query tiles per CTA
     const long long per_cta = use_tc ? 2LL * p.tile_tokens : p.tile_tokens;
@@ -827,7 +834,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, con
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     CUtensorMap k_rows{};
     if (!PA_PREFILL_TC ||
-        !encode_k_rows(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks)) {
+        !prefill_k_source(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks)) {
         // no tensor map for the prefix pass: the plain decode gives the same result
         pa::DecodeParams p = make_params(out, q, k_cache, v_cache, block_tables, context_lens, scale, sh);
         p.new_key = key;

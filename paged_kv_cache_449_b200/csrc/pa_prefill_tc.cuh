@@ -6,13 +6,17 @@
 //    tiles).  A query tile is 128 MMA rows, (query token, head of the GQA
 //    group) pairs, 128 / g tokens; in a softmax warpgroup thread t owns row t,
 //    which is tensor-memory lane t.  The two tiles share every K/V tile.
-//  * Key tiles of 64 keys (8, 4 or 2 pool blocks of 8, 16 or 32 tokens).  K
-//    arrives chunk-major, [D/8][64][8], by tile::gather4 loads (one 8-dim chunk
-//    of four pool blocks per load, two chunks of two blocks for 32-token
-//    blocks), so S = Q K^T is one N = 64 MMA per 16-dim step; V arrives as
-//    whole (block, head) tiles [D/8][B][8] by 1-D bulk copies, the MN-major B
-//    operand of O += P V as stored (with 8-token blocks one 16-key step reads
-//    two adjacent tiles).  K and V have three-stage rings of their own.
+//  * Key tiles of 64 keys (8, 4 or 2 pool blocks of 8, 16 or 32 tokens), so
+//    that S = Q K^T is one N = 64 MMA per 16-dim step.  With 16- and 32-token
+//    blocks K arrives chunk-major, [D/8][64][8], by tile::gather4 loads (one
+//    8-dim chunk of four pool blocks per load, two chunks of two blocks for
+//    32-token blocks); an 8-token block's (block, head) tile [D/8][8][8] is
+//    already one column of the operand's core matrices, so those tiles arrive
+//    whole by 1-D bulk copies and the MMA steps from block to block with a
+//    stride of one tile.  V arrives as whole (block, head) tiles [D/8][B][8]
+//    by 1-D bulk copies, the MN-major B operand of O += P V as stored (with
+//    8-token blocks one 16-key step reads two adjacent tiles).  K and V have
+//    three-stage rings of their own.
 //  * Warp roles: 0-3 and 4-7 softmax of query tile 0 and 1; 8 and 9 issue
 //    S = Q K^T for query tile 0 and 1 (Q and K in shared memory); 10 and 11
 //    issue O += P V for query tile 0 and 1 (P in tensor memory, V in shared
@@ -446,7 +450,20 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
 #pragma unroll
             for (int b = 0; b < kBlocks; ++b)
                 if ((tb + j) * kBlocks + b < nblk && !((ok >> b) & 1u)) flag_error(1 /* PA_DEVERR_BLOCK_ID */);
-            if (ok == 0u) {
+            if constexpr (B == 8) {
+                // 8-token blocks: a (block, head) tile, [D/8][8][8], is already a
+                // column of core matrices of the S MMA's K-major operand, so the
+                // stage holds whole tiles (block-major) by 1-D bulk copies and the
+                // MMA steps over blocks with a stride of one tile.  A refused or
+                // unneeded block is not fetched: its scores are masked.
+                mbar_arrive_expect_tx(&full[st], __popc(ok) * kTile);
+#pragma unroll
+                for (int b = 0; b < kBlocks; ++b) {
+                    if (!((ok >> b) & 1u)) continue;
+                    const long long off = (static_cast<long long>(ids[b]) * p.num_kv_heads + kvh) * kTile;
+                    tc::bulk_copy(dst + b * kTile, reinterpret_cast<const char*>(p.k_cache) + off, kTile, &full[st]);
+                }
+            } else if (ok == 0u) {
                 mbar_arrive_expect_tx(&full[st], 0);   // nothing to fetch: every key is masked
             } else {
                 // refused ids and blocks past the need read a fetched block instead
@@ -587,7 +604,9 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
 #pragma unroll
                         for (int kc = 0; kc < D / 16; ++kc)
                             tc::mma(qb, tc::smem_desc(qs + 2 * kc * 2048, 2048, 128),
-                                    tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128), idesc_s, kc > 0);
+                                    B == 8 ? tc::smem_desc(kbase + 2 * kc * 128, 128, kTile)    // block-major
+                                           : tc::smem_desc(kbase + 2 * kc * 1024, 1024, 128),  // chunk-major
+                                    idesc_s, kc > 0);
                     }
                     tc::commit(&s_full[q]);
                 }

@@ -48,6 +48,7 @@ CASES = [
     (torch.bfloat16, 64, 32, 8, 4, (60, 200), (60, 200)),
     (torch.bfloat16, 128, 32, 16, 4, (100, 300), (20, 200)),
     (torch.float16, 128, 32, 32, 8, (64, 64), (64, 64)),
+    (torch.float16, 64, 8, 8, 2, (30, 150), (5, 100)),
 ]
 
 
