@@ -103,8 +103,8 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
  * first, then seq_order[1], ...; a host scheduler that knows the context
  * lengths passes them longest first, so long sequences do not start last and
  * hold up the end of the launch.  Without it, a one-pass launch of many small
- * thread blocks (more than four per SM, blocks of 8 or 16 tokens) starts the
- * sequences of at least max_context_len / 4 tokens before the others.  The
+ * thread blocks (more than four per SM) starts the sequences of at least
+ * max_context_len / 4 tokens before the others.  The
  * results are bit-identical for every order.  An entry outside [0, num_seqs) sets PA_DEVERR_SEQ_ORDER and the
  * thread blocks it names do nothing; a repeated entry is the caller's error
  * (the sequences it leaves out are then not computed).

@@ -110,6 +110,14 @@ struct KindTuning<Kind::kWide, true> {
 };
 
 
+// 16-bit pools of 32-token blocks take wide CTAs of this many warps (one 16
+// KiB stage each): on the continuous-batching mix two warps per CTA with the
+// long sequences started first ran 40.1 us, four warps 41.7 us (and 43.2 with
+// the long sequences first), three 41.2, one 54.4.
+#ifndef PA_WIDE32_WARPS
+#define PA_WIDE32_WARPS 2
+#endif
+
 // FP8: the pools hold 1-byte e4m3 codes, so a stage is half the size of a
 // 16-bit one and the same ring bytes hold twice the stages.
 template <typename T, int D, int B, Kind K, bool FP8 = false>
@@ -118,7 +126,9 @@ struct DecodeConfig {
     static constexpr int kStageBytes = 2 * B * D * kElem;                       // K + V tile
     static constexpr int kRingCap = KindTuning<K, FP8>::kRingCap;                    // ring bytes per CTA at most
     static constexpr int kMaxWarps = kRingCap / kStageBytes;
-    static constexpr int kWarps = KindTuning<K, FP8>::kWarps < kMaxWarps ? KindTuning<K, FP8>::kWarps : kMaxWarps;
+    static constexpr int kWarpsWanted =
+        (K == Kind::kWide && !FP8 && B == 32 && sizeof(T) == 2) ? PA_WIDE32_WARPS : KindTuning<K, FP8>::kWarps;
+    static constexpr int kWarps = kWarpsWanted < kMaxWarps ? kWarpsWanted : kMaxWarps;
     static constexpr int kRaw = KindTuning<K, FP8>::kRing / kStageBytes;
     static constexpr int kFit = kRingCap / (kWarps * kStageBytes);
     static constexpr int kStages0 = kRaw < 1 ? 1 : (kRaw > 16 ? 16 : kRaw);
@@ -266,14 +276,12 @@ cudaError_t decode_dispatch(pa_dtype dt, int D, int B, const pa::DecodeParams& p
 // order from the host starts the long sequences first by running the grid
 // twice over: the first half takes the sequences of at least a quarter of
 // max_context_len tokens, the second half the others (CTAs start roughly in
-// blockIdx order; a CTA of the other class leaves at once).  Not for 32-token
-// blocks: there a wide CTA holds one 16 KiB stage per warp and three fit an
-// SM, and starting the long sequences first was measured slower.
+// blockIdx order; a CTA of the other class leaves at once).
 dim3 two_class_grid(pa::DecodeParams& p, dim3 grid, int max_context_len, int block_size, int threshold = -1) {
     const long long ctas = static_cast<long long>(grid.x) * grid.y * grid.z;
     const bool wide = ctas > static_cast<long long>(PA_DEEP_MAX_CTAS_PER_SM) * sm_count();
     if (threshold < 0) threshold = PA_TWO_CLASS && max_context_len >= 4 ? max_context_len / 4 : 0;
-    if (threshold <= 0 || !wide || block_size > 16 || p.seq_order != nullptr || 2LL * grid.z > 65535)
+    if (threshold <= 0 || !wide || p.seq_order != nullptr || 2LL * grid.z > 65535)
         return grid;
     p.class_threshold = threshold;
     grid.z *= 2;

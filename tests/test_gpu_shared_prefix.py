@@ -197,3 +197,30 @@ def test_host_side_refusals():
     assert e.value.status == 1
     with pytest.raises(ValueError):
         pa.pa_decode_shared_prefix(out, dev["q"], b.new_key.cuda(), None, *args[4:], 4)
+
+
+def test_a_shared_newest_block_is_not_written(orc):
+    """With reference counts given, a sequence whose newest token's block is
+    also another sequence's (a table that skipped copy-on-write) is not
+    written and sets DEVERR_SHARED_BLOCK, as with pa_decode_append; the other
+    sequences are written and attended as usual."""
+    b = _batch(4700, torch.bfloat16, 128, 16, 8, 2, 4, [5, 5, 20])
+    bt = b.block_tables.clone()
+    bt[1, 4] = bt[0, 4]                       # sequence 1's own block aliases sequence 0's
+    counts = torch.zeros(b.num_blocks, dtype=torch.int32)
+    for s in range(b.num_seqs):
+        for j in range((int(b.context_lens[s]) + 15) // 16):
+            counts[int(bt[s, j])] += 1
+    c = b.__class__(**{**b.__dict__, "block_tables": bt})
+    dev = _dev(c)
+    k0 = dev["k_cache"].clone()
+    pa.pa_get_device_error()
+    got = _shared_prefix(c, dev, True, ref_counts=counts.cuda())
+    assert pa.pa_get_device_error() & pa.DEVERR_SHARED_BLOCK
+    shared = int(bt[0, 4])
+    assert torch.equal(dev["k_cache"][shared], k0[shared])        # the shared block is untouched
+    kc, vc = b.k_cache.cpu().clone(), b.v_cache.cpu().clone()
+    slots = torch.tensor([-1, -1, int(b.slot_mapping[2])], dtype=torch.int64)
+    orc.reshape_and_cache(b.new_key.cpu(), b.new_value.cpu(), kc, vc, slots, 16)
+    ref = orc.decode(b.q.cpu(), kc, vc, bt, b.context_lens, b.scale, 16, b.num_kv_heads)
+    check_tolerance(as_f64(got), ref, b.dtype)      # 0 and 1 attend over the pool as it was
