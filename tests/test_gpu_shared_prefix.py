@@ -83,6 +83,8 @@ SMALL = [
     (torch.float16, 128, 8, 32, 8, 13, 33, (1, 70)),        # 8-token blocks, 104-key prefix
     (torch.bfloat16, 128, 16, 8, 2, 128, 3, (1, 50)),       # few sequences, long prefix: 16 key partitions
     (torch.float16, 64, 32, 4, 2, 40, 5, (1, 100)),         # 20 key partitions of one tile each
+    (torch.bfloat16, 128, 16, 8, 1, 7, 1, (1, 30)),         # one sequence, one kv head
+    (torch.float16, 128, 16, 8, 8, 3, 700, (1, 20)),        # group 1: three row CTAs, 188 rows in the last tile
 ]
 
 
