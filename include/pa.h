@@ -413,7 +413,9 @@ pa_status pa_decode_shared_prefix_workspace_size(int num_seqs, int num_q_heads, 
  *                  num_kv_heads, all zero before the first call, and left at
  *                  zero by every call (as pa_decode_splitk's; one array may
  *                  serve both entries on one stream); PA_ERR_WORKSPACE if
- *                  NULL or too short
+ *                  NULL or too short.  A call that returns PA_ERR_CUDA may
+ *                  have launched the first pass only: zero the counters again
+ *                  before the next call.
  *   ref_counts     as in pa_decode_append
  *   fp16 or bf16 only (PA_ERR_UNSUPPORTED for fp32).  Where the prefix pass
  *   would need a tensor map of the K pool that cannot be built (see
