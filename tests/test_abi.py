@@ -49,6 +49,37 @@ def test_header_declares_the_boundary():
         "pa_decode_shared_prefix", "pa_decode_shared_prefix_workspace_size"])
 
 
+def declared_signatures():
+    """(name, return type, [parameter declarations]) of every entry point in
+    include/pa.h, comments stripped."""
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "pa.h")).read(), flags=re.S)
+    out = []
+    for m in re.finditer(r"^\s*((?:const\s+)?\w+\s*\*?)\s*(pa_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M):
+        params = [" ".join(x.split()) for x in m.group(3).split(",") if x.strip() and x.strip() != "void"]
+        out.append((m.group(2), " ".join(m.group(1).split()), params))
+    return out
+
+
+def test_binding_argument_types_match_the_header(lib):
+    """Every ctypes declaration of the binding has the header's arity, a
+    pointer where the header has one and the same scalar type elsewhere, so
+    the binding cannot drift from the C ABI."""
+    c = ctypes
+    scalar = {"int": c.c_int, "int64_t": c.c_int64, "float": c.c_float, "size_t": c.c_size_t,
+              "pa_dtype": c.c_int, "pa_status": c.c_int}
+    sigs = declared_signatures()
+    assert sorted(n for n, _, _ in sigs) == declared_functions()
+    for name, ret, params in sigs:
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None and len(fn.argtypes) == len(params), name
+        for decl, ct in zip(params, fn.argtypes):
+            if "*" in decl:
+                assert ct is c.c_void_p or issubclass(ct, c._Pointer), (name, decl, ct)
+            else:
+                assert ct is scalar[decl.rsplit(" ", 1)[0].replace("const ", "")], (name, decl, ct)
+        assert fn.restype is (c.c_char_p if ret == "const char*" else c.c_int), name
+
+
 def test_library_exports_every_declared_symbol(lib):
     have = exported(pa.library_path())
     for name in declared_functions():
