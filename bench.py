@@ -900,7 +900,9 @@ def block_manager_step(seed, steps, warmup, world, peak):
             "frac_of_hbm_peak": round(gbs / world / peak, 4),
             "hbm_peak": f"{peak} GB/s, {measured_peaks()[1]} copy bandwidth",
             "kernel_ms": {k_: (round(v_, 5) if isinstance(v_, float) else v_) for k_, v_ in per_kernel.items()},
-            "kernel_ms_how": "torch.profiler CUDA activity records of one step after the timed ones",
+            "kernel_ms_how": ("torch.profiler CUDA activity records of one step after the timed ones; a "
+                              "kernel's grid may be resident before the launch ahead of it ends (it waits "
+                              "for that launch first), so a record can include that wait"),
             "gpu_launches": 3 * steps,
             "bytes_basis": ("K/V at the mean context length over the timed steps (each step appends a token to "
                             "every sequence) + q, out, the new rows, block-table entries and lengths"),
@@ -972,7 +974,9 @@ def config_lines(args, world, rank):
                                     ("pa_reshape_kernel", "pa_decode_kernel", "pa_merge_kernel"))
     two["kernel_ms"] = {k: (round(v, 5) if isinstance(v, float) else v) for k, v in per_kernel.items()}
     two["kernel_ms_how"] = ("torch.profiler CUDA activity records over min(steps, 20) steps on one input copy "
-                            "(L2 not flushed between them)")
+                            "(L2 not flushed between them); a kernel's grid may be resident before the launch "
+                            "ahead of it ends (it waits for that launch first), so a record can include that "
+                            "wait: the step time is the figure to compare")
     out["llama3_70b_long_two_kernel"] = two
     del b, st
     b = workloads.llama3_8b_decode(seed=seed, device="cuda")

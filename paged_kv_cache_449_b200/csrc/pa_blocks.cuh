@@ -66,6 +66,7 @@ __device__ __forceinline__ V cta_exclusive_scan(V x, V* total, V* sh) {
 // ---------------------------------------------------------------- init
 
 __global__ void __launch_bounds__(256) pa_blocks_init_kernel(const __grid_constant__ BlockState st) {
+    wait_for_prior_work();
     for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < st.num_blocks;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         st.free_ids[i] = static_cast<int32_t>(i);
@@ -128,6 +129,7 @@ constexpr int kRingWindow = 2048;
 // Launched with blockDim.x = a multiple of 32 up to kBlocksThreads (the
 // batch rounded up: a small batch syncs few warps).
 __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_append_kernel(const __grid_constant__ AppendParams p) {
+    wait_for_prior_work();
     __shared__ long long sh[33];
     __shared__ int shx[kBlocksThreads];
     __shared__ int32_t window[kRingWindow];
@@ -337,6 +339,7 @@ struct ForkParams {
 };
 
 __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_fork_kernel(const __grid_constant__ ForkParams p) {
+    wait_for_prior_work();
     __shared__ int parent_sh, child_sh, len_sh, nb_sh;
     const int tid = threadIdx.x;
     for (int k = 0; k < p.num_forks; ++k) {
@@ -392,6 +395,7 @@ struct ReleaseParams {
 };
 
 __global__ void __launch_bounds__(kBlocksThreads) pa_blocks_release_kernel(const __grid_constant__ ReleaseParams p) {
+    wait_for_prior_work();
     __shared__ long long sh[33];
     __shared__ int s_sh, nb_sh;
     const int tid = threadIdx.x;

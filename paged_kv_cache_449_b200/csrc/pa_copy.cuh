@@ -32,6 +32,7 @@ constexpr int kCopyUnroll = 4;
 constexpr int kChunkVecs = kCopyThreads * kCopyUnroll;  // 16 KiB
 
 __global__ void __launch_bounds__(kCopyThreads) pa_copy_blocks_kernel(const __grid_constant__ CopyParams p) {
+    wait_for_prior_work();
     const long long unit = blockIdx.x;
     const int chunk = static_cast<int>(unit % p.chunks);
     const long long rest = unit / p.chunks;

@@ -243,6 +243,8 @@ __global__ void __launch_bounds__(NW * 32, (PREFIX && NW <= 4) ? PA_PREFIX_MIN_C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int part = blockIdx.x, kvh = blockIdx.y;
     int s = blockIdx.z;
+    // (the shared-prefix form overlaps the prefix pass instead: see below)
+    if constexpr (!PREFIX) wait_for_prior_work();
     // Shared-prefix form: this grid may start while the prefix pass still runs
     // (the two meet only through the arrival counters).  CTA 0 waits for that
     // pass to complete before it leaves, so that this grid, and the work after
@@ -639,6 +641,7 @@ struct MergeParams {
 
 template <typename T, int D, bool LOG2>
 __global__ void __launch_bounds__(128) pa_merge_kernel(const __grid_constant__ MergeParams p) {
+    wait_for_prior_work();
     constexpr int kPer = D / 32;
     const int lane = threadIdx.x & 31;
     const long long gw = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);

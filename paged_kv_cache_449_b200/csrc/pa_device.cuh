@@ -212,6 +212,16 @@ struct Mma<__half> {
     }
 };
 
+// Every kernel is a programmatic dependent launch: its grid may become resident
+// before the work ahead of it on the stream has ended, so a kernel reads and
+// writes nothing before that work has completed (and its writes are visible),
+// and then lets the launch after it become resident early in turn.  Only the
+// launch latency is hidden; the order of the work is the stream's.
+__device__ __forceinline__ void wait_for_prior_work() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
 // ---------------------------------------------------------------- numerics
 
 // 2^x by the hardware approximation (MUFU); 2^-inf = +0.

@@ -74,6 +74,7 @@ struct PrefillSmem {
 
 template <typename T, int D, int B, int NW, int STAGES>
 __global__ void __launch_bounds__(NW * 32) pa_prefill_kernel(const __grid_constant__ PrefillParams p) {
+    wait_for_prior_work();
     using Smem = PrefillSmem<T, D, B, NW, STAGES>;
     constexpr int kTile = Smem::kTile;
     constexpr int kNt = B / 8;          // 8-token n-tiles per block

@@ -264,15 +264,15 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     volatile uint32_t* abort = misc + 1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    wait_for_prior_work();   // (the shared-prefix form's decode pass may then start: it overlaps this grid)
     // PREFIX: the table of row 0 holds the shared prefix; blockIdx.z is the key partition
     const int kvh = blockIdx.y, s = PREFIX ? 0 : static_cast<int>(blockIdx.z);
     const int group = p.group;
 
     int q0, Q, L, tb = 0;   // tb: the first key tile of this CTA
     if constexpr (PREFIX) {
-        // the decode pass of the sequences' own blocks may start its CTAs now
-        // (it shares nothing with this grid but the arrival counters)
-        asm volatile("griddepcontrol.launch_dependents;");
+        // (the decode pass of the sequences' own blocks shares nothing with
+        // this grid but the arrival counters)
         // every sequence's decode query is one "token" of the chunk, and all of
         // the prefix is visible to it
         q0 = 0;

@@ -27,6 +27,7 @@ struct ReshapeParams {
 };
 
 __global__ void __launch_bounds__(256) pa_reshape_kernel(const __grid_constant__ ReshapeParams p) {
+    wait_for_prior_work();
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const long long per_token = static_cast<long long>(p.num_kv_heads) * p.vecs_per_row;
     if (idx >= p.num_tokens * per_token) return;
@@ -70,6 +71,7 @@ struct ReshapeE4m3Params {
 
 template <typename T>
 __global__ void __launch_bounds__(256) pa_reshape_e4m3_kernel(const __grid_constant__ ReshapeE4m3Params p) {
+    wait_for_prior_work();
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int words = p.head_dim / 4;   // four words per 16-dim vector
     const long long per_token = static_cast<long long>(p.num_kv_heads) * words;
