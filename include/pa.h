@@ -23,7 +23,11 @@
  *   keeps no state except one device-side error word per GPU (see
  *   pa_get_device_error).  All calls are asynchronous on `stream` (a
  *   cudaStream_t passed as void*; NULL = the legacy default stream) and return
- *   once the work is enqueued.
+ *   once the work is enqueued.  Every kernel is launched as a programmatic
+ *   dependent launch: its thread blocks may take their places on the SMs
+ *   while the work ahead of it on the stream still runs, but each first waits
+ *   for that work to complete, so the stream's order and memory visibility
+ *   are those of ordinary launches.
  * Alignment.  q, out, key, value, both pools and the workspace must be
  *   16-byte aligned; slot_mapping 8-byte, block_tables and context_lens
  *   4-byte aligned.
