@@ -35,8 +35,10 @@
 //    (block-table read, first copies) and final merge overlap other CTAs'
 //    streaming; best for grids of many short CTAs (split-K partitions,
 //    batches of short sequences).
+// (12 warps: with the launches made early, the Llama-3-8B step 48.0 -> 46.9
+// us against 8 warps; 10 and 11 warps lie between)
 #ifndef PA_DEEP_WARPS
-#define PA_DEEP_WARPS 8
+#define PA_DEEP_WARPS 12
 #endif
 #ifndef PA_DEEP_RING
 #define PA_DEEP_RING 16384
