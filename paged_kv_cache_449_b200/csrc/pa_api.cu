@@ -454,13 +454,27 @@ bool prefill_k_source(CUtensorMap* map, const void* k_cache, pa_dtype dt, int B,
     return B == 8 || encode_k_rows(map, k_cache, dt, B, D, Hkv, num_blocks);
 }
 
+// Query tiles (of 128 MMA rows) per tensor-core prefill CTA: 2 (one CTA per
+// SM, the two tiles sharing every K/V tile) or 1 (two CTAs per SM, each with
+// its own K/V stream).  On the chunked-prefill workload one tile per CTA ran
+// 197.4 against 208.6 us at 32-token blocks, but 228.0 against 221.1 at 16 and
+// 273.2 against 236.6 at 8 (twice the copies per SM), and the shared-prefix
+// step 44.3 against 36.1 us; so 32-token blocks take one (PA_PF_QT32).
+#ifndef PA_PF_QT32
+#define PA_PF_QT32 1
+#endif
+constexpr int prefill_tiles_per_cta(int block_size, bool prefix) {
+    return (block_size == 32 && !prefix) ? PA_PF_QT32 : 2;
+}
+
 template <typename T, int D, int B, bool PREFIX = false>
 cudaError_t launch_prefill_tc(const pa::PrefillParams& p, const CUtensorMap& k_rows, dim3 grid, cudaStream_t st) {
-    using Sm = pa::PrefillTcSmem<T, D, B>;
-    auto kernel = pa::pa_prefill_tc_kernel<T, D, B, PREFIX>;
+    constexpr int kQT = prefill_tiles_per_cta(B, PREFIX);
+    using Sm = pa::PrefillTcSmem<T, D, B, kQT>;
+    auto kernel = pa::pa_prefill_tc_kernel<T, D, B, PREFIX, kQT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
-    return launch_early(kernel, grid, dim3(448), Sm::kTotal, st, PA_EARLY_LAUNCH, p, k_rows);
+    return launch_early(kernel, grid, dim3((6 * kQT + 2) * 32), Sm::kTotal, st, PA_EARLY_LAUNCH, p, k_rows);
 }
 
 template <typename T, int D, int B>
@@ -808,8 +822,9 @@ pa_status pa_prefill(void* out, const void* q, const void* k_cache, const void* 
     const bool use_tc = PA_PREFILL_TC &&
                         prefill_k_source(&k_rows, k_cache, dtype, block_size, head_dim, num_kv_heads, num_blocks);
     p.tile_tokens = (use_tc ? 128 : kPrefillWarps * 16) / p.group;
-    // the tensor-core kernel takes two query tiles per CTA
-    const long long per_cta = use_tc ? 2LL * p.tile_tokens : p.tile_tokens;
+    // the tensor-core kernel takes one or two query tiles per CTA
+    const long long per_cta =
+        use_tc ? static_cast<long long>(prefill_tiles_per_cta(block_size, false)) * p.tile_tokens : p.tile_tokens;
     const long long tiles = (static_cast<long long>(max_query_len) + per_cta - 1) / per_cta;
     if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
     const dim3 grid(static_cast<unsigned>(tiles), num_kv_heads, num_seqs);
@@ -876,7 +891,8 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, const void* key, con
     // key partitions spread over the SMs, unnormalised partials to the workspace.
     const int group = num_q_heads / num_kv_heads;
     const int tile_tokens = 128 / group;
-    const long long row_ctas = (static_cast<long long>(num_seqs) + 2 * tile_tokens - 1) / (2 * tile_tokens);
+    const int qt = prefill_tiles_per_cta(block_size, true);
+    const long long row_ctas = (static_cast<long long>(num_seqs) + qt * tile_tokens - 1) / (qt * tile_tokens);
     const long long per_part = row_ctas * num_kv_heads;
     long long want = (PA_PREFIX_CTAS > 0 ? PA_PREFIX_CTAS : sm_count() / 3) / per_part;
     want = want < 1 ? 1 : (want > tiles ? tiles : want);

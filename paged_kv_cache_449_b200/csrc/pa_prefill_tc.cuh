@@ -3,9 +3,10 @@
 // causal attention of each sequence's newest Q tokens over its paged context).
 //
 //  * One CTA (448 threads, one per SM) per (sequence, kv head, pair of query
-//    tiles).  A query tile is 128 MMA rows, (query token, head of the GQA
-//    group) pairs, 128 / g tokens; in a softmax warpgroup thread t owns row t,
-//    which is tensor-memory lane t.  The two tiles share every K/V tile.
+//    tiles), or with QT = 1 two CTAs per SM (256 threads) of one query tile
+//    each.  A query tile is 128 MMA rows, (query token, head of the GQA group)
+//    pairs, 128 / g tokens; in a softmax warpgroup thread t owns row t, which
+//    is tensor-memory lane t.  The tiles of a CTA share every K/V tile.
 //  * Key tiles of 64 keys (8, 4 or 2 pool blocks of 8, 16 or 32 tokens), so
 //    that S = Q K^T is one N = 64 MMA per 16-dim step.  With 16- and 32-token
 //    blocks K arrives chunk-major, [D/8][64][8], by tile::gather4 loads (one
@@ -195,7 +196,7 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 // holds the tile chunk-major, [D/8][64 keys][8], gathered from the pool's
 // (block, head) tiles by tile::gather4 loads (one 8-dim chunk of four blocks
 // per load), so that one N = 64 MMA covers all of the tile's keys.
-template <typename T, int D, int B>
+template <typename T, int D, int B, int QT = 2>
 struct PrefillTcSmem {
     static constexpr int kKeys = 64;
     static constexpr int kBlocks = kKeys / B;             // blocks per key tile
@@ -204,16 +205,17 @@ struct PrefillTcSmem {
 #ifndef PA_PF_STAGES
 #define PA_PF_STAGES 3
 #endif
-    static constexpr int kKStages = D == 128 ? PA_PF_STAGES : PA_PF_STAGES + 2;
+    // (one query tile per CTA: two CTAs share an SM, so two stages each)
+    static constexpr int kKStages = QT == 2 ? (D == 128 ? PA_PF_STAGES : PA_PF_STAGES + 2) : (D == 128 ? 2 : 4);
     static constexpr int kVStages = kKStages;
     static constexpr int kQ = 128 * D * 2;                // one query tile, core-matrix layout
     static constexpr int kKOff = 0;
     static constexpr int kVOff = kKStages * kStage;
     static constexpr int kQOff = kVOff + kVStages * kStage;   // [query tile]
-    static constexpr int kBarOff = kQOff + 2 * kQ;
+    static constexpr int kBarOff = kQOff + QT * kQ;
     static constexpr int kMiscOff = kBarOff + 48 * 8;     // tmem base, abort
     static constexpr int kTotal = kMiscOff + 16;
-    static_assert(kTotal <= 232448, "shared memory per CTA");
+    static_assert(kTotal <= (QT == 2 ? 232448 : 115712), "shared memory per CTA");
     static_assert(kKStages <= 6, "barrier slots");
 };
 
@@ -235,16 +237,20 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 
 // Warps 0-3 and 4-7: softmax of query tile 0 and 1 (thread = row = tensor-memory
 // lane); warps 8 / 9 issue S = Q K^T and 10 / 11 O += P V for query tile 0 / 1;
-// warps 12 and 13 fetch K and V.
-template <typename T, int D, int B, bool PREFIX = false>
-__global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
+// warps 12 and 13 fetch K and V (QT = 1: warps 0-3, 4, 5, 6 and 7).
+template <typename T, int D, int B, bool PREFIX = false, int QT = 2>
+__global__ void __launch_bounds__((6 * QT + 2) * 32, QT == 2 ? 1 : 2) pa_prefill_tc_kernel(const __grid_constant__ PrefillParams p,
                                                                 const __grid_constant__ CUtensorMap k_rows) {
-    using Sm = PrefillTcSmem<T, D, B>;
+    using Sm = PrefillTcSmem<T, D, B, QT>;
     constexpr int kKeys = Sm::kKeys, kBlocks = Sm::kBlocks, kTile = Sm::kTile;
     constexpr int KS = Sm::kKStages, VS = Sm::kVStages;
     // tensor memory, per query tile q (256 columns at q * 256): S [0, 64),
     // O [64, 64 + D), P (16-bit pairs per column, two buffers of 32 columns)
-    constexpr uint32_t kTmemCols = 512;
+    constexpr uint32_t kTmemCols = QT * 256;
+    // warp roles: softmax [0, 4 QT), S issuers [4 QT, 5 QT), O += P V issuers
+    // [5 QT, 6 QT), K producer 6 QT, V producer 6 QT + 1
+    constexpr int kThreads = (6 * QT + 2) * 32;
+    constexpr int kSoftWarps = 4 * QT, kSIss = 4 * QT, kPVIss = 5 * QT, kProdK = 6 * QT, kProdV = 6 * QT + 1;
     constexpr uint32_t kOCol = kKeys, kPCol = kKeys + D;
     static_assert(kPCol + kKeys <= 256, "tensor memory budget");
     static_assert(B == 8 || B == 16 || B == 32, "8-, 16- or 32-token blocks");
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     const int tile = PA_PF_HEAVY_FIRST ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-        tok0[q] = (2 * tile + q) * p.tile_tokens;
+        tok0[q] = q < QT ? (QT * tile + q) * p.tile_tokens : Q;
         tok1[q] = min(Q, tok0[q] + p.tile_tokens);
         if constexpr (PREFIX) {
             nt[q] = tok0[q] < Q ? min(p.prefix_tiles, (L + kKeys - 1) / kKeys - tb) : 0;
@@ -316,10 +322,10 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     // The K ring holds the list of sequences this CTA merges.
     auto prefix_finish = [&](bool empty) {
         if constexpr (PREFIX) {
-            const int seq_end = min(Q, tok0[0] + 2 * p.tile_tokens);
+            const int seq_end = min(Q, tok0[0] + QT * p.tile_tokens);
             const int rows = (seq_end - tok0[0]) * group;
             if (empty) {
-                for (int i = tid; i < rows * (D + 2); i += 448) {
+                for (int i = tid; i < rows * (D + 2); i += kThreads) {
                     const int r = i / (D + 2), e = i % (D + 2);
                     const long long slot = (static_cast<long long>(tok0[0] + r / group) * p.num_q_heads +
                                             kvh * group + r % group) * p.num_partitions + blockIdx.z;
@@ -332,7 +338,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             if (tid == 0) *n_merge = 0u;
             __threadfence();   // this CTA's partials before its arrivals
             __syncthreads();
-            for (int t = tok0[0] + tid; t < seq_end; t += 448) {
+            for (int t = tok0[0] + tid; t < seq_end; t += kThreads) {
                 const int old = atomicAdd(p.counters + static_cast<long long>(t) * p.num_kv_heads + kvh, 1);
                 if (old == p.num_partitions - 1) merge_list[atomicAdd(const_cast<uint32_t*>(n_merge), 1u)] = t;
             }
@@ -343,13 +349,13 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
                 // two outputs per thread and step (eight loads in flight)
                 constexpr int kU = 2;
                 const int slices = group * D / 4;
-                for (int w0 = tid; w0 < n * slices; w0 += kU * 448) {
+                for (int w0 = tid; w0 < n * slices; w0 += kU * kThreads) {
                     long long row[kU];
                     int c[kU];
                     bool use[kU], zero[kU];
 #pragma unroll
                     for (int u = 0; u < kU; ++u) {
-                        const int w = w0 + u * 448;
+                        const int w = w0 + u * kThreads;
                         use[u] = w < n * slices;
                         const int t = use[u] ? merge_list[w / slices] : 0, v = w % slices;
                         int Lt = use[u] ? p.context_lens[t] : 0;
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
                     }
                     merge_shared_prefix<T, D, kU>(p.out, p.part_acc, p.part_ml, p.num_partitions, row, c, use, zero);
                 }
-                for (int i = tid; i < n; i += 448)
+                for (int i = tid; i < n; i += kThreads)
                     p.counters[static_cast<long long>(merge_list[i]) * p.num_kv_heads + kvh] = 0;
             }
         }
@@ -376,14 +382,14 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
         return;
     }
 
-    if (tid == 256) {
+    if (tid == kSIss * 32) {
         for (int i = 0; i < KS; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 2);
+            mbar_init(&k_empty[i], QT);
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 2);
+            mbar_init(&v_empty[i], QT);
         }
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < QT; ++q) {
             mbar_init(&s_full[q], 1);
             mbar_init(&s_free[q], 4);
             for (int b = 0; b < 2; ++b) {
@@ -391,11 +397,11 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
                 mbar_init(&p_free[q * 2 + b], 1);
             }
         }
-        for (int d = 0; d < 4; ++d) mbar_init(&drain[d], 1);
+        for (int d = 0; d < 2 * QT; ++d) mbar_init(&drain[d], 1);
         *abort = 0u;
         fence_barrier_init();
     }
-    if (warp == 8) {
+    if (warp == kSIss) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -433,8 +439,8 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     };
 
     // ---- producers: warp 12 lane 0 fetches K tiles, warp 13 lane 0 V tiles
-    const bool is_producer = (warp == 12 || warp == 13) && lane == 0;
-    const bool v_side = warp == 13;
+    const bool is_producer = (warp == kProdK || warp == kProdV) && lane == 0;
+    const bool v_side = warp == kProdV;
     const char* vpool = reinterpret_cast<const char*>(p.v_cache);
     uint64_t* full = v_side ? v_full : k_full;
     uint64_t* empty = v_side ? v_empty : k_empty;
@@ -536,10 +542,10 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     const int my_tok1 = qt == 1 ? tok1[1] : tok1[0];
     const int my_nt = qt == 1 ? nt[1] : nt[0];
     const int row = tid & 127;
-    const bool softmax_warp = warp < 8 && my_nt > 0;
+    const bool softmax_warp = warp < kSoftWarps && my_nt > 0;
     const int row_tok = my_tok0 + row / group;
     const int row_head = kvh * group + row % group;
-    const bool row_ok = warp < 8 && row_tok < my_tok1;
+    const bool row_ok = warp < kSoftWarps && row_tok < my_tok1;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t qbase = tmem + static_cast<uint32_t>(qt & 1) * 256u;
     const uint32_t s_tmem = qbase, o_tmem = qbase + kOCol, p_tmem = qbase + kPCol;
@@ -567,7 +573,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     tc::fence_after();
 
     bool failed = false;
-    if (warp == 12 || warp == 13) {
+    if (warp == kProdK || warp == kProdV) {
         // ---------------- producers
         if (is_producer) {
             for (int j = nst; j < ntiles; ++j) {
@@ -581,9 +587,9 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             for (int k = issued > nst ? issued - nst : 0; k < issued; ++k)
                 mbar_wait_bounded(&full[k % nst], (k / nst) & 1, kWaitLimitNs);
         }
-    } else if (warp == 8 || warp == 9) {
+    } else if (warp >= kSIss && warp < kSIss + QT) {
         // ---------------- S = Q K^T issue (lane 0), one warp per query tile
-        const int q = warp - 8;
+        const int q = warp - kSIss;
         if (lane == 0) {
             const uint32_t idesc_s = tc::instr_desc<T>(kKeys, false);
             const uint32_t k_ring = smem_u32(smem + Sm::kKOff);
@@ -615,10 +621,10 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             tc::commit(&drain[q]);
             mbar_wait_bounded(&drain[q], 0, kWaitLimitNs);
         }
-    } else if (warp == 10 || warp == 11) {
+    } else if (warp >= kPVIss && warp < kPVIss + QT) {
         // ---------------- O += P V issue (lane 0), one warp per query tile; each warp
         //                  zeroes V rows past the context (the same zeros: harmless twice)
-        const int q = warp - 10;
+        const int q = warp - kPVIss;
         const uint32_t idesc_o = tc::instr_desc<T>(D, true);
         const uint32_t v_ring = smem_u32(smem + Sm::kVOff);
         int id_n = lane_id(0);
@@ -671,8 +677,8 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
             if (lane == 0) tc::commit(&v_empty[vst]);
         }
         if (lane == 0) {
-            tc::commit(&drain[2 + q]);
-            mbar_wait_bounded(&drain[2 + q], 0, kWaitLimitNs);
+            tc::commit(&drain[QT + q]);
+            mbar_wait_bounded(&drain[QT + q], 0, kWaitLimitNs);
         }
         __syncwarp();
     } else if (softmax_warp) {
@@ -858,7 +864,7 @@ __global__ void __launch_bounds__(448, 1) pa_prefill_tc_kernel(const __grid_cons
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kSIss) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
     }
     prefix_finish(false);
