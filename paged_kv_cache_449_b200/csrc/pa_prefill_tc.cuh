@@ -217,6 +217,9 @@ struct PrefillTcSmem {
     static constexpr int kTotal = kMiscOff + 16;
     static_assert(kTotal <= (QT == 2 ? 232448 : 115712), "shared memory per CTA");
     static_assert(kKStages <= 6, "barrier slots");
+    // the barrier set-up and both producers index the K and V rings with one
+    // stage count
+    static_assert(kVStages == kKStages, "K and V rings of one depth");
 };
 
 // Bounded mbarrier wait that also gives up when another role of the CTA has
