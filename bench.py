@@ -150,13 +150,13 @@ NCU_TRAFFIC = {
         ("llama3_8b_decode_bf16+e4m3", "append"): 146.823e6 + 3.909e6,
         ("llama3_70b_long_bf16+e4m3", "splitk"): 1.260385e9 + 6.494e6,
     },
-    "e3b791ccb47c4530": {
+    "507e69b3acbb29e4": {
         ("chunked_prefill_bfloat16", "prefill"): 118.626e6 + 19.744e6,
         ("chunked_prefill_bfloat16_B8", "prefill"): 118.361e6 + 20.244e6,
         ("chunked_prefill_bfloat16_B32", "prefill"): 118.734e6 + 20.894e6,
     },
     # the shared-prefix step: its prefix pass plus its decode pass
-    "b83eb7e217d369ee": {
+    "83e5129f3fabb696": {
         ("prefix_sharing_f16_p1024", "shared_prefix"): 5.319e6 + 0.0 + 153.313e6 + 0.180e6,
     },
 }
