@@ -117,6 +117,10 @@ def cuda_runtime():
         fn = lib.cudaMemcpyAsync
         fn.restype = ctypes.c_int
         fn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+        lib.cudaEventRecord.restype = ctypes.c_int
+        lib.cudaEventRecord.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        lib.cudaStreamWaitEvent.restype = ctypes.c_int
+        lib.cudaStreamWaitEvent.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
         return lib
     return None
 
@@ -585,27 +589,42 @@ def run_gpu(args, world, rank, local):
             up = [torch.cuda.Event() for _ in range(n)]
             done = [torch.cuda.Event() for _ in range(n)]
             down = [torch.cuda.Event() for _ in range(n)]
+            for e in up + done + down:   # created (on first record) before the timed region
+                e.record(stream)
+            torch.cuda.synchronize()
+            if cudart is not None:   # the runtime's own calls on the raw handles: a few us of host time less a step
+                def rec(e, s_):
+                    rcs.append(cudart.cudaEventRecord(e.cuda_event, s_.cuda_stream))
+
+                def wait(s_, e):
+                    rcs.append(cudart.cudaStreamWaitEvent(s_.cuda_stream, e.cuda_event, 0))
+            else:
+                def rec(e, s_):
+                    e.record(s_)
+
+                def wait(s_, e):
+                    s_.wait_event(e)
             up_s.wait_stream(stream)
             down_s.wait_stream(stream)
             ev0.record(up_s)
             upload(steps[0], up_s)
-            up[0].record(up_s)
+            rec(up[0], up_s)
             for i in range(n):
                 st = steps[i % R]
-                stream.wait_event(up[i])
+                wait(stream, up[i])
                 if i - R >= 0:
-                    stream.wait_event(down[i - R])
+                    wait(stream, down[i - R])
                 st.reshape(stream)
                 st.decode(stream)
-                done[i].record(stream)
+                rec(done[i], stream)
                 if i + 1 < n:
                     if i + 1 - R >= 0:
-                        up_s.wait_event(done[i + 1 - R])
+                        wait(up_s, done[i + 1 - R])
                     upload(steps[(i + 1) % R], up_s)
-                    up[i + 1].record(up_s)
-                down_s.wait_event(done[i])
+                    rec(up[i + 1], up_s)
+                wait(down_s, done[i])
                 download(st, i, down_s)
-                down[i].record(down_s)
+                rec(down[i], down_s)
             stream.wait_stream(up_s)
             stream.wait_stream(down_s)
             ev1.record(stream)
@@ -652,7 +671,8 @@ def run_gpu(args, world, rank, local):
                "how": ("step i+1's inputs uploaded on a copy stream while step i computes; step i's output "
                        "read back on another copy stream when its kernels end" if "pipelined" in e2e_modes
                        else "upload, step, read-back serialised on one stream")
-                      + ("; copies by cudaMemcpyAsync, the step by its prepared C-ABI call" if cudart is not None
+                      + ("; copies and event records / waits by the CUDA runtime's own calls, the step by its "
+                         "prepared C-ABI call" if cudart is not None
                          else "; copies by torch tensor copies, the step by its prepared C-ABI call"),
                "serial_ms_per_step": e2e_serial_ms_max}
 
