@@ -276,7 +276,10 @@ class Prepared:
     def __init__(self, name, args, device, tensors):
         self._fn = getattr(load(), name)
         self._name = name
-        self._args = tuple(args)
+        # each argument already of its ctypes type, so a call converts nothing
+        # but the stream
+        types = self._fn.argtypes[:len(args)]
+        self._args = tuple(a if isinstance(a, t) else t(a) for a, t in zip(args, types))
         self._device = device.index
         self._tensors = tensors
 
