@@ -157,3 +157,59 @@ def test_graph_replay_shared_prefix():
     assert int(counters[0].abs().sum()) == 0 and int(counters[1].abs().sum()) == 0   # left at zero
     assert pa.pa_get_device_error() == 0
     del g
+
+
+def test_graph_replay_of_a_block_manager_step():
+    """A serving step of three launches -- pa_blocks_append, pa_copy_blocks,
+    pa_decode_append, each a programmatic dependent launch of the one before --
+    captured once and replayed: after the same number of steps the block
+    manager's state, the pools and the output are bit-identical to an eager
+    twin's."""
+    b = workloads.llama3_8b_decode(seed=34, device="cuda", num_seqs=16, num_blocks=2048)
+    B, N, S = b.block_size, b.num_blocks, b.num_seqs
+    mb = b.max_blocks_per_seq + 2
+    lens0 = (b.context_lens - 1).to(torch.int64)
+
+    def state():
+        tables = torch.full((S, mb), -1, dtype=torch.int32)
+        ref = torch.zeros(N, dtype=torch.int32)
+        for s in range(S):
+            n = int((lens0[s] + B - 1) // B)
+            tables[s, :n] = b.block_tables[s, :n]
+            ref[b.block_tables[s, :n].long()] = 1
+        free = torch.nonzero(ref == 0).flatten().to(torch.int32)
+        ring = torch.full((N,), -1, dtype=torch.int32)
+        ring[:free.numel()] = free
+        return dict(tables=tables.cuda(), lens=lens0.to(torch.int32).cuda(), ref=ref.cuda(), ring=ring.cuda(),
+                    state=torch.tensor([0, free.numel()], dtype=torch.int64, device="cuda"),
+                    ones=torch.ones(S, dtype=torch.int32, device="cuda"),
+                    slots=torch.empty(S, dtype=torch.int64, device="cuda"),
+                    pairs=torch.empty((S, 2), dtype=torch.int64, device="cuda"),
+                    k=b.k_cache.cuda().clone(), v=b.v_cache.cuda().clone(), q=b.q.cuda(),
+                    nk=b.new_key.cuda(), nv=b.new_value.cuda(), out=torch.empty_like(b.q.cuda()))
+
+    def step(d):
+        pa.pa_blocks_append(d["tables"], d["lens"], d["ones"], d["ref"], d["ring"], d["state"], d["slots"],
+                            d["pairs"], B)
+        pa.pa_copy_blocks(d["k"], d["v"], d["k"], d["v"], d["pairs"])
+        pa.pa_decode_append(d["out"], d["q"], d["nk"], d["nv"], d["k"], d["v"], d["tables"], d["lens"], b.scale,
+                            max_context_len=mb * B, ref_counts=d["ref"])
+
+    eager, graphed = state(), state()
+    pa.pa_get_device_error()
+    step(graphed)                      # the uncaptured first step
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(graphed)
+    step(eager)
+    for _ in range(2):
+        step(eager)
+        g.replay()
+    torch.cuda.synchronize()
+    for key in ("tables", "lens", "ref", "ring", "state", "slots", "pairs"):
+        assert torch.equal(graphed[key], eager[key]), key
+    assert torch.equal(_bits(graphed["out"]), _bits(eager["out"]))
+    assert torch.equal(_bits(graphed["k"]), _bits(eager["k"])) and torch.equal(_bits(graphed["v"]), _bits(eager["v"]))
+    assert pa.pa_get_device_error() == 0
+    del g
